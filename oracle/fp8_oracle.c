@@ -247,7 +247,13 @@ int orc_compute_scale_mu(double amax, int fmt, int margin, double mu, double *to
 {
     double s_g;
     int rc = orc_compute_scale(mu * amax, fmt, margin, &s_g);
-    *total_scale = mu * s_g;
+    /* reading: the combined multiplier is itself kept a normal binary32 */
+    double t = mu * s_g;
+    if (t < ldexp(1.0, -126))
+        t = ldexp(1.0, -126);
+    if (t > ldexp(1.0, 126))
+        t = ldexp(1.0, 126);
+    *total_scale = t;
     return rc;
 }
 

@@ -22,7 +22,7 @@ MUTATIONS = {
     "f16_bias": ("ldexp((double)(1024 + Mt), E - 25)", "ldexp((double)(1024 + Mt), E - 24)"),
     "floor_at_tie": ("return (a <= f) ? (r - p) : (r - p - 1);", "return (a < f) ? (r - p) : (r - p - 1);"),
     "margin_sign": ("orc_fmt_max(fmt)) - margin;", "orc_fmt_max(fmt)) + margin;"),
-    "mu_dropped": ("*total_scale = mu * s_g;", "*total_scale = s_g;"),
+    "mu_dropped": ("double t = mu * s_g;", "double t = s_g;"),
     "gemm_transposed_b": ("orc_fp8_decode(fb, B[j * b_sj + k * b_sk])", "orc_fp8_decode(fb, B[k * b_sj + j * b_sk])"),
     "gemm_descale_dropped": ("C[ij] = s * inv_sa * inv_sb", "C[ij] = s * inv_sa"),
     "adam_bias_correction_dropped": ("double mhat = m[i] / bc1;", "double mhat = m[i];"),

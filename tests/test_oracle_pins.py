@@ -214,6 +214,8 @@ def test_scale_closed_forms():
     # clamping keeps s and 1/s normal binary32
     assert oracle.compute_scale(1e-45, E4, 0) == (0, 2.0 ** 126)
     assert oracle.compute_scale(1e38, E4, 10) == (0, 2.0 ** -126)
+    # total multiplier mu * s_g = 2^103 * 2^32 is clamped to 2^126 as well
+    assert oracle.compute_scale(1e-38, E4, 0, mu=2.0 ** 32) == (0, 2.0 ** 126)
 
 
 def test_scale_rule_brute_force():
@@ -245,6 +247,7 @@ def test_scale_invariants_and_mu():
                 if margin == 0:
                     assert a * s > mx / 2
             # mu invariance for powers of two: the total scale does not depend on mu
+            # (the combined multiplier is clamped to normal binary32 like any scale)
             base = oracle.compute_scale(a, fmt, 0, mu=1.0)[1]
             for mu in (2.0 ** 10, 2.0 ** -4, 2.0 ** 3):
                 assert oracle.compute_scale(a, fmt, 0, mu=mu)[1] == base
