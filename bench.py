@@ -1,0 +1,428 @@
+"""Benchmark of the FP8 mixed-precision training hot path on B200.
+
+One step = one pass of the whole path over one batch of the GPT-7B
+transformer block's four linears (tokens 4096 = batch 2 x seq 2048, hidden
+4096: QKV 4096->12288, out-proj 4096->4096, FFN 4096->16384->4096):
+
+  for each linear:  amax/scale/cast X (E4M3), W (E4M3), dY (E5M2, mu-scaled)
+                    fwd   Y  = Xq Wq^T     (bf16 out, fused amax)
+                    dgrad dX = dYq Wq      (bf16 out, fused amax)
+                    wgrad dW = dYq^T Xq    (fp32 out, fused amax)
+                    grad  gq = E5M2(mu s_g dW)
+  then one precision-decoupled FP8 Adam step over the 4 weight tensors
+  (201,326,592 parameters: E5M2 grad, E4M3 m1, FP16 m2, FP16 master).
+
+`value` is the step's algorithmic GEMM work (3 x 2MNK per linear, 4.948
+TFLOP) divided by the device time of the whole step, inputs resident in HBM.
+Inputs are seeded synthetic tensors (bf16 activations ~N(0,1), weights
+~N(0,0.02), output gradients ~N(0,1e-4)); every step touches several GB, far
+more than the 126 MB L2, so no explicit L2 flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from fp8_mixed_precision_tensor_b200 import synth  # noqa: E402
+
+METRIC = "FP8 linear fwd+bwd TFLOP/s (% FP8 peak); cast & Adam GB/s (% HBM peak)"
+WORKLOAD = "gpt7b_block_linears_fp8_train_step"
+MU = 2.0 ** 10
+HP = dict(lr=1e-4, beta1=0.9, beta2=0.95, eps=1e-8)
+# Algorithmic bytes per element / parameter (reads + writes of the definition).
+CAST_BYTES_BF16 = 2 + 2 + 1   # amax read + cast read + code write
+GRAD_CAST_BYTES = 4 + 1       # fp32 dW read (amax fused in the GEMM) + code write
+ADAM_BYTES = 11               # read g1 m1 v2 w2, write m1 v2 w2
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        p = json.load(open(path))
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sus=p["bf16_tflops_sustained"],
+                    src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.samples, self.reasons = [], set()
+        self.period = period_s
+        self.stop_ev = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        names = {
+            getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8): "hw_slowdown",
+            getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40): "hw_thermal_slowdown",
+            getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20): "sw_thermal_slowdown",
+            getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4): "sw_power_cap",
+            0x80: "hw_power_brake_slowdown",
+        }
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in names.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self.stop_ev.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- the step
+class Block7BStep:
+    """Device buffers and the launch sequence of one training step."""
+
+    def __init__(self, device, seed: int = 0, linears=None, tokens=None, w_std=None):
+        from fp8_mixed_precision_tensor_b200 import fp8
+
+        self.fp8 = fp8
+        self.dev = device
+        self.linears = linears or synth.GPT7B_LINEARS
+        self.M = tokens or synth.GPT7B_TOKENS
+        w_std = w_std or synth.GPT7B_W_STD
+        f32 = dict(dtype=torch.float32, device=device)
+        u8 = dict(dtype=torch.uint8, device=device)
+        self.L = []
+        for li, (name, K, N) in enumerate(self.linears):
+            M = self.M
+            d = dict(name=name, M=M, N=N, K=K)
+            d["X"] = synth.device_normal((M, K), synth.ACT_STD, seed * 1000 + 10 * li + 1, torch.bfloat16, device)
+            d["W"] = synth.device_normal((N, K), w_std, seed * 1000 + 10 * li + 2, torch.bfloat16, device)
+            d["dY"] = synth.device_normal((M, N), synth.GRAD_STD, seed * 1000 + 10 * li + 3, torch.bfloat16, device)
+            d["xq"], d["wq"], d["dyq"] = (torch.empty(s, **u8) for s in ((M, K), (N, K), (M, N)))
+            d["y"] = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+            d["dx"] = torch.empty((M, K), dtype=torch.bfloat16, device=device)
+            d["dw"] = torch.empty((N, K), **f32)
+            d["gq"] = torch.empty((N, K), **u8)
+            # scalars: amax, scale, inv for x, w, dy, g; fused amaxes of y, dx, dw
+            d["sc"] = torch.zeros(16, **f32)
+            # Adam state: master from W (tensor-scaled FP16), zero moments
+            d["m"] = torch.zeros((N, K), **u8)
+            d["v"] = torch.zeros((N, K), dtype=torch.int16, device=device)
+            d["wh"] = torch.empty((N, K), dtype=torch.int16, device=device)
+            d["st"] = torch.ones(4, **f32)  # m_scale, v_scale, w_scale, spare
+            tmp = torch.zeros(3, **f32)
+            fp8.fp8_amax(d["W"], tmp[0:1])
+            fp8.fp8_compute_scale(tmp[0:1], fp8.FP8_F16S, 0, 1.0, d["st"][2:3], tmp[1:2])
+            fp8.fp8_cast(d["W"], fp8.FP8_F16S, d["st"][2:3], d["wh"])
+            self.L.append(d)
+        self.chunks = fp8.pack_adam_chunks([
+            fp8.AdamChunk(d["gq"], d["sc"][11:12], d["m"], d["st"][0:1], d["v"], d["st"][1:2], d["wh"],
+                          d["st"][2:3]) for d in self.L])
+        self.ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(self.L)) // 4 + 64, **f32)
+        self.t = 0
+        self.flops = sum(3 * 2 * d["M"] * d["N"] * d["K"] for d in self.L)
+        self.cast_elems = sum(d["M"] * d["K"] + d["N"] * d["K"] + d["M"] * d["N"] for d in self.L)
+        self.params = sum(d["N"] * d["K"] for d in self.L)
+        self.launches_per_step = 4 * (3 * 3 + 3 + 2) + 3  # amax/scale/cast x3, GEMMs, grad scale+cast; Adam
+
+    def quantise(self, x, fmt, sc, i, mu=1.0, out=None):
+        fp8 = self.fp8
+        fp8.fp8_amax(x, sc[i:i + 1])
+        fp8.fp8_compute_scale(sc[i:i + 1], fmt, 0, mu, sc[i + 1:i + 2], sc[i + 2:i + 3])
+        fp8.fp8_cast(x, fmt, sc[i + 1:i + 2], out)
+
+    def step(self, ev=None):
+        """Enqueue one step.  ev: optional dict name -> list of (start, end)
+        events recorded around the GEMM / cast / Adam launches."""
+        fp8 = self.fp8
+
+        def mark(kind):
+            if ev is None:
+                return None
+            e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            e[0].record()
+            ev.setdefault(kind, []).append(e)
+            return e
+
+        for d in self.L:
+            sc = d["sc"]
+            e = mark("cast")
+            self.quantise(d["X"], fp8.FP8_E4M3, sc, 0, out=d["xq"])
+            self.quantise(d["W"], fp8.FP8_E4M3, sc, 3, out=d["wq"])
+            self.quantise(d["dY"], fp8.FP8_E5M2, sc, 6, mu=MU, out=d["dyq"])
+            if e: e[1].record()
+            e = mark("gemm")
+            fp8.fp8_linear_fwd(d["xq"], sc[2:3], d["wq"], sc[5:6], d["y"], sc[12:13])
+            fp8.fp8_linear_dgrad(d["dyq"], sc[8:9], d["wq"], sc[5:6], d["dx"], sc[13:14])
+            fp8.fp8_linear_wgrad(d["dyq"], sc[8:9], d["xq"], sc[2:3], d["dw"], sc[14:15])
+            if e: e[1].record()
+            e = mark("grad_cast")
+            fp8.fp8_compute_scale(sc[14:15], fp8.FP8_E5M2, 0, MU, sc[10:11], sc[11:12])
+            fp8.fp8_cast(d["dw"], fp8.FP8_E5M2, sc[10:11], d["gq"])
+            if e: e[1].record()
+        self.t += 1
+        e = mark("adam")
+        fp8.fp8_adam_step(self.chunks, step=self.t, margin=0, workspace=self.ws, **HP)
+        if e: e[1].record()
+
+    def result_scalars(self):
+        return torch.cat([d["sc"] for d in self.L] + [d["st"] for d in self.L])
+
+
+def timed_steps(runner, steps, ev=None):
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        runner.step(ev)
+    end.record()
+    end.synchronize()
+    return start.elapsed_time(end)
+
+
+def sum_events(ev, kind):
+    return sum(a.elapsed_time(b) for a, b in ev.get(kind, []))
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+def oracle_step_estimate(budget_s: float = 12.0):
+    """Times the CPU oracle on bounded samples of one step's work and
+    extrapolates to a full step (seconds).  Returns (seconds, cores, sample text)."""
+    import oracle
+
+    cores = oracle.num_threads()
+    t_total = 0.0
+    parts = []
+    rows = 4
+    for name, K, N in synth.GPT7B_LINEARS:
+        M = synth.GPT7B_TOKENS
+        g = synth.rng("bench-oracle", name)
+        # codes for a row block: fwd uses rows of X, dgrad rows of dY, wgrad rows of dW (cols of dY)
+        xq = g.integers(0, 0x7E, (rows, K), dtype=np.uint8)
+        wq = g.integers(0, 0x7E, (N, K), dtype=np.uint8)
+        t0 = time.perf_counter()
+        oracle.linear_fwd(xq, 1.0, wq, 1.0, rows, N, K)
+        t_fwd = (time.perf_counter() - t0) * M / rows
+        # dgrad and wgrad have the same MNK product: scale the fwd row-block rate
+        t_total += 3 * t_fwd
+        parts.append(f"{name}: {rows}x{N}x{K} fwd row block")
+    n = 1 << 21
+    xb = synth.normal_bf16((n,), 1.0, "bench-oracle", "cast")
+    t0 = time.perf_counter()
+    a = oracle.amax(xb, oracle.DT_BF16, parallel=True)
+    _, s = oracle.compute_scale(a, oracle.E4M3, 0)
+    oracle.cast(xb, oracle.E4M3, s, oracle.DT_BF16)
+    t_cast = (time.perf_counter() - t0) / n
+    elems = sum(synth.GPT7B_TOKENS * K + N * K + synth.GPT7B_TOKENS * N for _, K, N in synth.GPT7B_LINEARS)
+    params = sum(N * K for _, K, N in synth.GPT7B_LINEARS)
+    t_total += t_cast * (elems + params)  # activation/weight/grad casts + gradient cast
+    na = 1 << 20
+    gq = np.random.default_rng(0).integers(0, 0x7B, na, dtype=np.uint8)
+    w = np.full(na, 0x2C00, np.uint16)
+    t0 = time.perf_counter()
+    oracle.adam_step(gq, 1e-6, np.zeros(na, np.uint8), 1.0, np.zeros(na, np.uint16), 1.0, w, 1.0,
+                     t=1, margin=0, **HP)
+    t_adam = (time.perf_counter() - t0) / na
+    t_total += t_adam * params
+    sample = (f"oracle timed on: {'; '.join(parts)}; amax+scale+cast of 2^21 bf16; Adam on 2^20 params; "
+              f"extrapolated to the full step by units")
+    return t_total, cores, sample
+
+
+# ---------------------------------------------------------------- arms
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    vals = []
+    t_all = []
+    for i in range(args.warmup + args.steps):
+        t, cores, sample = oracle_step_estimate()
+        if i >= args.warmup:
+            t_all.append(t)
+    t = statistics.median(t_all)
+    flops = sum(3 * 2 * synth.GPT7B_TOKENS * N * K for _, K, N in synth.GPT7B_LINEARS)
+    v = flops / t / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "tokens": synth.GPT7B_TOKENS, "hidden": 4096,
+                       "linears": [l[0] for l in synth.GPT7B_LINEARS], "adam_params": 201326592},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_gpu(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    from fp8_mixed_precision_tensor_b200 import fp8
+
+    peaks = load_peaks()
+    runner = Block7BStep(dev, seed=rank)
+    for _ in range(args.warmup):
+        runner.step()
+    barrier()
+
+    # ---- device-timed region: inputs resident, whole step
+    sampler = ClockSampler(local)
+    with sampler:
+        barrier()
+        ms = timed_steps(runner, args.steps)
+        barrier()
+    ms_step = ms / args.steps
+    if dist is not None:
+        t = torch.tensor([ms_step], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = t.item()
+    status = fp8.fp8_get_status()
+
+    # ---- per-kernel breakdown (separate pass with events between phases)
+    ev = {}
+    timed_steps(runner, args.steps, ev)
+    t_gemm = sum_events(ev, "gemm") / args.steps
+    t_cast = sum_events(ev, "cast") / args.steps
+    t_gcast = sum_events(ev, "grad_cast") / args.steps
+    t_adam = sum_events(ev, "adam") / args.steps
+
+    # ---- end to end: host inputs (pinned) copied in, result scalars read back
+    host_in = [(d["X"].cpu().pin_memory(), d["dY"].cpu().pin_memory()) for d in runner.L]
+    res = torch.empty(runner.result_scalars().numel(), dtype=torch.float32).pin_memory()
+    h2d = sum(x.numel() * x.element_size() + y.numel() * y.element_size() for x, y in host_in)
+    d2h = res.numel() * 4
+
+    def e2e_step():
+        for d, (x, y) in zip(runner.L, host_in):
+            d["X"].copy_(x, non_blocking=True)
+            d["dY"].copy_(y, non_blocking=True)
+        runner.step()
+        res.copy_(runner.result_scalars(), non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    s1.record()
+    s1.synchronize()
+    e2e_ms = s0.elapsed_time(s1) / args.steps
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+
+    value = runner.flops * world / (ms_step * 1e-3) / 1e12
+    fp8_peak = 2.0 * peaks["bf16_sus"]  # FP8 dense = 2 x bf16 dense (nominal ratio), sustained
+    gemm_tflops = runner.flops / (t_gemm * 1e-3) / 1e12
+    cast_gbs = runner.cast_elems * CAST_BYTES_BF16 / (t_cast * 1e-3) / 1e9
+    gcast_gbs = runner.params * GRAD_CAST_BYTES / (t_gcast * 1e-3) / 1e9
+    adam_gbs = runner.params * ADAM_BYTES / (t_adam * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8(e4m3/e5m2)->f32 accum; f32 elementwise", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tokens": runner.M, "hidden": 4096,
+                   "linears": [d["name"] for d in runner.L], "adam_params": runner.params,
+                   "gemm_flops_per_step": runner.flops, "l2": "inputs larger than L2 (no flush)",
+                   "parallelism": f"replicas{world}" if world > 1 else "single"},
+        "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
+                     "frac": gemm_tflops / fp8_peak, "traffic": None,
+                     "kernel": "k_gemm (fwd+dgrad+wgrad, flop-weighted over the 12 launches)",
+                     "peak_src": f"2 x bf16_tflops_sustained ({peaks['src']})"},
+        "kernels": {
+            "gemm": {"ms": t_gemm, "TFLOP/s": gemm_tflops, "frac_fp8_peak": gemm_tflops / fp8_peak},
+            "amax_scale_cast": {"ms": t_cast, "GB/s": cast_gbs, "frac_hbm": cast_gbs / peaks["hbm"]},
+            "grad_cast": {"ms": t_gcast, "GB/s": gcast_gbs, "frac_hbm": gcast_gbs / peaks["hbm"]},
+            "adam": {"ms": t_adam, "GB/s": adam_gbs, "frac_hbm": adam_gbs / peaks["hbm"],
+                     "bytes_per_param_algorithmic": ADAM_BYTES},
+        },
+        "e2e": {"value": runner.flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": runner.launches_per_step * args.steps,
+        "clocks": sampler.summary(),
+        "device_status": status,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t_cpu, cores, sample = oracle_step_estimate()
+        line["cpu_baseline"] = {"value": runner.flops / t_cpu / 1e12, "unit": "TFLOP/s", "cores": cores,
+                                "kind": "oracle", "sample": sample}
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

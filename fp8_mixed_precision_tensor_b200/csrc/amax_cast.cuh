@@ -1,0 +1,186 @@
+// amax_cast.cuh -- per-tensor amax, scale and cast kernels (HBM-bound).
+//
+// "Training and inference of large language models using 8-bit floating
+// point", 제안 방법: the scaling bias of every weight, activation and gradient
+// tensor comes from its maximum absolute value; the tensor is scaled and then
+// cast to FP8.  "FP8-LM: Training FP8 Large Language Models", 提案手法 O1,
+// Eq. 3: gradients are auto-scaled by mu before the cast.
+//
+// Design: grid-stride streaming kernels over 16-byte vectors with several
+// independent loads in flight per thread; amax reduces |x| as integer bit
+// patterns (warp redux -> block -> one atomicMax per block); the cast reads
+// its scale from device memory so amax -> scale -> cast chains with no host
+// round-trip.
+#pragma once
+
+#include "common.cuh"
+
+namespace fp8lib {
+
+constexpr int kStreamThreads = 256;
+
+// 16 elements of a high-precision tensor as floats.
+template <int DT>
+struct Vec16 {
+  static constexpr int kBytes = DT == FP8_DT_F32 ? 64 : 32;
+};
+
+template <int DT>
+__device__ __forceinline__ void load16(const void *base, size_t group, float (&f)[16]) {
+  if constexpr (DT == FP8_DT_F32) {
+    const uint4 *p = reinterpret_cast<const uint4 *>(base) + group * 4;
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      uint4 v = __ldcs(p + j);
+      f[4 * j + 0] = __uint_as_float(v.x);
+      f[4 * j + 1] = __uint_as_float(v.y);
+      f[4 * j + 2] = __uint_as_float(v.z);
+      f[4 * j + 3] = __uint_as_float(v.w);
+    }
+  } else {
+    const uint4 *p = reinterpret_cast<const uint4 *>(base) + group * 2;
+#pragma unroll
+    for (int j = 0; j < 2; j++) {
+      uint4 v = __ldcs(p + j);
+      uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; k++) {
+        if constexpr (DT == FP8_DT_BF16) {
+          f[8 * j + 2 * k] = __uint_as_float(w[k] << 16);
+          f[8 * j + 2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+        } else {
+          float2 t = h2f2(w[k]);
+          f[8 * j + 2 * k] = t.x;
+          f[8 * j + 2 * k + 1] = t.y;
+        }
+      }
+    }
+  }
+}
+
+template <int DT>
+__device__ __forceinline__ float load1(const void *base, size_t i) {
+  if constexpr (DT == FP8_DT_F32) return reinterpret_cast<const float *>(base)[i];
+  uint32_t h = reinterpret_cast<const uint16_t *>(base)[i];
+  if constexpr (DT == FP8_DT_BF16) return __uint_as_float(h << 16);
+  return __half2float(__ushort_as_half((unsigned short)h));
+}
+
+// ---------------------------------------------------------------------------
+// amax.  Magnitudes are compared as unsigned bit patterns: for bf16 and f32
+// that is the raw |bits|; fp16 halves are widened to f32 first.
+template <int DT>
+__device__ __forceinline__ uint32_t group_absmax(const void *base, size_t group) {
+  if constexpr (DT == FP8_DT_BF16) {
+    // 16 bf16 = 2 x uint4; SIMD max over 16-bit halves of |bits|.
+    const uint4 *p = reinterpret_cast<const uint4 *>(base) + group * 2;
+    uint4 a = __ldcg(p), b = __ldcg(p + 1);
+    uint32_t m = __vmaxu2(__vmaxu2(a.x & 0x7fff7fffu, a.y & 0x7fff7fffu),
+                          __vmaxu2(a.z & 0x7fff7fffu, a.w & 0x7fff7fffu));
+    m = __vmaxu2(m, __vmaxu2(__vmaxu2(b.x & 0x7fff7fffu, b.y & 0x7fff7fffu),
+                             __vmaxu2(b.z & 0x7fff7fffu, b.w & 0x7fff7fffu)));
+    uint32_t hi = m >> 16, lo = m & 0xffffu;
+    return (hi > lo ? hi : lo) << 16;  // bf16 -> f32 bits
+  } else if constexpr (DT == FP8_DT_F32) {
+    const uint4 *p = reinterpret_cast<const uint4 *>(base) + group * 4;
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      uint4 v = __ldcg(p + j);
+      m = max(m, max(max(v.x & 0x7fffffffu, v.y & 0x7fffffffu), max(v.z & 0x7fffffffu, v.w & 0x7fffffffu)));
+    }
+    return m;
+  } else {
+    const uint4 *p = reinterpret_cast<const uint4 *>(base) + group * 2;
+    uint4 a = __ldcg(p), b = __ldcg(p + 1);
+    uint32_t m = __vmaxu2(__vmaxu2(a.x & 0x7fff7fffu, a.y & 0x7fff7fffu),
+                          __vmaxu2(a.z & 0x7fff7fffu, a.w & 0x7fff7fffu));
+    m = __vmaxu2(m, __vmaxu2(__vmaxu2(b.x & 0x7fff7fffu, b.y & 0x7fff7fffu),
+                             __vmaxu2(b.z & 0x7fff7fffu, b.w & 0x7fff7fffu)));
+    uint32_t hi = m >> 16, lo = m & 0xffffu;
+    uint32_t h = hi > lo ? hi : lo;  // largest |half| bits (NaN above inf)
+    return absbits_f32(__half2float(__ushort_as_half((unsigned short)h)));
+  }
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kStreamThreads) k_amax(const void *__restrict__ x, size_t n,
+                                                         float *__restrict__ amax) {
+  __shared__ uint32_t red[32];
+  const size_t groups = n / 16;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+  for (; g + 3 * stride < groups; g += 4 * stride) {
+    m0 = max(m0, group_absmax<DT>(x, g));
+    m1 = max(m1, group_absmax<DT>(x, g + stride));
+    m2 = max(m2, group_absmax<DT>(x, g + 2 * stride));
+    m3 = max(m3, group_absmax<DT>(x, g + 3 * stride));
+  }
+  for (; g < groups; g += stride) m0 = max(m0, group_absmax<DT>(x, g));
+  uint32_t m = max(max(m0, m1), max(m2, m3));
+  if (blockIdx.x == 0) {  // ragged tail (< 16 elements)
+    for (size_t i = groups * 16 + threadIdx.x; i < n; i += blockDim.x)
+      m = max(m, absbits_f32(load1<DT>(x, i)));
+  }
+  m = block_max_u32(m, red);
+  if (threadIdx.x == 0) atomic_max_bits(amax, m);
+}
+
+// ---------------------------------------------------------------------------
+// scale: one thread.
+__global__ void k_compute_scale(const float *__restrict__ amax, float fmax, int margin, int log2mu,
+                                float *__restrict__ scale, float *__restrict__ inv_scale) {
+  int k;
+  if (!scale_exponent(*amax, fmax, margin, log2mu, k)) atomicOr(&g_status, FP8_STATUS_NONFINITE);
+  *scale = pow2f(k);
+  *inv_scale = pow2f(-k);
+}
+
+// ---------------------------------------------------------------------------
+// cast: 16 elements per thread-iteration, one 16-byte store of codes
+// (or two of halves for the scaled-FP16 format).
+template <int DT, int FMT>
+__device__ __forceinline__ void cast_group(const void *x, size_t g, float s, void *q) {
+  float f[16];
+  load16<DT>(x, g, f);
+#pragma unroll
+  for (int j = 0; j < 16; j++) f[j] *= s;
+  if constexpr (FMT == FP8_F16S) {
+    uint4 lo = make_uint4(f16x2(f[0], f[1]), f16x2(f[2], f[3]), f16x2(f[4], f[5]), f16x2(f[6], f[7]));
+    uint4 hi = make_uint4(f16x2(f[8], f[9]), f16x2(f[10], f[11]), f16x2(f[12], f[13]), f16x2(f[14], f[15]));
+    uint4 *p = reinterpret_cast<uint4 *>(q) + g * 2;
+    __stcs(p, lo);
+    __stcs(p + 1, hi);
+  } else {
+    uint4 o = make_uint4(enc4<FMT>(f[0], f[1], f[2], f[3]), enc4<FMT>(f[4], f[5], f[6], f[7]),
+                         enc4<FMT>(f[8], f[9], f[10], f[11]), enc4<FMT>(f[12], f[13], f[14], f[15]));
+    __stcs(reinterpret_cast<uint4 *>(q) + g, o);
+  }
+}
+
+template <int DT, int FMT>
+__global__ void __launch_bounds__(kStreamThreads) k_cast(const void *__restrict__ x, size_t n,
+                                                         const float *__restrict__ scale,
+                                                         void *__restrict__ q) {
+  const float s = *scale;
+  const size_t groups = n / 16;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (; g + stride < groups; g += 2 * stride) {
+    cast_group<DT, FMT>(x, g, s, q);
+    cast_group<DT, FMT>(x, g + stride, s, q);
+  }
+  if (g < groups) cast_group<DT, FMT>(x, g, s, q);
+  if (blockIdx.x == 0) {
+    for (size_t i = groups * 16 + threadIdx.x; i < n; i += blockDim.x) {
+      float y = load1<DT>(x, i) * s;
+      if constexpr (FMT == FP8_F16S)
+        reinterpret_cast<uint16_t *>(q)[i] = __half_as_ushort(__float2half_rn(y));
+      else
+        reinterpret_cast<uint8_t *>(q)[i] = (uint8_t)(enc2<FMT>(y, 0.0f) & 0xffu);
+    }
+  }
+}
+
+}  // namespace fp8lib

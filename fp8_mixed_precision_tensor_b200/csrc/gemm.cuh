@@ -1,0 +1,433 @@
+// gemm.cuh -- FP8 x FP8 -> FP32 GEMM on the 5th-generation tensor cores
+// (tcgen05.mma kind::f8f6f4, accumulator in TMEM, operands staged by TMA).
+//
+// "Training and inference of large language models using 8-bit floating
+// point", 제안 방법: the linear layer multiplies FP8 operands (E4M3 weights
+// and activations, E5M2 gradients) and the per-tensor scaling is undone after
+// the matmul; "FP8-LM: Training FP8 Large Language Models", 新規性: FP8 in the
+// linear-layer GEMMs (forward, dgrad, wgrad).
+//
+// One kernel serves all three products.  The output is C[rows, cols] =
+// sum_k A(r, k) B(c, k), with each operand either K-major (the reduction
+// index is contiguous in memory) or MN-major (the output index is
+// contiguous): fwd reads X and W K-major; dgrad reads dY K-major and W
+// MN-major; wgrad reads dY and X MN-major.  No operand is ever transposed in
+// memory: the MN-major forms are legal tcgen05 operands for 8-bit types.
+//
+// Structure (one CTA per SM, persistent over output tiles of 128 x BN):
+//   warp 0      TMA producer: 128 x 128-byte tiles of A and BN x 128-byte
+//               tiles of B into a STAGES-deep shared-memory ring (128-byte
+//               swizzle), completion tracked by mbarriers.
+//   warp 1      allocates TMEM (two BN-column fp32 accumulators) and issues
+//               tcgen05.mma from one thread; tcgen05.commit frees ring slots
+//               and hands finished accumulators to the epilogue.
+//   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes, descale by the
+//               two inverse scales, + bias, round to the output type, store,
+//               and reduce the amax of the stored values (one atomicMax per
+//               warp and tile).  Double-buffered TMEM lets tile i's epilogue
+//               overlap tile i+1's MMAs.
+// Every mbarrier wait is bounded (wall clock, %globaltimer): on timeout the
+// kernel raises FP8_STATUS_TIMEOUT, lets in-flight copies and MMAs finish,
+// frees TMEM and returns.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace fp8lib {
+namespace gemm {
+
+constexpr int BM = 128;            // tile rows (TMEM lanes)
+constexpr int BK = 128;            // k per stage: 128 one-byte elements = one 128B swizzle row
+constexpr int UMMA_K = 32;         // k per tcgen05.mma for 8-bit inputs
+constexpr int kThreads = 192;      // 6 warps
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s: far above any legitimate wait
+
+template <int BN>
+struct Cfg {
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int A_BYTES = BM * BK;
+  static constexpr int B_BYTES = BN * BK;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;  // two accumulators
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
+};
+
+struct Args {
+  int rows, cols, K;           // output [rows, cols], reduction length K
+  int num_m_blocks, num_n_blocks, num_tiles, num_k_blocks;
+  uint32_t idesc;              // tcgen05 instruction descriptor
+  const float *inv_a, *inv_b;  // descale factors (device scalars)
+  const void *bias;            // [cols] or null
+  int bias_dtype;
+  void *out;                   // row-major [rows, cols]
+  int out_dtype;
+  float *out_amax;             // amax of the stored output (pre-zeroed) or null
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers.
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait on one phase of an mbarrier.  Returns false on timeout (after
+// raising the status bit and the CTA's abort flag) or when another role of
+// the CTA has already aborted.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kTimeoutNs) {
+        atomicOr(&g_status, FP8_STATUS_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// A wait used only while tearing down after an abort: bounded, no flag check.
+__device__ __noinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kTimeoutNs) return;
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 lanes x 32 consecutive fp32 columns: thread t of the warp gets row
+// (lane base + t), columns [col, col + 32).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), version 1.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Descriptor of the k-th 32-deep slice of an operand tile.
+//   K-major tile: rows of 128 bytes (the k extent), 8-row groups 1024 B apart;
+//     the slice starts 32 bytes further along each row.
+//   MN-major tile: 128-byte-wide columns of the MN extent (one per 128
+//     outputs), each holding BK rows of k; 8-row groups of k 1024 B apart,
+//     neighbouring 128-wide MN chunks BK*128 bytes apart; the slice starts
+//     32 rows (4096 B) further down.
+template <bool MN_MAJOR>
+__device__ __forceinline__ uint64_t operand_desc(uint32_t tile_base, int kslice) {
+  if constexpr (MN_MAJOR)
+    return smem_desc(tile_base + kslice * (UMMA_K * 128), BK * 128, 1024);
+  else
+    return smem_desc(tile_base + kslice * UMMA_K, 16, 1024);
+}
+
+__device__ __forceinline__ float load_bias(const void *bias, int dt, int c) {
+  if (dt == FP8_DT_F32) return reinterpret_cast<const float *>(bias)[c];
+  uint32_t h = reinterpret_cast<const uint16_t *>(bias)[c];
+  if (dt == FP8_DT_BF16) return __uint_as_float(h << 16);
+  return __half2float(__ushort_as_half((unsigned short)h));
+}
+
+// ---------------------------------------------------------------------------
+template <int BN, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+           const Args args) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;  // 1024-aligned for the 128B swizzle
+  uint8_t *base_ptr = smem_raw + (base - raw);
+  const uint32_t bar0 = base + C::STAGES * C::STAGE_BYTES;
+  // barrier layout: full[S], empty[S], tfull[2], tempty[2], drain, then tmem slot + abort flag
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 2 + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * C::STAGES + 4);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + C::STAGES * C::STAGE_BYTES + 8 * (2 * C::STAGES + 5));
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; s++) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; b++) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 4);  // one arrive per epilogue warp
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int stage = 0;
+    uint32_t phase = 0;
+    // parity of the last load issued into each stage (for the abort drain)
+    uint32_t issued_mask = 0, issued_par = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < args.num_tiles && ok; tile += gridDim.x) {
+      const int mb = tile % args.num_m_blocks, nb = tile / args.num_m_blocks;
+      for (int kb = 0; kb < args.num_k_blocks; kb++) {
+        bool got = lane == 0 ? mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag) : true;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) { ok = false; break; }
+        if (lane == 0) {
+          const uint32_t sa = base + stage * C::STAGE_BYTES, sb = sa + C::A_BYTES;
+          mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
+          if (A_MN) tma_load_2d(sa, &tmA, mb * BM, kb * BK, full_bar(stage));
+          else      tma_load_2d(sa, &tmA, kb * BK, mb * BM, full_bar(stage));
+          if (B_MN) {
+#pragma unroll
+            for (int h = 0; h < BN / 128; h++)
+              tma_load_2d(sb + h * (128 * BK), &tmB, nb * BN + h * 128, kb * BK, full_bar(stage));
+          } else {
+            tma_load_2d(sb, &tmB, kb * BK, nb * BN, full_bar(stage));
+          }
+          issued_mask |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        }
+        __syncwarp();
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (!ok && lane == 0) {
+      // let every issued copy land before the CTA can exit
+      for (int s = 0; s < C::STAGES; s++)
+        if (issued_mask & (1u << s)) mbar_wait_drain(full_bar(s), (issued_par >> s) & 1u);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true, issued_any = false;
+    for (int tile = blockIdx.x; tile < args.num_tiles && ok; tile += gridDim.x) {
+      bool got = lane == 0 ? mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag) : true;
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * BN;
+      for (int kb = 0; kb < args.num_k_blocks; kb++) {
+        got = lane == 0 ? mbar_wait(full_bar(stage), phase, abort_flag) : true;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) { ok = false; break; }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t sa = base + stage * C::STAGE_BYTES, sb = sa + C::A_BYTES;
+#pragma unroll
+          for (int ks = 0; ks < BK / UMMA_K; ks++) {
+            tc_mma(d_tmem, operand_desc<A_MN>(sa, ks), operand_desc<B_MN>(sb, ks), args.idesc,
+                   (kb | ks) != 0 ? 1u : 0u);
+          }
+          tc_commit(empty_bar(stage));  // ring slot free once these MMAs have read it
+          issued_any = true;
+        }
+        __syncwarp();
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      if (lane == 0) tc_commit(tfull_bar(acc));  // accumulator complete
+      __syncwarp();
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    if (!ok && lane == 0 && issued_any) {
+      tc_commit(drain_bar);  // arrives once every MMA issued so far has completed
+      mbar_wait_drain(drain_bar, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const float inv_a = *args.inv_a, inv_b = *args.inv_b;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x) {
+      const int mb = tile % args.num_m_blocks, nb = tile / args.num_m_blocks;
+      bool got = lane == 0 ? mbar_wait(tfull_bar(acc), acc_phase, abort_flag) : true;
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) break;
+      tc_fence_after();
+      const int row = mb * BM + q * 32 + lane;
+      const bool row_ok = row < args.rows;
+      uint32_t amax_bits = 0;
+#pragma unroll 1
+      for (int cc = 0; cc < BN / 32; cc++) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + cc * 32, r);
+        const int col0 = nb * BN + cc * 32;
+        float y[32];
+#pragma unroll
+        for (int j = 0; j < 32; j++) y[j] = __fmul_rn(__fmul_rn(__uint_as_float(r[j]), inv_a), inv_b);
+        if (args.bias != nullptr) {
+#pragma unroll
+          for (int j = 0; j < 32; j++)
+            if (col0 + j < args.cols) y[j] = __fadd_rn(y[j], load_bias(args.bias, args.bias_dtype, col0 + j));
+        }
+        if (args.out_dtype == FP8_DT_F32) {
+          float *orow = reinterpret_cast<float *>(args.out) + (size_t)row * args.cols;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            if (row_ok && col0 + j < args.cols) {
+              *reinterpret_cast<float4 *>(orow + col0 + j) = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
+              amax_bits = max(amax_bits, max(max(absbits_f32(y[j]), absbits_f32(y[j + 1])),
+                                             max(absbits_f32(y[j + 2]), absbits_f32(y[j + 3]))));
+            }
+          }
+        } else {
+          uint16_t *orow = reinterpret_cast<uint16_t *>(args.out) + (size_t)row * args.cols;
+          const bool bf = args.out_dtype == FP8_DT_BF16;
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            uint32_t p[4];
+            uint32_t mx = 0;
+#pragma unroll
+            for (int t = 0; t < 4; t++) {
+              uint32_t lo, hi;
+              if (bf) {
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(y[j + 2 * t], y[j + 2 * t + 1]);
+                p[t] = *reinterpret_cast<uint32_t *>(&h2);
+                lo = (p[t] & 0x7fffu) << 16;
+                hi = p[t] & 0x7fff0000u;
+              } else {
+                p[t] = f16x2(y[j + 2 * t], y[j + 2 * t + 1]);
+                float2 back = h2f2(p[t]);
+                lo = absbits_f32(back.x);
+                hi = absbits_f32(back.y);
+              }
+              mx = max(mx, max(lo, hi));
+            }
+            if (row_ok && col0 + j < args.cols) {
+              *reinterpret_cast<uint4 *>(orow + col0 + j) = make_uint4(p[0], p[1], p[2], p[3]);
+              amax_bits = max(amax_bits, mx);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if (args.out_amax != nullptr) {
+        amax_bits = warp_max_u32(amax_bits);
+        if (lane == 0) atomic_max_bits(args.out_amax, amax_bits);
+      }
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+}  // namespace gemm
+}  // namespace fp8lib

@@ -1,0 +1,333 @@
+// libfp8.cu -- the C ABI of include/fp8.h: argument checks, TMA descriptor
+// encoding and kernel launches.  All device code lives in the headers
+// included below; this is the library's single translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/fp8.h"
+#include "adam.cuh"
+#include "amax_cast.cuh"
+#include "common.cuh"
+#include "gemm.cuh"
+
+using namespace fp8lib;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sms = 0;
+  int adam_blocks_per_sm = 1;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA; }
+
+template <typename K>
+int set_smem(K kernel, int bytes) {
+  return cuda_rc(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+}
+
+// One-time per-device set-up: SM count, occupancy, kernel attributes.
+int device_info(DeviceInfo **out) {
+  int dev;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP8_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo &d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    int bps = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k_adam<2>, kAdamThreads, 0) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    d.adam_blocks_per_sm = bps > 0 ? bps : 1;
+    int rc = FP8_OK;
+    rc |= set_smem(gemm::k_gemm<256, false, false>, gemm::Cfg<256>::SMEM_BYTES);
+    rc |= set_smem(gemm::k_gemm<256, false, true>, gemm::Cfg<256>::SMEM_BYTES);
+    rc |= set_smem(gemm::k_gemm<256, true, true>, gemm::Cfg<256>::SMEM_BYTES);
+    if (rc) return FP8_ERR_CUDA;
+    if (!g_encode) {
+      cudaDriverEntryPointQueryResult q;
+      void *fn = nullptr;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return FP8_ERR_CUDA;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    d.ready = true;
+  }
+  *out = &d;
+  return FP8_OK;
+}
+
+int launch_rc() { return cuda_rc(cudaGetLastError()); }
+
+bool valid_dtype(int dt) { return dt == FP8_DT_F32 || dt == FP8_DT_BF16 || dt == FP8_DT_F16; }
+bool valid_fmt(int f) { return f == FP8_E4M3 || f == FP8_E5M2 || f == FP8_F16S; }
+size_t dtype_bytes(int dt) { return dt == FP8_DT_F32 ? 4 : 2; }
+
+unsigned grid_for(size_t work_items, int per_block, int cap) {
+  size_t b = (work_items + per_block - 1) / per_block;
+  if (b < 1) b = 1;
+  if (b > (size_t)cap) b = cap;
+  return (unsigned)b;
+}
+
+// 2-D row-major uint8 tensor [outer, inner] -> TMA map with a box of
+// 128 bytes x box_outer rows and the 128-byte swizzle.
+int make_map(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer, uint32_t box_outer) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {128, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(ptr), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8_OK : FP8_ERR_CUDA;
+}
+
+// C[rows, cols] = sum_k A(r, k) B(c, k), operand majorness as template flags.
+// A is [rows, K] (K-major) or [K, rows] (MN-major); B likewise with cols.
+template <bool A_MN, bool B_MN>
+int run_gemm(const uint8_t *A, int fmt_a, const float *inv_a, const uint8_t *B, int fmt_b,
+             const float *inv_b, const void *bias, int bias_dtype, void *out, int out_dtype,
+             float *out_amax, int rows, int cols, int K, cudaStream_t stream) {
+  if (!A || !B || !inv_a || !inv_b || !out) return FP8_ERR_INVALID_ARG;
+  if (rows < 0 || cols < 0 || K < 0) return FP8_ERR_INVALID_ARG;
+  if (!valid_dtype(out_dtype) || (bias && !valid_dtype(bias_dtype))) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(out)) return FP8_ERR_UNALIGNED;
+  if (rows == 0 || cols == 0) {
+    if (out_amax) return cuda_rc(cudaMemsetAsync(out_amax, 0, sizeof(float), stream));
+    return FP8_OK;
+  }
+  if (K == 0 || rows % 16 || cols % 16 || K % 16) return FP8_ERR_UNSUPPORTED;
+  DeviceInfo *d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  constexpr int BN = 256;
+  CUtensorMap ma, mb;
+  if (A_MN) rc = make_map(&ma, A, (uint64_t)rows, (uint64_t)K, gemm::BK);
+  else      rc = make_map(&ma, A, (uint64_t)K, (uint64_t)rows, gemm::BM);
+  if (rc) return rc;
+  if (B_MN) rc = make_map(&mb, B, (uint64_t)cols, (uint64_t)K, gemm::BK);
+  else      rc = make_map(&mb, B, (uint64_t)K, (uint64_t)cols, BN);
+  if (rc) return rc;
+  gemm::Args a;
+  a.rows = rows;
+  a.cols = cols;
+  a.K = K;
+  a.num_m_blocks = (rows + gemm::BM - 1) / gemm::BM;
+  a.num_n_blocks = (cols + BN - 1) / BN;
+  a.num_tiles = a.num_m_blocks * a.num_n_blocks;
+  a.num_k_blocks = (K + gemm::BK - 1) / gemm::BK;
+  a.idesc = (1u << 4)                       // accumulate in F32
+            | ((uint32_t)fmt_a << 7)         // A: 0 = E4M3, 1 = E5M2
+            | ((uint32_t)fmt_b << 10)        // B
+            | ((uint32_t)(A_MN ? 1 : 0) << 15) | ((uint32_t)(B_MN ? 1 : 0) << 16)
+            | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(gemm::BM >> 4) << 24);
+  a.inv_a = inv_a;
+  a.inv_b = inv_b;
+  a.bias = bias;
+  a.bias_dtype = bias_dtype;
+  a.out = out;
+  a.out_dtype = out_dtype;
+  a.out_amax = out_amax;
+  if (out_amax && (rc = cuda_rc(cudaMemsetAsync(out_amax, 0, sizeof(float), stream)))) return rc;
+  unsigned grid = (unsigned)(a.num_tiles < d->sms ? a.num_tiles : d->sms);
+  gemm::k_gemm<BN, A_MN, B_MN><<<grid, gemm::kThreads, gemm::Cfg<BN>::SMEM_BYTES, stream>>>(ma, mb, a);
+  return launch_rc();
+}
+
+template <int DT>
+void launch_amax(const void *x, size_t n, float *amax, cudaStream_t s, int sms) {
+  unsigned grid = grid_for(n / 16, kStreamThreads * 4, sms * 8);
+  k_amax<DT><<<grid, kStreamThreads, 0, s>>>(x, n, amax);
+}
+
+template <int DT, int FMT>
+void launch_cast(const void *x, size_t n, const float *scale, void *q, cudaStream_t s, int sms) {
+  unsigned grid = grid_for(n / 16, kStreamThreads * 2, sms * 8);
+  k_cast<DT, FMT><<<grid, kStreamThreads, 0, s>>>(x, n, scale, q);
+}
+
+template <int DT>
+void launch_cast_dt(int fmt, const void *x, size_t n, const float *scale, void *q, cudaStream_t s, int sms) {
+  if (fmt == FP8_E4M3) launch_cast<DT, FP8_E4M3>(x, n, scale, q, s, sms);
+  else if (fmt == FP8_E5M2) launch_cast<DT, FP8_E5M2>(x, n, scale, q, s, sms);
+  else launch_cast<DT, FP8_F16S>(x, n, scale, q, s, sms);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp8_amax(const void *x, int dtype, size_t n, float *amax_dev, void *stream) {
+  if (!amax_dev || !valid_dtype(dtype) || (n > 0 && !x)) return FP8_ERR_INVALID_ARG;
+  if (n > 0 && !aligned16(x)) return FP8_ERR_UNALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int rc = cuda_rc(cudaMemsetAsync(amax_dev, 0, sizeof(float), s));
+  if (rc || n == 0) return rc;
+  DeviceInfo *d;
+  if ((rc = device_info(&d))) return rc;
+  if (dtype == FP8_DT_F32) launch_amax<FP8_DT_F32>(x, n, amax_dev, s, d->sms);
+  else if (dtype == FP8_DT_BF16) launch_amax<FP8_DT_BF16>(x, n, amax_dev, s, d->sms);
+  else launch_amax<FP8_DT_F16>(x, n, amax_dev, s, d->sms);
+  return launch_rc();
+}
+
+int fp8_compute_scale(const float *amax_dev, int fmt, int margin, float mu, float *scale_dev,
+                      float *inv_scale_dev, void *stream) {
+  if (!amax_dev || !scale_dev || !inv_scale_dev || !valid_fmt(fmt)) return FP8_ERR_INVALID_ARG;
+  if (margin < 0 || margin > 64) return FP8_ERR_INVALID_ARG;
+  int e2;
+  float frac = frexpf(mu, &e2);
+  if (!(mu > 0.0f) || frac != 0.5f || e2 - 1 < -32 || e2 - 1 > 32) return FP8_ERR_INVALID_ARG;
+  k_compute_scale<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(amax_dev, fmt_max_of(fmt), margin,
+                                                                 e2 - 1, scale_dev, inv_scale_dev);
+  return launch_rc();
+}
+
+int fp8_cast(const void *x, int dtype, size_t n, int fmt, const float *scale_dev, void *q, void *stream) {
+  if (!valid_dtype(dtype) || !valid_fmt(fmt) || !scale_dev) return FP8_ERR_INVALID_ARG;
+  if (n == 0) return FP8_OK;
+  if (!x || !q) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(q)) return FP8_ERR_UNALIGNED;
+  DeviceInfo *d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == FP8_DT_F32) launch_cast_dt<FP8_DT_F32>(fmt, x, n, scale_dev, q, s, d->sms);
+  else if (dtype == FP8_DT_BF16) launch_cast_dt<FP8_DT_BF16>(fmt, x, n, scale_dev, q, s, d->sms);
+  else launch_cast_dt<FP8_DT_F16>(fmt, x, n, scale_dev, q, s, d->sms);
+  return launch_rc();
+}
+
+int fp8_linear_fwd(const uint8_t *xq, const float *x_inv, const uint8_t *wq, const float *w_inv,
+                   const void *bias, int bias_dtype, void *y, int y_dtype, float *y_amax, int M,
+                   int N, int K, void *stream) {
+  return run_gemm<false, false>(xq, FP8_E4M3, x_inv, wq, FP8_E4M3, w_inv, bias, bias_dtype, y,
+                                y_dtype, y_amax, M, N, K, static_cast<cudaStream_t>(stream));
+}
+
+int fp8_linear_dgrad(const uint8_t *dyq, const float *dy_inv, const uint8_t *wq,
+                     const float *w_inv, void *dx, int dx_dtype, float *dx_amax, int M, int N,
+                     int K, void *stream) {
+  // dX[M,K] = dY[M,N] . W[N,K]: rows M, cols K, reduction N; W is MN-major.
+  return run_gemm<false, true>(dyq, FP8_E5M2, dy_inv, wq, FP8_E4M3, w_inv, nullptr, 0, dx,
+                               dx_dtype, dx_amax, M, K, N, static_cast<cudaStream_t>(stream));
+}
+
+int fp8_linear_wgrad(const uint8_t *dyq, const float *dy_inv, const uint8_t *xq,
+                     const float *x_inv, void *dw, int dw_dtype, float *dw_amax, int M, int N,
+                     int K, void *stream) {
+  // dW[N,K] = dY[M,N]^T . X[M,K]: rows N, cols K, reduction M; both MN-major.
+  return run_gemm<true, true>(dyq, FP8_E5M2, dy_inv, xq, FP8_E4M3, x_inv, nullptr, 0, dw,
+                              dw_dtype, dw_amax, N, K, M, static_cast<cudaStream_t>(stream));
+}
+
+size_t fp8_adam_workspace_bytes(int nchunks) {
+  if (nchunks <= 0) return 0;
+  return (size_t)nchunks * kAdamWsFloatsPerChunk * sizeof(float);
+}
+
+int fp8_adam_step(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp,
+                  void *workspace, size_t ws_bytes, void *stream) {
+  if (!chunks || !hp || nchunks <= 0 || !workspace) return FP8_ERR_INVALID_ARG;
+  if (ws_bytes < fp8_adam_workspace_bytes(nchunks)) return FP8_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FP8_ERR_UNALIGNED;
+  if (!(hp->lr >= 0.0f) || !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) ||
+      !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f) || !(hp->eps >= 0.0f) || hp->step < 1 ||
+      hp->margin < 0 || hp->margin > 64)
+    return FP8_ERR_INVALID_ARG;
+  for (int i = 0; i < nchunks; i++) {
+    const fp8_adam_chunk &c = chunks[i];
+    if (!c.g_inv || !c.m_scale || !c.v_scale || !c.w_scale) return FP8_ERR_INVALID_ARG;
+    if (c.n > 0 && (!c.g || !c.m || !c.v || !c.w)) return FP8_ERR_INVALID_ARG;
+    if (c.n > 0 && (!aligned16(c.g) || !aligned16(c.m) || !aligned16(c.v) || !aligned16(c.w)))
+      return FP8_ERR_UNALIGNED;
+  }
+  DeviceInfo *d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = cuda_rc(cudaMemsetAsync(workspace, 0, fp8_adam_workspace_bytes(nchunks), s)))) return rc;
+
+  static thread_local AdamLaunch L;  // ~20 KB: kept off the stack
+  L.margin = hp->margin;
+  L.lr = hp->lr;
+  L.beta1 = hp->beta1;
+  L.beta2 = hp->beta2;
+  L.eps = hp->eps;
+  L.inv_bc1 = (float)(1.0 / (1.0 - pow((double)hp->beta1, (double)hp->step)));
+  L.inv_bc2 = (float)(1.0 / (1.0 - pow((double)hp->beta2, (double)hp->step)));
+  const unsigned cap = (unsigned)(d->sms * d->adam_blocks_per_sm);
+  for (int first = 0; first < nchunks; first += kAdamMaxChunksPerLaunch) {
+    const int cnt = nchunks - first < kAdamMaxChunksPerLaunch ? nchunks - first : kAdamMaxChunksPerLaunch;
+    unsigned long long tiles = 0;
+    for (int i = 0; i < cnt; i++) {
+      const fp8_adam_chunk &c = chunks[first + i];
+      AdamChunkDev &e = L.c[i];
+      e.g = c.g; e.g_inv = c.g_inv; e.m = c.m; e.m_scale = c.m_scale;
+      e.v = c.v; e.v_scale = c.v_scale; e.w = c.w; e.w_scale = c.w_scale;
+      e.n = c.n;
+      e.tile_begin = tiles;
+      tiles += (c.n + kAdamTile - 1) / kAdamTile;
+    }
+    L.nchunks = cnt;
+    L.total_tiles = tiles;
+    L.ws = reinterpret_cast<float *>(workspace) + (size_t)first * kAdamWsFloatsPerChunk;
+    const unsigned grid = tiles == 0 ? 1u : (unsigned)(tiles < cap ? tiles : cap);
+    k_adam<1><<<grid, kAdamThreads, 0, s>>>(L);
+    if ((rc = launch_rc())) return rc;
+    k_adam_finalize<<<1, 256, 0, s>>>(L);
+    if ((rc = launch_rc())) return rc;
+    k_adam<2><<<grid, kAdamThreads, 0, s>>>(L);
+    if ((rc = launch_rc())) return rc;
+  }
+  return FP8_OK;
+}
+
+int fp8_get_status(unsigned *host_out, void *stream) {
+  if (!host_out) return FP8_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_status, sizeof(v), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return FP8_ERR_CUDA;
+  if (cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return FP8_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FP8_ERR_CUDA;
+  *host_out = v;
+  return FP8_OK;
+}
+
+const char *fp8_strerror(int code) {
+  switch (code) {
+    case FP8_OK: return "ok";
+    case FP8_ERR_INVALID_ARG: return "invalid argument";
+    case FP8_ERR_UNALIGNED: return "pointer not 16-byte aligned";
+    case FP8_ERR_UNSUPPORTED: return "unsupported shape (GEMM dims must be multiples of 16)";
+    case FP8_ERR_CUDA: return "CUDA error";
+    case FP8_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case FP8_ERR_NONFINITE: return "non-finite amax";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

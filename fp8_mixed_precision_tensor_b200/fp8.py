@@ -1,0 +1,194 @@
+"""ctypes binding of libfp8 (the C ABI in include/fp8.h).
+
+Argument marshalling only: every function takes torch tensors that already
+live on the current CUDA device, passes their data pointers, sizes and the
+current stream to the entry point of the same name, and raises FP8Error on a
+non-zero status.  All arithmetic happens in the CUDA kernels of libfp8.so;
+there is no fallback, and importing this module fails loudly when the library
+has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp8.so")
+
+# status codes / enums (include/fp8.h)
+FP8_OK, FP8_ERR_INVALID_ARG, FP8_ERR_UNALIGNED, FP8_ERR_UNSUPPORTED = 0, 1, 2, 3
+FP8_ERR_CUDA, FP8_ERR_TIMEOUT, FP8_ERR_NONFINITE = 4, 5, 6
+FP8_STATUS_NONFINITE, FP8_STATUS_TIMEOUT = 1, 2
+FP8_DT_F32, FP8_DT_BF16, FP8_DT_F16 = 0, 1, 2
+FP8_E4M3, FP8_E5M2, FP8_F16S = 0, 1, 2
+
+_DT = {torch.float32: FP8_DT_F32, torch.bfloat16: FP8_DT_BF16, torch.float16: FP8_DT_F16}
+
+SYMBOLS = ("fp8_amax", "fp8_compute_scale", "fp8_cast", "fp8_linear_fwd", "fp8_linear_dgrad",
+           "fp8_linear_wgrad", "fp8_adam_workspace_bytes", "fp8_adam_step", "fp8_get_status",
+           "fp8_strerror")
+
+
+class FP8Error(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {fp8_strerror(code)} (status {code})")
+        self.code = code
+
+
+class _Chunk(ctypes.Structure):
+    _fields_ = [("g", ctypes.c_void_p), ("g_inv", ctypes.c_void_p), ("m", ctypes.c_void_p),
+                ("m_scale", ctypes.c_void_p), ("v", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
+                ("w", ctypes.c_void_p), ("w_scale", ctypes.c_void_p), ("n", ctypes.c_size_t)]
+
+
+class _HParams(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("step", ctypes.c_int), ("margin", ctypes.c_int)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libfp8.so and declare the signatures of every entry point."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libfp8.so not built ({path}); run python -m fp8_mixed_precision_tensor_b200.build")
+    lib = ctypes.CDLL(path)
+    p, i, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    lib.fp8_amax.argtypes = [p, i, sz, p, p]
+    lib.fp8_compute_scale.argtypes = [p, i, i, f, p, p, p]
+    lib.fp8_cast.argtypes = [p, i, sz, i, p, p, p]
+    lib.fp8_linear_fwd.argtypes = [p, p, p, p, p, i, p, i, p, i, i, i, p]
+    lib.fp8_linear_dgrad.argtypes = [p, p, p, p, p, i, p, i, i, i, p]
+    lib.fp8_linear_wgrad.argtypes = [p, p, p, p, p, i, p, i, i, i, p]
+    lib.fp8_adam_workspace_bytes.argtypes, lib.fp8_adam_workspace_bytes.restype = [i], sz
+    lib.fp8_adam_step.argtypes = [ctypes.POINTER(_Chunk), i, ctypes.POINTER(_HParams), p, sz, p]
+    lib.fp8_get_status.argtypes = [ctypes.POINTER(ctypes.c_uint), p]
+    lib.fp8_strerror.argtypes, lib.fp8_strerror.restype = [i], ctypes.c_char_p
+    for name in SYMBOLS:
+        if name not in ("fp8_adam_workspace_bytes", "fp8_strerror"):
+            getattr(lib, name).restype = i
+    _lib = lib
+    return lib
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libfp8 takes device tensors")
+    return t.data_ptr()
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != FP8_OK:
+        raise FP8Error(rc, what)
+
+
+def fp8_strerror(code: int) -> str:
+    return load_library().fp8_strerror(code).decode()
+
+
+# ---------------------------------------------------------------- amax / scale / cast
+def fp8_amax(x: torch.Tensor, amax_out: torch.Tensor, stream=None) -> None:
+    """amax_out[0] = max |x| (float32 device scalar)."""
+    _check(load_library().fp8_amax(_ptr(x), _DT[x.dtype], x.numel(), _ptr(amax_out), _stream(stream)),
+           "fp8_amax")
+
+
+def fp8_compute_scale(amax: torch.Tensor, fmt: int, margin: int, mu: float, scale_out: torch.Tensor,
+                      inv_scale_out: torch.Tensor, stream=None) -> None:
+    _check(load_library().fp8_compute_scale(_ptr(amax), fmt, margin, mu, _ptr(scale_out),
+                                            _ptr(inv_scale_out), _stream(stream)), "fp8_compute_scale")
+
+
+def fp8_cast(x: torch.Tensor, fmt: int, scale: torch.Tensor, q_out: torch.Tensor, stream=None) -> None:
+    """q_out = enc_fmt(x * scale): uint8 codes, or 16-bit halves for FP8_F16S."""
+    _check(load_library().fp8_cast(_ptr(x), _DT[x.dtype], x.numel(), fmt, _ptr(scale), _ptr(q_out),
+                                   _stream(stream)), "fp8_cast")
+
+
+# ---------------------------------------------------------------- GEMMs
+def fp8_linear_fwd(xq, x_inv, wq, w_inv, y, y_amax=None, bias=None, stream=None) -> None:
+    """y[M,N] = (xq[M,K] . wq[N,K]^T) * x_inv * w_inv (+ bias)."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    _check(load_library().fp8_linear_fwd(_ptr(xq), _ptr(x_inv), _ptr(wq), _ptr(w_inv), _ptr(bias),
+                                         _DT[bias.dtype] if bias is not None else 0, _ptr(y), _DT[y.dtype],
+                                         _ptr(y_amax), M, N, K, _stream(stream)), "fp8_linear_fwd")
+
+
+def fp8_linear_dgrad(dyq, dy_inv, wq, w_inv, dx, dx_amax=None, stream=None) -> None:
+    """dx[M,K] = (dyq[M,N] . wq[N,K]) * dy_inv * w_inv."""
+    M, N = dyq.shape
+    K = wq.shape[1]
+    _check(load_library().fp8_linear_dgrad(_ptr(dyq), _ptr(dy_inv), _ptr(wq), _ptr(w_inv), _ptr(dx),
+                                           _DT[dx.dtype], _ptr(dx_amax), M, N, K, _stream(stream)),
+           "fp8_linear_dgrad")
+
+
+def fp8_linear_wgrad(dyq, dy_inv, xq, x_inv, dw, dw_amax=None, stream=None) -> None:
+    """dw[N,K] = (dyq[M,N]^T . xq[M,K]) * dy_inv * x_inv."""
+    M, N = dyq.shape
+    K = xq.shape[1]
+    _check(load_library().fp8_linear_wgrad(_ptr(dyq), _ptr(dy_inv), _ptr(xq), _ptr(x_inv), _ptr(dw),
+                                           _DT[dw.dtype], _ptr(dw_amax), M, N, K, _stream(stream)),
+           "fp8_linear_wgrad")
+
+
+# ---------------------------------------------------------------- Adam
+@dataclass
+class AdamChunk:
+    """Stored state of one tensor: E5M2 grad codes + g_inv, E4M3 m1 codes +
+    scale, FP16 m2 bits + scale, FP16 master bits + scale (device tensors)."""
+    g: torch.Tensor
+    g_inv: torch.Tensor
+    m: torch.Tensor
+    m_scale: torch.Tensor
+    v: torch.Tensor
+    v_scale: torch.Tensor
+    w: torch.Tensor
+    w_scale: torch.Tensor
+
+
+def fp8_adam_workspace_bytes(nchunks: int) -> int:
+    return load_library().fp8_adam_workspace_bytes(nchunks)
+
+
+def pack_adam_chunks(chunks: list[AdamChunk]):
+    """Host array of fp8_adam_chunk (reusable across steps)."""
+    arr = (_Chunk * len(chunks))()
+    for i, c in enumerate(chunks):
+        arr[i] = _Chunk(_ptr(c.g), _ptr(c.g_inv), _ptr(c.m), _ptr(c.m_scale), _ptr(c.v), _ptr(c.v_scale),
+                        _ptr(c.w), _ptr(c.w_scale), c.g.numel())
+    return arr
+
+
+def fp8_adam_step(chunks, lr: float, beta1: float, beta2: float, eps: float, step: int, margin: int,
+                  workspace: torch.Tensor, stream=None) -> None:
+    """One decoupled FP8 Adam step over every chunk (in place).  `chunks` is a
+    list of AdamChunk or the array returned by pack_adam_chunks."""
+    arr = chunks if isinstance(chunks, ctypes.Array) else pack_adam_chunks(chunks)
+    hp = _HParams(lr, beta1, beta2, eps, step, margin)
+    _check(load_library().fp8_adam_step(arr, len(arr), ctypes.byref(hp), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _stream(stream)),
+           "fp8_adam_step")
+
+
+def fp8_get_status(stream=None) -> int:
+    """Wait for the stream, read and clear the device status word."""
+    out = ctypes.c_uint(0)
+    _check(load_library().fp8_get_status(ctypes.byref(out), _stream(stream)), "fp8_get_status")
+    return out.value

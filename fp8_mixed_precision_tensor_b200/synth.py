@@ -1,8 +1,8 @@
 """Seeded synthetic inputs shared by the tests, the smoke check and the benchmark.
 
 This module draws random numbers and nothing else: it holds none of the FP8
-method's arithmetic (no scaling, casting, GEMM or optimizer math), so both the
-CUDA path and the CPU oracle can be fed from it.  Host arrays come from numpy
+method's arithmetic (no scaling, casting, GEMM or optimizer math), so the same
+seeded bytes can feed the CUDA path and any independent CPU checker.  Host arrays come from numpy
 PCG64 generators keyed by (workload, tensor, step); large device-resident
 benchmark inputs come from torch's seeded CUDA generator with the same value
 distributions.  fp32 -> bf16 input rounding is round-to-nearest-even.

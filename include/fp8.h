@@ -1,0 +1,207 @@
+/*
+ * fp8.h -- C ABI of libfp8, the B200 (sm_100a) hot path of FP8 mixed-precision
+ * LLM training: per-tensor dynamically scaled FP8 linear layers and the
+ * precision-decoupled FP8 Adam step.
+ *
+ * Sources (by page title and section):
+ *   [FP8-AMAX] "Training and inference of large language models using 8-bit
+ *              floating point" (paper review), 제안 방법: per-tensor scaling
+ *              bias from the amax of each weight, activation and gradient
+ *              tensor (log2 of fmt_max / amax with a configurable margin);
+ *              scale before the FP8 cast, undo the scaling after the matmul;
+ *              E4M3 for weights and activations, E5M2 for gradients.
+ *   [FP8-LM]   "FP8-LM: Training FP8 Large Language Models" (paper memo),
+ *              提案手法: O1 gradient auto-scaling g' = mu * g (Eq. 3);
+ *              O2 Adam with FP8 first moment, FP16 second moment and FP16
+ *              master weights with tensor scaling.
+ *
+ * Conventions shared by every entry point
+ *   - Ownership: the caller owns every buffer.  The library allocates and
+ *     frees nothing and never synchronises the stream (fp8_get_status is the
+ *     one exception and says so).  Every call only enqueues work on `stream`
+ *     (a cudaStream_t; NULL = the legacy default stream) and returns.
+ *   - "dev" pointers are device memory of the current CUDA device; "host"
+ *     pointers are host memory.  Scalars that chain one call into the next
+ *     (amax, scale, inverse scale) stay in device memory as float.
+ *   - Bulk tensors are dense and contiguous; their pointers must be 16-byte
+ *     aligned (FP8_ERR_UNALIGNED otherwise).  Any element count is allowed.
+ *   - Errors found on the host are returned at once and nothing is enqueued.
+ *     Conditions found on the device (a non-finite amax, a pipeline wait that
+ *     ran out of time) set bits of a device status word read by
+ *     fp8_get_status.
+ */
+#ifndef FP8_B200_H
+#define FP8_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ----------------------------------------------------- */
+#define FP8_OK 0
+#define FP8_ERR_INVALID_ARG 1 /* null pointer, bad enum, bad hyper-parameter */
+#define FP8_ERR_UNALIGNED 2   /* a bulk pointer is not 16-byte aligned */
+#define FP8_ERR_UNSUPPORTED 3 /* a GEMM shape the kernel cannot tile (see below) */
+#define FP8_ERR_CUDA 4        /* a CUDA runtime call or kernel launch failed */
+#define FP8_ERR_TIMEOUT 5     /* device status: a pipeline wait ran out of time */
+#define FP8_ERR_NONFINITE 6   /* device status: an amax was NaN or inf */
+
+/* Device status word bits (fp8_get_status). */
+#define FP8_STATUS_NONFINITE 1u
+#define FP8_STATUS_TIMEOUT 2u
+
+/* ---- element types of high-precision tensors -------------------------- */
+#define FP8_DT_F32 0
+#define FP8_DT_BF16 1
+#define FP8_DT_F16 2
+
+/* ---- storage formats ---------------------------------------------------
+ * FP8_E4M3: OCP E4M3, max 448, no infinities (weights, activations, Adam m1).
+ * FP8_E5M2: OCP E5M2, max 57344 (gradients).
+ * FP8_F16S: IEEE binary16 with a per-tensor power-of-two scale, max 65504
+ *           ("FP16 with tensor scaling": Adam m2 and master weights). */
+#define FP8_E4M3 0
+#define FP8_E5M2 1
+#define FP8_F16S 2
+
+/*
+ * fp8_amax -- amax = max_i |x_i| over n elements, written to *amax_dev as a
+ * float ([FP8-AMAX] 제안 방법).  Exact: the maximum is taken over bit
+ * patterns.  Any NaN element gives a NaN amax; otherwise any inf gives +inf.
+ * n == 0 writes 0.
+ *   x        dev, n elements of `dtype`, 16-byte aligned
+ *   amax_dev dev, one float, overwritten
+ */
+int fp8_amax(const void *x, int dtype, size_t n, float *amax_dev, void *stream);
+
+/*
+ * fp8_compute_scale -- the per-tensor power-of-two scale of [FP8-AMAX]
+ * 제안 방법 with the gradient auto-scaling factor of [FP8-LM] O1 (Eq. 3):
+ *     e     = floor(log2(fmt_max / (mu * amax)))   (exact integer arithmetic)
+ *     s_g   = 2^(clamp(e - margin, -126, 126))
+ *     scale = mu * s_g,   inv_scale = 1 / (mu * s_g).
+ * `scale` multiplies the raw tensor before the cast; `inv_scale` undoes it
+ * after a GEMM (or when decoding).  amax == 0 gives s_g = 1.  A NaN or inf
+ * amax gives s_g = 1 and sets FP8_STATUS_NONFINITE.
+ *   amax_dev      dev, one float (typically written by fp8_amax or by a
+ *                 GEMM's fused output amax)
+ *   fmt           FP8_E4M3 (fmt_max 448), FP8_E5M2 (57344), FP8_F16S (65504)
+ *   margin        integer >= 0; each unit halves the scale (headroom)
+ *   mu            host float, a power of two in [2^-32, 2^32] (1 = off)
+ *   scale_dev, inv_scale_dev  dev, one float each, overwritten
+ */
+int fp8_compute_scale(const float *amax_dev, int fmt, int margin, float mu, float *scale_dev,
+                      float *inv_scale_dev, void *stream);
+
+/*
+ * fp8_cast -- q_i = enc_fmt(x_i * scale) ([FP8-AMAX] 제안 방법: scale, then
+ * cast).  FP8 formats: round to nearest even, saturating at +-max; +-inf
+ * saturates too; NaN becomes 0x7F with the input's sign bit.  FP8_F16S:
+ * IEEE round to nearest even.  With a scale from fp8_compute_scale on the
+ * tensor's own amax nothing saturates.
+ *   x          dev, n elements of `dtype`, 16-byte aligned
+ *   scale_dev  dev, one float (power of two times mu)
+ *   q          dev, n bytes (E4M3/E5M2) or n uint16 (F16S), 16-byte aligned
+ */
+int fp8_cast(const void *x, int dtype, size_t n, int fmt, const float *scale_dev, void *q,
+             void *stream);
+
+/*
+ * FP8 linear layer GEMMs ([FP8-AMAX] 제안 방법: matmul on FP8 operands, the
+ * scaling undone on the output; [FP8-LM] 新規性: FP8 in the linear layers).
+ * Shapes follow nn.Linear: X[M,K], W[N,K], Y[M,N]; all row-major, dense.
+ * Every operand is read in place (no transposed copies): dgrad reads W and
+ * wgrad reads dY and X along their rows as MN-major tensor-core operands.
+ * The epilogue multiplies by the two inverse scales, adds the bias (fwd),
+ * rounds to the output type and, when out_amax is not NULL, writes the amax
+ * of the output *as stored* (overwritten, not accumulated).
+ * Shape rule: M, N, K must each be a multiple of 16 (TMA row pitch);
+ * otherwise FP8_ERR_UNSUPPORTED.  M == 0 or N == 0 is a no-op that writes an
+ * amax of 0.  Output types: FP8_DT_F32, FP8_DT_BF16, FP8_DT_F16.
+ * A mis-tiled pipeline cannot hang: every wait is bounded, and a wait that
+ * runs out sets FP8_STATUS_TIMEOUT and the kernel returns.
+ */
+
+/* Y[M,N] = (Xq . Wq^T) * x_inv * w_inv (+ bias[N]).
+ *   xq  dev [M,K] E4M3,  wq dev [N,K] E4M3,  x_inv/w_inv dev floats
+ *   bias dev [N] of bias_dtype or NULL;  y dev [M,N] of y_dtype */
+int fp8_linear_fwd(const uint8_t *xq, const float *x_inv, const uint8_t *wq, const float *w_inv,
+                   const void *bias, int bias_dtype, void *y, int y_dtype, float *y_amax, int M,
+                   int N, int K, void *stream);
+
+/* dX[M,K] = (dYq . Wq) * dy_inv * w_inv.
+ *   dyq dev [M,N] E5M2,  wq dev [N,K] E4M3;  dx dev [M,K] of dx_dtype */
+int fp8_linear_dgrad(const uint8_t *dyq, const float *dy_inv, const uint8_t *wq,
+                     const float *w_inv, void *dx, int dx_dtype, float *dx_amax, int M, int N,
+                     int K, void *stream);
+
+/* dW[N,K] = (dYq^T . Xq) * dy_inv * x_inv.
+ *   dyq dev [M,N] E5M2,  xq dev [M,K] E4M3;  dw dev [N,K] of dw_dtype */
+int fp8_linear_wgrad(const uint8_t *dyq, const float *dy_inv, const uint8_t *xq,
+                     const float *x_inv, void *dw, int dw_dtype, float *dw_amax, int M, int N,
+                     int K, void *stream);
+
+/*
+ * Precision-decoupled FP8 Adam ([FP8-LM] 提案手法 O2): per parameter 6 bytes
+ * of state -- FP8 E5M2 gradient (1 B), FP8 E4M3 first moment (1 B), FP16
+ * second moment (2 B) and FP16 master weight (2 B) -- each tensor with its
+ * own power-of-two scale.  One call updates every chunk (tensor) in place:
+ *   g  = dec_E5M2(g) * g_inv                 (g_inv = 1 / (mu * s_g))
+ *   m0 = dec_E4M3(m) / m_scale,  v0 = half(v) / v_scale,  w0 = half(w) / w_scale
+ *   m  = b1 m0 + (1 - b1) g,     v  = b2 v0 + (1 - b2) g^2
+ *   w  = w0 - lr * (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps)
+ * then new per-chunk scales from the amax of the new m, v, w (same rule as
+ * fp8_compute_scale with `margin`, fmt_max 448 / 65504 / 65504) and the state
+ * is re-encoded with them; the new scales replace m_scale, v_scale, w_scale.
+ * Arithmetic is float32.  A non-finite new amax sets FP8_STATUS_NONFINITE and
+ * that scale to 1.
+ * Pointers g, m, v, w are dev and 16-byte aligned; the scale pointers are dev
+ * floats.  Chunks must not overlap.  `chunks` is a HOST array of nchunks.
+ */
+typedef struct {
+  const uint8_t *g;    /* dev [n] E5M2 gradient codes */
+  const float *g_inv;  /* dev float: 1 / (mu * s_g) */
+  uint8_t *m;          /* dev [n] E4M3 first-moment codes (in/out) */
+  float *m_scale;      /* dev float (in/out) */
+  uint16_t *v;         /* dev [n] FP16 second moment, scaled (in/out) */
+  float *v_scale;      /* dev float (in/out) */
+  uint16_t *w;         /* dev [n] FP16 master weight, scaled (in/out) */
+  float *w_scale;      /* dev float (in/out) */
+  size_t n;            /* parameters in this chunk (0 allowed) */
+} fp8_adam_chunk;
+
+typedef struct {
+  float lr, beta1, beta2, eps; /* lr > 0, 0 <= beta < 1, eps >= 0 */
+  int step;                    /* t >= 1 (bias correction) */
+  int margin;                  /* scale margin, >= 0 */
+} fp8_adam_hparams;
+
+/* Bytes of device workspace fp8_adam_step needs for nchunks chunks. */
+size_t fp8_adam_workspace_bytes(int nchunks);
+
+/*
+ * fp8_adam_step -- one step over all chunks.  workspace: dev, at least
+ * fp8_adam_workspace_bytes(nchunks) bytes, 256-byte aligned, owned by the
+ * caller, not touched by anything else while the step runs (it holds the
+ * per-chunk amax accumulators and the old scales between the two passes).
+ */
+int fp8_adam_step(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp,
+                  void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * fp8_get_status -- waits for `stream`, then reads the device status word
+ * (OR of FP8_STATUS_* bits raised since the last read) into *host_out and
+ * clears it.  Returns FP8_ERR_CUDA if the stream reported an error.
+ */
+int fp8_get_status(unsigned *host_out, void *stream);
+
+/* Human-readable message of a status code (static string). */
+const char *fp8_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FP8_B200_H */

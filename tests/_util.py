@@ -1,0 +1,57 @@
+"""Helpers shared by the GPU parity tests (comparison rules, device copies)."""
+import numpy as np
+import torch
+
+# GEMM tolerance: |gpu - oracle| <= 1e-3 * sum_k |a_ik b_kj| (plus half an ULP
+# of a 16-bit output type for the final rounding).
+GEMM_REL = 1e-3
+
+
+def to_dev(a: np.ndarray, dtype=None) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    return t if dtype is None else t.view(dtype)
+
+
+def bf16_dev(bits: np.ndarray) -> torch.Tensor:
+    return to_dev(bits.view(np.int16)).view(torch.bfloat16)
+
+
+def code_rank(c: np.ndarray) -> np.ndarray:
+    """Monotone integer order of FP8 codes (-0 and +0 share rank 0)."""
+    c = np.asarray(c).astype(np.int64)
+    return np.where(c < 128, c, 128 - c)
+
+
+def f16_vals(bits: np.ndarray) -> np.ndarray:
+    return np.asarray(bits).view(np.uint16).view(np.float16).astype(np.float64)
+
+
+def f16_ulp(vals: np.ndarray) -> np.ndarray:
+    return np.spacing(np.abs(vals).astype(np.float16)).astype(np.float64)
+
+
+def half_ulp_out(ref: np.ndarray, out_dtype: torch.dtype) -> np.ndarray:
+    if out_dtype == torch.float32:
+        return np.zeros_like(ref)
+    if out_dtype == torch.float16:
+        return 0.5 * f16_ulp(ref)
+    # bf16: 8 significant bits
+    e = np.floor(np.log2(np.maximum(np.abs(ref), 1e-300)))
+    return 0.5 * 2.0 ** (e - 7)
+
+
+def assert_gemm_close(gpu: np.ndarray, ref: np.ndarray, rabs: np.ndarray, out_dtype, what=""):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    err = np.abs(gpu - ref)
+    bound = GEMM_REL * rabs + half_ulp_out(ref, out_dtype)
+    bad = err > bound
+    if np.any(bad):
+        i = np.argmax(err - bound)
+        raise AssertionError(f"{what}: {np.count_nonzero(bad)} outputs outside tolerance; worst at flat {i}: "
+                             f"gpu {gpu.flat[i]!r} oracle {ref.flat[i]!r} bound {bound.flat[i]!r}")
+
+
+def tensor_to_np(t: torch.Tensor) -> np.ndarray:
+    if t.dtype == torch.bfloat16:
+        return t.float().cpu().numpy().astype(np.float64)
+    return t.cpu().numpy()

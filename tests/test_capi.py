@@ -1,0 +1,93 @@
+"""The C-ABI library loads and exports every entry point include/fp8.h
+declares; host-side argument checks answer without touching a GPU; the
+product path has no route to the oracle and fails loudly without the library."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8.h")
+PKG = os.path.join(ROOT, "fp8_mixed_precision_tensor_b200")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from fp8_mixed_precision_tensor_b200 import build
+
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(fp8_[a-z_0-9]+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_hot_path():
+    names = declared_functions()
+    for n in ("fp8_amax", "fp8_compute_scale", "fp8_cast", "fp8_linear_fwd", "fp8_linear_dgrad",
+              "fp8_linear_wgrad", "fp8_adam_step", "fp8_adam_workspace_bytes", "fp8_get_status",
+              "fp8_strerror"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_binding_symbol_list_matches_header():
+    from fp8_mixed_precision_tensor_b200 import fp8
+
+    assert sorted(fp8.SYMBOLS) == declared_functions()
+
+
+def test_strerror_and_workspace_size(lib):
+    lib.fp8_strerror.restype = ctypes.c_char_p
+    assert lib.fp8_strerror(0) == b"ok"
+    assert b"aligned" in lib.fp8_strerror(2)
+    lib.fp8_adam_workspace_bytes.restype = ctypes.c_size_t
+    assert lib.fp8_adam_workspace_bytes(3) == 3 * 64
+    assert lib.fp8_adam_workspace_bytes(0) == 0
+
+
+def test_host_side_validation_without_gpu(lib):
+    p, i, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    lib.fp8_amax.argtypes = [p, i, sz, p, p]
+    lib.fp8_cast.argtypes = [p, i, sz, i, p, p, p]
+    lib.fp8_compute_scale.argtypes = [p, i, i, f, p, p, p]
+    lib.fp8_linear_fwd.argtypes = [p, p, p, p, p, i, p, i, p, i, i, i, p]
+    fake = 0x10000  # never dereferenced: every call below fails its host checks first
+    assert lib.fp8_amax(fake, 1, 10, None, None) == 1                # null amax
+    assert lib.fp8_amax(fake, 9, 10, fake, None) == 1                # bad dtype
+    assert lib.fp8_amax(fake + 2, 1, 10, fake, None) == 2            # unaligned
+    assert lib.fp8_cast(fake, 1, 10, 5, fake, fake, None) == 1       # bad format
+    assert lib.fp8_cast(fake, 1, 10, 0, fake, fake + 8, None) == 2   # unaligned output
+    assert lib.fp8_compute_scale(fake, 0, 0, 3.0, fake, fake, None) == 1   # mu not a power of two
+    assert lib.fp8_compute_scale(fake, 0, -1, 1.0, fake, fake, None) == 1  # negative margin
+    # GEMM dims that are not multiples of 16
+    assert lib.fp8_linear_fwd(fake, fake, fake, fake, None, 0, fake, 0, None, 32, 32, 24, None) == 3
+    assert lib.fp8_linear_fwd(fake, fake, fake, fake, None, 0, fake, 7, None, 32, 32, 32, None) == 1
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    from fp8_mixed_precision_tensor_b200 import fp8
+
+    saved = fp8._lib
+    fp8._lib = None
+    try:
+        with pytest.raises(ImportError):
+            fp8.load_library(str(tmp_path / "missing.so"))
+    finally:
+        fp8._lib = saved
+
+
+def test_product_never_touches_the_oracle():
+    for dirpath, _, files in os.walk(PKG):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, fn)).read()
+                assert not re.search(r"\boracle\b", text), f"{fn} mentions the oracle"

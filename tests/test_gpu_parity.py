@@ -1,0 +1,401 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Bars: amax, scales and cast bytes bit-exact; GEMM outputs within
+1e-3 * sum_k |a b| (+ half an output ULP for 16-bit outputs); fused output
+amax bit-exact against the oracle's amax of the GPU's own output; Adam master
+weights and second moment within 1 FP16 ULP, first-moment codes within 1 code,
+scales bit-equal.  Each stage is fed the GPU's own upstream values.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp8_mixed_precision_tensor_b200 import fp8, synth
+from _util import (assert_gemm_close, bf16_dev, code_rank, f16_ulp, f16_vals, tensor_to_np, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+F32 = dict(dtype=torch.float32, device="cuda")
+ODT = {fp8.FP8_DT_F32: oracle.DT_F32, fp8.FP8_DT_BF16: oracle.DT_BF16, fp8.FP8_DT_F16: oracle.DT_F16}
+OFMT = {fp8.FP8_E4M3: oracle.E4M3, fp8.FP8_E5M2: oracle.E5M2, fp8.FP8_F16S: oracle.F16}
+
+
+def scalar():
+    return torch.zeros(1, **F32)
+
+
+def host_input(n, dt, key, specials=False):
+    """(host array for the oracle, oracle dtype code, device tensor)."""
+    b = synth.lognormal_outliers_bf16(n, *key)
+    x = synth.bf16_bits_to_f32(b)
+    if specials and n >= 8:
+        x = x.copy()
+        x[[1, n // 2, n - 1]] = [-0.0, 3.0e38 if dt == fp8.FP8_DT_F32 else 60000.0, -7.5]
+    if dt == fp8.FP8_DT_F32:
+        return x, oracle.DT_F32, to_dev(x)
+    if dt == fp8.FP8_DT_BF16:
+        bits = synth.to_bf16_bits(x)
+        return bits, oracle.DT_BF16, bf16_dev(bits)
+    h = np.clip(x, -60000, 60000).astype(np.float16)
+    return h.view(np.uint16), oracle.DT_F16, to_dev(h)
+
+
+# ---------------------------------------------------------------- amax
+@pytest.mark.parametrize("dt", [fp8.FP8_DT_F32, fp8.FP8_DT_BF16, fp8.FP8_DT_F16])
+@pytest.mark.parametrize("n", [1, 7, 16, 17, 4096 + 5, (1 << 20) + 3])
+def test_amax_bit_exact(dt, n):
+    h, odt, d = host_input(n, dt, ("amax", dt, n), specials=True)
+    a = scalar()
+    fp8.fp8_amax(d, a)
+    assert a.item() == oracle.amax(h, odt)
+
+
+def test_amax_empty_and_specials():
+    a = scalar()
+    a.fill_(5.0)
+    fp8.fp8_amax(torch.empty(0, **F32), a)
+    assert a.item() == 0.0
+    x = torch.tensor([1.0, -float("inf"), 2.0] * 11, **F32)
+    fp8.fp8_amax(x, a)
+    assert a.item() == math.inf
+    x[5] = float("nan")
+    fp8.fp8_amax(x, a)
+    assert math.isnan(a.item())
+    x = torch.tensor([-0.0, 0.0] * 20, **F32)
+    fp8.fp8_amax(x, a)
+    assert a.item() == 0.0 and math.copysign(1, a.item()) == 1.0
+
+
+def test_amax_rejects_unaligned():
+    x = torch.zeros(100, **F32)
+    with pytest.raises(fp8.FP8Error) as e:
+        fp8.fp8_amax(x[1:], scalar())
+    assert e.value.code == fp8.FP8_ERR_UNALIGNED
+
+
+# ---------------------------------------------------------------- scale
+def test_compute_scale_bit_exact_sweep():
+    g = synth.rng("scale", "sweep")
+    amaxes = list(np.exp(g.uniform(-95, 95, 300)).astype(np.float32))
+    amaxes += [0.0, 448.0, 57344.0, 65504.0, 1.0, 1e-45, 1.17e-38, 3.0e38,
+               float(np.nextafter(np.float32(448), np.float32(1e9))), float(np.float32(448 * 0.75))]
+    am = torch.tensor(amaxes, **F32)
+    for fmt in (fp8.FP8_E4M3, fp8.FP8_E5M2, fp8.FP8_F16S):
+        for margin in (0, 1, 3):
+            for mu in (1.0, 2.0 ** 10, 2.0 ** -4):
+                s, inv = torch.zeros_like(am), torch.zeros_like(am)
+                for i in range(am.numel()):
+                    fp8.fp8_compute_scale(am[i:i + 1], fmt, margin, mu, s[i:i + 1], inv[i:i + 1])
+                s_h, inv_h = s.cpu().numpy(), inv.cpu().numpy()
+                for i, a in enumerate(amaxes):
+                    rc, ref = oracle.compute_scale(float(np.float32(a)), OFMT[fmt], margin, mu=mu)
+                    assert rc == 0
+                    assert s_h[i] == ref and inv_h[i] == 1.0 / ref, (fmt, margin, mu, a, s_h[i], ref)
+    assert fp8.fp8_get_status() == 0
+
+
+def test_compute_scale_nonfinite_sets_status():
+    fp8.fp8_get_status()
+    for bad in (float("inf"), float("nan")):
+        a = torch.tensor([bad], **F32)
+        s, inv = scalar(), scalar()
+        fp8.fp8_compute_scale(a, fp8.FP8_E4M3, 0, 1.0, s, inv)
+        assert s.item() == 1.0 and inv.item() == 1.0
+        assert fp8.fp8_get_status() & fp8.FP8_STATUS_NONFINITE
+    assert fp8.fp8_get_status() == 0
+
+
+def test_compute_scale_rejects_bad_mu_and_margin():
+    a, s, inv = scalar(), scalar(), scalar()
+    for mu, margin in ((3.0, 0), (0.0, 0), (-2.0, 0), (2.0 ** 40, 0), (1.0, -1)):
+        with pytest.raises(fp8.FP8Error) as e:
+            fp8.fp8_compute_scale(a, fp8.FP8_E4M3, margin, mu, s, inv)
+        assert e.value.code == fp8.FP8_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------------- cast
+@pytest.mark.parametrize("dt", [fp8.FP8_DT_F32, fp8.FP8_DT_BF16, fp8.FP8_DT_F16])
+@pytest.mark.parametrize("fmt", [fp8.FP8_E4M3, fp8.FP8_E5M2, fp8.FP8_F16S])
+@pytest.mark.parametrize("margin", [0, 1])
+def test_amax_scale_cast_chain_bit_exact(dt, fmt, margin):
+    n = (1 << 18) + 13
+    h, odt, d = host_input(n, dt, ("cast", dt, fmt), specials=True)
+    a, s, inv = scalar(), scalar(), scalar()
+    q = torch.empty(n, dtype=torch.int16 if fmt == fp8.FP8_F16S else torch.uint8, device="cuda")
+    fp8.fp8_amax(d, a)
+    fp8.fp8_compute_scale(a, fmt, margin, 1.0, s, inv)
+    fp8.fp8_cast(d, fmt, s, q)
+    rc, s_ref = oracle.compute_scale(oracle.amax(h, odt), OFMT[fmt], margin)
+    assert s.item() == s_ref
+    ref = oracle.cast(h, OFMT[fmt], s_ref, odt)
+    got = q.cpu().numpy()
+    if fmt == fp8.FP8_F16S:
+        got = got.view(np.uint16)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("fmt", [fp8.FP8_E4M3, fp8.FP8_E5M2])
+def test_cast_saturation_and_specials(fmt):
+    vals = np.array([0.0, -0.0, 1.0, -1.0, 448.0, 464.0, 500.0, 57344.0, 61440.0, 1e6, -1e6, np.inf, -np.inf,
+                     np.nan, -np.nan, 1e-9, -1e-9, 2.0 ** -9, 2.0 ** -10, 3 * 2.0 ** -11, 2.0 ** -16,
+                     2.0 ** -17, 3.0e38] * 3, dtype=np.float32)
+    d = to_dev(vals)
+    s = torch.ones(1, **F32)
+    q = torch.empty(vals.size, dtype=torch.uint8, device="cuda")
+    fp8.fp8_cast(d, fmt, s, q)
+    got = q.cpu().numpy()
+    ref = oracle.cast(vals, OFMT[fmt], 1.0)
+    nan = np.isnan(vals)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert np.all((got[nan] & 0x7F) == 0x7F)  # NaN stays NaN
+
+
+def test_cast_mu_invariance():
+    g = synth.normal_f32(((1 << 16) + 3,), 1e-3, "mu")
+    d = to_dev(g)
+    a = scalar()
+    fp8.fp8_amax(d, a)
+    codes = []
+    for mu in (1.0, 2.0 ** 10, 2.0 ** -4):
+        s, inv = scalar(), scalar()
+        q = torch.empty(g.size, dtype=torch.uint8, device="cuda")
+        fp8.fp8_compute_scale(a, fp8.FP8_E5M2, 0, mu, s, inv)
+        fp8.fp8_cast(d, fp8.FP8_E5M2, s, q)
+        codes.append(q.cpu().numpy())
+        assert s.item() == oracle.compute_scale(oracle.amax(g), oracle.E5M2, 0, mu=mu)[1]
+    assert all(np.array_equal(codes[0], c) for c in codes[1:])
+
+
+def test_cast_rejects_unaligned_and_bad_enums():
+    x = torch.zeros(64, **F32)
+    q = torch.zeros(64, dtype=torch.uint8, device="cuda")
+    s = torch.ones(1, **F32)
+    with pytest.raises(fp8.FP8Error) as e:
+        fp8.fp8_cast(x[1:], fp8.FP8_E4M3, s, q)
+    assert e.value.code == fp8.FP8_ERR_UNALIGNED
+    with pytest.raises(fp8.FP8Error) as e:
+        fp8.fp8_cast(x, 7, s, q)
+    assert e.value.code == fp8.FP8_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------------- GEMMs
+def quantised_linear(M, N, K, key, x_std=1.0, w_std=0.02, dy_std=1e-4):
+    """E4M3 X, W and E5M2 dY codes + scales, made by the GPU cast chain."""
+    X, W, dY = synth.linear_inputs_f32(M, N, K, x_std, w_std, dy_std, *key)
+    out = {}
+    for name, host, fmt in (("x", X, fp8.FP8_E4M3), ("w", W, fp8.FP8_E4M3), ("dy", dY, fp8.FP8_E5M2)):
+        d = to_dev(host)
+        a, s, inv = scalar(), scalar(), scalar()
+        q = torch.empty(host.shape, dtype=torch.uint8, device="cuda")
+        fp8.fp8_amax(d, a)
+        fp8.fp8_compute_scale(a, fmt, 0, 1.0, s, inv)
+        fp8.fp8_cast(d, fmt, s, q)
+        out[name] = (q, inv)
+    return out
+
+
+OUT_DT = {fp8.FP8_DT_F32: torch.float32, fp8.FP8_DT_BF16: torch.bfloat16, fp8.FP8_DT_F16: torch.float16}
+
+SHAPES = [(256, 256, 256), (128, 256, 128), (16, 16, 16), (272, 400, 208), (384, 528, 1040),
+          (1024, 768, 4096)]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("out_dt", [fp8.FP8_DT_F32, fp8.FP8_DT_BF16])
+def test_linear_gemms_vs_oracle(shape, out_dt):
+    M, N, K = shape
+    q = quantised_linear(M, N, K, ("gemm", shape))
+    (xq, xi), (wq, wi), (dyq, dyi) = q["x"], q["w"], q["dy"]
+    tdt = OUT_DT[out_dt]
+    y = torch.empty((M, N), dtype=tdt, device="cuda")
+    dx = torch.empty((M, K), dtype=tdt, device="cuda")
+    dw = torch.empty((N, K), dtype=tdt, device="cuda")
+    ya, dxa, dwa = scalar(), scalar(), scalar()
+    fp8.fp8_linear_fwd(xq, xi, wq, wi, y, ya)
+    fp8.fp8_linear_dgrad(dyq, dyi, wq, wi, dx, dxa)
+    fp8.fp8_linear_wgrad(dyq, dyi, xq, xi, dw, dwa)
+    assert fp8.fp8_get_status() == 0
+    h = {k: (v[0].cpu().numpy(), float(v[1].item())) for k, v in q.items()}
+    refs = {
+        "fwd": oracle.linear_fwd(h["x"][0], h["x"][1], h["w"][0], h["w"][1], M, N, K),
+        "dgrad": oracle.linear_dgrad(h["dy"][0], h["dy"][1], h["w"][0], h["w"][1], M, N, K),
+        "wgrad": oracle.linear_wgrad(h["dy"][0], h["dy"][1], h["x"][0], h["x"][1], M, N, K),
+    }
+    for name, out, amax in (("fwd", y, ya), ("dgrad", dx, dxa), ("wgrad", dw, dwa)):
+        ref, rabs = refs[name]
+        got = tensor_to_np(out)
+        assert_gemm_close(got, ref, rabs, tdt, f"{name} {shape}")
+        # fused amax == amax of the GPU's own stored output, bit-exact
+        assert amax.item() == float(np.max(np.abs(got))), name
+
+
+def test_linear_fwd_bias_f16_out():
+    M, N, K = 256, 272, 128
+    q = quantised_linear(M, N, K, ("bias",))
+    (xq, xi), (wq, wi) = q["x"], q["w"]
+    bias = synth.normal_f32((N,), 0.5, "bias", "b")
+    for bdt, tb in ((fp8.FP8_DT_F32, to_dev(bias)), (fp8.FP8_DT_BF16, to_dev(bias).bfloat16())):
+        y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+        ya = scalar()
+        fp8.fp8_linear_fwd(xq, xi, wq, wi, y, ya, bias=tb)
+        b_used = tb.double().cpu().numpy()
+        ref, rabs = oracle.linear_fwd(xq.cpu().numpy(), xi.item(), wq.cpu().numpy(), wi.item(), M, N, K,
+                                      bias=b_used)
+        got = y.double().cpu().numpy()
+        assert_gemm_close(got, ref, rabs, torch.float16, f"bias {bdt}")
+        assert ya.item() == float(np.max(np.abs(got)))
+
+
+def test_gemm_exact_integer_operands():
+    """Codes for +-1, +-2 only: every partial sum is an exact integer, so the
+    FP32 accumulation must equal the oracle exactly."""
+    M, N, K = 256, 256, 2048
+    g = synth.rng("gemm", "int")
+    pick = np.array([0x38, 0xB8, 0x40, 0xC0], np.uint8)
+    xq = pick[g.integers(0, 4, (M, K))]
+    wq = pick[g.integers(0, 4, (N, K))]
+    one = torch.ones(1, **F32)
+    y = torch.empty((M, N), **F32)
+    fp8.fp8_linear_fwd(to_dev(xq), one, to_dev(wq), one, y)
+    ref, _ = oracle.linear_fwd(xq, 1.0, wq, 1.0, M, N, K)
+    assert np.array_equal(y.cpu().numpy().astype(np.float64), ref)
+
+
+def test_gemm_rejects_unsupported_shapes():
+    a = torch.zeros((32, 24), dtype=torch.uint8, device="cuda")
+    b = torch.zeros((32, 24), dtype=torch.uint8, device="cuda")
+    y = torch.zeros((32, 32), **F32)
+    one = torch.ones(1, **F32)
+    with pytest.raises(fp8.FP8Error) as e:
+        fp8.fp8_linear_fwd(a, one, b, one, y)
+    assert e.value.code == fp8.FP8_ERR_UNSUPPORTED
+
+
+def test_gemm_empty_rows_writes_zero_amax():
+    a = torch.zeros((0, 32), dtype=torch.uint8, device="cuda")
+    b = torch.zeros((32, 32), dtype=torch.uint8, device="cuda")
+    y = torch.zeros((0, 32), **F32)
+    ya = torch.full((1,), 3.0, **F32)
+    one = torch.ones(1, **F32)
+    fp8.fp8_linear_fwd(a, one, b, one, y, ya)
+    assert ya.item() == 0.0
+
+
+# ---------------------------------------------------------------- Adam
+HP = dict(lr=1e-4, beta1=0.9, beta2=0.95, eps=1e-8)
+
+
+def make_adam_state(sizes, key, steps_done=0):
+    """Per chunk: E5M2 grads (mu = 2^10) and a stored state built by the GPU
+    cast chain from seeded fp32 tensors (zero moments when steps_done == 0)."""
+    chunks, host = [], []
+    for ci, n in enumerate(sizes):
+        gf = synth.adam_grad_f32(n, 1e-3, *key, ci, "g")
+        wf = synth.normal_f32((n,), 0.02, *key, ci, "w")
+        st = {}
+        for name, arr, fmt, mu in (("g", gf, fp8.FP8_E5M2, 2.0 ** 10), ("w", wf, fp8.FP8_F16S, 1.0)):
+            d = to_dev(arr)
+            a, s, inv = scalar(), scalar(), scalar()
+            q = torch.empty(n, dtype=torch.uint8 if fmt != fp8.FP8_F16S else torch.int16, device="cuda")
+            fp8.fp8_amax(d, a)
+            fp8.fp8_compute_scale(a, fmt, 0, mu, s, inv)
+            fp8.fp8_cast(d, fmt, s, q)
+            st[name] = (q, s, inv)
+        if steps_done:
+            mf = synth.normal_f32((n,), 1e-4, *key, ci, "m")
+            vf = np.abs(synth.normal_f32((n,), 1e-7, *key, ci, "v"))
+            for name, arr, fmt in (("m", mf, fp8.FP8_E4M3), ("v", vf, fp8.FP8_F16S)):
+                d = to_dev(arr)
+                a, s, inv = scalar(), scalar(), scalar()
+                q = torch.empty(n, dtype=torch.uint8 if fmt != fp8.FP8_F16S else torch.int16, device="cuda")
+                fp8.fp8_amax(d, a)
+                fp8.fp8_compute_scale(a, fmt, 0, 1.0, s, inv)
+                fp8.fp8_cast(d, fmt, s, q)
+                st[name] = (q, s)
+        else:
+            st["m"] = (torch.zeros(n, dtype=torch.uint8, device="cuda"), torch.ones(1, **F32))
+            st["v"] = (torch.zeros(n, dtype=torch.int16, device="cuda"), torch.ones(1, **F32))
+        c = fp8.AdamChunk(st["g"][0], st["g"][2], st["m"][0], st["m"][1], st["v"][0], st["v"][1],
+                          st["w"][0], st["w"][1])
+        chunks.append(c)
+    return chunks
+
+
+def snapshot(c):
+    return dict(g=c.g.cpu().numpy(), g_inv=c.g_inv.item(), m=c.m.cpu().numpy(), s_m=c.m_scale.item(),
+                v=c.v.cpu().numpy().view(np.uint16), s_v=c.v_scale.item(),
+                w=c.w.cpu().numpy().view(np.uint16), s_w=c.w_scale.item())
+
+
+def check_adam_chunk(before, c, step, margin=0):
+    out = oracle.adam_step(before["g"], before["g_inv"], before["m"], before["s_m"], before["v"],
+                           before["s_v"], before["w"], before["s_w"], t=step, margin=margin, **HP)
+    after = snapshot(c)
+    # scales bit-equal unless the oracle amax sits on a power-of-two threshold
+    for key, amax, fmax in (("s_m", out["amax"][0], 448.0), ("s_v", out["amax"][1], 65504.0),
+                            ("s_w", out["amax"][2], 65504.0)):
+        if after[key] != out[key]:
+            e = oracle.floor_log2_ratio(amax, fmax)
+            thresh = fmax * 2.0 ** (-e)
+            assert abs(amax - thresh) <= 4 * np.spacing(np.float32(thresh)), (key, after[key], out[key])
+            pytest.skip(f"tie: oracle amax {amax} on a scale threshold")
+    # master and second moment within 1 FP16 ULP of the dequantised oracle value
+    for key, skey in (("w", "s_w"), ("v", "s_v")):
+        ref = f16_vals(out[key]) / out[skey]
+        got = f16_vals(after[key]) / after[skey]
+        ulp = f16_ulp(f16_vals(out[key])) / out[skey]
+        bad = np.abs(got - ref) > ulp
+        assert not np.any(bad), (key, np.count_nonzero(bad), got[bad][:4], ref[bad][:4])
+    # first moment within 1 code (scales equal)
+    assert np.all(np.abs(code_rank(after["m"]) - code_rank(out["mq"])) <= 1)
+    return out
+
+
+@pytest.mark.parametrize("sizes", [[65536], [1, 7, 16, 4099, 65536 + 5, 0], [300000, 4096 * 3]])
+@pytest.mark.parametrize("steps_done", [0, 4])
+def test_adam_step_vs_oracle(sizes, steps_done):
+    chunks = make_adam_state(sizes, ("adam", len(sizes), steps_done), steps_done)
+    ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(chunks)) // 4, **F32)
+    step = steps_done + 1
+    before = [snapshot(c) for c in chunks]
+    fp8.fp8_adam_step(chunks, step=step, margin=0, workspace=ws, **HP)
+    assert fp8.fp8_get_status() == 0
+    for b, c in zip(before, chunks):
+        if b["g"].size:
+            check_adam_chunk(b, c, step)
+
+
+def test_adam_three_steps_stage_parity():
+    """Each step's oracle input is the GPU's own stored state from the step before."""
+    chunks = make_adam_state([50000, 12345], ("adam3",))
+    ws = torch.zeros(fp8.fp8_adam_workspace_bytes(2) // 4, **F32)
+    for step in (1, 2, 3):
+        before = [snapshot(c) for c in chunks]
+        fp8.fp8_adam_step(chunks, step=step, margin=1, workspace=ws, **HP)
+        for b, c in zip(before, chunks):
+            out = oracle.adam_step(b["g"], b["g_inv"], b["m"], b["s_m"], b["v"], b["s_v"], b["w"], b["s_w"],
+                                   t=step, margin=1, **HP)
+            a = snapshot(c)
+            assert (a["s_m"], a["s_v"], a["s_w"]) == (out["s_m"], out["s_v"], out["s_w"])
+
+
+def test_adam_many_chunks_multiple_launches():
+    sizes = [37 + 16 * i for i in range(300)]  # > 256 chunks: two launch groups
+    chunks = make_adam_state(sizes, ("adam-many",))
+    ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(chunks)) // 4, **F32)
+    before = [snapshot(c) for c in chunks]
+    fp8.fp8_adam_step(chunks, step=1, margin=0, workspace=ws, **HP)
+    for i in (0, 1, 255, 256, 299):
+        check_adam_chunk(before[i], chunks[i], 1)
+
+
+def test_adam_rejects_bad_args():
+    chunks = make_adam_state([64], ("adam-bad",))
+    ws = torch.zeros(16, **F32)
+    with pytest.raises(fp8.FP8Error):
+        fp8.fp8_adam_step(chunks, step=0, margin=0, workspace=ws, **HP)
+    with pytest.raises(fp8.FP8Error):
+        fp8.fp8_adam_step(chunks, step=1, margin=0, workspace=ws[:3], **HP)
