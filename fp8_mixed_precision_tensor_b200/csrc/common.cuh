@@ -65,21 +65,17 @@ __device__ __forceinline__ float pow2f(int k) {  // k in [-126, 127]
 
 __device__ __forceinline__ int clamp_exp(int k) { return k < -126 ? -126 : (k > 126 ? 126 : k); }
 
-// Exponent k of the scale 2^k for a tensor with this amax; log2mu = log2(mu).
-// Returns false (and k = 0) for a non-finite amax.
+// Exponent k of the total scale mu * s_g = 2^k for a tensor with this amax,
+// where s_g = 2^clamp(floor(log2(fmax / (mu * amax))) - margin) and
+// log2mu = log2(mu).  amax == 0 and a non-finite amax give s_g = 1; the
+// latter returns false.
 __device__ __forceinline__ bool scale_exponent(float amax, float fmax, int margin, int log2mu,
                                                int &k) {
-  if (!(fabsf(amax) <= 3.402823466e38f)) {  // NaN or inf
-    k = 0;
-    return false;
-  }
-  if (amax == 0.0f) {
-    k = 0;
-    return true;
-  }
-  int kg = clamp_exp(floor_log2_ratio(amax, fmax) - log2mu - margin);  // s_g = 2^kg
-  k = clamp_exp(kg + log2mu);                                          // mu * s_g
-  return true;
+  const bool finite = fabsf(amax) <= 3.402823466e38f;  // false for NaN and inf
+  int kg = 0;
+  if (finite && amax != 0.0f) kg = clamp_exp(floor_log2_ratio(amax, fmax) - log2mu - margin);
+  k = clamp_exp(kg + log2mu);
+  return finite;
 }
 
 // ---------------------------------------------------------------------------

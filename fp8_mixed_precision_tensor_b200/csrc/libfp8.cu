@@ -81,7 +81,6 @@ int launch_rc() { return cuda_rc(cudaGetLastError()); }
 
 bool valid_dtype(int dt) { return dt == FP8_DT_F32 || dt == FP8_DT_BF16 || dt == FP8_DT_F16; }
 bool valid_fmt(int f) { return f == FP8_E4M3 || f == FP8_E5M2 || f == FP8_F16S; }
-size_t dtype_bytes(int dt) { return dt == FP8_DT_F32 ? 4 : 2; }
 
 unsigned grid_for(size_t work_items, int per_block, int cap) {
   size_t b = (work_items + per_block - 1) / per_block;
@@ -109,14 +108,14 @@ template <bool A_MN, bool B_MN>
 int run_gemm(const uint8_t *A, int fmt_a, const float *inv_a, const uint8_t *B, int fmt_b,
              const float *inv_b, const void *bias, int bias_dtype, void *out, int out_dtype,
              float *out_amax, int rows, int cols, int K, cudaStream_t stream) {
-  if (!A || !B || !inv_a || !inv_b || !out) return FP8_ERR_INVALID_ARG;
   if (rows < 0 || cols < 0 || K < 0) return FP8_ERR_INVALID_ARG;
   if (!valid_dtype(out_dtype) || (bias && !valid_dtype(bias_dtype))) return FP8_ERR_INVALID_ARG;
-  if (!aligned16(A) || !aligned16(B) || !aligned16(out)) return FP8_ERR_UNALIGNED;
-  if (rows == 0 || cols == 0) {
+  if (rows == 0 || cols == 0) {  // empty output: operands may be null
     if (out_amax) return cuda_rc(cudaMemsetAsync(out_amax, 0, sizeof(float), stream));
     return FP8_OK;
   }
+  if (!A || !B || !inv_a || !inv_b || !out) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(out)) return FP8_ERR_UNALIGNED;
   if (K == 0 || rows % 16 || cols % 16 || K % 16) return FP8_ERR_UNSUPPORTED;
   DeviceInfo *d;
   int rc = device_info(&d);

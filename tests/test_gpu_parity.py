@@ -79,7 +79,7 @@ def test_amax_rejects_unaligned():
 # ---------------------------------------------------------------- scale
 def test_compute_scale_bit_exact_sweep():
     g = synth.rng("scale", "sweep")
-    amaxes = list(np.exp(g.uniform(-95, 95, 300)).astype(np.float32))
+    amaxes = list(np.exp(g.uniform(-87, 87, 300)).astype(np.float32))
     amaxes += [0.0, 448.0, 57344.0, 65504.0, 1.0, 1e-45, 1.17e-38, 3.0e38,
                float(np.nextafter(np.float32(448), np.float32(1e9))), float(np.float32(448 * 0.75))]
     am = torch.tensor(amaxes, **F32)
@@ -343,10 +343,10 @@ def check_adam_chunk(before, c, step, margin=0):
             assert abs(amax - thresh) <= 4 * np.spacing(np.float32(thresh)), (key, after[key], out[key])
             pytest.skip(f"tie: oracle amax {amax} on a scale threshold")
     # master and second moment within 1 FP16 ULP of the dequantised oracle value
-    for key, skey in (("w", "s_w"), ("v", "s_v")):
-        ref = f16_vals(out[key]) / out[skey]
+    for key, okey, skey in (("w", "wh", "s_w"), ("v", "vh", "s_v")):
+        ref = f16_vals(out[okey]) / out[skey]
         got = f16_vals(after[key]) / after[skey]
-        ulp = f16_ulp(f16_vals(out[key])) / out[skey]
+        ulp = f16_ulp(f16_vals(out[okey])) / out[skey]
         bad = np.abs(got - ref) > ulp
         assert not np.any(bad), (key, np.count_nonzero(bad), got[bad][:4], ref[bad][:4])
     # first moment within 1 code (scales equal)
