@@ -303,6 +303,38 @@ int fp8_adam_step(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hpar
   return FP8_OK;
 }
 
+// Scratch of fp8_adam_step_noalloc: one 64-byte slot per chunk, in a fixed
+// array so the call needs no memory from the caller.  Host code must not use
+// the array's name as an address (on the host it is only a stand-in); each
+// device's real address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) float
+    g_adam_noalloc_scratch[FP8_ADAM_NOALLOC_MAX_CHUNKS * kAdamWsFloatsPerChunk];
+static void *g_noalloc_addr[kMaxDevices];
+
+static int noalloc_scratch(void **out) {
+  int dev;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP8_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_adam_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return FP8_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return FP8_OK;
+}
+
+int fp8_adam_step_noalloc(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp,
+                          void *stream) {
+  if (nchunks <= 0 || nchunks > FP8_ADAM_NOALLOC_MAX_CHUNKS) return FP8_ERR_INVALID_ARG;
+  void *scratch = nullptr;
+  int rc = noalloc_scratch(&scratch);
+  if (rc) return rc;
+  return fp8_adam_step(chunks, nchunks, hp, scratch,
+                       (size_t)FP8_ADAM_NOALLOC_MAX_CHUNKS * kAdamWsFloatsPerChunk * sizeof(float), stream);
+}
+
 int fp8_get_status(unsigned *host_out, void *stream) {
   if (!host_out) return FP8_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

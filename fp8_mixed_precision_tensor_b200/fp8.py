@@ -28,8 +28,8 @@ FP8_E4M3, FP8_E5M2, FP8_F16S = 0, 1, 2
 _DT = {torch.float32: FP8_DT_F32, torch.bfloat16: FP8_DT_BF16, torch.float16: FP8_DT_F16}
 
 SYMBOLS = ("fp8_amax", "fp8_compute_scale", "fp8_cast", "fp8_linear_fwd", "fp8_linear_dgrad",
-           "fp8_linear_wgrad", "fp8_adam_workspace_bytes", "fp8_adam_step", "fp8_get_status",
-           "fp8_strerror")
+           "fp8_linear_wgrad", "fp8_adam_workspace_bytes", "fp8_adam_step", "fp8_adam_step_noalloc",
+           "fp8_get_status", "fp8_strerror")
 
 
 class FP8Error(RuntimeError):
@@ -69,6 +69,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fp8_linear_wgrad.argtypes = [p, p, p, p, p, i, p, i, i, i, p]
     lib.fp8_adam_workspace_bytes.argtypes, lib.fp8_adam_workspace_bytes.restype = [i], sz
     lib.fp8_adam_step.argtypes = [ctypes.POINTER(_Chunk), i, ctypes.POINTER(_HParams), p, sz, p]
+    lib.fp8_adam_step_noalloc.argtypes = [ctypes.POINTER(_Chunk), i, ctypes.POINTER(_HParams), p]
     lib.fp8_get_status.argtypes = [ctypes.POINTER(ctypes.c_uint), p]
     lib.fp8_strerror.argtypes, lib.fp8_strerror.restype = [i], ctypes.c_char_p
     for name in SYMBOLS:
@@ -185,6 +186,20 @@ def fp8_adam_step(chunks, lr: float, beta1: float, beta2: float, eps: float, ste
     _check(load_library().fp8_adam_step(arr, len(arr), ctypes.byref(hp), _ptr(workspace),
                                         workspace.numel() * workspace.element_size(), _stream(stream)),
            "fp8_adam_step")
+
+
+FP8_ADAM_NOALLOC_MAX_CHUNKS = 1024
+
+
+def fp8_adam_step_noalloc(chunks, lr: float, beta1: float, beta2: float, eps: float, step: int,
+                          margin: int, stream=None) -> None:
+    """fp8_adam_step for callers that cannot provide device memory: the
+    library's fixed per-device scratch array replaces the workspace (at most
+    FP8_ADAM_NOALLOC_MAX_CHUNKS chunks; calls overlapping on the GPU race)."""
+    arr = chunks if isinstance(chunks, ctypes.Array) else pack_adam_chunks(chunks)
+    hp = _HParams(lr, beta1, beta2, eps, step, margin)
+    _check(load_library().fp8_adam_step_noalloc(arr, len(arr), ctypes.byref(hp), _stream(stream)),
+           "fp8_adam_step_noalloc")
 
 
 def fp8_get_status(stream=None) -> int:

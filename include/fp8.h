@@ -192,6 +192,30 @@ int fp8_adam_step(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hpar
                   void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * fp8_adam_step_noalloc -- the same step as fp8_adam_step, for callers that
+ * cannot hand the library any device memory of their own: code running under
+ * a host framework whose caching allocator owns (and has already reserved)
+ * the GPU's memory, plugins whose host forbids raw cudaMalloc, and loops that
+ * must never hit the device-wide synchronisation cudaMalloc/cudaFree can
+ * cause.  The paper has no counterpart; this is a deployment convenience.
+ *
+ * The per-chunk scratch lives in a fixed array compiled into the library
+ * (FP8_ADAM_NOALLOC_MAX_CHUNKS x 64 bytes = 64 KiB on every GPU that loads
+ * the library, held until the process exits).  The call allocates and frees
+ * nothing.  nchunks above FP8_ADAM_NOALLOC_MAX_CHUNKS returns
+ * FP8_ERR_INVALID_ARG before any work is enqueued.
+ * The first call on a device looks up that device's copy of the array (a
+ * cudaGetSymbolAddress with the device current); make that first call before
+ * any stream capture.  Every call on a device shares the one array: the step
+ * clears the part it needs before use, and two calls whose work overlaps on
+ * the GPU (different streams, no ordering between them) race on it.
+ * Arguments, results and errors are otherwise those of fp8_adam_step.
+ */
+#define FP8_ADAM_NOALLOC_MAX_CHUNKS 1024
+int fp8_adam_step_noalloc(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp,
+                          void *stream);
+
+/*
  * fp8_get_status -- waits for `stream`, then reads the device status word
  * (OR of FP8_STATUS_* bits raised since the last read) into *host_out and
  * clears it.  Returns FP8_ERR_CUDA if the stream reported an error.
