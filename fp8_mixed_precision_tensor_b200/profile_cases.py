@@ -1,0 +1,114 @@
+"""Run one kernel family of the hot path on a chosen case (for profilers).
+
+    python -m fp8_mixed_precision_tensor_b200.profile_cases linear --M 4096 --N 16384 --K 4096
+    python -m fp8_mixed_precision_tensor_b200.profile_cases cast --n 268435456
+    python -m fp8_mixed_precision_tensor_b200.profile_cases adam --n 67108864
+
+Each case runs `--iters` passes after one warm-up pass on seeded synthetic
+inputs and prints the CUDA-event time per pass.  Launch order per pass:
+linear: amax/scale/cast of X, W, dY (9 launches), then fwd, dgrad, wgrad;
+cast: amax, scale, cast; adam: stats pass, finalize, update pass.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from fp8_mixed_precision_tensor_b200 import fp8, synth
+
+
+def _scalars(n):
+    return torch.zeros(n, dtype=torch.float32, device="cuda")
+
+
+def case_linear(a):
+    M, N, K = a.M, a.N, a.K
+    X = synth.device_normal((M, K), synth.ACT_STD, 1, torch.bfloat16, "cuda")
+    W = synth.device_normal((N, K), synth.GPT7B_W_STD, 2, torch.bfloat16, "cuda")
+    dY = synth.device_normal((M, N), synth.GRAD_STD, 3, torch.bfloat16, "cuda")
+    u8 = dict(dtype=torch.uint8, device="cuda")
+    xq, wq, dyq = torch.empty((M, K), **u8), torch.empty((N, K), **u8), torch.empty((M, N), **u8)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    dx = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    dw = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    sc = _scalars(16)
+
+    def one():
+        for t, q, i, fmt in ((X, xq, 0, fp8.FP8_E4M3), (W, wq, 3, fp8.FP8_E4M3), (dY, dyq, 6, fp8.FP8_E5M2)):
+            fp8.fp8_amax(t, sc[i:i + 1])
+            fp8.fp8_compute_scale(sc[i:i + 1], fmt, 0, 1.0, sc[i + 1:i + 2], sc[i + 2:i + 3])
+            fp8.fp8_cast(t, fmt, sc[i + 1:i + 2], q)
+        fp8.fp8_linear_fwd(xq, sc[2:3], wq, sc[5:6], y, sc[12:13])
+        fp8.fp8_linear_dgrad(dyq, sc[8:9], wq, sc[5:6], dx, sc[13:14])
+        fp8.fp8_linear_wgrad(dyq, sc[8:9], xq, sc[2:3], dw, sc[14:15])
+
+    return one
+
+
+def case_cast(a):
+    x = synth.device_normal((a.n,), 1.0, 4, torch.bfloat16, "cuda")
+    q = torch.empty(a.n, dtype=torch.uint8, device="cuda")
+    sc = _scalars(3)
+
+    def one():
+        fp8.fp8_amax(x, sc[0:1])
+        fp8.fp8_compute_scale(sc[0:1], fp8.FP8_E4M3, 0, 1.0, sc[1:2], sc[2:3])
+        fp8.fp8_cast(x, fp8.FP8_E4M3, sc[1:2], q)
+
+    return one
+
+
+def case_adam(a):
+    n = a.n
+    g = synth.device_normal((n,), 1e-3, 5, torch.float32, "cuda")
+    w = synth.device_normal((n,), 0.02, 6, torch.float32, "cuda")
+    sc = _scalars(8)
+    gq = torch.empty(n, dtype=torch.uint8, device="cuda")
+    wh = torch.empty(n, dtype=torch.int16, device="cuda")
+    fp8.fp8_amax(g, sc[0:1])
+    fp8.fp8_compute_scale(sc[0:1], fp8.FP8_E5M2, 0, 2.0 ** 10, sc[1:2], sc[2:3])
+    fp8.fp8_cast(g, fp8.FP8_E5M2, sc[1:2], gq)
+    fp8.fp8_amax(w, sc[3:4])
+    fp8.fp8_compute_scale(sc[3:4], fp8.FP8_F16S, 0, 1.0, sc[4:5], sc[5:6])
+    fp8.fp8_cast(w, fp8.FP8_F16S, sc[4:5], wh)
+    del g, w
+    m = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    v = torch.zeros(n, dtype=torch.int16, device="cuda")
+    st = torch.ones(2, dtype=torch.float32, device="cuda")
+    chunks = fp8.pack_adam_chunks([fp8.AdamChunk(gq, sc[2:3], m, st[0:1], v, st[1:2], wh, sc[4:5])])
+    ws = torch.zeros(64, dtype=torch.float32, device="cuda")
+    state = {"t": 0}
+
+    def one():
+        state["t"] += 1
+        fp8.fp8_adam_step(chunks, 1e-4, 0.9, 0.95, 1e-8, state["t"], 0, ws)
+
+    return one
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("case", choices=["linear", "cast", "adam"])
+    ap.add_argument("--M", type=int, default=4096)
+    ap.add_argument("--N", type=int, default=16384)
+    ap.add_argument("--K", type=int, default=4096)
+    ap.add_argument("--n", type=int, default=1 << 26)
+    ap.add_argument("--iters", type=int, default=2)
+    a = ap.parse_args()
+    one = {"linear": case_linear, "cast": case_cast, "adam": case_adam}[a.case](a)
+    one()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(a.iters):
+        one()
+    e.record()
+    e.synchronize()
+    status = fp8.fp8_get_status()
+    print(f"{a.case}: {s.elapsed_time(e) / a.iters:.4f} ms per pass, device status {status}")
+    return 0 if status == 0 else 1
+
+
+if __name__ == "__main__":
+    raise SystemExit(main())
