@@ -51,30 +51,57 @@ struct AdamLaunch {
   int nchunks;
   int margin;
   unsigned long long total_tiles;
-  float lr, beta1, beta2, eps;
-  float inv_bc1, inv_bc2;  // 1 / (1 - beta^t)
+  float beta1, beta2, eps;
+  float neg_lr_bc1;        // -lr / (1 - beta1^t)
+  float inv_bc2;           // 1 / (1 - beta2^t)
   float *ws;               // kAdamWsFloatsPerChunk floats per chunk of this launch
 };
 
-// The update of one parameter, float32.  Written with explicit round-to-
-// nearest intrinsics so both passes evaluate exactly the same operations.
+// Per-chunk constants of the update: the descales are folded into the Adam
+// coefficients, m = (b1/s_m) m~ + ((1-b1)/(mu s_g)) g~ and
+// v = (b2/s_v) v~ + ((1-b2)/(mu s_g)^2) g~^2, where ~ marks a decoded code.
 struct AdamScalars {
-  float g_inv, m_inv, v_inv, w_inv;
+  float cm, cgm;   // b1 / s_m,  (1 - b1) g_inv
+  float cv, cgv;   // b2 / s_v,  (1 - b2) g_inv^2
+  float w_inv;     // 1 / s_w
 };
 
+__device__ __forceinline__ AdamScalars adam_scalars(const AdamLaunch &L, float g_inv, float m_inv,
+                                                    float v_inv, float w_inv) {
+  AdamScalars s;
+  s.cm = __fmul_rn(L.beta1, m_inv);
+  s.cgm = __fmul_rn(__fsub_rn(1.0f, L.beta1), g_inv);
+  s.cv = __fmul_rn(L.beta2, v_inv);
+  s.cgv = __fmul_rn(__fmul_rn(__fsub_rn(1.0f, L.beta2), g_inv), g_inv);
+  s.w_inv = w_inv;
+  return s;
+}
+
+// Approximate (MUFU) square root and reciprocal: relative error ~1e-7 on the
+// step direction m_hat / (sqrt(v_hat) + eps), which moves the master weight by
+// lr * O(1) -- far below an FP16 ULP of the stored master.
+__device__ __forceinline__ float sqrt_approx(float x) {
+  float r;
+  asm("sqrt.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// The update of one parameter, float32, from decoded codes.  Written with
+// explicit round-to-nearest intrinsics so both passes evaluate exactly the
+// same operations (the stats pass must see the values the update pass
+// stores).  L.neg_lr_bc1 = -lr / (1 - b1^t), L.inv_bc2 = 1 / (1 - b2^t).
 __device__ __forceinline__ void adam_update(const AdamLaunch &L, float gd, float md, float vd,
                                             float wd, const AdamScalars &s, float &m, float &v,
                                             float &w) {
-  float g = __fmul_rn(gd, s.g_inv);
-  float m0 = __fmul_rn(md, s.m_inv);
-  float v0 = __fmul_rn(vd, s.v_inv);
-  float w0 = __fmul_rn(wd, s.w_inv);
-  m = __fadd_rn(__fmul_rn(L.beta1, m0), __fmul_rn(__fsub_rn(1.0f, L.beta1), g));
-  v = __fadd_rn(__fmul_rn(L.beta2, v0), __fmul_rn(__fsub_rn(1.0f, L.beta2), __fmul_rn(g, g)));
-  float mhat = __fmul_rn(m, L.inv_bc1);
-  float vhat = __fmul_rn(v, L.inv_bc2);
-  float denom = __fadd_rn(__fsqrt_rn(vhat), L.eps);
-  w = __fsub_rn(w0, __fdiv_rn(__fmul_rn(L.lr, mhat), denom));
+  m = __fmaf_rn(s.cm, md, __fmul_rn(s.cgm, gd));
+  v = __fmaf_rn(s.cv, vd, __fmul_rn(s.cgv, __fmul_rn(gd, gd)));
+  const float denom = __fadd_rn(sqrt_approx(__fmul_rn(v, L.inv_bc2)), L.eps);
+  w = __fmaf_rn(L.neg_lr_bc1, __fmul_rn(m, rcp_approx(denom)), __fmul_rn(wd, s.w_inv));
 }
 
 __device__ __forceinline__ int find_chunk(const AdamLaunch &L, unsigned long long tile) {
@@ -90,7 +117,7 @@ template <int PASS>
 __global__ void __launch_bounds__(kAdamThreads) k_adam(const __grid_constant__ AdamLaunch L) {
   uint32_t am = 0, av = 0, aw = 0;  // pass 1: running maxima of the current chunk
   int cur = -1;
-  AdamScalars sc{};
+  AdamScalars sc{};  // of the current chunk
   float new_m = 1.f, new_v = 1.f, new_w = 1.f;
 
   for (unsigned long long tile = blockIdx.x; tile < L.total_tiles; tile += gridDim.x) {
@@ -108,16 +135,10 @@ __global__ void __launch_bounds__(kAdamThreads) k_adam(const __grid_constant__ A
           }
           am = av = aw = 0;
         }
-        sc.g_inv = *C.g_inv;
-        sc.m_inv = 1.0f / *C.m_scale;
-        sc.v_inv = 1.0f / *C.v_scale;
-        sc.w_inv = 1.0f / *C.w_scale;
+        sc = adam_scalars(L, *C.g_inv, 1.0f / *C.m_scale, 1.0f / *C.v_scale, 1.0f / *C.w_scale);
       } else {
         const float *ws = L.ws + ci * kAdamWsFloatsPerChunk;
-        sc.g_inv = *C.g_inv;
-        sc.m_inv = ws[WS_OLDINV_M];
-        sc.v_inv = ws[WS_OLDINV_V];
-        sc.w_inv = ws[WS_OLDINV_W];
+        sc = adam_scalars(L, *C.g_inv, ws[WS_OLDINV_M], ws[WS_OLDINV_V], ws[WS_OLDINV_W]);
         new_m = ws[WS_NEW_M];
         new_v = ws[WS_NEW_V];
         new_w = ws[WS_NEW_W];

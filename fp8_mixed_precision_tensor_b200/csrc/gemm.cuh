@@ -58,6 +58,7 @@ struct Cfg {
 struct Args {
   int rows, cols, K;           // output [rows, cols], reduction length K
   int num_m_blocks, num_n_blocks, num_tiles, num_k_blocks;
+  int group_m;                 // tile order: groups of group_m row blocks, columns inside
   uint32_t idesc;              // tcgen05 instruction descriptor
   const float *inv_a, *inv_b;  // descale factors (device scalars)
   const void *bias;            // [cols] or null
@@ -215,6 +216,130 @@ __device__ __forceinline__ float load_bias(const void *bias, int dt, int c) {
   return __half2float(__ushort_as_half((unsigned short)h));
 }
 
+// Tile order: walk the output in bands of group_m row blocks, column-major
+// inside a band, so the CTAs running at the same time share a compact block
+// of A rows and B columns in L2.
+__device__ __forceinline__ void tile_coords(int t, const Args &a, int &mb, int &nb) {
+  const int per_band = a.group_m * a.num_n_blocks;
+  const int band = t / per_band;
+  const int first = band * a.group_m;
+  const int rows_in_band = min(a.num_m_blocks - first, a.group_m);
+  const int r = t - band * per_band;
+  mb = first + r % rows_in_band;
+  nb = r / rows_in_band;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of the same shared-memory word in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// TMA load whose completion is counted on a barrier that may live in the
+// peer CTA of the pair (cta_group::2 form; no multicast).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int c0, int c1,
+                                                 uint32_t cluster_bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(cluster_bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on the barrier at this offset in both CTAs of the pair once every
+// tcgen05 operation issued so far by this thread has completed.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"((uint16_t)3)
+      : "memory");
+}
+
+__device__ __forceinline__ void sleep_ns_bounded(uint32_t total_ns) {
+  uint64_t t0 = globaltimer_ns();
+  while (globaltimer_ns() - t0 < total_ns) __nanosleep(1000);
+}
+
+// Epilogue of one 32-column chunk: descale, bias, round, store, amax.
+__device__ __forceinline__ uint32_t store_chunk(const Args &args, const uint32_t (&r)[32], int row, int col0,
+                                                float inv_a, float inv_b) {
+  const bool row_ok = row < args.rows;
+  uint32_t amax_bits = 0;
+  float y[32];
+#pragma unroll
+  for (int j = 0; j < 32; j++) y[j] = __fmul_rn(__fmul_rn(__uint_as_float(r[j]), inv_a), inv_b);
+  if (args.bias != nullptr) {
+#pragma unroll
+    for (int j = 0; j < 32; j++)
+      if (col0 + j < args.cols) y[j] = __fadd_rn(y[j], load_bias(args.bias, args.bias_dtype, col0 + j));
+  }
+  if (args.out_dtype == FP8_DT_F32) {
+    float *orow = reinterpret_cast<float *>(args.out) + (size_t)row * args.cols;
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      if (row_ok && col0 + j < args.cols) {
+        *reinterpret_cast<float4 *>(orow + col0 + j) = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
+        amax_bits = max(amax_bits, max(max(absbits_f32(y[j]), absbits_f32(y[j + 1])),
+                                       max(absbits_f32(y[j + 2]), absbits_f32(y[j + 3]))));
+      }
+    }
+  } else {
+    uint16_t *orow = reinterpret_cast<uint16_t *>(args.out) + (size_t)row * args.cols;
+    const bool bf = args.out_dtype == FP8_DT_BF16;
+#pragma unroll
+    for (int j = 0; j < 32; j += 8) {
+      uint32_t p[4];
+      uint32_t mx = 0;
+#pragma unroll
+      for (int t = 0; t < 4; t++) {
+        uint32_t lo, hi;
+        if (bf) {
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(y[j + 2 * t], y[j + 2 * t + 1]);
+          p[t] = *reinterpret_cast<uint32_t *>(&h2);
+          lo = (p[t] & 0x7fffu) << 16;
+          hi = p[t] & 0x7fff0000u;
+        } else {
+          p[t] = f16x2(y[j + 2 * t], y[j + 2 * t + 1]);
+          float2 back = h2f2(p[t]);
+          lo = absbits_f32(back.x);
+          hi = absbits_f32(back.y);
+        }
+        mx = max(mx, max(lo, hi));
+      }
+      if (row_ok && col0 + j < args.cols) {
+        *reinterpret_cast<uint4 *>(orow + col0 + j) = make_uint4(p[0], p[1], p[2], p[3]);
+        amax_bits = max(amax_bits, mx);
+      }
+    }
+  }
+  return amax_bits;
+}
+
 // ---------------------------------------------------------------------------
 template <int BN, bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -271,7 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t issued_mask = 0, issued_par = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < args.num_tiles && ok; tile += gridDim.x) {
-      const int mb = tile % args.num_m_blocks, nb = tile / args.num_m_blocks;
+      int mb, nb;
+      tile_coords(tile, args, mb, nb);
       for (int kb = 0; kb < args.num_k_blocks; kb++) {
         bool got = lane == 0 ? mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag) : true;
         got = __shfl_sync(0xffffffffu, got, 0);
@@ -347,66 +473,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x) {
-      const int mb = tile % args.num_m_blocks, nb = tile / args.num_m_blocks;
+      int mb, nb;
+      tile_coords(tile, args, mb, nb);
       bool got = lane == 0 ? mbar_wait(tfull_bar(acc), acc_phase, abort_flag) : true;
       got = __shfl_sync(0xffffffffu, got, 0);
       if (!got) break;
       tc_fence_after();
       const int row = mb * BM + q * 32 + lane;
-      const bool row_ok = row < args.rows;
       uint32_t amax_bits = 0;
 #pragma unroll 1
       for (int cc = 0; cc < BN / 32; cc++) {
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + cc * 32, r);
-        const int col0 = nb * BN + cc * 32;
-        float y[32];
-#pragma unroll
-        for (int j = 0; j < 32; j++) y[j] = __fmul_rn(__fmul_rn(__uint_as_float(r[j]), inv_a), inv_b);
-        if (args.bias != nullptr) {
-#pragma unroll
-          for (int j = 0; j < 32; j++)
-            if (col0 + j < args.cols) y[j] = __fadd_rn(y[j], load_bias(args.bias, args.bias_dtype, col0 + j));
-        }
-        if (args.out_dtype == FP8_DT_F32) {
-          float *orow = reinterpret_cast<float *>(args.out) + (size_t)row * args.cols;
-#pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            if (row_ok && col0 + j < args.cols) {
-              *reinterpret_cast<float4 *>(orow + col0 + j) = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
-              amax_bits = max(amax_bits, max(max(absbits_f32(y[j]), absbits_f32(y[j + 1])),
-                                             max(absbits_f32(y[j + 2]), absbits_f32(y[j + 3]))));
-            }
-          }
-        } else {
-          uint16_t *orow = reinterpret_cast<uint16_t *>(args.out) + (size_t)row * args.cols;
-          const bool bf = args.out_dtype == FP8_DT_BF16;
-#pragma unroll
-          for (int j = 0; j < 32; j += 8) {
-            uint32_t p[4];
-            uint32_t mx = 0;
-#pragma unroll
-            for (int t = 0; t < 4; t++) {
-              uint32_t lo, hi;
-              if (bf) {
-                __nv_bfloat162 h2 = __floats2bfloat162_rn(y[j + 2 * t], y[j + 2 * t + 1]);
-                p[t] = *reinterpret_cast<uint32_t *>(&h2);
-                lo = (p[t] & 0x7fffu) << 16;
-                hi = p[t] & 0x7fff0000u;
-              } else {
-                p[t] = f16x2(y[j + 2 * t], y[j + 2 * t + 1]);
-                float2 back = h2f2(p[t]);
-                lo = absbits_f32(back.x);
-                hi = absbits_f32(back.y);
-              }
-              mx = max(mx, max(lo, hi));
-            }
-            if (row_ok && col0 + j < args.cols) {
-              *reinterpret_cast<uint4 *>(orow + col0 + j) = make_uint4(p[0], p[1], p[2], p[3]);
-              amax_bits = max(amax_bits, mx);
-            }
-          }
-        }
+        amax_bits = max(amax_bits, store_chunk(args, r, row, nb * BN + cc * 32, inv_a, inv_b));
       }
       tc_fence_before();
       __syncwarp();
@@ -425,6 +504,373 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// Pair kernel: a cluster of two CTAs on two SMs computes 256 x 256 output
+// tiles with tcgen05.mma.cta_group::2 (M = 256, N = 256).  Each CTA loads its
+// own 128 rows of A and its own 128 columns of B (32 KB per stage, 6 stages),
+// so every SM streams half the B bytes of the one-CTA kernel for the same
+// tensor-core work.  The even CTA (the leader) counts both CTAs' TMA bytes on
+// its "full" barriers and issues the MMAs, which read A and B from both
+// CTAs' shared memory and write each CTA's 128 accumulator rows into that
+// CTA's TMEM.  Commits are multicast to the same barrier in both CTAs; the
+// epilogue warps of both CTAs return the accumulator to the leader with a
+// remote arrive.  No TMA load is multicast.  Launched as clusters of two
+// CTAs (cudaLaunchAttributeClusterDimension = 2).
+constexpr int kPairBN = 256;     // output columns per pair tile
+constexpr int kPairHalf = 128;   // rows (and B columns) held by one CTA
+constexpr int kPairStages = 6;
+constexpr int kPairStageBytes = 2 * kPairHalf * BK;  // A 16 KB + B 16 KB
+constexpr int kPairTmemCols = 2 * kPairBN;
+constexpr int kPairSmemBytes = kPairStages * kPairStageBytes + 256 + 1024;
+
+template <bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+            const Args args) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *base_ptr = smem_raw + (base - raw);
+  const uint32_t bar0 = base + kPairStages * kPairStageBytes;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kPairStages + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * kPairStages + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * kPairStages + 2 + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * kPairStages + 4);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + kPairStages * kPairStageBytes + 8 * (2 * kPairStages + 5));
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; s++) {
+      mbar_init(full_bar(s), 1);   // leader: its producer's arrive + both CTAs' bytes
+      mbar_init(empty_bar(s), 1);  // one multicast commit per phase
+    }
+    for (int b = 0; b < 2; b++) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 8);  // leader: 4 epilogue warps x 2 CTAs
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"((uint32_t)kPairTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync();  // barriers of both CTAs initialised before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producers (both CTAs)
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true, issued = false;
+    for (int tile = pair; tile < args.num_tiles && ok; tile += num_pairs) {
+      int mb, nb;
+      tile_coords(tile, args, mb, nb);
+      const int arow = mb * (2 * kPairHalf) + (int)rank * kPairHalf;
+      const int bcol = nb * kPairBN + (int)rank * kPairHalf;
+      for (int kb = 0; kb < args.num_k_blocks; kb++) {
+        bool got = lane == 0 ? mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag) : true;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) { ok = false; break; }
+        if (lane == 0) {
+          const uint32_t sa = base + stage * kPairStageBytes, sb = sa + kPairHalf * BK;
+          const uint32_t fb = map_to_rank(full_bar(stage), 0);
+          if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * kPairStageBytes);
+          if (A_MN) tma_load_2d_pair(sa, &tmA, arow, kb * BK, fb);
+          else      tma_load_2d_pair(sa, &tmA, kb * BK, arow, fb);
+          if (B_MN) tma_load_2d_pair(sb, &tmB, bcol, kb * BK, fb);
+          else      tma_load_2d_pair(sb, &tmB, kb * BK, bcol, fb);
+          issued = true;
+        }
+        __syncwarp();
+        if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (!ok && issued && lane == 0) sleep_ns_bounded(50000);  // let copies in flight land
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true, issued_any = false;
+      for (int tile = pair; tile < args.num_tiles && ok; tile += num_pairs) {
+        bool got = lane == 0 ? mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag) : true;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kPairBN;
+        for (int kb = 0; kb < args.num_k_blocks; kb++) {
+          got = lane == 0 ? mbar_wait(full_bar(stage), phase, abort_flag) : true;
+          got = __shfl_sync(0xffffffffu, got, 0);
+          if (!got) { ok = false; break; }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t sa = base + stage * kPairStageBytes, sb = sa + kPairHalf * BK;
+#pragma unroll
+            for (int ks = 0; ks < BK / UMMA_K; ks++) {
+              tc_mma_pair(d_tmem, operand_desc<A_MN>(sa, ks), operand_desc<B_MN>(sb, ks), args.idesc,
+                          (kb | ks) != 0 ? 1u : 0u);
+            }
+            tc_commit_pair(empty_bar(stage));
+            issued_any = true;
+          }
+          __syncwarp();
+          if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        if (lane == 0) tc_commit_pair(tfull_bar(acc));
+        __syncwarp();
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok && lane == 0 && issued_any) {
+        asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(drain_bar)
+                     : "memory");
+        mbar_wait_drain(drain_bar, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const float inv_a = *args.inv_a, inv_b = *args.inv_b;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < args.num_tiles; tile += num_pairs) {
+      int mb, nb;
+      tile_coords(tile, args, mb, nb);
+      bool got = lane == 0 ? mbar_wait(tfull_bar(acc), acc_phase, abort_flag) : true;
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) break;
+      tc_fence_after();
+      const int row = mb * (2 * kPairHalf) + (int)rank * kPairHalf + q * 32 + lane;
+      uint32_t amax_bits = 0;
+#pragma unroll 1
+      for (int cc = 0; cc < kPairBN / 32; cc++) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * kPairBN + cc * 32, r);
+        amax_bits = max(amax_bits, store_chunk(args, r, row, nb * kPairBN + cc * 32, inv_a, inv_b));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(map_to_rank(tempty_bar(acc), 0));
+      if (args.out_amax != nullptr) {
+        amax_bits = warp_max_u32(amax_bits);
+        if (lane == 0) atomic_max_bits(args.out_amax, amax_bits);
+      }
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();  // the leader's MMAs no longer read this CTA's smem / TMEM
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"((uint32_t)kPairTmemCols)
+                 : "memory");
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// Wide pair kernel: a cluster of two CTAs computes 256 x 512 output tiles.
+// Per k-slice the leader issues two tcgen05.mma.cta_group::2 (M = 256,
+// N = 256), one into each of two accumulators that together fill all 512
+// TMEM columns.  Each CTA loads its 128 rows of A (16 KB) and 256 rows of B
+// (32 KB) per stage: the same A tile now feeds twice the tensor-core work,
+// so each SM streams 48 KB per 2 x 128x256x128 MACs instead of 32 KB per one.
+// Column bookkeeping: CTA r holds B rows (output columns) [r*256, r*256+256)
+// of the tile; the MMA reading B rows [0,128) of both CTAs produces tile
+// columns {0..127, 256..383} in accumulator 0, and rows [128,256) produce
+// {128..255, 384..511} in accumulator 1.  There is no room left in TMEM for a
+// second tile, so the epilogue (eight warps, one accumulator half each)
+// runs between tiles while the producer already refills the ring.
+constexpr int kWideBN = 512;
+constexpr int kWideStages = 4;
+constexpr int kWideStageBytes = kPairHalf * BK + 2 * kPairHalf * BK;  // A 16 KB + B 32 KB
+constexpr int kWideThreads = 320;                                     // 10 warps
+constexpr int kWideSmemBytes = kWideStages * kWideStageBytes + 256 + 1024;
+
+template <bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(kWideThreads, 1)
+    k_gemm3(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+            const Args args) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *base_ptr = smem_raw + (base - raw);
+  const uint32_t bar0 = base + kWideStages * kWideStageBytes;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kWideStages + s); };
+  const uint32_t tfull_bar = bar0 + 8u * (2 * kWideStages);
+  const uint32_t tempty_bar = bar0 + 8u * (2 * kWideStages + 1);
+  const uint32_t drain_bar = bar0 + 8u * (2 * kWideStages + 2);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + kWideStages * kWideStageBytes + 8 * (2 * kWideStages + 3));
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kWideStages; s++) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(tfull_bar, 1);
+    mbar_init(tempty_bar, 16);  // leader: 8 epilogue warps x 2 CTAs
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(512u)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producers (both CTAs)
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true, issued = false;
+    for (int tile = pair; tile < args.num_tiles && ok; tile += num_pairs) {
+      int mb, nb;
+      tile_coords(tile, args, mb, nb);
+      const int arow = mb * (2 * kPairHalf) + (int)rank * kPairHalf;
+      const int bcol = nb * kWideBN + (int)rank * (2 * kPairHalf);
+      for (int kb = 0; kb < args.num_k_blocks; kb++) {
+        bool got = lane == 0 ? mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag) : true;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) { ok = false; break; }
+        if (lane == 0) {
+          const uint32_t sa = base + stage * kWideStageBytes, sb = sa + kPairHalf * BK;
+          const uint32_t fb = map_to_rank(full_bar(stage), 0);
+          if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * kWideStageBytes);
+          if (A_MN) tma_load_2d_pair(sa, &tmA, arow, kb * BK, fb);
+          else      tma_load_2d_pair(sa, &tmA, kb * BK, arow, fb);
+          if (B_MN) {
+            tma_load_2d_pair(sb, &tmB, bcol, kb * BK, fb);
+            tma_load_2d_pair(sb + kPairHalf * BK, &tmB, bcol + kPairHalf, kb * BK, fb);
+          } else {
+            tma_load_2d_pair(sb, &tmB, kb * BK, bcol, fb);  // one box of 256 rows
+          }
+          issued = true;
+        }
+        __syncwarp();
+        if (++stage == kWideStages) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (!ok && issued && lane == 0) sleep_ns_bounded(50000);  // let copies in flight land
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (leader) {
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true, issued_any = false;
+      for (int tile = pair; tile < args.num_tiles && ok; tile += num_pairs) {
+        bool got = lane == 0 ? mbar_wait(tempty_bar, acc_phase ^ 1u, abort_flag) : true;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) { ok = false; break; }
+        tc_fence_after();
+        for (int kb = 0; kb < args.num_k_blocks; kb++) {
+          got = lane == 0 ? mbar_wait(full_bar(stage), phase, abort_flag) : true;
+          got = __shfl_sync(0xffffffffu, got, 0);
+          if (!got) { ok = false; break; }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t sa = base + stage * kWideStageBytes, sb = sa + kPairHalf * BK;
+#pragma unroll
+            for (int ks = 0; ks < BK / UMMA_K; ks++) {
+              const uint64_t ad = operand_desc<A_MN>(sa, ks);
+              const uint32_t accum = (kb | ks) != 0 ? 1u : 0u;
+              tc_mma_pair(tmem_base, ad, operand_desc<B_MN>(sb, ks), args.idesc, accum);
+              tc_mma_pair(tmem_base + 256, ad, operand_desc<B_MN>(sb + kPairHalf * BK, ks), args.idesc, accum);
+            }
+            tc_commit_pair(empty_bar(stage));
+            issued_any = true;
+          }
+          __syncwarp();
+          if (++stage == kWideStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        if (lane == 0) tc_commit_pair(tfull_bar);
+        __syncwarp();
+        acc_phase ^= 1u;
+      }
+      if (!ok && lane == 0 && issued_any) {
+        asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(drain_bar)
+                     : "memory");
+        mbar_wait_drain(drain_bar, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (8 warps, both CTAs)
+    const int q = warp & 3;         // TMEM lane quarter
+    const int h = (warp - 2) >> 2;  // accumulator half: 0 or 1
+    const float inv_a = *args.inv_a, inv_b = *args.inv_b;
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < args.num_tiles; tile += num_pairs) {
+      int mb, nb;
+      tile_coords(tile, args, mb, nb);
+      bool got = lane == 0 ? mbar_wait(tfull_bar, acc_phase, abort_flag) : true;
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) break;
+      tc_fence_after();
+      const int row = mb * (2 * kPairHalf) + (int)rank * kPairHalf + q * 32 + lane;
+      uint32_t amax_bits = 0;
+#pragma unroll 1
+      for (int cc = 0; cc < 8; cc++) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + h * 256 + cc * 32, r);
+        const int col0 = nb * kWideBN + (cc < 4 ? 0 : 256) + h * kPairHalf + (cc & 3) * 32;
+        amax_bits = max(amax_bits, store_chunk(args, r, row, col0, inv_a, inv_b));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(map_to_rank(tempty_bar, 0));
+      if (args.out_amax != nullptr) {
+        amax_bits = warp_max_u32(amax_bits);
+        if (lane == 0) atomic_max_bits(args.out_amax, amax_bits);
+      }
+      acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512u)
                  : "memory");
   }
 }

@@ -25,6 +25,8 @@ struct DeviceInfo {
   bool ready = false;
   int sms = 0;
   int adam_blocks_per_sm = 1;
+  int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair GEMM
+  int wide_clusters = 0;  // co-resident 2-CTA clusters of the wide pair GEMM
 };
 
 std::mutex g_mu;
@@ -62,7 +64,35 @@ int device_info(DeviceInfo **out) {
     rc |= set_smem(gemm::k_gemm<256, false, false>, gemm::Cfg<256>::SMEM_BYTES);
     rc |= set_smem(gemm::k_gemm<256, false, true>, gemm::Cfg<256>::SMEM_BYTES);
     rc |= set_smem(gemm::k_gemm<256, true, true>, gemm::Cfg<256>::SMEM_BYTES);
+    rc |= set_smem(gemm::k_gemm2<false, false>, gemm::kPairSmemBytes);
+    rc |= set_smem(gemm::k_gemm2<false, true>, gemm::kPairSmemBytes);
+    rc |= set_smem(gemm::k_gemm2<true, true>, gemm::kPairSmemBytes);
+    rc |= set_smem(gemm::k_gemm3<false, false>, gemm::kWideSmemBytes);
+    rc |= set_smem(gemm::k_gemm3<false, true>, gemm::kWideSmemBytes);
+    rc |= set_smem(gemm::k_gemm3<true, true>, gemm::kWideSmemBytes);
     if (rc) return FP8_ERR_CUDA;
+    {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = 2;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * (d.sms / 2));
+      cfg.blockDim = dim3(gemm::kThreads);
+      cfg.dynamicSmemBytes = gemm::kPairSmemBytes;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, gemm::k_gemm2<false, false>, &cfg) != cudaSuccess)
+        return FP8_ERR_CUDA;
+      d.pair_clusters = clusters;
+      cfg.blockDim = dim3(gemm::kWideThreads);
+      cfg.dynamicSmemBytes = gemm::kWideSmemBytes;
+      if (cudaOccupancyMaxActiveClusters(&clusters, gemm::k_gemm3<false, false>, &cfg) != cudaSuccess)
+        return FP8_ERR_CUDA;
+      d.wide_clusters = clusters;
+    }
     if (!g_encode) {
       cudaDriverEntryPointQueryResult q;
       void *fn = nullptr;
@@ -120,27 +150,38 @@ int run_gemm(const uint8_t *A, int fmt_a, const float *inv_a, const uint8_t *B, 
   DeviceInfo *d;
   int rc = device_info(&d);
   if (rc) return rc;
-  constexpr int BN = 256;
+  // Kernel choice: the widest tile that still gives every co-resident cluster
+  // at least one tile (256x512 pair tiles, then 256x256, then one CTA 128x256).
+  const int wide_tiles = ((rows + 255) / 256) * ((cols + 511) / 512);
+  const int pair_tiles = ((rows + 255) / 256) * ((cols + 255) / 256);
+  const int variant = (d->wide_clusters > 0 && wide_tiles >= d->wide_clusters) ? 3
+                      : (d->pair_clusters > 0 && pair_tiles >= d->pair_clusters) ? 2 : 1;
+  const int BN = variant == 3 ? 512 : 256;
+  const uint32_t a_box = variant == 1 ? (uint32_t)gemm::BM : 128u;  // rows of A per CTA
+  const uint32_t b_box = variant == 1 ? 256u : (variant == 2 ? 128u : 256u);  // B rows per CTA
   CUtensorMap ma, mb;
   if (A_MN) rc = make_map(&ma, A, (uint64_t)rows, (uint64_t)K, gemm::BK);
-  else      rc = make_map(&ma, A, (uint64_t)K, (uint64_t)rows, gemm::BM);
+  else      rc = make_map(&ma, A, (uint64_t)K, (uint64_t)rows, a_box);
   if (rc) return rc;
   if (B_MN) rc = make_map(&mb, B, (uint64_t)cols, (uint64_t)K, gemm::BK);
-  else      rc = make_map(&mb, B, (uint64_t)K, (uint64_t)cols, BN);
+  else      rc = make_map(&mb, B, (uint64_t)K, (uint64_t)cols, b_box);
   if (rc) return rc;
+  const int tile_rows = variant == 1 ? gemm::BM : 256;
   gemm::Args a;
   a.rows = rows;
   a.cols = cols;
   a.K = K;
-  a.num_m_blocks = (rows + gemm::BM - 1) / gemm::BM;
+  a.num_m_blocks = (rows + tile_rows - 1) / tile_rows;
   a.num_n_blocks = (cols + BN - 1) / BN;
   a.num_tiles = a.num_m_blocks * a.num_n_blocks;
   a.num_k_blocks = (K + gemm::BK - 1) / gemm::BK;
+  a.group_m = variant == 1 ? 16 : 8;
+  // one MMA instruction: M = 128 (one CTA) or 256 (pair), N = 256
   a.idesc = (1u << 4)                       // accumulate in F32
             | ((uint32_t)fmt_a << 7)         // A: 0 = E4M3, 1 = E5M2
             | ((uint32_t)fmt_b << 10)        // B
             | ((uint32_t)(A_MN ? 1 : 0) << 15) | ((uint32_t)(B_MN ? 1 : 0) << 16)
-            | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(gemm::BM >> 4) << 24);
+            | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(tile_rows >> 4) << 24);
   a.inv_a = inv_a;
   a.inv_b = inv_b;
   a.bias = bias;
@@ -149,8 +190,26 @@ int run_gemm(const uint8_t *A, int fmt_a, const float *inv_a, const uint8_t *B, 
   a.out_dtype = out_dtype;
   a.out_amax = out_amax;
   if (out_amax && (rc = cuda_rc(cudaMemsetAsync(out_amax, 0, sizeof(float), stream)))) return rc;
+  if (variant != 1) {
+    const int avail = variant == 3 ? d->wide_clusters : d->pair_clusters;
+    const int clusters = a.num_tiles < avail ? a.num_tiles : avail;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * clusters);
+    cfg.blockDim = dim3(variant == 3 ? gemm::kWideThreads : gemm::kThreads);
+    cfg.dynamicSmemBytes = variant == 3 ? gemm::kWideSmemBytes : gemm::kPairSmemBytes;
+    cfg.stream = stream;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    if (variant == 3) return cuda_rc(cudaLaunchKernelEx(&cfg, gemm::k_gemm3<A_MN, B_MN>, ma, mb, a));
+    return cuda_rc(cudaLaunchKernelEx(&cfg, gemm::k_gemm2<A_MN, B_MN>, ma, mb, a));
+  }
   unsigned grid = (unsigned)(a.num_tiles < d->sms ? a.num_tiles : d->sms);
-  gemm::k_gemm<BN, A_MN, B_MN><<<grid, gemm::kThreads, gemm::Cfg<BN>::SMEM_BYTES, stream>>>(ma, mb, a);
+  gemm::k_gemm<256, A_MN, B_MN><<<grid, gemm::kThreads, gemm::Cfg<256>::SMEM_BYTES, stream>>>(ma, mb, a);
   return launch_rc();
 }
 
@@ -270,11 +329,10 @@ int fp8_adam_step(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hpar
 
   static thread_local AdamLaunch L;  // ~20 KB: kept off the stack
   L.margin = hp->margin;
-  L.lr = hp->lr;
   L.beta1 = hp->beta1;
   L.beta2 = hp->beta2;
   L.eps = hp->eps;
-  L.inv_bc1 = (float)(1.0 / (1.0 - pow((double)hp->beta1, (double)hp->step)));
+  L.neg_lr_bc1 = (float)(-(double)hp->lr / (1.0 - pow((double)hp->beta1, (double)hp->step)));
   L.inv_bc2 = (float)(1.0 / (1.0 - pow((double)hp->beta2, (double)hp->step)));
   const unsigned cap = (unsigned)(d->sms * d->adam_blocks_per_sm);
   for (int first = 0; first < nchunks; first += kAdamMaxChunksPerLaunch) {

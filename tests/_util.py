@@ -55,3 +55,24 @@ def tensor_to_np(t: torch.Tensor) -> np.ndarray:
     if t.dtype == torch.bfloat16:
         return t.float().cpu().numpy().astype(np.float64)
     return t.cpu().numpy()
+
+
+def boundary_samples(rows: int, cols: int, n_random: int, key, tile_r=(128, 256), tile_c=(256,)):
+    """(row, col) sample positions: random ones plus every corner and the
+    first/last row and column of each tile edge (ragged edges included)."""
+    from fp8_mixed_precision_tensor_b200 import synth
+
+    g = synth.rng("samples", *key)
+    r = list(g.integers(0, rows, n_random))
+    c = list(g.integers(0, cols, n_random))
+    edge_r = sorted({x for t in tile_r for k in range(0, rows, t) for x in (k, min(k + t, rows) - 1)})
+    edge_c = sorted({x for t in tile_c for k in range(0, cols, t) for x in (k, min(k + t, cols) - 1)})
+    for er in edge_r:
+        for ec in g.choice(cols, min(cols, 8), replace=False).tolist() + [0, cols - 1]:
+            r.append(er)
+            c.append(ec)
+    for ec in edge_c:
+        for er in g.choice(rows, min(rows, 8), replace=False).tolist() + [0, rows - 1]:
+            r.append(er)
+            c.append(ec)
+    return np.asarray(r, dtype=np.int64), np.asarray(c, dtype=np.int64)

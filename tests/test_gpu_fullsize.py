@@ -1,0 +1,70 @@
+"""Full-size parity at the workloads' own shapes, in the launch configuration
+the benchmark times: the GPT-7B and GPT-175B block linears (fwd, dgrad,
+wgrad through the amax -> scale -> cast chain).  The oracle computes sampled
+outputs one by one (random positions plus every tile edge); the fused output
+amax is checked as a property that holds at any size (it equals the maximum
+magnitude of the stored output)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp8_mixed_precision_tensor_b200 import fp8, synth
+from _util import assert_gemm_close, boundary_samples, tensor_to_np
+
+pytestmark = pytest.mark.gpu
+
+F32 = dict(dtype=torch.float32, device="cuda")
+
+
+def _quantise(t, fmt, mu=1.0):
+    a, s, inv = (torch.zeros(1, **F32) for _ in range(3))
+    q = torch.empty(t.shape, dtype=torch.uint8, device="cuda")
+    fp8.fp8_amax(t, a)
+    fp8.fp8_compute_scale(a, fmt, 0, mu, s, inv)
+    fp8.fp8_cast(t, fmt, s, q)
+    return q, s, inv, a
+
+
+def _check_linear(M, K, N, w_std, seed):
+    X = synth.device_normal((M, K), synth.ACT_STD, seed + 1, torch.bfloat16, "cuda")
+    W = synth.device_normal((N, K), w_std, seed + 2, torch.bfloat16, "cuda")
+    dY = synth.device_normal((M, N), synth.GRAD_STD, seed + 3, torch.bfloat16, "cuda")
+    (xq, sx, xi, xa), (wq, sw, wi, wa), (dyq, sdy, dyi, dya) = (
+        _quantise(X, fp8.FP8_E4M3), _quantise(W, fp8.FP8_E4M3), _quantise(dY, fp8.FP8_E5M2, 2.0 ** 10))
+    # the scales are the oracle's for the amax the GPU found, and the amax is exact
+    for t, a, s, fmt, mu in ((X, xa, sx, oracle.E4M3, 1.0), (W, wa, sw, oracle.E4M3, 1.0),
+                             (dY, dya, sdy, oracle.E5M2, 2.0 ** 10)):
+        assert a.item() == t.abs().max().float().item()
+        assert s.item() == oracle.compute_scale(a.item(), fmt, 0, mu=mu)[1]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    dx = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    dw = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    ya, dxa, dwa = (torch.zeros(1, **F32) for _ in range(3))
+    fp8.fp8_linear_fwd(xq, xi, wq, wi, y, ya)
+    fp8.fp8_linear_dgrad(dyq, dyi, wq, wi, dx, dxa)
+    fp8.fp8_linear_wgrad(dyq, dyi, xq, xi, dw, dwa)
+    assert fp8.fp8_get_status() == 0
+    xh, wh, dyh = xq.cpu().numpy(), wq.cpu().numpy(), dyq.cpu().numpy()
+    for name, out, amax, (rows, cols), fn in (
+            ("fwd", y, ya, (M, N), lambda s: oracle.linear_fwd(xh, xi.item(), wh, wi.item(), M, N, K, samples=s)),
+            ("dgrad", dx, dxa, (M, K), lambda s: oracle.linear_dgrad(dyh, dyi.item(), wh, wi.item(), M, N, K,
+                                                                     samples=s)),
+            ("wgrad", dw, dwa, (N, K), lambda s: oracle.linear_wgrad(dyh, dyi.item(), xh, xi.item(), M, N, K,
+                                                                     samples=s))):
+        r, c = boundary_samples(rows, cols, 2000, (name, M, N, K), tile_c=(256, 512))
+        ref, rabs = fn((r, c))
+        got = tensor_to_np(out[torch.from_numpy(r).cuda(), torch.from_numpy(c).cuda()].contiguous())
+        assert_gemm_close(got, ref, rabs, out.dtype, f"{name} M{M} N{N} K{K}")
+        assert amax.item() == out.abs().max().float().item(), name
+    del X, W, dY, y, dx, dw
+
+
+@pytest.mark.parametrize("name,K,N", synth.GPT7B_LINEARS)
+def test_gpt7b_linears_full_size(name, K, N):
+    _check_linear(synth.GPT7B_TOKENS, K, N, synth.GPT7B_W_STD, 100)
+
+
+@pytest.mark.parametrize("name,K,N", synth.GPT175B_LINEARS)
+def test_gpt175b_linears_full_size(name, K, N):
+    _check_linear(synth.GPT175B_TOKENS, K, N, synth.GPT175B_W_STD, 200)

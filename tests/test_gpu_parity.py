@@ -14,7 +14,8 @@ import torch
 
 import oracle
 from fp8_mixed_precision_tensor_b200 import fp8, synth
-from _util import (assert_gemm_close, bf16_dev, code_rank, f16_ulp, f16_vals, tensor_to_np, to_dev)
+from _util import (assert_gemm_close, bf16_dev, boundary_samples, code_rank, f16_ulp, f16_vals, tensor_to_np,
+                   to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -229,6 +230,37 @@ def test_linear_gemms_vs_oracle(shape, out_dt):
         got = tensor_to_np(out)
         assert_gemm_close(got, ref, rabs, tdt, f"{name} {shape}")
         # fused amax == amax of the GPU's own stored output, bit-exact
+        assert amax.item() == float(np.max(np.abs(got))), name
+
+
+@pytest.mark.parametrize("shape", [(2320, 2064, 400), (2048, 4096, 512), (2320, 4624, 4112)])
+def test_linear_gemms_pair_kernel_sampled(shape):
+    """Shapes with enough 256x256 (first two) or 256x512 (last: all three
+    GEMMs) tiles to run the two-CTA kernels, ragged edges included; the oracle
+    computes sampled outputs one by one."""
+    M, N, K = shape
+    q = quantised_linear(M, N, K, ("gemm-pair", shape))
+    (xq, xi), (wq, wi), (dyq, dyi) = q["x"], q["w"], q["dy"]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    dx = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    dw = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    ya, dxa, dwa = scalar(), scalar(), scalar()
+    fp8.fp8_linear_fwd(xq, xi, wq, wi, y, ya)
+    fp8.fp8_linear_dgrad(dyq, dyi, wq, wi, dx, dxa)
+    fp8.fp8_linear_wgrad(dyq, dyi, xq, xi, dw, dwa)
+    assert fp8.fp8_get_status() == 0
+    h = {k: (v[0].cpu().numpy(), float(v[1].item())) for k, v in q.items()}
+    for name, out, amax, (rows, cols), fn in (
+            ("fwd", y, ya, (M, N), lambda smp: oracle.linear_fwd(h["x"][0], h["x"][1], h["w"][0], h["w"][1],
+                                                                 M, N, K, samples=smp)),
+            ("dgrad", dx, dxa, (M, K), lambda smp: oracle.linear_dgrad(h["dy"][0], h["dy"][1], h["w"][0],
+                                                                       h["w"][1], M, N, K, samples=smp)),
+            ("wgrad", dw, dwa, (N, K), lambda smp: oracle.linear_wgrad(h["dy"][0], h["dy"][1], h["x"][0],
+                                                                       h["x"][1], M, N, K, samples=smp))):
+        r, c = boundary_samples(rows, cols, 3000, (name, shape), tile_c=(256, 512))
+        ref, rabs = fn((r, c))
+        got = tensor_to_np(out)
+        assert_gemm_close(got[r, c], ref, rabs, out.dtype, f"{name} {shape}")
         assert amax.item() == float(np.max(np.abs(got))), name
 
 
