@@ -87,14 +87,19 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// One potentially blocking test of a barrier phase.  With the suspend-time
+// hint the thread sleeps until the phase completes (or the hint elapses)
+// instead of spinning, which keeps waiting warps off the issue slots and the
+// memory-instruction queue that the TMA and tcgen05 instructions also use.
+constexpr uint32_t kSuspendHintNs = 1000000;  // 1 ms per try; the caller bounds the total
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(done)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return done != 0;
 }
@@ -111,15 +116,13 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kTimeoutNs) {
-        atomicOr(&g_status, FP8_STATUS_TIMEOUT);
-        *abort_flag = 1;
-        return false;
-      }
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kTimeoutNs) {
+      atomicOr(&g_status, FP8_STATUS_TIMEOUT);
+      *abort_flag = 1;
+      return false;
     }
   }
 }
@@ -271,6 +274,28 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uin
       : "memory");
 }
 
+// Pair MMAs that share their A operand through the tensor core's collector
+// buffer: `fill` reads A from shared memory and keeps it, `lastuse` takes A
+// from the buffer (its descriptor is not read again) and releases it.
+__device__ __forceinline__ void tc_mma_pair_fill_a(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                   uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4.collector::a::fill [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair_lastuse_a(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                      uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4.collector::a::lastuse [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on the barrier at this offset in both CTAs of the pair once every
 // tcgen05 operation issued so far by this thread has completed.
 __device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
@@ -283,6 +308,36 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
 __device__ __forceinline__ void sleep_ns_bounded(uint32_t total_ns) {
   uint64_t t0 = globaltimer_ns();
   while (globaltimer_ns() - t0 < total_ns) __nanosleep(1000);
+}
+
+// Bulk tensor store of a 128B-swizzled shared-memory box to global memory
+// (bulk async-group completion; no mbarrier).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// Descale (+ bias) 32 accumulator columns of one row in place; columns at or
+// beyond `cols` are left as they are (zero: their B rows were zero-filled).
+__device__ __forceinline__ void descale_chunk(const Args &args, uint32_t (&r)[32], int col0, float inv_a,
+                                              float inv_b) {
+#pragma unroll
+  for (int j = 0; j < 32; j++) {
+    float y = __fmul_rn(__fmul_rn(__uint_as_float(r[j]), inv_a), inv_b);
+    if (args.bias != nullptr && col0 + j < args.cols) y = __fadd_rn(y, load_bias(args.bias, args.bias_dtype, col0 + j));
+    r[j] = __float_as_uint(y);
+  }
 }
 
 // Epilogue of one 32-column chunk: descale, bias, round, store, amax.
@@ -709,23 +764,25 @@ constexpr int kWideBN = 512;
 constexpr int kWideStages = 4;
 constexpr int kWideStageBytes = kPairHalf * BK + 2 * kPairHalf * BK;  // A 16 KB + B 32 KB
 constexpr int kWideThreads = 320;                                     // 10 warps
-constexpr int kWideSmemBytes = kWideStages * kWideStageBytes + 256 + 1024;
+constexpr int kWideStageOutBytes = 32 * 128;                             // per epilogue warp: 32 rows x 128 B
+constexpr int kWideSmemBytes = kWideStages * kWideStageBytes + 8 * kWideStageOutBytes + 256 + 1024;
 
 template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(kWideThreads, 1)
     k_gemm3(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-            const Args args) {
+            const __grid_constant__ CUtensorMap tmOut, const Args args) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t *base_ptr = smem_raw + (base - raw);
-  const uint32_t bar0 = base + kWideStages * kWideStageBytes;
+  const uint32_t out_stage0 = base + kWideStages * kWideStageBytes;  // 8 x 4 KB, 1024-aligned
+  const uint32_t bar0 = out_stage0 + 8 * kWideStageOutBytes;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (kWideStages + s); };
   const uint32_t tfull_bar = bar0 + 8u * (2 * kWideStages);
   const uint32_t tempty_bar = bar0 + 8u * (2 * kWideStages + 1);
   const uint32_t drain_bar = bar0 + 8u * (2 * kWideStages + 2);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + kWideStages * kWideStageBytes + 8 * (2 * kWideStages + 3));
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + (bar0 - base) + 8 * (2 * kWideStages + 3));
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -745,6 +802,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmOut);
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -812,8 +870,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             for (int ks = 0; ks < BK / UMMA_K; ks++) {
               const uint64_t ad = operand_desc<A_MN>(sa, ks);
               const uint32_t accum = (kb | ks) != 0 ? 1u : 0u;
-              tc_mma_pair(tmem_base, ad, operand_desc<B_MN>(sb, ks), args.idesc, accum);
-              tc_mma_pair(tmem_base + 256, ad, operand_desc<B_MN>(sb + kPairHalf * BK, ks), args.idesc, accum);
+              // the same A slice feeds both accumulators: read it from shared memory once
+              tc_mma_pair_fill_a(tmem_base, ad, operand_desc<B_MN>(sb, ks), args.idesc, accum);
+              tc_mma_pair_lastuse_a(tmem_base + 256, ad, operand_desc<B_MN>(sb + kPairHalf * BK, ks), args.idesc,
+                                    accum);
             }
             tc_commit_pair(empty_bar(stage));
             issued_any = true;
@@ -834,9 +894,16 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue (8 warps, both CTAs)
+    // Each warp drains 32 rows x 256 columns of one accumulator half in
+    // 128-byte-wide column blocks: tcgen05.ld -> descale/bias/round -> its own
+    // 4 KB staging box in shared memory (128B-swizzled rows) -> one bulk tensor
+    // store.  The store clips rows and columns outside the output.
     const int q = warp & 3;         // TMEM lane quarter
     const int h = (warp - 2) >> 2;  // accumulator half: 0 or 1
     const float inv_a = *args.inv_a, inv_b = *args.inv_b;
+    const uint32_t stg = out_stage0 + (warp - 2) * kWideStageOutBytes;
+    const bool f32out = args.out_dtype == FP8_DT_F32;
+    const bool bfout = args.out_dtype == FP8_DT_BF16;
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < args.num_tiles; tile += num_pairs) {
       int mb, nb;
@@ -845,24 +912,78 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       got = __shfl_sync(0xffffffffu, got, 0);
       if (!got) break;
       tc_fence_after();
-      const int row = mb * (2 * kPairHalf) + (int)rank * kPairHalf + q * 32 + lane;
+      const int row0 = mb * (2 * kPairHalf) + (int)rank * kPairHalf + q * 32;
+      const bool rows_in = row0 < args.rows;
       uint32_t amax_bits = 0;
+      // accumulator column c of half h holds output column
+      //   nb*512 + (c < 128 ? 0 : 256) + h*128 + (c mod 128)
+      const int cols_per_box = f32out ? 32 : 64;
 #pragma unroll 1
-      for (int cc = 0; cc < 8; cc++) {
+      for (int c = 0; c < 256; c += cols_per_box) {
+        const int col0 = nb * kWideBN + (c < 128 ? 0 : 256) + h * kPairHalf + (c & 127);
         uint32_t r[32];
-        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + h * 256 + cc * 32, r);
-        const int col0 = nb * kWideBN + (cc < 4 ? 0 : 256) + h * kPairHalf + (cc & 3) * 32;
-        amax_bits = max(amax_bits, store_chunk(args, r, row, col0, inv_a, inv_b));
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + h * 256 + c, r);
+        descale_chunk(args, r, col0, inv_a, inv_b);
+        uint32_t w[32];  // the row's 128 bytes as 32 words
+        if (f32out) {
+#pragma unroll
+          for (int j = 0; j < 32; j++) {
+            w[j] = r[j];
+            amax_bits = max(amax_bits, r[j] & 0x7fffffffu);
+          }
+        } else {
+          uint32_t r2[32];
+          tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + h * 256 + c + 32, r2);
+          descale_chunk(args, r2, col0 + 32, inv_a, inv_b);
+#pragma unroll
+          for (int j = 0; j < 16; j++) {
+            const float a0 = __uint_as_float(r[2 * j]), a1 = __uint_as_float(r[2 * j + 1]);
+            const float b0 = __uint_as_float(r2[2 * j]), b1 = __uint_as_float(r2[2 * j + 1]);
+            uint32_t pa, pb;
+            if (bfout) {
+              __nv_bfloat162 x = __floats2bfloat162_rn(a0, a1), y = __floats2bfloat162_rn(b0, b1);
+              pa = *reinterpret_cast<uint32_t *>(&x);
+              pb = *reinterpret_cast<uint32_t *>(&y);
+              amax_bits = max(amax_bits, max(max((pa & 0x7fffu) << 16, pa & 0x7fff0000u),
+                                             max((pb & 0x7fffu) << 16, pb & 0x7fff0000u)));
+            } else {
+              pa = f16x2(a0, a1);
+              pb = f16x2(b0, b1);
+              const float2 ba = h2f2(pa), bb = h2f2(pb);
+              amax_bits = max(amax_bits, max(max(absbits_f32(ba.x), absbits_f32(ba.y)),
+                                             max(absbits_f32(bb.x), absbits_f32(bb.y))));
+            }
+            w[j] = pa;
+            w[16 + j] = pb;
+          }
+        }
+        // the staging box must be free: the previous bulk store has read it
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+#pragma unroll
+        for (int ch = 0; ch < 8; ch++) {  // 16-byte chunk ch of this row, 128B swizzle
+          const uint32_t addr = stg + lane * 128 + ((ch ^ (lane & 7)) << 4);
+          st_shared_v4(addr, w[4 * ch], w[4 * ch + 1], w[4 * ch + 2], w[4 * ch + 3]);
+        }
+        fence_async_shared();
+        __syncwarp();
+        if (lane == 0 && rows_in && col0 < args.cols) {
+          tma_store_2d(&tmOut, stg, col0, row0);
+          bulk_commit();
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(map_to_rank(tempty_bar, 0));
+      if (row0 + lane >= args.rows) amax_bits = 0;  // a row past the output (holds only the bias)
       if (args.out_amax != nullptr) {
         amax_bits = warp_max_u32(amax_bits);
         if (lane == 0) atomic_max_bits(args.out_amax, amax_bits);
       }
       acc_phase ^= 1u;
     }
+    if (lane == 0) bulk_wait0();  // every store has landed before the CTA exits
+    __syncwarp();
   }
 
   tc_fence_before();

@@ -132,6 +132,23 @@ int make_map(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer, ui
   return r == CUDA_SUCCESS ? FP8_OK : FP8_ERR_CUDA;
 }
 
+// Row-major output [rows, cols] -> TMA map for 32-row boxes of 128 bytes
+// (32 fp32 or 64 16-bit columns) with the 128-byte swizzle (bulk stores).
+int make_out_map(CUtensorMap *m, void *out, int dtype, uint64_t rows, uint64_t cols) {
+  const CUtensorMapDataType t = dtype == FP8_DT_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                : dtype == FP8_DT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const uint64_t esz = dtype == FP8_DT_F32 ? 4 : 2;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * esz};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / esz), 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, t, 2, out, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8_OK : FP8_ERR_CUDA;
+}
+
 // C[rows, cols] = sum_k A(r, k) B(c, k), operand majorness as template flags.
 // A is [rows, K] (K-major) or [K, rows] (MN-major); B likewise with cols.
 template <bool A_MN, bool B_MN>
@@ -205,7 +222,11 @@ int run_gemm(const uint8_t *A, int fmt_a, const float *inv_a, const uint8_t *B, 
     cfg.stream = stream;
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
-    if (variant == 3) return cuda_rc(cudaLaunchKernelEx(&cfg, gemm::k_gemm3<A_MN, B_MN>, ma, mb, a));
+    if (variant == 3) {
+      CUtensorMap mo;
+      if ((rc = make_out_map(&mo, out, out_dtype, (uint64_t)rows, (uint64_t)cols))) return rc;
+      return cuda_rc(cudaLaunchKernelEx(&cfg, gemm::k_gemm3<A_MN, B_MN>, ma, mb, mo, a));
+    }
     return cuda_rc(cudaLaunchKernelEx(&cfg, gemm::k_gemm2<A_MN, B_MN>, ma, mb, a));
   }
   unsigned grid = (unsigned)(a.num_tiles < d->sms ? a.num_tiles : d->sms);
