@@ -4,13 +4,22 @@
 // power-of-two scale (6 bytes of state per parameter).
 //
 // The new scales are just-in-time: each comes from the amax of the *new*
-// values (the same rule as the linear layer's casts), so a step is two
-// streaming passes over all chunks plus a one-block finalize between them:
-//   pass 1 (stats):  decode, update in registers, reduce amax|m|, amax v,
-//                    amax|w| per chunk (nothing written but three scalars);
-//   finalize:        new scales from those amaxes; old inverse scales saved;
-//   pass 2 (update): decode, update again (bit-identical arithmetic),
-//                    re-encode with the new scales, write m, v, w.
+// values (the same rule as the linear layer's casts).  A step is
+//   pass 1 (stats):   decode, update in registers, reduce per chunk amax|m|,
+//                     amax v and either amax|w| (reading the master) or, when
+//                     the caller tracks the master's amax A0, the largest
+//                     step |dw| (not reading the master: 4 instead of 6 B);
+//   finalize 1:       new scales; with a tracked A0 the new master amax lies
+//                     in [A0 - U, A0 + U] and the scale exponent is taken from
+//                     that interval when it contains no scale threshold,
+//                     otherwise the chunk is flagged;
+//   pass 1b:          exact amax|w| for flagged chunks only (others skip);
+//   finalize 2:       remaining scales; publish all new scales;
+//   pass 2 (update):  decode, update again (bit-identical arithmetic), encode
+//                     m, v, w with the new scales, optionally write the E4M3
+//                     copy of the new stored master for the next forward GEMM,
+//                     and reduce the stored master's amax;
+//   finalize 3:       new tracked A0; consistency check of the inferred scale.
 // All chunks of one call share each launch: the chunk table travels in the
 // kernel parameters and tiles of 4096 parameters are mapped to chunks by a
 // binary search over the chunks' first-tile indices.
@@ -26,11 +35,17 @@ constexpr int kAdamTile = kAdamThreads * kAdamPerThread;  // parameters per tile
 constexpr int kAdamMaxChunksPerLaunch = 256;
 constexpr int kAdamWsFloatsPerChunk = 16;  // workspace slots per chunk (64 bytes)
 
-// Workspace slots of one chunk.
+// Workspace slots of one chunk (float bits; amax slots are max-reduced as
+// unsigned bit patterns).
 enum : int {
   WS_AMAX_M = 0, WS_AMAX_V = 1, WS_AMAX_W = 2,
   WS_OLDINV_M = 3, WS_OLDINV_V = 4, WS_OLDINV_W = 5,
   WS_NEW_M = 6, WS_NEW_V = 7, WS_NEW_W = 8,
+  WS_STEP_MAX = 9,     // max |dw| of the update (tracked-master path)
+  WS_FLAGS = 10,       // bit 0: needs the exact master pass; bit 1: tracked path
+  WS_NEW_WQ = 11,      // scale of the E4M3 master copy
+  WS_STORED_W = 12,    // max |stored FP16 master| (as f32 bits of the half)
+  WS_CHECK_W = 13,     // exact amax|w| of the new f32 master (pass 2)
 };
 
 struct AdamChunkDev {
@@ -42,6 +57,9 @@ struct AdamChunkDev {
   float *v_scale;
   uint16_t *w;
   float *w_scale;
+  float *w_amax;  // optional tracked amax of the stored master
+  uint8_t *wq;    // optional E4M3 copy of the new master
+  float *wq_scale, *wq_inv;
   unsigned long long n;
   unsigned long long tile_begin;
 };
@@ -52,18 +70,18 @@ struct AdamLaunch {
   int margin;
   unsigned long long total_tiles;
   float beta1, beta2, eps;
-  float neg_lr_bc1;        // -lr / (1 - beta1^t)
-  float inv_bc2;           // 1 / (1 - beta2^t)
-  float *ws;               // kAdamWsFloatsPerChunk floats per chunk of this launch
+  float neg_lr_bc1;  // -lr / (1 - beta1^t)
+  float inv_bc2;     // 1 / (1 - beta2^t)
+  float *ws;         // kAdamWsFloatsPerChunk floats per chunk of this launch
 };
 
 // Per-chunk constants of the update: the descales are folded into the Adam
 // coefficients, m = (b1/s_m) m~ + ((1-b1)/(mu s_g)) g~ and
 // v = (b2/s_v) v~ + ((1-b2)/(mu s_g)^2) g~^2, where ~ marks a decoded code.
 struct AdamScalars {
-  float cm, cgm;   // b1 / s_m,  (1 - b1) g_inv
-  float cv, cgv;   // b2 / s_v,  (1 - b2) g_inv^2
-  float w_inv;     // 1 / s_w
+  float cm, cgm;  // b1 / s_m,  (1 - b1) g_inv
+  float cv, cgv;  // b2 / s_v,  (1 - b2) g_inv^2
+  float w_inv;    // 1 / s_w
 };
 
 __device__ __forceinline__ AdamScalars adam_scalars(const AdamLaunch &L, float g_inv, float m_inv,
@@ -91,17 +109,20 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return r;
 }
 
-// The update of one parameter, float32, from decoded codes.  Written with
-// explicit round-to-nearest intrinsics so both passes evaluate exactly the
-// same operations (the stats pass must see the values the update pass
-// stores).  L.neg_lr_bc1 = -lr / (1 - b1^t), L.inv_bc2 = 1 / (1 - b2^t).
-__device__ __forceinline__ void adam_update(const AdamLaunch &L, float gd, float md, float vd,
-                                            float wd, const AdamScalars &s, float &m, float &v,
-                                            float &w) {
+// The new moments and the master step dw = -lr m_hat / (sqrt(v_hat) + eps)
+// of one parameter, float32, from decoded codes.  Explicit round-to-nearest
+// intrinsics keep every pass on exactly the same operations.
+__device__ __forceinline__ void adam_moments(const AdamLaunch &L, float gd, float md, float vd,
+                                             const AdamScalars &s, float &m, float &v, float &dw) {
   m = __fmaf_rn(s.cm, md, __fmul_rn(s.cgm, gd));
   v = __fmaf_rn(s.cv, vd, __fmul_rn(s.cgv, __fmul_rn(gd, gd)));
   const float denom = __fadd_rn(sqrt_approx(__fmul_rn(v, L.inv_bc2)), L.eps);
-  w = __fmaf_rn(L.neg_lr_bc1, __fmul_rn(m, rcp_approx(denom)), __fmul_rn(wd, s.w_inv));
+  dw = __fmul_rn(L.neg_lr_bc1, __fmul_rn(m, rcp_approx(denom)));
+}
+
+// w = w0 + dw as one rounding (the master's new value).
+__device__ __forceinline__ float adam_master(float wd, float dw, const AdamScalars &s) {
+  return __fadd_rn(__fmul_rn(wd, s.w_inv), dw);
 }
 
 __device__ __forceinline__ int find_chunk(const AdamLaunch &L, unsigned long long tile) {
@@ -113,38 +134,68 @@ __device__ __forceinline__ int find_chunk(const AdamLaunch &L, unsigned long lon
   return lo;
 }
 
+__device__ __forceinline__ float ws_get(const AdamLaunch &L, int ci, int slot) {
+  return L.ws[ci * kAdamWsFloatsPerChunk + slot];
+}
+__device__ __forceinline__ uint32_t ws_flags(const AdamLaunch &L, int ci) {
+  return __float_as_uint(L.ws[ci * kAdamWsFloatsPerChunk + WS_FLAGS]);
+}
+
+// Warp-reduce three running maxima and fold them into a chunk's slots.
+__device__ __forceinline__ void flush_max3(const AdamLaunch &L, int ci, int s0, uint32_t a0, int s1,
+                                           uint32_t a1, int s2, uint32_t a2) {
+  a0 = warp_max_u32(a0);
+  a1 = warp_max_u32(a1);
+  a2 = warp_max_u32(a2);
+  if ((threadIdx.x & 31) == 0) {
+    float *ws = L.ws + ci * kAdamWsFloatsPerChunk;
+    atomic_max_bits(ws + s0, a0);
+    atomic_max_bits(ws + s1, a1);
+    atomic_max_bits(ws + s2, a2);
+  }
+}
+
+// PASS 1: stats.  PASS 3: exact master amax of flagged chunks.  PASS 2: update.
 template <int PASS>
 __global__ void __launch_bounds__(kAdamThreads) k_adam(const __grid_constant__ AdamLaunch L) {
-  uint32_t am = 0, av = 0, aw = 0;  // pass 1: running maxima of the current chunk
+  uint32_t am = 0, av = 0, aw = 0;  // running maxima of the current chunk
   int cur = -1;
-  AdamScalars sc{};  // of the current chunk
-  float new_m = 1.f, new_v = 1.f, new_w = 1.f;
+  bool tracked = false, active = true, want_wq = false;
+  AdamScalars sc{};
+  float new_m = 1.f, new_v = 1.f, new_w = 1.f, new_wq = 1.f, inv_new_w = 1.f;
 
   for (unsigned long long tile = blockIdx.x; tile < L.total_tiles; tile += gridDim.x) {
     const int ci = find_chunk(L, tile);  // uniform across the block
     const AdamChunkDev &C = L.c[ci];
     if (ci != cur) {
-      if constexpr (PASS == 1) {
-        if (cur >= 0) {
-          am = warp_max_u32(am); av = warp_max_u32(av); aw = warp_max_u32(aw);
-          if ((threadIdx.x & 31) == 0) {
-            float *ws = L.ws + cur * kAdamWsFloatsPerChunk;
-            atomic_max_bits(ws + WS_AMAX_M, am);
-            atomic_max_bits(ws + WS_AMAX_V, av);
-            atomic_max_bits(ws + WS_AMAX_W, aw);
-          }
-          am = av = aw = 0;
-        }
-        sc = adam_scalars(L, *C.g_inv, 1.0f / *C.m_scale, 1.0f / *C.v_scale, 1.0f / *C.w_scale);
-      } else {
-        const float *ws = L.ws + ci * kAdamWsFloatsPerChunk;
-        sc = adam_scalars(L, *C.g_inv, ws[WS_OLDINV_M], ws[WS_OLDINV_V], ws[WS_OLDINV_W]);
-        new_m = ws[WS_NEW_M];
-        new_v = ws[WS_NEW_V];
-        new_w = ws[WS_NEW_W];
+      if (cur >= 0) {
+        if constexpr (PASS == 1)
+          flush_max3(L, cur, WS_AMAX_M, am, WS_AMAX_V, av, tracked ? WS_STEP_MAX : WS_AMAX_W, aw);
+        if constexpr (PASS == 3)
+          if (active) flush_max3(L, cur, WS_AMAX_W, aw, WS_AMAX_W, aw, WS_AMAX_W, aw);
+        if constexpr (PASS == 2) flush_max3(L, cur, WS_STORED_W, am, WS_CHECK_W, aw, WS_CHECK_W, aw);
+        am = av = aw = 0;
       }
       cur = ci;
+      if constexpr (PASS == 1) {
+        tracked = C.w_amax != nullptr && *C.w_amax >= 0.0f;
+        sc = adam_scalars(L, *C.g_inv, 1.0f / *C.m_scale, 1.0f / *C.v_scale, 1.0f / *C.w_scale);
+      } else {
+        const uint32_t fl = ws_flags(L, ci);
+        tracked = (fl & 2u) != 0;
+        active = PASS == 2 || (fl & 1u) != 0;
+        sc = adam_scalars(L, *C.g_inv, ws_get(L, ci, WS_OLDINV_M), ws_get(L, ci, WS_OLDINV_V),
+                          ws_get(L, ci, WS_OLDINV_W));
+        new_m = ws_get(L, ci, WS_NEW_M);
+        new_v = ws_get(L, ci, WS_NEW_V);
+        new_w = ws_get(L, ci, WS_NEW_W);
+        inv_new_w = 1.0f / new_w;
+        want_wq = C.wq != nullptr;
+        new_wq = want_wq ? ws_get(L, ci, WS_NEW_WQ) : 1.0f;
+      }
     }
+    if (!active) continue;  // pass 1b: chunk not flagged
+    const bool read_w = PASS != 1 || !tracked;
     const unsigned long long base =
         (tile - C.tile_begin) * kAdamTile + (unsigned long long)threadIdx.x * kAdamPerThread;
     if (base >= C.n) continue;
@@ -155,31 +206,50 @@ __global__ void __launch_bounds__(kAdamThreads) k_adam(const __grid_constant__ A
       uint4 mq = __ldcs(reinterpret_cast<const uint4 *>(C.m) + grp);
       uint4 vq0 = __ldcs(reinterpret_cast<const uint4 *>(C.v) + 2 * grp);
       uint4 vq1 = __ldcs(reinterpret_cast<const uint4 *>(C.v) + 2 * grp + 1);
-      uint4 wq0 = __ldcs(reinterpret_cast<const uint4 *>(C.w) + 2 * grp);
-      uint4 wq1 = __ldcs(reinterpret_cast<const uint4 *>(C.w) + 2 * grp + 1);
+      uint4 wq0 = make_uint4(0, 0, 0, 0), wq1 = make_uint4(0, 0, 0, 0);
+      if (read_w) {
+        wq0 = __ldcs(reinterpret_cast<const uint4 *>(C.w) + 2 * grp);
+        wq1 = __ldcs(reinterpret_cast<const uint4 *>(C.w) + 2 * grp + 1);
+      }
       const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
       const uint32_t mw[4] = {mq.x, mq.y, mq.z, mq.w};
       const uint32_t vw[8] = {vq0.x, vq0.y, vq0.z, vq0.w, vq1.x, vq1.y, vq1.z, vq1.w};
       const uint32_t ww[8] = {wq0.x, wq0.y, wq0.z, wq0.w, wq1.x, wq1.y, wq1.z, wq1.w};
-      uint32_t mo[4], vo[8], wo[8];
+      uint32_t mo[4], vo[8], wo[8], qo[4];
 #pragma unroll
       for (int p = 0; p < 8; p++) {  // pairs of parameters
         const uint32_t g2 = (gw[p >> 1] >> ((p & 1) * 16)) & 0xffffu;
         const uint32_t m2 = (mw[p >> 1] >> ((p & 1) * 16)) & 0xffffu;
-        float2 gd = dec2<FP8_E5M2>(g2), md = dec2<FP8_E4M3>(m2);
-        float2 vd = h2f2(vw[p]), wd = h2f2(ww[p]);
-        float m_a, v_a, w_a, m_b, v_b, w_b;
-        adam_update(L, gd.x, md.x, vd.x, wd.x, sc, m_a, v_a, w_a);
-        adam_update(L, gd.y, md.y, vd.y, wd.y, sc, m_b, v_b, w_b);
+        const float2 gd = dec2<FP8_E5M2>(g2), md = dec2<FP8_E4M3>(m2);
+        const float2 vd = h2f2(vw[p]), wd = h2f2(ww[p]);
+        float m_a, v_a, d_a, m_b, v_b, d_b;
+        adam_moments(L, gd.x, md.x, vd.x, sc, m_a, v_a, d_a);
+        adam_moments(L, gd.y, md.y, vd.y, sc, m_b, v_b, d_b);
         if constexpr (PASS == 1) {
           am = max(am, max(absbits_f32(m_a), absbits_f32(m_b)));
           av = max(av, max(absbits_f32(v_a), absbits_f32(v_b)));
-          aw = max(aw, max(absbits_f32(w_a), absbits_f32(w_b)));
+          if (tracked) {
+            aw = max(aw, max(absbits_f32(d_a), absbits_f32(d_b)));
+          } else {
+            aw = max(aw, max(absbits_f32(adam_master(wd.x, d_a, sc)), absbits_f32(adam_master(wd.y, d_b, sc))));
+          }
+        } else if constexpr (PASS == 3) {
+          aw = max(aw, max(absbits_f32(adam_master(wd.x, d_a, sc)), absbits_f32(adam_master(wd.y, d_b, sc))));
         } else {
+          const float w_a = adam_master(wd.x, d_a, sc), w_b = adam_master(wd.y, d_b, sc);
+          aw = max(aw, max(absbits_f32(w_a), absbits_f32(w_b)));
           const uint32_t mc = enc2<FP8_E4M3>(__fmul_rn(m_a, new_m), __fmul_rn(m_b, new_m));
           if (p & 1) mo[p >> 1] |= mc << 16; else mo[p >> 1] = mc;
           vo[p] = f16x2(__fmul_rn(v_a, new_v), __fmul_rn(v_b, new_v));
           wo[p] = f16x2(__fmul_rn(w_a, new_w), __fmul_rn(w_b, new_w));
+          const float2 st = h2f2(wo[p]);  // the stored master (scaled)
+          am = max(am, max(absbits_f32(st.x), absbits_f32(st.y)));
+          if (want_wq) {
+            // E4M3 copy of the stored master: (h / s_w) * s_q, exact in f32
+            const uint32_t qc = enc2<FP8_E4M3>(__fmul_rn(__fmul_rn(st.x, inv_new_w), new_wq),
+                                               __fmul_rn(__fmul_rn(st.y, inv_new_w), new_wq));
+            if (p & 1) qo[p >> 1] |= qc << 16; else qo[p >> 1] = qc;
+          }
         }
       }
       if constexpr (PASS == 2) {
@@ -188,60 +258,126 @@ __global__ void __launch_bounds__(kAdamThreads) k_adam(const __grid_constant__ A
         __stcs(reinterpret_cast<uint4 *>(C.v) + 2 * grp + 1, make_uint4(vo[4], vo[5], vo[6], vo[7]));
         __stcs(reinterpret_cast<uint4 *>(C.w) + 2 * grp, make_uint4(wo[0], wo[1], wo[2], wo[3]));
         __stcs(reinterpret_cast<uint4 *>(C.w) + 2 * grp + 1, make_uint4(wo[4], wo[5], wo[6], wo[7]));
+        if (want_wq) __stcs(reinterpret_cast<uint4 *>(C.wq) + grp, make_uint4(qo[0], qo[1], qo[2], qo[3]));
       }
     } else {
       // Ragged end of a chunk: element by element.
       for (unsigned long long i = base; i < C.n; i++) {
-        float gd = dec2<FP8_E5M2>(C.g[i]).x, md = dec2<FP8_E4M3>(C.m[i]).x;
-        float vd = __half2float(__ushort_as_half(C.v[i])), wd = __half2float(__ushort_as_half(C.w[i]));
-        float m, v, w;
-        adam_update(L, gd, md, vd, wd, sc, m, v, w);
+        const float gd = dec2<FP8_E5M2>(C.g[i]).x, md = dec2<FP8_E4M3>(C.m[i]).x;
+        const float vd = __half2float(__ushort_as_half(C.v[i]));
+        const float wd = read_w ? __half2float(__ushort_as_half(C.w[i])) : 0.0f;
+        float m, v, d;
+        adam_moments(L, gd, md, vd, sc, m, v, d);
         if constexpr (PASS == 1) {
           am = max(am, absbits_f32(m));
           av = max(av, absbits_f32(v));
-          aw = max(aw, absbits_f32(w));
+          aw = max(aw, tracked ? absbits_f32(d) : absbits_f32(adam_master(wd, d, sc)));
+        } else if constexpr (PASS == 3) {
+          aw = max(aw, absbits_f32(adam_master(wd, d, sc)));
         } else {
+          const float w = adam_master(wd, d, sc);
+          aw = max(aw, absbits_f32(w));
           C.m[i] = (uint8_t)(enc2<FP8_E4M3>(__fmul_rn(m, new_m), 0.0f) & 0xffu);
           C.v[i] = __half_as_ushort(__float2half_rn(__fmul_rn(v, new_v)));
-          C.w[i] = __half_as_ushort(__float2half_rn(__fmul_rn(w, new_w)));
+          const __half h = __float2half_rn(__fmul_rn(w, new_w));
+          C.w[i] = __half_as_ushort(h);
+          const float st = __half2float(h);
+          am = max(am, absbits_f32(st));
+          if (want_wq)
+            C.wq[i] = (uint8_t)(enc2<FP8_E4M3>(__fmul_rn(__fmul_rn(st, inv_new_w), new_wq), 0.0f) & 0xffu);
         }
       }
     }
   }
-  if constexpr (PASS == 1) {
-    // cur is block-uniform, so the whole warp takes this branch together.
-    if (cur >= 0) {
-      am = warp_max_u32(am); av = warp_max_u32(av); aw = warp_max_u32(aw);
-      if ((threadIdx.x & 31) == 0) {
-        float *ws = L.ws + cur * kAdamWsFloatsPerChunk;
-        atomic_max_bits(ws + WS_AMAX_M, am);
-        atomic_max_bits(ws + WS_AMAX_V, av);
-        atomic_max_bits(ws + WS_AMAX_W, aw);
-      }
-    }
+  // cur is block-uniform, so whole warps take these branches together.
+  if (cur >= 0) {
+    if constexpr (PASS == 1)
+      flush_max3(L, cur, WS_AMAX_M, am, WS_AMAX_V, av, tracked ? WS_STEP_MAX : WS_AMAX_W, aw);
+    if constexpr (PASS == 3)
+      if (active) flush_max3(L, cur, WS_AMAX_W, aw, WS_AMAX_W, aw, WS_AMAX_W, aw);
+    if constexpr (PASS == 2) flush_max3(L, cur, WS_STORED_W, am, WS_CHECK_W, aw, WS_CHECK_W, aw);
   }
 }
 
-// Between the passes: new scales from the new amaxes, old inverse scales
-// saved for pass 2, new scales published to the caller's scale slots.
+// Exponent of the E4M3 copy's scale from an amax of the stored master: the
+// stored value of x is fp16(x s_w) / s_w (monotone in x).
+__device__ __forceinline__ float stored_value(float x, float s_w) {
+  return __fmul_rn(__half2float(__float2half_rn(__fmul_rn(x, s_w))), 1.0f / s_w);
+}
+
+// STAGE 1: after pass 1.  STAGE 2: after pass 1b.  STAGE 3: after pass 2.
+// STAGE 12: stages 1 and 2 in one launch (no chunk tracks its master amax,
+// so no chunk can be flagged and pass 1b has nothing to do).
+template <int STAGE>
 __global__ void k_adam_finalize(const __grid_constant__ AdamLaunch L) {
   for (int ci = threadIdx.x; ci < L.nchunks; ci += blockDim.x) {
     float *ws = L.ws + ci * kAdamWsFloatsPerChunk;
     const AdamChunkDev &C = L.c[ci];
-    int km, kv, kw;
-    bool ok = scale_exponent(ws[WS_AMAX_M], kMaxE4M3, L.margin, 0, km);
-    ok &= scale_exponent(ws[WS_AMAX_V], kMaxF16, L.margin, 0, kv);
-    ok &= scale_exponent(ws[WS_AMAX_W], kMaxF16, L.margin, 0, kw);
-    if (!ok) atomicOr(&g_status, FP8_STATUS_NONFINITE);
-    ws[WS_OLDINV_M] = 1.0f / *C.m_scale;
-    ws[WS_OLDINV_V] = 1.0f / *C.v_scale;
-    ws[WS_OLDINV_W] = 1.0f / *C.w_scale;
-    ws[WS_NEW_M] = pow2f(km);
-    ws[WS_NEW_V] = pow2f(kv);
-    ws[WS_NEW_W] = pow2f(kw);
-    *C.m_scale = pow2f(km);
-    *C.v_scale = pow2f(kv);
-    *C.w_scale = pow2f(kw);
+    uint32_t flags = __float_as_uint(ws[WS_FLAGS]);
+    if constexpr (STAGE == 1 || STAGE == 12) {
+      int km, kv, kw = 0, kq = 0;
+      bool ok = scale_exponent(ws[WS_AMAX_M], kMaxE4M3, L.margin, 0, km);
+      ok &= scale_exponent(ws[WS_AMAX_V], kMaxF16, L.margin, 0, kv);
+      ws[WS_OLDINV_M] = 1.0f / *C.m_scale;
+      ws[WS_OLDINV_V] = 1.0f / *C.v_scale;
+      ws[WS_OLDINV_W] = 1.0f / *C.w_scale;
+      ws[WS_NEW_M] = pow2f(km);
+      ws[WS_NEW_V] = pow2f(kv);
+      const bool tracked = C.w_amax != nullptr && *C.w_amax >= 0.0f;
+      bool exact = !tracked;
+      if (tracked) {
+        // amax|w_new| lies in [A0 - U, A0 + U], widened for the one rounding of w0 + dw
+        const float a0 = *C.w_amax, u = ws[WS_STEP_MAX];
+        const float hi = __fmul_rn(__fadd_ru(a0, u), 1.0f + 0x1p-20f);
+        const float lo = __fmul_rn(__fsub_rd(a0, u), 1.0f - 0x1p-20f);
+        int klo, khi;
+        bool known = lo > 0.0f && scale_exponent(lo, kMaxF16, L.margin, 0, klo) &&
+                     scale_exponent(hi, kMaxF16, L.margin, 0, khi) && klo == khi;
+        if (known) {
+          kw = klo;
+          if (C.wq != nullptr) {
+            const float s = pow2f(kw);
+            int qlo, qhi;
+            known = scale_exponent(stored_value(lo, s), kMaxE4M3, L.margin, 0, qlo) &&
+                    scale_exponent(stored_value(hi, s), kMaxE4M3, L.margin, 0, qhi) && qlo == qhi;
+            kq = qlo;
+          }
+        }
+        flags = 2u | (known ? 0u : 1u);
+        exact = !known;
+      }
+      if (!exact) {
+        ws[WS_NEW_W] = pow2f(kw);
+        ws[WS_NEW_WQ] = pow2f(kq);
+      }
+      if (!ok) atomicOr(&g_status, FP8_STATUS_NONFINITE);
+      ws[WS_FLAGS] = __uint_as_float(flags);
+    }
+    if constexpr (STAGE == 2 || STAGE == 12) {
+      // exact master amax: untracked chunks (pass 1) or flagged ones (pass 1b)
+      if (!(flags & 2u) || (flags & 1u)) {
+        int kw, kq = 0;
+        bool ok = scale_exponent(ws[WS_AMAX_W], kMaxF16, L.margin, 0, kw);
+        if (C.wq != nullptr) ok &= scale_exponent(stored_value(ws[WS_AMAX_W], pow2f(kw)), kMaxE4M3, L.margin, 0, kq);
+        if (!ok) atomicOr(&g_status, FP8_STATUS_NONFINITE);
+        ws[WS_NEW_W] = pow2f(kw);
+        ws[WS_NEW_WQ] = pow2f(kq);
+      }
+      *C.m_scale = ws[WS_NEW_M];
+      *C.v_scale = ws[WS_NEW_V];
+      *C.w_scale = ws[WS_NEW_W];
+      if (C.wq != nullptr) {
+        *C.wq_scale = ws[WS_NEW_WQ];
+        *C.wq_inv = 1.0f / ws[WS_NEW_WQ];
+      }
+    }
+    if constexpr (STAGE == 3) {
+      // the exact new amax must give the scale that was used
+      int kw;
+      if (scale_exponent(ws[WS_CHECK_W], kMaxF16, L.margin, 0, kw) && pow2f(kw) != ws[WS_NEW_W])
+        atomicOr(&g_status, FP8_STATUS_INTERNAL);
+      if (C.w_amax != nullptr) *C.w_amax = __fmul_rn(ws[WS_STORED_W], 1.0f / ws[WS_NEW_W]);
+    }
   }
 }
 

@@ -338,8 +338,10 @@ int fp8_adam_step(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hpar
   for (int i = 0; i < nchunks; i++) {
     const fp8_adam_chunk &c = chunks[i];
     if (!c.g_inv || !c.m_scale || !c.v_scale || !c.w_scale) return FP8_ERR_INVALID_ARG;
+    if (c.wq && (!c.wq_scale || !c.wq_inv)) return FP8_ERR_INVALID_ARG;
     if (c.n > 0 && (!c.g || !c.m || !c.v || !c.w)) return FP8_ERR_INVALID_ARG;
-    if (c.n > 0 && (!aligned16(c.g) || !aligned16(c.m) || !aligned16(c.v) || !aligned16(c.w)))
+    if (c.n > 0 && (!aligned16(c.g) || !aligned16(c.m) || !aligned16(c.v) || !aligned16(c.w) ||
+                    (c.wq && !aligned16(c.wq))))
       return FP8_ERR_UNALIGNED;
   }
   DeviceInfo *d;
@@ -364,6 +366,7 @@ int fp8_adam_step(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hpar
       AdamChunkDev &e = L.c[i];
       e.g = c.g; e.g_inv = c.g_inv; e.m = c.m; e.m_scale = c.m_scale;
       e.v = c.v; e.v_scale = c.v_scale; e.w = c.w; e.w_scale = c.w_scale;
+      e.w_amax = c.w_amax; e.wq = c.wq; e.wq_scale = c.wq_scale; e.wq_inv = c.wq_inv;
       e.n = c.n;
       e.tile_begin = tiles;
       tiles += (c.n + kAdamTile - 1) / kAdamTile;
@@ -372,11 +375,18 @@ int fp8_adam_step(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hpar
     L.total_tiles = tiles;
     L.ws = reinterpret_cast<float *>(workspace) + (size_t)first * kAdamWsFloatsPerChunk;
     const unsigned grid = tiles == 0 ? 1u : (unsigned)(tiles < cap ? tiles : cap);
-    k_adam<1><<<grid, kAdamThreads, 0, s>>>(L);
-    if ((rc = launch_rc())) return rc;
-    k_adam_finalize<<<1, 256, 0, s>>>(L);
-    if ((rc = launch_rc())) return rc;
-    k_adam<2><<<grid, kAdamThreads, 0, s>>>(L);
+    bool tracked = false;
+    for (int i = 0; i < cnt; i++) tracked |= L.c[i].w_amax != nullptr;
+    k_adam<1><<<grid, kAdamThreads, 0, s>>>(L);        // stats
+    if (tracked) {
+      k_adam_finalize<1><<<1, 256, 0, s>>>(L);
+      k_adam<3><<<grid, kAdamThreads, 0, s>>>(L);      // exact master amax, flagged chunks only
+      k_adam_finalize<2><<<1, 256, 0, s>>>(L);
+    } else {
+      k_adam_finalize<12><<<1, 256, 0, s>>>(L);
+    }
+    k_adam<2><<<grid, kAdamThreads, 0, s>>>(L);        // update
+    if (tracked) k_adam_finalize<3><<<1, 256, 0, s>>>(L);
     if ((rc = launch_rc())) return rc;
   }
   return FP8_OK;

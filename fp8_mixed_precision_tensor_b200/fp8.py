@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libfp8.so")
 # status codes / enums (include/fp8.h)
 FP8_OK, FP8_ERR_INVALID_ARG, FP8_ERR_UNALIGNED, FP8_ERR_UNSUPPORTED = 0, 1, 2, 3
 FP8_ERR_CUDA, FP8_ERR_TIMEOUT, FP8_ERR_NONFINITE = 4, 5, 6
-FP8_STATUS_NONFINITE, FP8_STATUS_TIMEOUT = 1, 2
+FP8_STATUS_NONFINITE, FP8_STATUS_TIMEOUT, FP8_STATUS_INTERNAL = 1, 2, 4
 FP8_DT_F32, FP8_DT_BF16, FP8_DT_F16 = 0, 1, 2
 FP8_E4M3, FP8_E5M2, FP8_F16S = 0, 1, 2
 
@@ -41,7 +41,9 @@ class FP8Error(RuntimeError):
 class _Chunk(ctypes.Structure):
     _fields_ = [("g", ctypes.c_void_p), ("g_inv", ctypes.c_void_p), ("m", ctypes.c_void_p),
                 ("m_scale", ctypes.c_void_p), ("v", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
-                ("w", ctypes.c_void_p), ("w_scale", ctypes.c_void_p), ("n", ctypes.c_size_t)]
+                ("w", ctypes.c_void_p), ("w_scale", ctypes.c_void_p), ("n", ctypes.c_size_t),
+                ("w_amax", ctypes.c_void_p), ("wq", ctypes.c_void_p), ("wq_scale", ctypes.c_void_p),
+                ("wq_inv", ctypes.c_void_p)]
 
 
 class _HParams(ctypes.Structure):
@@ -153,7 +155,9 @@ def fp8_linear_wgrad(dyq, dy_inv, xq, x_inv, dw, dw_amax=None, stream=None) -> N
 @dataclass
 class AdamChunk:
     """Stored state of one tensor: E5M2 grad codes + g_inv, E4M3 m1 codes +
-    scale, FP16 m2 bits + scale, FP16 master bits + scale (device tensors)."""
+    scale, FP16 m2 bits + scale, FP16 master bits + scale (device tensors).
+    Optional: w_amax (tracked amax of the stored master, -1 = unknown) and
+    wq, wq_scale, wq_inv (E4M3 copy of the new master and its scales)."""
     g: torch.Tensor
     g_inv: torch.Tensor
     m: torch.Tensor
@@ -162,6 +166,10 @@ class AdamChunk:
     v_scale: torch.Tensor
     w: torch.Tensor
     w_scale: torch.Tensor
+    w_amax: torch.Tensor | None = None
+    wq: torch.Tensor | None = None
+    wq_scale: torch.Tensor | None = None
+    wq_inv: torch.Tensor | None = None
 
 
 def fp8_adam_workspace_bytes(nchunks: int) -> int:
@@ -173,7 +181,8 @@ def pack_adam_chunks(chunks: list[AdamChunk]):
     arr = (_Chunk * len(chunks))()
     for i, c in enumerate(chunks):
         arr[i] = _Chunk(_ptr(c.g), _ptr(c.g_inv), _ptr(c.m), _ptr(c.m_scale), _ptr(c.v), _ptr(c.v_scale),
-                        _ptr(c.w), _ptr(c.w_scale), c.g.numel())
+                        _ptr(c.w), _ptr(c.w_scale), c.g.numel(), _ptr(c.w_amax), _ptr(c.wq),
+                        _ptr(c.wq_scale), _ptr(c.wq_inv))
     return arr
 
 

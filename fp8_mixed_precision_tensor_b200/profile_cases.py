@@ -2,7 +2,7 @@
 
     python -m fp8_mixed_precision_tensor_b200.profile_cases linear --M 4096 --N 16384 --K 4096
     python -m fp8_mixed_precision_tensor_b200.profile_cases cast --n 268435456
-    python -m fp8_mixed_precision_tensor_b200.profile_cases adam --n 67108864
+    python -m fp8_mixed_precision_tensor_b200.profile_cases adam --n 67108864 [--track]
 
 Each case runs `--iters` passes after one warm-up pass on seeded synthetic
 inputs and prints the CUDA-event time per pass.  Launch order per pass:
@@ -75,8 +75,10 @@ def case_adam(a):
     del g, w
     m = torch.zeros(n, dtype=torch.uint8, device="cuda")
     v = torch.zeros(n, dtype=torch.int16, device="cuda")
-    st = torch.ones(2, dtype=torch.float32, device="cuda")
-    chunks = fp8.pack_adam_chunks([fp8.AdamChunk(gq, sc[2:3], m, st[0:1], v, st[1:2], wh, sc[4:5])])
+    st = torch.ones(3, dtype=torch.float32, device="cuda")
+    st[2] = -1.0  # tracked master amax: unknown until the first step
+    chunks = fp8.pack_adam_chunks([fp8.AdamChunk(gq, sc[2:3], m, st[0:1], v, st[1:2], wh, sc[4:5],
+                                                 w_amax=st[2:3] if a.track else None)])
     ws = torch.zeros(64, dtype=torch.float32, device="cuda")
     state = {"t": 0}
 
@@ -95,6 +97,7 @@ def main():
     ap.add_argument("--K", type=int, default=4096)
     ap.add_argument("--n", type=int, default=1 << 26)
     ap.add_argument("--iters", type=int, default=2)
+    ap.add_argument("--track", action="store_true", help="adam: track the master amax across steps")
     a = ap.parse_args()
     one = {"linear": case_linear, "cast": case_cast, "adam": case_adam}[a.case](a)
     one()

@@ -52,6 +52,7 @@ extern "C" {
 /* Device status word bits (fp8_get_status). */
 #define FP8_STATUS_NONFINITE 1u
 #define FP8_STATUS_TIMEOUT 2u
+#define FP8_STATUS_INTERNAL 4u /* a kernel's own consistency check failed */
 
 /* ---- element types of high-precision tensors -------------------------- */
 #define FP8_DT_F32 0
@@ -158,8 +159,19 @@ int fp8_linear_wgrad(const uint8_t *dyq, const float *dy_inv, const uint8_t *xq,
  * is re-encoded with them; the new scales replace m_scale, v_scale, w_scale.
  * Arithmetic is float32.  A non-finite new amax sets FP8_STATUS_NONFINITE and
  * that scale to 1.
- * Pointers g, m, v, w are dev and 16-byte aligned; the scale pointers are dev
- * floats.  Chunks must not overlap.  `chunks` is a HOST array of nchunks.
+ * Tracked master amax (optional; the first pass then moves 4 instead of 6
+ * bytes per parameter): when w_amax points to the exact amax of the
+ * dequantised stored master (a value >= 0), the new master amax is bounded by
+ * that value -/+ the largest step |w - w0|, and the master is re-read only
+ * when the interval holds a scale threshold.  Every step rewrites *w_amax; a
+ * negative value means "unknown" (the step re-reads the master).  After
+ * changing w or w_scale by other means, set *w_amax to -1.
+ * E4M3 master copy (optional; the next forward pass's weight cast fused into
+ * the update): when wq is not NULL the step also writes
+ * wq = E4M3(stored master * s_q), s_q from the amax of the stored master with
+ * fmt_max 448 and the same margin, and s_q, 1/s_q to *wq_scale, *wq_inv.
+ * Pointers g, m, v, w, wq are dev and 16-byte aligned; the scale pointers are
+ * dev floats.  Chunks must not overlap.  `chunks` is a HOST array of nchunks.
  */
 typedef struct {
   const uint8_t *g;    /* dev [n] E5M2 gradient codes */
@@ -171,6 +183,10 @@ typedef struct {
   uint16_t *w;         /* dev [n] FP16 master weight, scaled (in/out) */
   float *w_scale;      /* dev float (in/out) */
   size_t n;            /* parameters in this chunk (0 allowed) */
+  float *w_amax;       /* dev float or NULL: tracked amax of the stored master (in/out) */
+  uint8_t *wq;         /* dev [n] or NULL: E4M3 copy of the new stored master (out) */
+  float *wq_scale;     /* dev float, required with wq (out) */
+  float *wq_inv;       /* dev float, required with wq (out) */
 } fp8_adam_chunk;
 
 typedef struct {

@@ -236,6 +236,19 @@ def adam_step(gq, g_inv, mq, s_m, vh, s_v, wh, s_w, lr, beta1, beta2, eps, t, ma
                 amax=tuple(am))
 
 
+def adam_master_e4m3(wh, s_w: float, margin: int):
+    """E4M3 copy of a stored FP16 master for the next forward pass ("FP8-LM",
+    提案手法 O2 master weights, cast as in "Training and inference of large
+    language models using 8-bit floating point", 제안 방법): the dequantised
+    master is dec_f16(wh) / s_w; its E4M3 scale s_q comes from its amax with
+    fmt_max 448; codes = enc_E4M3(dec_f16(wh) / s_w * s_q), where the product
+    s_q / s_w is an exact power of two.  Returns (codes, s_q)."""
+    wh = np.ascontiguousarray(wh).view(np.uint16)
+    a = amax(wh, DT_F16) / s_w
+    rc, s_q = compute_scale(a, E4M3, margin)
+    return cast(wh, E4M3, s_q / s_w, DT_F16), s_q
+
+
 def num_threads() -> int:
     return _load().orc_num_threads()
 

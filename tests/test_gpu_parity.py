@@ -431,3 +431,76 @@ def test_adam_rejects_bad_args():
         fp8.fp8_adam_step(chunks, step=0, margin=0, workspace=ws, **HP)
     with pytest.raises(fp8.FP8Error):
         fp8.fp8_adam_step(chunks, step=1, margin=0, workspace=ws[:3], **HP)
+
+
+# ---------------------------------------------------------------- Adam: tracked master amax, E4M3 copy
+def _with_tracking(chunks, wq=False):
+    out = []
+    for c in chunks:
+        n = c.g.numel()
+        extra = dict(w_amax=torch.full((1,), -1.0, **F32))
+        if wq:
+            extra.update(wq=torch.empty(n, dtype=torch.uint8, device="cuda"), wq_scale=scalar(), wq_inv=scalar())
+        out.append(fp8.AdamChunk(c.g, c.g_inv, c.m, c.m_scale, c.v, c.v_scale, c.w, c.w_scale, **extra))
+    return out
+
+
+def _stored_amax(snap):
+    return float(np.max(np.abs(f16_vals(snap["w"])))) / snap["s_w"]
+
+
+@pytest.mark.parametrize("sizes", [[65536, 4099], [300000, 7, 16]])
+def test_adam_tracked_master_amax_matches_untracked(sizes):
+    """Step 1 with the tracked amax unknown (full path), steps 2-3 with it known
+    (the first pass skips the master): every step leaves exactly the state of
+    the untracked step, and the tracked value is the amax of the stored master."""
+    ref = make_adam_state(sizes, ("adam-track",))
+    trk = _with_tracking(make_adam_state(sizes, ("adam-track",)), wq=True)
+    ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(ref)) // 4, **F32)
+    for step in (1, 2, 3):
+        before = [snapshot(c) for c in trk]
+        fp8.fp8_adam_step(ref, step=step, margin=0, workspace=ws, **HP)
+        fp8.fp8_adam_step(trk, step=step, margin=0, workspace=ws, **HP)
+        assert fp8.fp8_get_status() == 0
+        for b, r, t in zip(before, ref, trk):
+            sr, st = snapshot(r), snapshot(t)
+            for k in ("m", "v", "w", "s_m", "s_v", "s_w"):
+                assert np.array_equal(np.asarray(sr[k]), np.asarray(st[k])), (step, k)
+            assert t.w_amax.item() == _stored_amax(st)
+            q, s_q = oracle.adam_master_e4m3(st["w"], st["s_w"], 0)
+            assert t.wq_scale.item() == s_q and t.wq_inv.item() == 1.0 / s_q
+            assert np.array_equal(t.wq.cpu().numpy(), q)
+            if b["g"].size:
+                check_adam_chunk(b, t, step)
+
+
+def test_adam_tracked_amax_straddling_a_threshold_takes_the_exact_pass():
+    """Master amax just below an FP16 scale threshold with steps large enough
+    to cross it: the bounds cannot fix the exponent, so the master is re-read;
+    the result must still equal the oracle's."""
+    n = 8192
+    thresh = 65504.0 * 2.0 ** -17  # new scale 2^17 below it, 2^16 above
+    w = synth.normal_f32((n,), 0.1, "straddle", "w")
+    w[17] = np.float32(thresh * (1 - 2e-4))
+    chunks = make_adam_state([n], ("straddle",))
+    c = chunks[0]
+    d = to_dev(w)
+    a, s, inv = scalar(), scalar(), scalar()
+    fp8.fp8_amax(d, a)
+    fp8.fp8_compute_scale(a, fp8.FP8_F16S, 0, 1.0, c.w_scale, inv)
+    fp8.fp8_cast(d, fp8.FP8_F16S, c.w_scale, c.w)
+    trk = _with_tracking(chunks)
+    trk[0].w_amax.fill_(_stored_amax(snapshot(trk[0])))
+    before = snapshot(trk[0])
+    hp = dict(HP, lr=1e-1)  # step |dw| ~ 0.1 >> distance to the threshold
+    ws = torch.zeros(fp8.fp8_adam_workspace_bytes(1) // 4, **F32)
+    fp8.fp8_adam_step(trk, step=1, margin=0, workspace=ws, **hp)
+    assert fp8.fp8_get_status() == 0
+    out = oracle.adam_step(before["g"], before["g_inv"], before["m"], before["s_m"], before["v"], before["s_v"],
+                           before["w"], before["s_w"], t=1, margin=0, **hp)
+    after = snapshot(trk[0])
+    assert (after["s_m"], after["s_v"], after["s_w"]) == (out["s_m"], out["s_v"], out["s_w"])
+    ref = f16_vals(out["wh"]) / out["s_w"]
+    got = f16_vals(after["w"]) / after["s_w"]
+    assert np.all(np.abs(got - ref) <= f16_ulp(f16_vals(out["wh"])) / out["s_w"])
+    assert trk[0].w_amax.item() == _stored_amax(after)

@@ -448,6 +448,21 @@ def _check_ties(ours, ref, exact, dec):
         assert abs(exact[i] - mid) <= 1e-12 * abs(mid), (i, exact[i], a, b)
 
 
+def test_adam_master_e4m3_copy_matches_independent_route():
+    """E4M3 copy of the stored master == torch float8 of (numpy-decoded half /
+    s_w * s_q) with s_q from the brute-force exponent of the decoded amax."""
+    w = synth.normal_f32((3001,), 0.02, "pin", "wq")
+    _, s_w = oracle.compute_scale(oracle.amax(w), oracle.F16, 0)
+    wh = oracle.cast(w, oracle.F16, s_w)
+    for margin in (0, 2):
+        q, s_q = oracle.adam_master_e4m3(wh, s_w, margin)
+        dec = wh.view(np.float16).astype(np.float64) / s_w
+        e = _brute_exponent(float(np.max(np.abs(dec))), 448.0) - margin
+        assert s_q == 2.0 ** e
+        ref = torch.from_numpy(dec * s_q).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        assert np.array_equal(q, ref)
+
+
 def test_adam_state_bytes_per_param():
     """[FP8-LM] O2: FP8 grad 1 B + FP8 m1 1 B + FP16 m2 2 B + FP16 master 2 B = 6 B/param."""
     n = 1000
