@@ -74,6 +74,16 @@ def _bind(lib):
     lib.orc_adam_step.argtypes = [sz, p, d, p, ctypes.POINTER(d), p, ctypes.POINTER(d), p,
                                   ctypes.POINTER(d), d, d, d, d, i, i, p, p]
     lib.orc_adam_step.restype = i
+    lib.orc_adam_step_amax.argtypes = [sz, p, d, p, ctypes.POINTER(d), p, ctypes.POINTER(d), p,
+                                       ctypes.POINTER(d), d, d, d, d, i, i, p, p, p]
+    lib.orc_adam_step_amax.restype = i
+    u64p = ctypes.POINTER(ctypes.c_ulonglong)
+    lib.orc_cast_counts.argtypes, lib.orc_cast_counts.restype = [p, i, sz, i, d, p, u64p], None
+    lib.orc_grad_scale.argtypes, lib.orc_grad_scale.restype = [d, i, i, d, ctypes.POINTER(d)], i
+    lib.orc_sum_codes.argtypes, lib.orc_sum_codes.restype = [p, i, sz, sz, i, p, u64p], None
+    lib.orc_mu_update.argtypes = [ctypes.POINTER(d), ctypes.POINTER(i), ctypes.c_ulonglong, ctypes.c_ulonglong,
+                                  d, i, d, d]
+    lib.orc_mu_update.restype = None
     lib.orc_num_threads.argtypes, lib.orc_num_threads.restype = [], i
     lib.orc_set_num_threads.argtypes, lib.orc_set_num_threads.restype = [i], None
     return lib
@@ -216,10 +226,12 @@ def adam_update_f64(g, m0, v0, w0, lr, beta1, beta2, eps, t):
     return m, v, w
 
 
-def adam_step(gq, g_inv, mq, s_m, vh, s_v, wh, s_w, lr, beta1, beta2, eps, t, margin):
+def adam_step(gq, g_inv, mq, s_m, vh, s_v, wh, s_w, lr, beta1, beta2, eps, t, margin, amax_in=None):
     """One decoupled Adam step on one tensor's stored state (copies; inputs untouched).
 
     Returns dict(rc, mq, s_m, vh, s_v, wh, s_w, amax=(|m|, v, |w|) of the new float64 values).
+    amax_in: optional (|m|, v, |w|) amaxes the new scales are taken from instead
+    of this call's own (a slice of a larger tensor, see adam_step_sharded).
     """
     n = np.asarray(gq).size
     gq = np.ascontiguousarray(gq, dtype=np.uint8)
@@ -229,11 +241,46 @@ def adam_step(gq, g_inv, mq, s_m, vh, s_v, wh, s_w, lr, beta1, beta2, eps, t, ma
     sm, sv, sw = ctypes.c_double(s_m), ctypes.c_double(s_v), ctypes.c_double(s_w)
     work = np.empty(7 * max(n, 1), dtype=np.float64)
     am = np.zeros(3, dtype=np.float64)
-    rc = _load().orc_adam_step(n, _ptr(gq), float(g_inv), _ptr(mq), ctypes.byref(sm), _ptr(vh),
-                               ctypes.byref(sv), _ptr(wh), ctypes.byref(sw), lr, beta1, beta2, eps,
-                               t, margin, _ptr(work), _ptr(am))
+    if amax_in is None:
+        rc = _load().orc_adam_step(n, _ptr(gq), float(g_inv), _ptr(mq), ctypes.byref(sm), _ptr(vh),
+                                   ctypes.byref(sv), _ptr(wh), ctypes.byref(sw), lr, beta1, beta2, eps,
+                                   t, margin, _ptr(work), _ptr(am))
+    else:
+        ain = np.array(amax_in, dtype=np.float64)
+        rc = _load().orc_adam_step_amax(n, _ptr(gq), float(g_inv), _ptr(mq), ctypes.byref(sm), _ptr(vh),
+                                        ctypes.byref(sv), _ptr(wh), ctypes.byref(sw), lr, beta1, beta2,
+                                        eps, t, margin, _ptr(work), _ptr(ain), _ptr(am))
     return dict(rc=rc, mq=mq, s_m=sm.value, vh=vh, s_v=sv.value, wh=wh, s_w=sw.value,
                 amax=tuple(am))
+
+
+def _nan_max(values):
+    r = 0.0
+    for x in values:
+        if np.isnan(x):
+            return float("nan")
+        r = max(r, x)
+    return r
+
+
+def adam_step_sharded(gq, g_inv, mq, s_m, vh, s_v, wh, s_w, lr, beta1, beta2, eps, t, margin, bounds):
+    """The step of adam_step with the tensor's elements split into slices
+    [lo, hi) ("FP8-LM", 提案手法 O3: optimizer state partitioned ZeRO-style
+    over data-parallel ranks): every slice first yields the amaxes of its new
+    values; the tensor's amax is their maximum (a NaN wins); every slice is
+    then requantised with the scales of that maximum.  Returns the
+    concatenated state in the form adam_step returns it."""
+    gq, mq, vh, wh = (np.asarray(a).reshape(-1) for a in (gq, mq, vh, wh))
+    args = (lr, beta1, beta2, eps, t, margin)
+    parts = [(lo, hi) for lo, hi in bounds]
+    stats = [adam_step(gq[lo:hi], g_inv, mq[lo:hi], s_m, vh[lo:hi], s_v, wh[lo:hi], s_w, *args)["amax"]
+             for lo, hi in parts]
+    glob = tuple(_nan_max([s[j] for s in stats]) for j in range(3))
+    outs = [adam_step(gq[lo:hi], g_inv, mq[lo:hi], s_m, vh[lo:hi], s_v, wh[lo:hi], s_w, *args, amax_in=glob)
+            for lo, hi in parts]
+    cat = {k: np.concatenate([o[k] for o in outs]) for k in ("mq", "vh", "wh")}
+    return dict(rc=max(o["rc"] for o in outs), s_m=outs[0]["s_m"], s_v=outs[0]["s_v"], s_w=outs[0]["s_w"],
+                amax=glob, **cat)
 
 
 def adam_master_e4m3(wh, s_w: float, margin: int):
@@ -247,6 +294,63 @@ def adam_master_e4m3(wh, s_w: float, margin: int):
     a = amax(wh, DT_F16) / s_w
     rc, s_q = compute_scale(a, E4M3, margin)
     return cast(wh, E4M3, s_q / s_w, DT_F16), s_q
+
+
+# ---------------------------------------------------------------- scaling variants, FP8 all-reduce
+def cast_counts(x, fmt: int, scale: float, dtype: int | None = None):
+    """(codes, (underflows, overflows)) of cast(x, fmt, scale)."""
+    x = np.ascontiguousarray(x)
+    q = np.empty(x.shape, dtype=np.uint16 if fmt == F16 else np.uint8)
+    counts = (ctypes.c_ulonglong * 2)(0, 0)
+    _load().orc_cast_counts(_ptr(x), _dtype_code(x, dtype), x.size, fmt, float(scale), _ptr(q), counts)
+    return q, (counts[0], counts[1])
+
+
+def grad_scale(amax_value: float, fmt: int, margin: int, mu: float) -> tuple[int, float]:
+    """(status, S) with S = mu * 2^(floor(log2(fmt_max/amax)) - margin): the
+    shared payload scale of the FP8 gradient all-reduce."""
+    out = ctypes.c_double(0.0)
+    rc = _load().orc_grad_scale(float(amax_value), fmt, margin, float(mu), ctypes.byref(out))
+    return rc, out.value
+
+
+def sum_codes(rows, fmt: int):
+    """rows: [nranks, n] uint8 codes with one shared scale.  Returns (codes of
+    the exact sum re-encoded, (underflows, overflows))."""
+    rows = np.ascontiguousarray(rows, dtype=np.uint8)
+    nranks, n = rows.shape
+    out = np.empty(n, dtype=np.uint8)
+    counts = (ctypes.c_ulonglong * 2)(0, 0)
+    _load().orc_sum_codes(_ptr(rows), nranks, n, n, fmt, _ptr(out), counts)
+    return out, (counts[0], counts[1])
+
+
+def mu_update(mu: float, clean: int, overflows: int, n: int, theta: float, interval: int,
+              mu_min: float, mu_max: float) -> tuple[float, int]:
+    """The auto-scaling rule for mu: returns (mu, clean steps) after one step."""
+    m, c = ctypes.c_double(mu), ctypes.c_int(clean)
+    _load().orc_mu_update(ctypes.byref(m), ctypes.byref(c), overflows, n, float(theta), interval,
+                          float(mu_min), float(mu_max))
+    return m.value, c.value
+
+
+def fp8_allreduce(grads, fmt: int, margin: int, mu: float):
+    """The FP8 gradient all-reduce over len(grads) ranks ("FP8-LM", 提案手法
+    O1): the amax over all ranks, the shared scale S = grad_scale(amax, mu),
+    every rank's payload cast with S, the exact sum of the payloads
+    re-encoded at S.  Returns dict(codes, S, rc, cast_counts, sum_counts);
+    the reduced gradient is dec(codes) / S (a sum over ranks, not a mean)."""
+    grads = [np.ascontiguousarray(g, dtype=np.float32).reshape(-1) for g in grads]
+    a = amax(np.stack(grads).reshape(-1)) if grads[0].size else 0.0
+    rc, S = grad_scale(a, fmt, margin, mu)
+    rows, cc = [], [0, 0]
+    for g in grads:
+        q, c = cast_counts(g, fmt, S)
+        rows.append(q)
+        cc[0] += c[0]
+        cc[1] += c[1]
+    codes, sc = sum_codes(np.stack(rows), fmt)
+    return dict(codes=codes, S=S, rc=rc, cast_counts=tuple(cc), sum_counts=sc, payloads=np.stack(rows))
 
 
 def num_threads() -> int:

@@ -275,6 +275,107 @@ void orc_cast(const void *x, int dtype, size_t n, int fmt, double scale, void *q
     }
 }
 
+/* ------------------------------------------------------------------------
+ * Underflow / overflow counters.  [FP8-LM] アブレーション研究 compares the
+ * gradient scaling variants by their underflow and overflow rates; [FP8-AMAX]
+ * 실험 결과 (research question RQ3) asks which scaling keeps weights,
+ * activations and gradients clear of both.  reading: an element underflows when it is a non-zero number and
+ * its code is zero; it overflows when |x * s| exceeds the format's largest
+ * finite value (the cast saturates it; inf included, NaN in neither).
+ * counts[0] += underflows, counts[1] += overflows.
+ * ---------------------------------------------------------------------- */
+void orc_cast_counts(const void *x, int dtype, size_t n, int fmt, double scale, void *q,
+                     unsigned long long *counts)
+{
+    orc_cast(x, dtype, n, fmt, scale, q);
+    double fmax = orc_fmt_max(fmt);
+    unsigned long long under = 0, over = 0;
+    for (size_t i = 0; i < n; i++) {
+        double v = load_elem(x, dtype, i);
+        unsigned c = fmt == ORC_F16 ? ((const uint16_t *)q)[i] : ((const uint8_t *)q)[i];
+        if (!isnan(v) && v != 0.0 && code_value(fmt, c) == 0.0)
+            under++;
+        if (fabs(v * scale) > fmax)
+            over++;
+    }
+    counts[0] += under;
+    counts[1] += over;
+}
+
+/*
+ * Shared payload scale of the FP8 gradient all-reduce ([FP8-LM] 提案手法 O1,
+ * Eq. 3).  reading: every rank casts its gradient with one scale taken from
+ * the amax over all ranks' gradients before auto-scaling, times mu:
+ *     S = mu * 2^(floor(log2(fmt_max / amax)) - margin),
+ * so that mu < 1 leaves headroom for the sum of the ranks' payloads.  The
+ * exponent rule, its clamps and amax == 0 / non-finite as in
+ * orc_compute_scale; mu is a power of two and S is clamped to
+ * [2^-126, 2^126].
+ */
+int orc_grad_scale(double amax, int fmt, int margin, double mu, double *scale)
+{
+    double s;
+    int rc = orc_compute_scale(amax, fmt, margin, &s);
+    double t = mu * s;
+    if (t < ldexp(1.0, -126))
+        t = ldexp(1.0, -126);
+    if (t > ldexp(1.0, 126))
+        t = ldexp(1.0, 126);
+    *scale = t;
+    return rc;
+}
+
+/*
+ * Reduction of the ranks' FP8 payloads ([FP8-LM] 提案手法 O1: gradients
+ * all-reduced in FP8).  in holds nranks rows of ld codes, all cast with the
+ * same scale; out_i = enc(sum_r dec(in[r * ld + i])): the exact sum (every
+ * FP8 value is a multiple of the format's smallest subnormal, so float64 adds
+ * them without rounding), re-encoded once in the same format and scale.
+ * readings: the sum starts at +0, so a zero sum is code 0x00; a NaN sum (a
+ * NaN code, or +inf and -inf) gives code 0x7F.
+ * counts as in orc_cast_counts, on the sums: [0] non-zero sums with a zero
+ * code, [1] sums beyond fmt_max (saturated).
+ */
+void orc_sum_codes(const uint8_t *in, int nranks, size_t ld, size_t n, int fmt, uint8_t *out,
+                   unsigned long long *counts)
+{
+    double fmax = orc_fmt_max(fmt);
+    for (size_t i = 0; i < n; i++) {
+        double sum = 0.0;
+        for (int r = 0; r < nranks; r++)
+            sum += orc_fp8_decode(fmt, in[(size_t)r * ld + i]);
+        unsigned c = isnan(sum) ? 0x7Fu : orc_fp8_encode(fmt, sum);
+        out[i] = (uint8_t)c;
+        if (!isnan(sum) && sum != 0.0 && orc_fp8_decode(fmt, c) == 0.0)
+            counts[0]++;
+        if (fabs(sum) > fmax)
+            counts[1]++;
+    }
+}
+
+/*
+ * Auto-scaling update of mu between steps ([FP8-LM] 提案手法 O1: mu changes
+ * dynamically).  The pages give no rule; this one is the build's own, in the
+ * manner of dynamic loss scaling: when more than theta * n of the n reduced
+ * gradient elements overflowed, mu halves (not below mu_min) and the count
+ * of clean steps restarts; otherwise the count grows, and after `interval`
+ * clean steps in a row mu doubles (not above mu_max) and the count restarts.
+ */
+void orc_mu_update(double *mu, int *clean, unsigned long long overflows, unsigned long long n,
+                   double theta, int interval, double mu_min, double mu_max)
+{
+    if ((double)overflows > theta * (double)n) {
+        *mu = (*mu * 0.5 < mu_min) ? mu_min : *mu * 0.5;
+        *clean = 0;
+        return;
+    }
+    *clean += 1;
+    if (*clean >= interval) {
+        *mu = (*mu * 2.0 > mu_max) ? mu_max : *mu * 2.0;
+        *clean = 0;
+    }
+}
+
 /* amax over all cores: the same definition as orc_amax, split into ranges. */
 double orc_amax_parallel(const void *x, int dtype, size_t n)
 {
@@ -406,11 +507,15 @@ static double max_abs(const double *x, size_t n)
  *   vh (FP16, scale *s_v), wh (FP16, scale *s_w).
  * Scratch: 7 arrays of n doubles supplied by the caller (work).
  * amax_out[0..2] receives amax|m|, amax v, amax|w| of the new float64 values.
- * Returns ORC_ERR_NONFINITE if any new amax is not finite.
+ * amax_in: NULL, or the three amaxes the new scales are taken from instead
+ * (those of the whole tensor when this call updates one slice of it, as in
+ * the element-sharded optimizer of "FP8-LM", 提案手法 O3).
+ * Returns ORC_ERR_NONFINITE if any amax the scales come from is not finite.
  */
-int orc_adam_step(size_t n, const uint8_t *gq, double g_inv, uint8_t *mq, double *s_m,
-                  uint16_t *vh, double *s_v, uint16_t *wh, double *s_w, double lr, double beta1,
-                  double beta2, double eps, int t, int margin, double *work, double *amax_out)
+int orc_adam_step_amax(size_t n, const uint8_t *gq, double g_inv, uint8_t *mq, double *s_m,
+                       uint16_t *vh, double *s_v, uint16_t *wh, double *s_w, double lr, double beta1,
+                       double beta2, double eps, int t, int margin, double *work,
+                       const double *amax_in, double *amax_out)
 {
     double *g = work, *m0 = work + n, *v0 = work + 2 * n, *w0 = work + 3 * n;
     double *m = work + 4 * n, *v = work + 5 * n, *w = work + 6 * n;
@@ -430,6 +535,11 @@ int orc_adam_step(size_t n, const uint8_t *gq, double g_inv, uint8_t *mq, double
     amax_out[0] = am;
     amax_out[1] = av;
     amax_out[2] = aw;
+    if (amax_in) {
+        am = amax_in[0];
+        av = amax_in[1];
+        aw = amax_in[2];
+    }
     int rc = ORC_OK;
     rc |= orc_compute_scale(am, ORC_E4M3, margin, s_m);
     rc |= orc_compute_scale(av, ORC_F16, margin, s_v);
@@ -443,6 +553,14 @@ int orc_adam_step(size_t n, const uint8_t *gq, double g_inv, uint8_t *mq, double
         wh[i] = (uint16_t)orc_f16_encode(w[i] * sw);
     }
     return rc ? ORC_ERR_NONFINITE : ORC_OK;
+}
+
+int orc_adam_step(size_t n, const uint8_t *gq, double g_inv, uint8_t *mq, double *s_m,
+                  uint16_t *vh, double *s_v, uint16_t *wh, double *s_w, double lr, double beta1,
+                  double beta2, double eps, int t, int margin, double *work, double *amax_out)
+{
+    return orc_adam_step_amax(n, gq, g_inv, mq, s_m, vh, s_v, wh, s_w, lr, beta1, beta2, eps, t,
+                              margin, work, NULL, amax_out);
 }
 
 int orc_num_threads(void)

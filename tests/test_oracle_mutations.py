@@ -32,6 +32,16 @@ MUTATIONS = {
     "adam_wrong_scale_format": ("rc |= orc_compute_scale(am, ORC_E4M3, margin, s_m);",
                                 "rc |= orc_compute_scale(am, ORC_F16, margin, s_m);"),
     "amax_nan_ignored": ("return saw_nan ? NAN : m;", "return m;"),
+    "sharded_slice_amax_used": ("    if (amax_in) {", "    if (0 && amax_in) {"),
+    "grad_scale_mu_dropped": ("    double t = mu * s;\n", "    double t = s;\n"),
+    "sum_overflow_inclusive": ("        if (fabs(sum) > fmax)\n", "        if (fabs(sum) >= fmax)\n"),
+    "cast_underflow_counts_zeros": ("if (!isnan(v) && v != 0.0 && code_value(fmt, c) == 0.0)",
+                                    "if (!isnan(v) && code_value(fmt, c) == 0.0)"),
+    "mu_quartered": ("*mu = (*mu * 0.5 < mu_min) ? mu_min : *mu * 0.5;",
+                     "*mu = (*mu * 0.25 < mu_min) ? mu_min : *mu * 0.25;"),
+    "mu_growth_late": ("    if (*clean >= interval) {", "    if (*clean > interval) {"),
+    "sum_rounded_through_float": ("            sum += orc_fp8_decode(fmt, in[(size_t)r * ld + i]);",
+                                  "            sum = (float)(sum + orc_fp8_decode(fmt, in[(size_t)r * ld + i]));"),
 }
 
 PINS = [
@@ -48,6 +58,13 @@ PINS = [
     lambda: pins.test_gemm_fwd_dgrad_wgrad_vs_numpy((3, 5, 7)),
     lambda: pins.test_adam_update_matches_torch_optim(2),
     pins.test_adam_step_composition_with_independent_pieces,
+    pins.test_adam_sharded_equals_whole_tensor_step,
+    lambda: pins.test_cast_counts_closed_forms(oracle.E5M2),
+    pins.test_grad_scale_closed_forms,
+    lambda: pins.test_sum_codes_vs_torch(oracle.E5M2, 3),
+    pins.test_sum_codes_specials,
+    pins.test_mu_update_hand_traced,
+    pins.test_fp8_allreduce_pre_post_auto_hand_built,
 ]
 
 

@@ -463,6 +463,43 @@ def test_adam_master_e4m3_copy_matches_independent_route():
         assert np.array_equal(q, ref)
 
 
+def test_adam_sharded_equals_whole_tensor_step():
+    """[FP8-LM] 提案手法 O3 (ZeRO-partitioned optimizer state): splitting a
+    tensor into slices, taking the max of the slices' amaxes and requantising
+    every slice with the scales of that max leaves exactly the state of the
+    whole-tensor step.  Outliers in the first and the last slice make the
+    slices' own scales differ from the tensor's."""
+    n = 4099
+    gf = synth.normal_f32((n,), 1e-3, "pin", "shard", "g")
+    gf[5] = 0.03      # m and v amax in the first slice
+    w_init = synth.normal_f32((n,), 0.02, "pin", "shard", "w")
+    w_init[n - 3] = 0.9   # master amax in the last slice
+    _, sg = oracle.compute_scale(oracle.amax(gf), oracle.E5M2, 0, mu=2.0 ** 10)
+    gq = oracle.cast(gf, oracle.E5M2, sg)
+    _, s_w = oracle.compute_scale(oracle.amax(w_init), oracle.F16, 0)
+    wh = oracle.cast(w_init, oracle.F16, s_w)
+    m_prev = synth.normal_f32((n,), 1e-4, "pin", "shard", "m")
+    _, s_m = oracle.compute_scale(oracle.amax(m_prev), oracle.E4M3, 0)
+    mq = oracle.cast(m_prev, oracle.E4M3, s_m)
+    v_prev = np.abs(synth.normal_f32((n,), 1e-7, "pin", "shard", "v"))
+    _, s_v = oracle.compute_scale(oracle.amax(v_prev), oracle.F16, 0)
+    vh = oracle.cast(v_prev, oracle.F16, s_v)
+    state = (gq, 1 / sg, mq, s_m, vh, s_v, wh, s_w)
+    whole = oracle.adam_step(*state, t=2, margin=0, **HP)
+    splits = [[(0, 2048), (2048, n)], [(0, 1024), (1024, 3072), (3072, n), (n, n)],
+              [(i * 512, min(n, (i + 1) * 512)) for i in range(9)]]
+    for bounds in splits:
+        own = [oracle.adam_step(gq[lo:hi], 1 / sg, mq[lo:hi], s_m, vh[lo:hi], s_v, wh[lo:hi], s_w,
+                                t=2, margin=0, **HP) for lo, hi in bounds if hi > lo]
+        assert len({(o["s_m"], o["s_v"], o["s_w"]) for o in own}) > 1  # slices alone disagree
+        shard = oracle.adam_step_sharded(*state, t=2, margin=0, bounds=bounds, **HP)
+        for k in ("s_m", "s_v", "s_w", "rc"):
+            assert shard[k] == whole[k], k
+        for k in ("mq", "vh", "wh"):
+            assert np.array_equal(shard[k], whole[k]), k
+        assert shard["amax"] == whole["amax"]
+
+
 def test_adam_state_bytes_per_param():
     """[FP8-LM] O2: FP8 grad 1 B + FP8 m1 1 B + FP16 m2 2 B + FP16 master 2 B = 6 B/param."""
     n = 1000
@@ -470,3 +507,156 @@ def test_adam_state_bytes_per_param():
            + np.zeros(n, np.uint16).nbytes + np.zeros(n, np.uint16).nbytes) / n
     assert per == 6.0
     assert 16 / per == pytest.approx(2.67, abs=0.01)
+
+
+# ---------------------------------------------------------------- scaling variants and the FP8 all-reduce
+MIN_SUB = {oracle.E4M3: 2.0 ** -9, oracle.E5M2: 2.0 ** -16, oracle.F16: 2.0 ** -24}  # [OFP8], IEEE binary16
+MAXV = {oracle.E4M3: 448.0, oracle.E5M2: 57344.0, oracle.F16: 65504.0}
+
+
+@pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2, oracle.F16])
+def test_cast_counts_closed_forms(fmt):
+    """Underflow: a non-zero value whose code is zero; overflow: |x s| above
+    the format's largest finite value.  Hand-placed values with scale 1."""
+    t, mx = MIN_SUB[fmt], MAXV[fmt]
+    x = np.array([0.0, -0.0, t / 2, -t / 2, t / 4, t * 0.5000001, t, mx, -mx, mx * (1 + 2 ** -20), -2 * mx,
+                  np.inf, -np.inf, np.nan, 1.0], dtype=np.float32)
+    q, (under, over) = oracle.cast_counts(x, fmt, 1.0)
+    x = x.astype(np.float64)
+    # t/2 and -t/2 are ties that round to the even code 0; t/4 rounds to 0
+    assert under == 3
+    # just above max, 2 max, +-inf
+    assert over == 4
+    # the same elements by an independent route: torch / numpy casts
+    if fmt == oracle.F16:
+        with np.errstate(over="ignore"):
+            ref = x.astype(np.float16).astype(np.float64)
+    else:
+        ref = torch.from_numpy(np.clip(x, -mx, mx)).to(TORCH_FP8[fmt]).double().numpy()
+    assert under == int(np.sum((x != 0) & ~np.isnan(x) & (ref == 0)))
+    assert over == int(np.sum(np.abs(x) > mx))
+
+
+def test_cast_counts_random_vs_torch():
+    x = synth.normal_f32((20000,), 1.0, "pin", "counts")
+    x[::7] *= 1e-6
+    for fmt in (oracle.E4M3, oracle.E5M2):
+        for s in (2.0 ** -8, 1.0, 2.0 ** 9):
+            q, (under, over) = oracle.cast_counts(x, fmt, s)
+            y = x.astype(np.float64) * s
+            ref = torch.from_numpy(np.clip(y, -MAXV[fmt], MAXV[fmt])).to(TORCH_FP8[fmt]).double().numpy()
+            assert under == int(np.sum((x != 0) & (ref == 0)))
+            assert over == int(np.sum(np.abs(y) > MAXV[fmt]))
+
+
+def test_grad_scale_closed_forms():
+    """S = mu * 2^(floor(log2(fmt_max/amax)) - margin): the exponent by brute
+    force, mu applied after it (it does not cancel, unlike the cast scale)."""
+    assert oracle.grad_scale(1.0, oracle.E5M2, 0, 1.0) == (0, 2.0 ** 15)
+    assert oracle.grad_scale(1.0, oracle.E5M2, 0, 2.0 ** -3) == (0, 2.0 ** 12)
+    assert oracle.grad_scale(1.0, oracle.E5M2, 1, 2.0 ** -3) == (0, 2.0 ** 11)
+    assert oracle.grad_scale(0.0, oracle.E4M3, 0, 2.0 ** -2) == (0, 2.0 ** -2)
+    assert oracle.grad_scale(float("inf"), oracle.E4M3, 0, 1.0)[0] != 0
+    assert oracle.grad_scale(1e-38, oracle.E5M2, 0, 2.0 ** 8)[1] == 2.0 ** 126
+    r = synth.rng("pin", "gscale")
+    for a in np.exp(r.uniform(-40, 40, 200)):
+        for fmt in (oracle.E4M3, oracle.E5M2):
+            for mu_e in (-5, 0, 3):
+                e = _brute_exponent(float(a), MAXV[fmt])
+                rc, S = oracle.grad_scale(float(a), fmt, 0, 2.0 ** mu_e)
+                assert S == 2.0 ** max(-126, min(126, max(-126, min(126, e)) + mu_e))
+                # with mu = 1 the payload of the largest element fits, doubled it would not
+                if mu_e == 0 and -126 < e < 126:
+                    assert a * S <= MAXV[fmt] < 2 * a * S
+
+
+def _finite_codes(shape, fmt, *key):
+    c = synth.rng(*key).integers(0, 256, size=shape, dtype=np.uint8)
+    bad = (c & 0x7F) == 0x7F if fmt == oracle.E4M3 else (c & 0x7C) == 0x7C
+    c[bad] &= 0x83  # finite, small
+    return c
+
+
+@pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2])
+@pytest.mark.parametrize("nranks", [1, 2, 3, 8])
+def test_sum_codes_vs_torch(fmt, nranks):
+    rows = _finite_codes((nranks, 5000), fmt, "pin", "sum", fmt, nranks)
+    out, (under, over) = oracle.sum_codes(rows, fmt)
+    exact = torch.from_numpy(rows).view(TORCH_FP8[fmt]).double().sum(0).numpy()
+    # brute force: nearest finite code by a scan of the whole table, ties to the
+    # even code, saturating (torch's own double -> float8 path rounds through
+    # float32 first, which double-rounds sums like 45055.9997)
+    codes = np.arange(256, dtype=np.uint8)
+    table = torch.from_numpy(codes).view(TORCH_FP8[fmt]).double().numpy()
+    ok = np.isfinite(table)
+    codes, table = codes[ok], table[ok]
+    y = np.clip(exact, -MAXV[fmt], MAXV[fmt])
+    d = np.abs(table[None, :] - y[:, None])
+    best = d.min(1, keepdims=True)
+    cand = np.where(d == best, codes[None, :].astype(int), 999)
+    even = np.where(cand % 2 == 0, cand, 999).min(1)
+    pick = np.where((cand != 999).sum(1) > 1, even, cand.min(1))
+    # equal-distance pairs are +0 and -0 only when y == 0: take +0
+    pick = np.where(y == 0, 0, pick)
+    assert np.array_equal(out, pick.astype(np.uint8))
+    assert over == int((np.abs(exact) > MAXV[fmt]).sum())
+    assert under == 0
+    if nranks == 1:  # one rank: the codes come back, a negative zero as +0 (the sum starts at +0)
+        assert np.array_equal(out, np.where(rows[0] == 0x80, 0, rows[0]))
+
+
+def test_sum_codes_specials():
+    E5, E4 = oracle.E5M2, oracle.E4M3
+    cases = [  # (fmt, codes of the ranks, expected code, expected overflow)
+        (E5, [0x7B, 0x7B], 0x7B, 1),   # max + max saturates
+        (E5, [0x7B, 0x00], 0x7B, 0),   # exactly max: no overflow
+        (E5, [0x01, 0x81], 0x00, 0),   # +-min subnormal cancel: an exact zero is no underflow
+        (E5, [0x7C, 0x3C], 0x7B, 1),   # +inf + 1 -> +inf, saturated
+        (E5, [0x7C, 0xFC], 0x7F, 0),   # +inf + -inf -> NaN
+        (E5, [0x7E, 0x00], 0x7F, 0),   # NaN
+        (E4, [0xFF, 0x38], 0x7F, 0),   # NaN (negative NaN code) -> 0x7F
+        (E4, [0x7E, 0x7E, 0xFE], 0x7E, 0),  # 448 + 448 - 448 = 448
+        (E4, [0x01] * 3, 0x03, 0),     # 3 x 2^-9: an exact subnormal
+        (E5, [0x3D] * 3, 0x44, 0),     # 3 x 1.25 = 3.75, halfway between 3.5 (0x43) and 4 (0x44): even
+    ]
+    for fmt, codes, want, want_over in cases:
+        out, (under, over) = oracle.sum_codes(np.array(codes, dtype=np.uint8).reshape(-1, 1), fmt)
+        assert (int(out[0]), over, under) == (want, want_over, 0), (fmt, codes)
+
+
+def test_mu_update_hand_traced():
+    args = dict(theta=1e-3, interval=3, mu_min=2.0 ** -4, mu_max=4.0)
+    mu, clean = 1.0, 0
+    trace = []
+    for over in (0, 0, 0, 2, 1, 0, 0, 0, 0, 0, 0, 0, 0, 0):
+        mu, clean = oracle.mu_update(mu, clean, over, 1000, **args)
+        trace.append((mu, clean))
+    assert trace == [(1.0, 1), (1.0, 2), (2.0, 0),    # three clean steps: doubles
+                     (1.0, 0),                          # 2 > 1e-3 * 1000: halves
+                     (1.0, 1),                          # 1 is not above the threshold
+                     (1.0, 2), (2.0, 0), (2.0, 1), (2.0, 2), (4.0, 0),
+                     (4.0, 1), (4.0, 2), (4.0, 0), (4.0, 1)]  # held at mu_max
+    mu, clean = 2.0 ** -4, 5
+    assert oracle.mu_update(mu, clean, 10 ** 6, 1000, **args) == (2.0 ** -4, 0)  # held at mu_min
+    assert oracle.mu_update(1.0, 0, 0, 0, **args) == (1.0, 1)  # empty tensor: no overflow
+
+
+def test_fp8_allreduce_pre_post_auto_hand_built():
+    """[FP8-LM] アブレーション研究: dividing by the rank count after the sum
+    (post-scaling, mu = 1) overflows where the ranks agree in sign; dividing
+    before the cast (pre-scaling, mu = 1/N) underflows small gradients.
+    Four ranks, E5M2, amax 1 on every rank."""
+    N = 4
+    g = np.zeros((N, 4), dtype=np.float32)
+    g[:, 0] = 1.0                 # sum 4 x payload: overflows at mu = 1
+    g[:, 1] = 2.0 ** -30          # payload 2^-15 at mu = 1, 2^-17 (a tie to 0) at mu = 1/4
+    g[:, 2] = [0.5, -0.5, 0.25, -0.25]   # cancels exactly
+    g[:, 3] = [0.75, 0.0, 0.0, 0.0]
+    post = oracle.fp8_allreduce(list(g), oracle.E5M2, 0, 1.0)
+    pre = oracle.fp8_allreduce(list(g), oracle.E5M2, 0, 1.0 / N)
+    assert post["S"] == 2.0 ** 15 and pre["S"] == 2.0 ** 13
+    assert post["cast_counts"] == (0, 0) and post["sum_counts"] == (0, 1)
+    assert pre["cast_counts"] == (4, 0) and pre["sum_counts"] == (0, 0)
+    val = lambda r: _torch_dec(r["codes"], oracle.E5M2) / r["S"]
+    np.testing.assert_array_equal(val(post), [1.75, 4 * 2.0 ** -30, 0.0, 0.75])   # element 0 saturated
+    np.testing.assert_array_equal(val(pre), [4.0, 0.0, 0.0, 0.75])                # element 1 lost
