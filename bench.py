@@ -48,6 +48,21 @@ GRAD_CAST_BYTES = 4 + 1       # fp32 dW read (amax fused in the GEMM) + code wri
 ADAM_BYTES = 11               # read g1 m1 v2 w2, write m1 v2 w2
 
 
+def gemm_traffic():
+    """Mean DRAM bytes per GEMM launch of this step from the committed ncu
+    capture, valid while the GEMM kernel source is the one that was measured."""
+    import hashlib
+
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "gemm_step_traffic.json")))
+        src = open(os.path.join(ROOT, "fp8_mixed_precision_tensor_b200", "csrc", "gemm.cuh"), "rb").read()
+        if hashlib.sha256(src).hexdigest() == rec["gemm_source_sha256"]:
+            return rec["dram_bytes_per_launch_mean"]
+    except Exception:
+        pass
+    return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -162,13 +177,12 @@ class Block7BStep:
         self.flops = sum(3 * 2 * d["M"] * d["N"] * d["K"] for d in self.L)
         self.cast_elems = sum(d["M"] * d["K"] + d["N"] * d["K"] + d["M"] * d["N"] for d in self.L)
         self.params = sum(d["N"] * d["K"] for d in self.L)
-        self.launches_per_step = 4 * (3 * 3 + 3 + 2) + 3  # amax/scale/cast x3, GEMMs, grad scale+cast; Adam
+        self.launches_per_step = 4 * (3 * 2 + 3 + 1) + 3  # (amax, scale+cast) x3, GEMMs, grad scale+cast; Adam
 
     def quantise(self, x, fmt, sc, i, mu=1.0, out=None):
         fp8 = self.fp8
         fp8.fp8_amax(x, sc[i:i + 1])
-        fp8.fp8_compute_scale(sc[i:i + 1], fmt, 0, mu, sc[i + 1:i + 2], sc[i + 2:i + 3])
-        fp8.fp8_cast(x, fmt, sc[i + 1:i + 2], out)
+        fp8.fp8_scale_cast(x, fmt, sc[i:i + 1], 0, mu, sc[i + 1:i + 2], sc[i + 2:i + 3], out)
 
     def step(self, ev=None):
         """Enqueue one step.  ev: optional dict name -> list of (start, end)
@@ -196,8 +210,7 @@ class Block7BStep:
             fp8.fp8_linear_wgrad(d["dyq"], sc[8:9], d["xq"], sc[2:3], d["dw"], sc[14:15])
             if e: e[1].record()
             e = mark("grad_cast")
-            fp8.fp8_compute_scale(sc[14:15], fp8.FP8_E5M2, 0, MU, sc[10:11], sc[11:12])
-            fp8.fp8_cast(d["dw"], fp8.FP8_E5M2, sc[10:11], d["gq"])
+            fp8.fp8_scale_cast(d["dw"], fp8.FP8_E5M2, sc[14:15], 0, MU, sc[10:11], sc[11:12], d["gq"])
             if e: e[1].record()
         self.t += 1
         e = mark("adam")
@@ -383,8 +396,9 @@ def run_gpu(args):
                    "gemm_flops_per_step": runner.flops, "l2": "inputs larger than L2 (no flush)",
                    "parallelism": f"replicas{world}" if world > 1 else "single"},
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
-                     "frac": gemm_tflops / fp8_peak, "traffic": None,
-                     "kernel": "k_gemm (fwd+dgrad+wgrad, flop-weighted over the 12 launches)",
+                     "frac": gemm_tflops / fp8_peak, "traffic": gemm_traffic(),
+                     "kernel": "k_gemm3 (fwd+dgrad+wgrad; achieved = GEMM flops per step / summed GEMM "
+                               "time; traffic = mean DRAM bytes per launch)",
                      "peak_src": f"2 x bf16_tflops_sustained ({peaks['src']})"},
         "kernels": {
             "gemm": {"ms": t_gemm, "TFLOP/s": gemm_tflops, "frac_fp8_peak": gemm_tflops / fp8_peak},

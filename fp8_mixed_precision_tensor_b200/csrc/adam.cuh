@@ -182,7 +182,9 @@ __global__ void __launch_bounds__(kAdamThreads) k_adam(const __grid_constant__ A
         sc = adam_scalars(L, *C.g_inv, 1.0f / *C.m_scale, 1.0f / *C.v_scale, 1.0f / *C.w_scale);
       } else {
         const uint32_t fl = ws_flags(L, ci);
-        tracked = (fl & 2u) != 0;
+        // pass 2: keep the stored-master amax (and its check) for every chunk
+        // that tracks it, including the step that first establishes it
+        tracked = PASS == 2 ? C.w_amax != nullptr : (fl & 2u) != 0;
         active = PASS == 2 || (fl & 1u) != 0;
         sc = adam_scalars(L, *C.g_inv, ws_get(L, ci, WS_OLDINV_M), ws_get(L, ci, WS_OLDINV_V),
                           ws_get(L, ci, WS_OLDINV_W));
@@ -237,14 +239,17 @@ __global__ void __launch_bounds__(kAdamThreads) k_adam(const __grid_constant__ A
           aw = max(aw, max(absbits_f32(adam_master(wd.x, d_a, sc)), absbits_f32(adam_master(wd.y, d_b, sc))));
         } else {
           const float w_a = adam_master(wd.x, d_a, sc), w_b = adam_master(wd.y, d_b, sc);
-          aw = max(aw, max(absbits_f32(w_a), absbits_f32(w_b)));
+          if (tracked) aw = max(aw, max(absbits_f32(w_a), absbits_f32(w_b)));
           const uint32_t mc = enc2<FP8_E4M3>(__fmul_rn(m_a, new_m), __fmul_rn(m_b, new_m));
           if (p & 1) mo[p >> 1] |= mc << 16; else mo[p >> 1] = mc;
           vo[p] = f16x2(__fmul_rn(v_a, new_v), __fmul_rn(v_b, new_v));
           wo[p] = f16x2(__fmul_rn(w_a, new_w), __fmul_rn(w_b, new_w));
-          const float2 st = h2f2(wo[p]);  // the stored master (scaled)
-          am = max(am, max(absbits_f32(st.x), absbits_f32(st.y)));
+          if (tracked) {  // amax of the stored master (scaled), for the tracked value
+            const uint32_t h = __vmaxu2(wo[p] & 0x7fff7fffu, 0u);
+            am = max(am, absbits_f32(__half2float(__ushort_as_half((unsigned short)max(h & 0xffffu, h >> 16)))));
+          }
           if (want_wq) {
+            const float2 st = h2f2(wo[p]);  // the stored master (scaled)
             // E4M3 copy of the stored master: (h / s_w) * s_q, exact in f32
             const uint32_t qc = enc2<FP8_E4M3>(__fmul_rn(__fmul_rn(st.x, inv_new_w), new_wq),
                                                __fmul_rn(__fmul_rn(st.y, inv_new_w), new_wq));
@@ -276,13 +281,13 @@ __global__ void __launch_bounds__(kAdamThreads) k_adam(const __grid_constant__ A
           aw = max(aw, absbits_f32(adam_master(wd, d, sc)));
         } else {
           const float w = adam_master(wd, d, sc);
-          aw = max(aw, absbits_f32(w));
+          if (tracked) aw = max(aw, absbits_f32(w));
           C.m[i] = (uint8_t)(enc2<FP8_E4M3>(__fmul_rn(m, new_m), 0.0f) & 0xffu);
           C.v[i] = __half_as_ushort(__float2half_rn(__fmul_rn(v, new_v)));
           const __half h = __float2half_rn(__fmul_rn(w, new_w));
           C.w[i] = __half_as_ushort(h);
           const float st = __half2float(h);
-          am = max(am, absbits_f32(st));
+          if (tracked) am = max(am, absbits_f32(st));
           if (want_wq)
             C.wq[i] = (uint8_t)(enc2<FP8_E4M3>(__fmul_rn(__fmul_rn(st, inv_new_w), new_wq), 0.0f) & 0xffu);
         }
@@ -372,11 +377,13 @@ __global__ void k_adam_finalize(const __grid_constant__ AdamLaunch L) {
       }
     }
     if constexpr (STAGE == 3) {
-      // the exact new amax must give the scale that was used
-      int kw;
-      if (scale_exponent(ws[WS_CHECK_W], kMaxF16, L.margin, 0, kw) && pow2f(kw) != ws[WS_NEW_W])
-        atomicOr(&g_status, FP8_STATUS_INTERNAL);
-      if (C.w_amax != nullptr) *C.w_amax = __fmul_rn(ws[WS_STORED_W], 1.0f / ws[WS_NEW_W]);
+      if (C.w_amax != nullptr) {
+        // the exact new amax must give the scale that was used
+        int kw;
+        if (scale_exponent(ws[WS_CHECK_W], kMaxF16, L.margin, 0, kw) && pow2f(kw) != ws[WS_NEW_W])
+          atomicOr(&g_status, FP8_STATUS_INTERNAL);
+        *C.w_amax = __fmul_rn(ws[WS_STORED_W], 1.0f / ws[WS_NEW_W]);
+      }
     }
   }
 }

@@ -159,27 +159,119 @@ __device__ __forceinline__ void cast_group(const void *x, size_t g, float s, voi
   }
 }
 
+// Scale source of a cast: a precomputed scale, or the amax from which every
+// block derives it (fused scale + cast; block 0 also publishes scale and
+// 1/scale).  With `mu` set (the payload of the FP8 gradient all-reduce) the
+// scale is *mu * 2^(floor(log2(fmax / amax)) - margin), mu read from device
+// memory and applied after the exponent rule, so it does not cancel.
+struct CastScale {
+  const float *scale;  // used when amax == nullptr
+  const float *amax;
+  float fmax;
+  int margin, log2mu;
+  float *scale_out, *inv_out;
+  const float *mu;
+};
+
+__device__ __forceinline__ float cast_scale(const CastScale &cs) {
+  if (cs.amax == nullptr) return *cs.scale;
+  int k;
+  bool finite;
+  if (cs.mu != nullptr) {
+    int kg;
+    finite = scale_exponent(*cs.amax, cs.fmax, cs.margin, 0, kg);
+    k = clamp_exp(kg + device_log2mu(*cs.mu));
+  } else {
+    finite = scale_exponent(*cs.amax, cs.fmax, cs.margin, cs.log2mu, k);
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    *cs.scale_out = pow2f(k);
+    *cs.inv_out = pow2f(-k);
+    if (!finite) atomicOr(&g_status, FP8_STATUS_NONFINITE);
+  }
+  return pow2f(k);
+}
+
+// The same cast with the under/overflow counts of its 16 elements: an
+// element underflows when it is a non-zero number whose code is zero, and
+// overflows when |x * s| exceeds fmax (inf included, NaN in neither).
 template <int DT, int FMT>
+__device__ __forceinline__ void cast_group_count(const void *x, size_t g, float s, float fmax, void *q,
+                                                 uint32_t &under, uint32_t &over) {
+  float f[16];
+  load16<DT>(x, g, f);
+  uint32_t nz = 0;
+#pragma unroll
+  for (int j = 0; j < 16; j++) {
+    nz |= (f[j] != 0.0f && f[j] == f[j]) ? (1u << j) : 0u;
+    f[j] *= s;
+    over += fabsf(f[j]) > fmax ? 1u : 0u;
+  }
+  if constexpr (FMT == FP8_F16S) {
+    uint32_t h[8];
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+      h[j] = f16x2(f[2 * j], f[2 * j + 1]);
+      under += ((nz >> (2 * j)) & 1u) && (h[j] & 0x7fffu) == 0u;
+      under += ((nz >> (2 * j + 1)) & 1u) && (h[j] & 0x7fff0000u) == 0u;
+    }
+    uint4 *p = reinterpret_cast<uint4 *>(q) + g * 2;
+    __stcs(p, make_uint4(h[0], h[1], h[2], h[3]));
+    __stcs(p + 1, make_uint4(h[4], h[5], h[6], h[7]));
+  } else {
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      w[j] = enc4<FMT>(f[4 * j], f[4 * j + 1], f[4 * j + 2], f[4 * j + 3]);
+#pragma unroll
+      for (int b = 0; b < 4; b++) under += ((nz >> (4 * j + b)) & 1u) && ((w[j] >> (8 * b)) & 0x7fu) == 0u;
+    }
+    __stcs(reinterpret_cast<uint4 *>(q) + g, make_uint4(w[0], w[1], w[2], w[3]));
+  }
+}
+
+template <int DT, int FMT, bool COUNT>
 __global__ void __launch_bounds__(kStreamThreads) k_cast(const void *__restrict__ x, size_t n,
-                                                         const float *__restrict__ scale,
-                                                         void *__restrict__ q) {
-  const float s = *scale;
+                                                         const CastScale cs, void *__restrict__ q,
+                                                         unsigned long long *__restrict__ counts) {
+  const float s = cast_scale(cs);
   const size_t groups = n / 16;
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  for (; g + stride < groups; g += 2 * stride) {
-    cast_group<DT, FMT>(x, g, s, q);
-    cast_group<DT, FMT>(x, g + stride, s, q);
+  uint32_t under = 0, over = 0;
+  const float fmax = FMT == FP8_E4M3 ? 448.0f : (FMT == FP8_E5M2 ? 57344.0f : 65504.0f);
+  if constexpr (COUNT) {
+    for (; g < groups; g += stride) cast_group_count<DT, FMT>(x, g, s, fmax, q, under, over);
+  } else {
+    for (; g + stride < groups; g += 2 * stride) {
+      cast_group<DT, FMT>(x, g, s, q);
+      cast_group<DT, FMT>(x, g + stride, s, q);
+    }
+    if (g < groups) cast_group<DT, FMT>(x, g, s, q);
   }
-  if (g < groups) cast_group<DT, FMT>(x, g, s, q);
   if (blockIdx.x == 0) {
     for (size_t i = groups * 16 + threadIdx.x; i < n; i += blockDim.x) {
-      float y = load1<DT>(x, i) * s;
-      if constexpr (FMT == FP8_F16S)
-        reinterpret_cast<uint16_t *>(q)[i] = __half_as_ushort(__float2half_rn(y));
-      else
-        reinterpret_cast<uint8_t *>(q)[i] = (uint8_t)(enc2<FMT>(y, 0.0f) & 0xffu);
+      const float xi = load1<DT>(x, i);
+      const float y = xi * s;
+      uint32_t code;
+      if constexpr (FMT == FP8_F16S) {
+        code = __half_as_ushort(__float2half_rn(y));
+        reinterpret_cast<uint16_t *>(q)[i] = (uint16_t)code;
+        code &= 0x7fffu;
+      } else {
+        code = enc2<FMT>(y, 0.0f) & 0xffu;
+        reinterpret_cast<uint8_t *>(q)[i] = (uint8_t)code;
+        code &= 0x7fu;
+      }
+      if constexpr (COUNT) {
+        under += (xi != 0.0f && xi == xi && code == 0u) ? 1u : 0u;
+        over += fabsf(y) > fmax ? 1u : 0u;
+      }
     }
+  }
+  if constexpr (COUNT) {
+    __shared__ uint32_t red[64];
+    block_add_counts(under, over, red, counts);
   }
 }
 

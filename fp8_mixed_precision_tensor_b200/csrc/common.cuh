@@ -82,11 +82,11 @@ __device__ __forceinline__ bool scale_exponent(float amax, float fmax, int margi
 // Encoding.  Finite values: round to nearest even with saturation (the
 // hardware cvt with .satfinite).  Specials are fixed up explicitly so the
 // result does not depend on the cvt's special-value conventions:
-// +-inf -> +-max, NaN -> 0x7F with the input's sign bit.
+// +-inf -> +-max, NaN -> 0x7F (a NaN's sign is not kept).
 __device__ __forceinline__ uint32_t fix_special(uint32_t code, float y, int fmt) {
   uint32_t u = __float_as_uint(y);
   uint32_t sign = (u >> 24) & 0x80u;
-  if ((u & 0x7fffffffu) > 0x7f800000u) return sign | 0x7Fu;  // NaN
+  if ((u & 0x7fffffffu) > 0x7f800000u) return 0x7Fu;  // NaN
   if ((u & 0x7fffffffu) == 0x7f800000u) return sign | top_code(fmt);
   return code;
 }
@@ -154,6 +154,42 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t *red) {
   if (threadIdx.x == 0) red[0] = r;
   __syncthreads();
   return red[0];
+}
+
+// Block-wide sum of two per-thread counts added to dst[0], dst[1] (one
+// atomic each per block).  `red` holds >= 64 words.
+__device__ __forceinline__ void block_add_counts(uint32_t a, uint32_t b, uint32_t *red,
+                                                 unsigned long long *dst) {
+  a = __reduce_add_sync(0xffffffffu, a);
+  b = __reduce_add_sync(0xffffffffu, b);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) {
+    red[warp] = a;
+    red[32 + warp] = b;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long sa = 0, sb = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); w++) {
+      sa += red[w];
+      sb += red[32 + w];
+    }
+    if (sa) atomicAdd(dst, sa);
+    if (sb) atomicAdd(dst + 1, sb);
+  }
+}
+
+// log2 of a device-side mu that must be a power of two in [2^-32, 2^32];
+// anything else raises FP8_STATUS_BAD_MU and counts as mu = 1.
+__device__ __forceinline__ int device_log2mu(float mu) {
+  const uint32_t u = __float_as_uint(mu);
+  const int e = (int)(u >> 23) - 127;
+  if ((u & 0x807fffffu) != 0u || e < -32 || e > 32) {
+    atomicOr(&g_status, FP8_STATUS_BAD_MU);
+    return 0;
+  }
+  return e;
 }
 
 }  // namespace fp8lib

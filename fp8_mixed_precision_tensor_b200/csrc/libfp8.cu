@@ -10,7 +10,10 @@
 #include <mutex>
 
 #include "../../include/fp8.h"
+#include <type_traits>
+
 #include "adam.cuh"
+#include "allreduce.cuh"
 #include "amax_cast.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
@@ -241,16 +244,39 @@ void launch_amax(const void *x, size_t n, float *amax, cudaStream_t s, int sms) 
 }
 
 template <int DT, int FMT>
-void launch_cast(const void *x, size_t n, const float *scale, void *q, cudaStream_t s, int sms) {
+void launch_cast(const void *x, size_t n, const CastScale &cs, void *q, unsigned long long *counts,
+                 cudaStream_t s, int sms) {
   unsigned grid = grid_for(n / 16, kStreamThreads * 2, sms * 8);
-  k_cast<DT, FMT><<<grid, kStreamThreads, 0, s>>>(x, n, scale, q);
+  if (counts) k_cast<DT, FMT, true><<<grid, kStreamThreads, 0, s>>>(x, n, cs, q, counts);
+  else k_cast<DT, FMT, false><<<grid, kStreamThreads, 0, s>>>(x, n, cs, q, nullptr);
 }
 
 template <int DT>
-void launch_cast_dt(int fmt, const void *x, size_t n, const float *scale, void *q, cudaStream_t s, int sms) {
-  if (fmt == FP8_E4M3) launch_cast<DT, FP8_E4M3>(x, n, scale, q, s, sms);
-  else if (fmt == FP8_E5M2) launch_cast<DT, FP8_E5M2>(x, n, scale, q, s, sms);
-  else launch_cast<DT, FP8_F16S>(x, n, scale, q, s, sms);
+void launch_cast_dt(int fmt, const void *x, size_t n, const CastScale &cs, void *q, unsigned long long *counts,
+                    cudaStream_t s, int sms) {
+  if (fmt == FP8_E4M3) launch_cast<DT, FP8_E4M3>(x, n, cs, q, counts, s, sms);
+  else if (fmt == FP8_E5M2) launch_cast<DT, FP8_E5M2>(x, n, cs, q, counts, s, sms);
+  else launch_cast<DT, FP8_F16S>(x, n, cs, q, counts, s, sms);
+}
+
+int cast_common(const void *x, int dtype, size_t n, int fmt, const CastScale &cs, void *q, cudaStream_t s,
+                unsigned long long *counts = nullptr) {
+  DeviceInfo *d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  if (dtype == FP8_DT_F32) launch_cast_dt<FP8_DT_F32>(fmt, x, n, cs, q, counts, s, d->sms);
+  else if (dtype == FP8_DT_BF16) launch_cast_dt<FP8_DT_BF16>(fmt, x, n, cs, q, counts, s, d->sms);
+  else launch_cast_dt<FP8_DT_F16>(fmt, x, n, cs, q, counts, s, d->sms);
+  return launch_rc();
+}
+
+// mu must be a power of two in [2^-32, 2^32]; its log2 on success.
+bool mu_log2(float mu, int *log2mu) {
+  int e2;
+  float frac = frexpf(mu, &e2);
+  if (!(mu > 0.0f) || frac != 0.5f || e2 - 1 < -32 || e2 - 1 > 32) return false;
+  *log2mu = e2 - 1;
+  return true;
 }
 
 }  // namespace
@@ -274,12 +300,10 @@ int fp8_amax(const void *x, int dtype, size_t n, float *amax_dev, void *stream) 
 int fp8_compute_scale(const float *amax_dev, int fmt, int margin, float mu, float *scale_dev,
                       float *inv_scale_dev, void *stream) {
   if (!amax_dev || !scale_dev || !inv_scale_dev || !valid_fmt(fmt)) return FP8_ERR_INVALID_ARG;
-  if (margin < 0 || margin > 64) return FP8_ERR_INVALID_ARG;
-  int e2;
-  float frac = frexpf(mu, &e2);
-  if (!(mu > 0.0f) || frac != 0.5f || e2 - 1 < -32 || e2 - 1 > 32) return FP8_ERR_INVALID_ARG;
+  int log2mu;
+  if (margin < 0 || margin > 64 || !mu_log2(mu, &log2mu)) return FP8_ERR_INVALID_ARG;
   k_compute_scale<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(amax_dev, fmt_max_of(fmt), margin,
-                                                                 e2 - 1, scale_dev, inv_scale_dev);
+                                                                 log2mu, scale_dev, inv_scale_dev);
   return launch_rc();
 }
 
@@ -288,14 +312,76 @@ int fp8_cast(const void *x, int dtype, size_t n, int fmt, const float *scale_dev
   if (n == 0) return FP8_OK;
   if (!x || !q) return FP8_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(q)) return FP8_ERR_UNALIGNED;
+  CastScale cs = {scale_dev, nullptr, 0.0f, 0, 0, nullptr, nullptr, nullptr};
+  return cast_common(x, dtype, n, fmt, cs, q, static_cast<cudaStream_t>(stream));
+}
+
+int fp8_cast_count(const void *x, int dtype, size_t n, int fmt, const float *scale_dev, void *q,
+                   unsigned long long *counts_dev, void *stream) {
+  if (!valid_dtype(dtype) || !valid_fmt(fmt) || !scale_dev || !counts_dev) return FP8_ERR_INVALID_ARG;
+  if (n == 0) return FP8_OK;
+  if (!x || !q) return FP8_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(q)) return FP8_ERR_UNALIGNED;
+  CastScale cs = {scale_dev, nullptr, 0.0f, 0, 0, nullptr, nullptr, nullptr};
+  return cast_common(x, dtype, n, fmt, cs, q, static_cast<cudaStream_t>(stream), counts_dev);
+}
+
+int fp8_grad_cast(const void *g, int dtype, size_t n, int fmt, const float *amax_dev, int margin,
+                  const float *mu_dev, float *scale_dev, float *inv_scale_dev, uint8_t *q,
+                  unsigned long long *counts_dev, void *stream) {
+  if (!valid_dtype(dtype) || (fmt != FP8_E4M3 && fmt != FP8_E5M2)) return FP8_ERR_INVALID_ARG;
+  if (!amax_dev || !mu_dev || !scale_dev || !inv_scale_dev || margin < 0 || margin > 64)
+    return FP8_ERR_INVALID_ARG;
+  if (n > 0 && (!g || !q)) return FP8_ERR_INVALID_ARG;
+  if (n > 0 && (!aligned16(g) || !aligned16(q))) return FP8_ERR_UNALIGNED;
+  CastScale cs = {nullptr, amax_dev, fmt_max_of(fmt), margin, 0, scale_dev, inv_scale_dev, mu_dev};
+  return cast_common(g, dtype, n, fmt, cs, q, static_cast<cudaStream_t>(stream), counts_dev);
+}
+
+int fp8_sum_codes(const uint8_t *in, int nranks, size_t ld, size_t n, int fmt, uint8_t *out,
+                  const float *inv_scale_dev, float *g_inv_dev, unsigned long long *counts_dev,
+                  void *stream) {
+  if ((fmt != FP8_E4M3 && fmt != FP8_E5M2) || nranks < 1 || nranks > kSumMaxRanks || ld < n)
+    return FP8_ERR_INVALID_ARG;
+  if (g_inv_dev && !inv_scale_dev) return FP8_ERR_INVALID_ARG;
+  if (n > 0 && (!in || !out)) return FP8_ERR_INVALID_ARG;
+  if (n > 0 && (!aligned16(in) || !aligned16(out) || ld % 16)) return FP8_ERR_UNALIGNED;
+  if (n == 0 && !g_inv_dev) return FP8_OK;
   DeviceInfo *d;
   int rc = device_info(&d);
   if (rc) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (dtype == FP8_DT_F32) launch_cast_dt<FP8_DT_F32>(fmt, x, n, scale_dev, q, s, d->sms);
-  else if (dtype == FP8_DT_BF16) launch_cast_dt<FP8_DT_BF16>(fmt, x, n, scale_dev, q, s, d->sms);
-  else launch_cast_dt<FP8_DT_F16>(fmt, x, n, scale_dev, q, s, d->sms);
+  const unsigned grid = grid_for(n / 16, kSumThreads, d->sms * 8);
+  if (fmt == FP8_E5M2)
+    k_sum_codes<FP8_E5M2><<<grid, kSumThreads, 0, s>>>(in, nranks, ld, n, out, inv_scale_dev, g_inv_dev, counts_dev);
+  else
+    k_sum_codes<FP8_E4M3><<<grid, kSumThreads, 0, s>>>(in, nranks, ld, n, out, inv_scale_dev, g_inv_dev, counts_dev);
   return launch_rc();
+}
+
+int fp8_mu_update(float *mu_dev, int *clean_dev, unsigned long long *counts_dev, unsigned long long n,
+                  const fp8_mu_rule *rule, void *stream) {
+  if (!mu_dev || !clean_dev || !counts_dev || !rule) return FP8_ERR_INVALID_ARG;
+  int lo, hi;
+  if (!(rule->theta >= 0.0f) || rule->interval < 1 || !mu_log2(rule->mu_min, &lo) ||
+      !mu_log2(rule->mu_max, &hi) || lo > hi)
+    return FP8_ERR_INVALID_ARG;
+  k_mu_update<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(mu_dev, clean_dev, counts_dev, n,
+                                                               (double)rule->theta, rule->interval,
+                                                               rule->mu_min, rule->mu_max);
+  return launch_rc();
+}
+
+int fp8_scale_cast(const void *x, int dtype, size_t n, int fmt, const float *amax_dev, int margin, float mu,
+                   float *scale_dev, float *inv_scale_dev, void *q, void *stream) {
+  int log2mu;
+  if (!valid_dtype(dtype) || !valid_fmt(fmt) || !amax_dev || !scale_dev || !inv_scale_dev)
+    return FP8_ERR_INVALID_ARG;
+  if (margin < 0 || margin > 64 || !mu_log2(mu, &log2mu)) return FP8_ERR_INVALID_ARG;
+  if (n > 0 && (!x || !q)) return FP8_ERR_INVALID_ARG;
+  if (n > 0 && (!aligned16(x) || !aligned16(q))) return FP8_ERR_UNALIGNED;
+  CastScale cs = {nullptr, amax_dev, fmt_max_of(fmt), margin, log2mu, scale_dev, inv_scale_dev, nullptr};
+  return cast_common(x, dtype, n, fmt, cs, q, static_cast<cudaStream_t>(stream));
 }
 
 int fp8_linear_fwd(const uint8_t *xq, const float *x_inv, const uint8_t *wq, const float *w_inv,
@@ -326,8 +412,16 @@ size_t fp8_adam_workspace_bytes(int nchunks) {
   return (size_t)nchunks * kAdamWsFloatsPerChunk * sizeof(float);
 }
 
-int fp8_adam_step(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp,
-                  void *workspace, size_t ws_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// The Adam step in phases: PH_STATS runs the stats pass into the workspace,
+// PH_APPLY finalizes the scales from it and runs the update, PH_ALL both.
+enum { PH_STATS = 1, PH_APPLY = 2, PH_ALL = 3 };
+
+int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp, void *workspace,
+             size_t ws_bytes, void *stream, int phases) {
   if (!chunks || !hp || nchunks <= 0 || !workspace) return FP8_ERR_INVALID_ARG;
   if (ws_bytes < fp8_adam_workspace_bytes(nchunks)) return FP8_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FP8_ERR_UNALIGNED;
@@ -339,6 +433,7 @@ int fp8_adam_step(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hpar
     const fp8_adam_chunk &c = chunks[i];
     if (!c.g_inv || !c.m_scale || !c.v_scale || !c.w_scale) return FP8_ERR_INVALID_ARG;
     if (c.wq && (!c.wq_scale || !c.wq_inv)) return FP8_ERR_INVALID_ARG;
+    if (phases != PH_ALL && c.w_amax) return FP8_ERR_INVALID_ARG;  // tracking needs the whole step
     if (c.n > 0 && (!c.g || !c.m || !c.v || !c.w)) return FP8_ERR_INVALID_ARG;
     if (c.n > 0 && (!aligned16(c.g) || !aligned16(c.m) || !aligned16(c.v) || !aligned16(c.w) ||
                     (c.wq && !aligned16(c.wq))))
@@ -348,9 +443,11 @@ int fp8_adam_step(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hpar
   int rc = device_info(&d);
   if (rc) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if ((rc = cuda_rc(cudaMemsetAsync(workspace, 0, fp8_adam_workspace_bytes(nchunks), s)))) return rc;
+  if ((phases & PH_STATS) &&
+      (rc = cuda_rc(cudaMemsetAsync(workspace, 0, fp8_adam_workspace_bytes(nchunks), s))))
+    return rc;
 
-  static thread_local AdamLaunch L;  // ~20 KB: kept off the stack
+  static thread_local AdamLaunch L;  // ~29 KB: kept off the stack
   L.margin = hp->margin;
   L.beta1 = hp->beta1;
   L.beta2 = hp->beta2;
@@ -377,19 +474,40 @@ int fp8_adam_step(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hpar
     const unsigned grid = tiles == 0 ? 1u : (unsigned)(tiles < cap ? tiles : cap);
     bool tracked = false;
     for (int i = 0; i < cnt; i++) tracked |= L.c[i].w_amax != nullptr;
-    k_adam<1><<<grid, kAdamThreads, 0, s>>>(L);        // stats
-    if (tracked) {
-      k_adam_finalize<1><<<1, 256, 0, s>>>(L);
-      k_adam<3><<<grid, kAdamThreads, 0, s>>>(L);      // exact master amax, flagged chunks only
-      k_adam_finalize<2><<<1, 256, 0, s>>>(L);
-    } else {
-      k_adam_finalize<12><<<1, 256, 0, s>>>(L);
+    if (phases & PH_STATS) k_adam<1><<<grid, kAdamThreads, 0, s>>>(L);  // stats
+    if (phases & PH_APPLY) {
+      if (tracked) {
+        k_adam_finalize<1><<<1, 256, 0, s>>>(L);
+        k_adam<3><<<grid, kAdamThreads, 0, s>>>(L);  // exact master amax, flagged chunks only
+        k_adam_finalize<2><<<1, 256, 0, s>>>(L);
+      } else {
+        k_adam_finalize<12><<<1, 256, 0, s>>>(L);
+      }
+      k_adam<2><<<grid, kAdamThreads, 0, s>>>(L);    // update
+      if (tracked) k_adam_finalize<3><<<1, 256, 0, s>>>(L);
     }
-    k_adam<2><<<grid, kAdamThreads, 0, s>>>(L);        // update
-    if (tracked) k_adam_finalize<3><<<1, 256, 0, s>>>(L);
     if ((rc = launch_rc())) return rc;
   }
   return FP8_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp8_adam_step(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp,
+                  void *workspace, size_t ws_bytes, void *stream) {
+  return adam_run(chunks, nchunks, hp, workspace, ws_bytes, stream, PH_ALL);
+}
+
+int fp8_adam_stats(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp,
+                   void *workspace, size_t ws_bytes, void *stream) {
+  return adam_run(chunks, nchunks, hp, workspace, ws_bytes, stream, PH_STATS);
+}
+
+int fp8_adam_apply(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp,
+                   void *workspace, size_t ws_bytes, void *stream) {
+  return adam_run(chunks, nchunks, hp, workspace, ws_bytes, stream, PH_APPLY);
 }
 
 // Scratch of fp8_adam_step_noalloc: one 64-byte slot per chunk, in a fixed

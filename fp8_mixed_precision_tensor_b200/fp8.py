@@ -21,14 +21,16 @@ LIB_PATH = os.path.join(_HERE, "libfp8.so")
 # status codes / enums (include/fp8.h)
 FP8_OK, FP8_ERR_INVALID_ARG, FP8_ERR_UNALIGNED, FP8_ERR_UNSUPPORTED = 0, 1, 2, 3
 FP8_ERR_CUDA, FP8_ERR_TIMEOUT, FP8_ERR_NONFINITE = 4, 5, 6
-FP8_STATUS_NONFINITE, FP8_STATUS_TIMEOUT, FP8_STATUS_INTERNAL = 1, 2, 4
+FP8_STATUS_NONFINITE, FP8_STATUS_TIMEOUT, FP8_STATUS_INTERNAL, FP8_STATUS_BAD_MU = 1, 2, 4, 8
 FP8_DT_F32, FP8_DT_BF16, FP8_DT_F16 = 0, 1, 2
 FP8_E4M3, FP8_E5M2, FP8_F16S = 0, 1, 2
 
 _DT = {torch.float32: FP8_DT_F32, torch.bfloat16: FP8_DT_BF16, torch.float16: FP8_DT_F16}
 
-SYMBOLS = ("fp8_amax", "fp8_compute_scale", "fp8_cast", "fp8_linear_fwd", "fp8_linear_dgrad",
-           "fp8_linear_wgrad", "fp8_adam_workspace_bytes", "fp8_adam_step", "fp8_adam_step_noalloc",
+SYMBOLS = ("fp8_amax", "fp8_compute_scale", "fp8_cast", "fp8_scale_cast", "fp8_cast_count", "fp8_grad_cast",
+           "fp8_sum_codes", "fp8_mu_update", "fp8_linear_fwd", "fp8_linear_dgrad",
+           "fp8_linear_wgrad", "fp8_adam_workspace_bytes", "fp8_adam_step", "fp8_adam_stats",
+           "fp8_adam_apply", "fp8_adam_step_noalloc",
            "fp8_get_status", "fp8_strerror")
 
 
@@ -44,6 +46,11 @@ class _Chunk(ctypes.Structure):
                 ("w", ctypes.c_void_p), ("w_scale", ctypes.c_void_p), ("n", ctypes.c_size_t),
                 ("w_amax", ctypes.c_void_p), ("wq", ctypes.c_void_p), ("wq_scale", ctypes.c_void_p),
                 ("wq_inv", ctypes.c_void_p)]
+
+
+class _MuRule(ctypes.Structure):
+    _fields_ = [("theta", ctypes.c_float), ("interval", ctypes.c_int), ("mu_min", ctypes.c_float),
+                ("mu_max", ctypes.c_float)]
 
 
 class _HParams(ctypes.Structure):
@@ -66,11 +73,17 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fp8_amax.argtypes = [p, i, sz, p, p]
     lib.fp8_compute_scale.argtypes = [p, i, i, f, p, p, p]
     lib.fp8_cast.argtypes = [p, i, sz, i, p, p, p]
+    lib.fp8_scale_cast.argtypes = [p, i, sz, i, p, i, f, p, p, p, p]
+    lib.fp8_cast_count.argtypes = [p, i, sz, i, p, p, p, p]
+    lib.fp8_grad_cast.argtypes = [p, i, sz, i, p, i, p, p, p, p, p, p]
+    lib.fp8_sum_codes.argtypes = [p, i, sz, sz, i, p, p, p, p, p]
+    lib.fp8_mu_update.argtypes = [p, p, p, ctypes.c_ulonglong, ctypes.POINTER(_MuRule), p]
     lib.fp8_linear_fwd.argtypes = [p, p, p, p, p, i, p, i, p, i, i, i, p]
     lib.fp8_linear_dgrad.argtypes = [p, p, p, p, p, i, p, i, i, i, p]
     lib.fp8_linear_wgrad.argtypes = [p, p, p, p, p, i, p, i, i, i, p]
     lib.fp8_adam_workspace_bytes.argtypes, lib.fp8_adam_workspace_bytes.restype = [i], sz
-    lib.fp8_adam_step.argtypes = [ctypes.POINTER(_Chunk), i, ctypes.POINTER(_HParams), p, sz, p]
+    for name in ("fp8_adam_step", "fp8_adam_stats", "fp8_adam_apply"):
+        getattr(lib, name).argtypes = [ctypes.POINTER(_Chunk), i, ctypes.POINTER(_HParams), p, sz, p]
     lib.fp8_adam_step_noalloc.argtypes = [ctypes.POINTER(_Chunk), i, ctypes.POINTER(_HParams), p]
     lib.fp8_get_status.argtypes = [ctypes.POINTER(ctypes.c_uint), p]
     lib.fp8_strerror.argtypes, lib.fp8_strerror.restype = [i], ctypes.c_char_p
@@ -121,6 +134,49 @@ def fp8_cast(x: torch.Tensor, fmt: int, scale: torch.Tensor, q_out: torch.Tensor
     """q_out = enc_fmt(x * scale): uint8 codes, or 16-bit halves for FP8_F16S."""
     _check(load_library().fp8_cast(_ptr(x), _DT[x.dtype], x.numel(), fmt, _ptr(scale), _ptr(q_out),
                                    _stream(stream)), "fp8_cast")
+
+
+def fp8_scale_cast(x: torch.Tensor, fmt: int, amax: torch.Tensor, margin: int, mu: float,
+                   scale_out: torch.Tensor, inv_scale_out: torch.Tensor, q_out: torch.Tensor,
+                   stream=None) -> None:
+    """fp8_compute_scale + fp8_cast in one launch."""
+    _check(load_library().fp8_scale_cast(_ptr(x), _DT[x.dtype], x.numel(), fmt, _ptr(amax), margin, mu,
+                                         _ptr(scale_out), _ptr(inv_scale_out), _ptr(q_out),
+                                         _stream(stream)), "fp8_scale_cast")
+
+
+# ---------------------------------------------------------------- scaling variants, FP8 all-reduce
+def fp8_cast_count(x: torch.Tensor, fmt: int, scale: torch.Tensor, q_out: torch.Tensor, counts: torch.Tensor,
+                   stream=None) -> None:
+    """fp8_cast, adding (underflows, overflows) to counts (2 x int64, device)."""
+    _check(load_library().fp8_cast_count(_ptr(x), _DT[x.dtype], x.numel(), fmt, _ptr(scale), _ptr(q_out),
+                                         _ptr(counts), _stream(stream)), "fp8_cast_count")
+
+
+def fp8_grad_cast(g: torch.Tensor, fmt: int, amax: torch.Tensor, margin: int, mu: torch.Tensor,
+                  scale_out: torch.Tensor, inv_scale_out: torch.Tensor, q_out: torch.Tensor,
+                  counts: torch.Tensor | None = None, stream=None) -> None:
+    """Payload cast of the FP8 gradient all-reduce: S = mu * 2^(floor(log2(fmax/amax)) - margin)."""
+    _check(load_library().fp8_grad_cast(_ptr(g), _DT[g.dtype], g.numel(), fmt, _ptr(amax), margin, _ptr(mu),
+                                        _ptr(scale_out), _ptr(inv_scale_out), _ptr(q_out), _ptr(counts),
+                                        _stream(stream)), "fp8_grad_cast")
+
+
+def fp8_sum_codes(rows: torch.Tensor, n: int, fmt: int, out: torch.Tensor, inv_scale: torch.Tensor | None = None,
+                  g_inv_out: torch.Tensor | None = None, counts: torch.Tensor | None = None,
+                  stream=None) -> None:
+    """out[:n] = enc(sum over the rows of rows[:, :n]), rows = [nranks, ld] uint8."""
+    nranks, ld = rows.shape
+    _check(load_library().fp8_sum_codes(_ptr(rows), nranks, ld, n, fmt, _ptr(out), _ptr(inv_scale),
+                                        _ptr(g_inv_out), _ptr(counts), _stream(stream)), "fp8_sum_codes")
+
+
+def fp8_mu_update(mu: torch.Tensor, clean: torch.Tensor, counts: torch.Tensor, n: int, theta: float,
+                  interval: int, mu_min: float, mu_max: float, stream=None) -> None:
+    """The auto-scaling rule for mu (device state; clears counts)."""
+    rule = _MuRule(theta, interval, mu_min, mu_max)
+    _check(load_library().fp8_mu_update(_ptr(mu), _ptr(clean), _ptr(counts), n, ctypes.byref(rule),
+                                        _stream(stream)), "fp8_mu_update")
 
 
 # ---------------------------------------------------------------- GEMMs
@@ -195,6 +251,27 @@ def fp8_adam_step(chunks, lr: float, beta1: float, beta2: float, eps: float, ste
     _check(load_library().fp8_adam_step(arr, len(arr), ctypes.byref(hp), _ptr(workspace),
                                         workspace.numel() * workspace.element_size(), _stream(stream)),
            "fp8_adam_step")
+
+
+def _adam_half(name, chunks, lr, beta1, beta2, eps, step, margin, workspace, stream):
+    arr = chunks if isinstance(chunks, ctypes.Array) else pack_adam_chunks(chunks)
+    hp = _HParams(lr, beta1, beta2, eps, step, margin)
+    _check(getattr(load_library(), name)(arr, len(arr), ctypes.byref(hp), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream(stream)), name)
+
+
+def fp8_adam_stats(chunks, lr: float, beta1: float, beta2: float, eps: float, step: int, margin: int,
+                   workspace: torch.Tensor, stream=None) -> None:
+    """First half of an element-sharded step: amax of this rank's new m, v, w
+    per chunk into `workspace` (state unchanged)."""
+    _adam_half("fp8_adam_stats", chunks, lr, beta1, beta2, eps, step, margin, workspace, stream)
+
+
+def fp8_adam_apply(chunks, lr: float, beta1: float, beta2: float, eps: float, step: int, margin: int,
+                   workspace: torch.Tensor, stream=None) -> None:
+    """Second half: new scales from the (rank-reduced) workspace, then the
+    in-place update of this rank's slices."""
+    _adam_half("fp8_adam_apply", chunks, lr, beta1, beta2, eps, step, margin, workspace, stream)
 
 
 FP8_ADAM_NOALLOC_MAX_CHUNKS = 1024

@@ -6,8 +6,8 @@
 
 Each case runs `--iters` passes after one warm-up pass on seeded synthetic
 inputs and prints the CUDA-event time per pass.  Launch order per pass:
-linear: amax/scale/cast of X, W, dY (9 launches), then fwd, dgrad, wgrad;
-cast: amax, scale, cast; adam: stats pass, finalize, update pass.
+linear: amax and fused scale+cast of X, W, dY (6 launches), then fwd, dgrad,
+wgrad; cast: amax, fused scale+cast; adam: stats pass, finalize, update pass.
 """
 from __future__ import annotations
 
@@ -37,8 +37,7 @@ def case_linear(a):
     def one():
         for t, q, i, fmt in ((X, xq, 0, fp8.FP8_E4M3), (W, wq, 3, fp8.FP8_E4M3), (dY, dyq, 6, fp8.FP8_E5M2)):
             fp8.fp8_amax(t, sc[i:i + 1])
-            fp8.fp8_compute_scale(sc[i:i + 1], fmt, 0, 1.0, sc[i + 1:i + 2], sc[i + 2:i + 3])
-            fp8.fp8_cast(t, fmt, sc[i + 1:i + 2], q)
+            fp8.fp8_scale_cast(t, fmt, sc[i:i + 1], 0, 1.0, sc[i + 1:i + 2], sc[i + 2:i + 3], q)
         fp8.fp8_linear_fwd(xq, sc[2:3], wq, sc[5:6], y, sc[12:13])
         fp8.fp8_linear_dgrad(dyq, sc[8:9], wq, sc[5:6], dx, sc[13:14])
         fp8.fp8_linear_wgrad(dyq, sc[8:9], xq, sc[2:3], dw, sc[14:15])
@@ -53,8 +52,7 @@ def case_cast(a):
 
     def one():
         fp8.fp8_amax(x, sc[0:1])
-        fp8.fp8_compute_scale(sc[0:1], fp8.FP8_E4M3, 0, 1.0, sc[1:2], sc[2:3])
-        fp8.fp8_cast(x, fp8.FP8_E4M3, sc[1:2], q)
+        fp8.fp8_scale_cast(x, fp8.FP8_E4M3, sc[0:1], 0, 1.0, sc[1:2], sc[2:3], q)
 
     return one
 

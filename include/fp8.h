@@ -53,6 +53,7 @@ extern "C" {
 #define FP8_STATUS_NONFINITE 1u
 #define FP8_STATUS_TIMEOUT 2u
 #define FP8_STATUS_INTERNAL 4u /* a kernel's own consistency check failed */
+#define FP8_STATUS_BAD_MU 8u   /* a device mu was not a power of two in [2^-32, 2^32]; 1 was used */
 
 /* ---- element types of high-precision tensors -------------------------- */
 #define FP8_DT_F32 0
@@ -100,15 +101,114 @@ int fp8_compute_scale(const float *amax_dev, int fmt, int margin, float mu, floa
 /*
  * fp8_cast -- q_i = enc_fmt(x_i * scale) ([FP8-AMAX] 제안 방법: scale, then
  * cast).  FP8 formats: round to nearest even, saturating at +-max; +-inf
- * saturates too; NaN becomes 0x7F with the input's sign bit.  FP8_F16S:
- * IEEE round to nearest even.  With a scale from fp8_compute_scale on the
- * tensor's own amax nothing saturates.
+ * saturates too; NaN becomes 0x7F (its sign is not kept).  FP8_F16S:
+ * IEEE round to nearest even; NaN becomes 0x7FFF.  With a scale from
+ * fp8_compute_scale on the tensor's own amax nothing saturates.
  *   x          dev, n elements of `dtype`, 16-byte aligned
  *   scale_dev  dev, one float (power of two times mu)
  *   q          dev, n bytes (E4M3/E5M2) or n uint16 (F16S), 16-byte aligned
  */
 int fp8_cast(const void *x, int dtype, size_t n, int fmt, const float *scale_dev, void *q,
              void *stream);
+
+/*
+ * fp8_scale_cast -- fp8_compute_scale followed by fp8_cast in one launch
+ * (same definitions, same results): every block derives the scale from
+ * *amax_dev itself and the first block also writes scale_dev and
+ * inv_scale_dev.  Arguments as in those two calls; n == 0 only writes the
+ * scales.
+ */
+int fp8_scale_cast(const void *x, int dtype, size_t n, int fmt, const float *amax_dev, int margin,
+                   float mu, float *scale_dev, float *inv_scale_dev, void *q, void *stream);
+
+/*
+ * fp8_cast_count -- fp8_cast plus its underflow and overflow counts, the
+ * measure by which [FP8-LM] アブレーション研究 compares scaling variants
+ * (and [FP8-AMAX] 실험 결과, RQ3, dynamic against constant scaling): an
+ * element underflows when it is a non-zero number whose code is zero, and
+ * overflows when |x * scale| exceeds fmt_max (the cast saturates it; inf
+ * counts, NaN counts as neither).  A constant scaling bias (FP8-CSCALE of
+ * [FP8-AMAX]) is this cast with a scale of 2^bias that the caller keeps.
+ *   counts_dev  dev, two uint64: [0] += underflows, [1] += overflows
+ *               (accumulated; the caller zeroes them)
+ * Other arguments as fp8_cast.
+ */
+int fp8_cast_count(const void *x, int dtype, size_t n, int fmt, const float *scale_dev, void *q,
+                   unsigned long long *counts_dev, void *stream);
+
+/*
+ * FP8 gradient all-reduce ([FP8-LM] 提案手法 O1: gradients communicated in
+ * FP8 with auto-scaling g' = mu * g, Eq. 3).  Every rank casts its gradient
+ * with ONE shared scale taken from the amax over all ranks, so that the
+ * ranks' codes can be summed as they are; mu sets the headroom the sum
+ * needs.  A rank's part of one all-reduce:
+ *   amax of its gradient (fp8_amax, or a GEMM's output amax)
+ *   <caller> MAX all-reduce of the amax over the ranks
+ *   fp8_grad_cast   payload codes with S = mu * 2^(floor(log2(fmt_max/amax)) - margin)
+ *   <caller> exchange: rank j receives every rank's codes of its slice j
+ *   fp8_sum_codes   exact sum of those codes, re-encoded at S (rank j's
+ *                   slice of the summed gradient) and g_inv = 1 / (S * nranks)
+ *   <caller> SUM all-reduce of the counts, then fp8_mu_update.
+ * With mu = 1 (post-scaling: divide by the rank count after the sum) the
+ * sum can saturate; with mu = 1/nranks (pre-scaling: divide before the
+ * cast) small gradients underflow; fp8_mu_update moves mu between those.
+ */
+
+/*
+ * fp8_grad_cast -- the payload cast: S = mu * 2^(clamp(floor(log2(fmt_max /
+ * amax)) - margin)), clamped to [2^-126, 2^126]; q_i = enc_fmt(g_i * S).
+ * Unlike fp8_compute_scale, mu multiplies the scale after the exponent rule
+ * (it does not cancel).  amax == 0 gives the exponent 0; a NaN or inf amax
+ * too, and sets FP8_STATUS_NONFINITE.
+ *   g              dev, n elements of `dtype`, 16-byte aligned
+ *   fmt            FP8_E5M2 (gradients) or FP8_E4M3
+ *   amax_dev       dev float: the amax over all ranks
+ *   mu_dev         dev float: a power of two in [2^-32, 2^32] (else 1 is used
+ *                  and FP8_STATUS_BAD_MU is set)
+ *   scale_dev, inv_scale_dev  dev floats, overwritten with S and 1/S
+ *   q              dev, n bytes, 16-byte aligned
+ *   counts_dev     dev two uint64 (as fp8_cast_count) or NULL
+ * n == 0 only writes the scales.
+ */
+int fp8_grad_cast(const void *g, int dtype, size_t n, int fmt, const float *amax_dev, int margin,
+                  const float *mu_dev, float *scale_dev, float *inv_scale_dev, uint8_t *q,
+                  unsigned long long *counts_dev, void *stream);
+
+/*
+ * fp8_sum_codes -- out_i = enc_fmt(sum_r dec(in[r * ld + i])) for i < n: the
+ * ranks' payload codes (all cast at one scale) summed exactly and rounded
+ * once (nearest even, saturating at +-fmt_max).  A zero sum is code 0x00; a
+ * NaN code, or +inf with -inf, gives 0x7F; an inf saturates.
+ *   in             dev, nranks rows of ld bytes (ld >= n, a multiple of 16),
+ *                  16-byte aligned; 1 <= nranks <= 4096
+ *   out            dev, n bytes, 16-byte aligned
+ *   inv_scale_dev  dev float 1/S (read when g_inv_dev is not NULL)
+ *   g_inv_dev      dev float or NULL: receives inv_scale * (1 / nranks) (both
+ *                  rounded to binary32), the descale of the mean gradient
+ *   counts_dev     dev two uint64 (as fp8_cast_count, on the sums) or NULL
+ */
+int fp8_sum_codes(const uint8_t *in, int nranks, size_t ld, size_t n, int fmt, uint8_t *out,
+                  const float *inv_scale_dev, float *g_inv_dev, unsigned long long *counts_dev,
+                  void *stream);
+
+/*
+ * fp8_mu_update -- the auto-scaling rule for mu between steps ([FP8-LM] O1
+ * says mu changes dynamically but gives no rule; this one is the library's
+ * own, after dynamic loss scaling): if counts_dev[1] (overflows of the
+ * summed gradient, over all ranks) > theta * n, mu halves (not below mu_min)
+ * and *clean_dev restarts at 0; otherwise *clean_dev grows by one and at
+ * `interval` mu doubles (not above mu_max) and *clean_dev restarts.  Then
+ * counts_dev[0..1] are set to 0.  All state stays on the device.
+ *   rule   host: theta >= 0, interval >= 1, mu_min <= mu_max powers of two
+ *          in [2^-32, 2^32]
+ */
+typedef struct {
+  float theta;
+  int interval;
+  float mu_min, mu_max;
+} fp8_mu_rule;
+int fp8_mu_update(float *mu_dev, int *clean_dev, unsigned long long *counts_dev, unsigned long long n,
+                  const fp8_mu_rule *rule, void *stream);
 
 /*
  * FP8 linear layer GEMMs ([FP8-AMAX] 제안 방법: matmul on FP8 operands, the
@@ -206,6 +306,33 @@ size_t fp8_adam_workspace_bytes(int nchunks);
  */
 int fp8_adam_step(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp,
                   void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Element-sharded step ([FP8-LM] 提案手法 O3: FP8 optimizer state under a
+ * ZeRO-style partition).  fp8_adam_step in two halves so that ranks which
+ * each hold a contiguous slice of every tensor agree on its per-tensor
+ * scales:
+ *   fp8_adam_stats  clears the workspace and writes the amax of the new
+ *                   m, v, w of this rank's slices (nothing else changes);
+ *   <caller>        element-wise MAX of the workspace over the ranks, taken
+ *                   on its 32-bit words read as int32 (every word is the bit
+ *                   pattern of a float >= 0 or of +NaN, so integer order is
+ *                   the amax order and a NaN wins);
+ *   fp8_adam_apply  derives the new scales from the reduced workspace and
+ *                   updates this rank's slices in place.
+ * Chunk i must be a slice of the same tensor on every rank, with the same
+ * m_scale, v_scale, w_scale values; every rank then writes the same new
+ * scales, and the slices end up exactly as one fp8_adam_step over the whole
+ * tensor would leave them.  Both calls take the same chunks, hparams and
+ * workspace (contents kept between them); tracked master amax is not
+ * available here (w_amax must be NULL, else FP8_ERR_INVALID_ARG).  A slice
+ * may be empty (n = 0).  Without the reduction in between (one rank), the
+ * pair equals fp8_adam_step.
+ */
+int fp8_adam_stats(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp,
+                   void *workspace, size_t ws_bytes, void *stream);
+int fp8_adam_apply(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp,
+                   void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * fp8_adam_step_noalloc -- the same step as fp8_adam_step, for callers that

@@ -152,13 +152,14 @@ static unsigned nearest_code(int fmt, double a)
 /*
  * Encode a real number as E4M3 / E5M2: round to nearest, ties to even,
  * saturating at +-max ("scale before the cast", [FP8-AMAX] 제안 방법).
- * reading: +-inf saturates to +-max as well; NaN becomes 0x7F with the
- * input's sign bit (parity unpinned).
+ * readings: +-inf saturates to +-max as well; NaN becomes the positive NaN
+ * code 0x7F whatever its sign bit (a NaN's sign carries no meaning, and the
+ * scaling multiply before the cast does not keep it) -- parity unpinned.
  */
 unsigned orc_fp8_encode(int fmt, double y)
 {
     if (isnan(y))
-        return signbit(y) ? 0xFFu : 0x7Fu;
+        return 0x7Fu;
     unsigned sign = signbit(y) ? 0x80u : 0u;
     double a = fabs(y);
     unsigned top = top_code(fmt);
@@ -167,11 +168,12 @@ unsigned orc_fp8_encode(int fmt, double y)
     return sign | nearest_code(fmt, a);
 }
 
-/* IEEE binary16 round-to-nearest-even; overflow past 65520 gives inf. */
+/* IEEE binary16 round-to-nearest-even; overflow past 65520 gives inf.
+ * reading: NaN becomes the positive all-ones NaN 0x7FFF (see orc_fp8_encode). */
 unsigned orc_f16_encode(double y)
 {
     if (isnan(y))
-        return signbit(y) ? 0xFE00u : 0x7E00u;
+        return 0x7FFFu;
     unsigned sign = signbit(y) ? 0x8000u : 0u;
     double a = fabs(y);
     if (a >= 65520.0)

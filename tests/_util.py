@@ -76,3 +76,17 @@ def boundary_samples(rows: int, cols: int, n_random: int, key, tile_r=(128, 256)
             r.append(er)
             c.append(ec)
     return np.asarray(r, dtype=np.int64), np.asarray(c, dtype=np.int64)
+
+
+def assert_codes_equal(got: np.ndarray, ref: np.ndarray, inputs=None, what=""):
+    """Bit-exact comparison of code arrays; on failure the first mismatches
+    with their inputs (bit patterns) are in the message."""
+    got, ref = np.asarray(got).reshape(-1), np.asarray(ref).reshape(-1)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    bad = np.nonzero(got != ref)[0]
+    if bad.size:
+        rows = []
+        for i in bad[:8]:
+            x = "" if inputs is None else f" input {np.asarray(inputs).reshape(-1)[i]!r}"
+            rows.append(f"[{i}] gpu {int(got[i]):#x} oracle {int(ref[i]):#x}{x}")
+        raise AssertionError(f"{what}: {bad.size} of {got.size} codes differ; " + "; ".join(rows))
