@@ -18,7 +18,14 @@ Inputs are seeded synthetic tensors (bf16 activations ~N(0,1), weights
 ~N(0,0.02), output gradients ~N(0,1e-4)); every step touches several GB, far
 more than the 126 MB L2, so no explicit L2 flush is needed between steps.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+The step's launches run on three streams by default (--schedule overlap):
+the casts of all four linears run ahead beside the GEMMs, wgrad and the
+gradient cast run beside fwd/dgrad, Adam joins them.  --schedule serial runs
+the same launches in order on one stream.  The per-kernel breakdown
+(`kernels`, `roofline`) always comes from a serial pass with CUDA events
+around each phase.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--schedule serial]
 """
 from __future__ import annotations
 
@@ -217,15 +224,59 @@ class Block7BStep:
         fp8.fp8_adam_step(self.chunks, step=self.t, margin=0, workspace=self.ws, **HP)
         if e: e[1].record()
 
+    def step_overlapped(self):
+        """The same launches as step(), on three streams: the casts of every
+        linear run ahead on a cast stream (HBM-bound work beside the
+        tensor-bound GEMMs, whose CTAs leave room for one cast block per SM),
+        forward and dgrad run on the current stream, wgrad and the gradient
+        cast on an auxiliary stream (one GEMM's last wave overlaps the next
+        GEMM); Adam joins them on the current stream.  Every buffer of a
+        step is written once, and the next step's casts start only after this
+        step's Adam (the cast stream waits for an event recorded at the start
+        of the next step on the current stream)."""
+        fp8 = self.fp8
+        main = torch.cuda.current_stream()
+        if not hasattr(self, "s_cast"):
+            self.s_cast, self.s_aux = torch.cuda.Stream(self.dev), torch.cuda.Stream(self.dev)
+            self.ev_start = torch.cuda.Event()
+            self.ev_cast = [torch.cuda.Event() for _ in self.L]
+            self.ev_grad = torch.cuda.Event()
+        self.ev_start.record(main)
+        self.s_cast.wait_event(self.ev_start)
+        self.s_aux.wait_event(self.ev_start)
+        with torch.cuda.stream(self.s_cast):
+            for d, e in zip(self.L, self.ev_cast):
+                sc = d["sc"]
+                self.quantise(d["X"], fp8.FP8_E4M3, sc, 0, out=d["xq"])
+                self.quantise(d["W"], fp8.FP8_E4M3, sc, 3, out=d["wq"])
+                self.quantise(d["dY"], fp8.FP8_E5M2, sc, 6, mu=MU, out=d["dyq"])
+                e.record(self.s_cast)
+        for d, e in zip(self.L, self.ev_cast):
+            sc = d["sc"]
+            main.wait_event(e)
+            fp8.fp8_linear_fwd(d["xq"], sc[2:3], d["wq"], sc[5:6], d["y"], sc[12:13])
+            fp8.fp8_linear_dgrad(d["dyq"], sc[8:9], d["wq"], sc[5:6], d["dx"], sc[13:14])
+            self.s_aux.wait_event(e)
+            with torch.cuda.stream(self.s_aux):
+                fp8.fp8_linear_wgrad(d["dyq"], sc[8:9], d["xq"], sc[2:3], d["dw"], sc[14:15])
+                fp8.fp8_scale_cast(d["dw"], fp8.FP8_E5M2, sc[14:15], 0, MU, sc[10:11], sc[11:12], d["gq"])
+        self.ev_grad.record(self.s_aux)
+        main.wait_event(self.ev_grad)
+        self.t += 1
+        fp8.fp8_adam_step(self.chunks, step=self.t, margin=0, workspace=self.ws, **HP)
+
     def result_scalars(self):
         return torch.cat([d["sc"] for d in self.L] + [d["st"] for d in self.L])
 
 
-def timed_steps(runner, steps, ev=None):
+def timed_steps(runner, steps, ev=None, overlap=False):
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record()
     for _ in range(steps):
-        runner.step(ev)
+        if overlap:
+            runner.step_overlapped()
+        else:
+            runner.step(ev)
     end.record()
     end.synchronize()
     return start.elapsed_time(end)
@@ -328,15 +379,16 @@ def run_gpu(args):
 
     peaks = load_peaks()
     runner = Block7BStep(dev, seed=rank)
+    overlap = args.schedule == "overlap"
     for _ in range(args.warmup):
-        runner.step()
+        runner.step_overlapped() if overlap else runner.step()
     barrier()
 
     # ---- device-timed region: inputs resident, whole step
     sampler = ClockSampler(local)
     with sampler:
         barrier()
-        ms = timed_steps(runner, args.steps)
+        ms = timed_steps(runner, args.steps, overlap=overlap)
         barrier()
     ms_step = ms / args.steps
     if dist is not None:
@@ -363,7 +415,7 @@ def run_gpu(args):
         for d, (x, y) in zip(runner.L, host_in):
             d["X"].copy_(x, non_blocking=True)
             d["dY"].copy_(y, non_blocking=True)
-        runner.step()
+        runner.step_overlapped() if overlap else runner.step()
         res.copy_(runner.result_scalars(), non_blocking=True)
 
     for _ in range(2):
@@ -394,6 +446,7 @@ def run_gpu(args):
         "config": {"workload": WORKLOAD, "tokens": runner.M, "hidden": 4096,
                    "linears": [d["name"] for d in runner.L], "adam_params": runner.params,
                    "gemm_flops_per_step": runner.flops, "l2": "inputs larger than L2 (no flush)",
+                   "schedule": args.schedule,
                    "parallelism": f"replicas{world}" if world > 1 else "single"},
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
                      "frac": gemm_tflops / fp8_peak, "traffic": gemm_traffic(),
@@ -432,6 +485,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--schedule", default="overlap", choices=["overlap", "serial"],
+                    help="overlap: casts / GEMMs / wgrad on three streams; serial: one stream")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

@@ -340,7 +340,7 @@ __global__ void k_adam_finalize(const __grid_constant__ AdamLaunch L) {
                      scale_exponent(hi, kMaxF16, L.margin, 0, khi) && klo == khi;
         if (known) {
           kw = klo;
-          if (C.wq != nullptr) {
+          if (C.wq_scale != nullptr) {
             const float s = pow2f(kw);
             int qlo, qhi;
             known = scale_exponent(stored_value(lo, s), kMaxE4M3, L.margin, 0, qlo) &&
@@ -363,7 +363,8 @@ __global__ void k_adam_finalize(const __grid_constant__ AdamLaunch L) {
       if (!(flags & 2u) || (flags & 1u)) {
         int kw, kq = 0;
         bool ok = scale_exponent(ws[WS_AMAX_W], kMaxF16, L.margin, 0, kw);
-        if (C.wq != nullptr) ok &= scale_exponent(stored_value(ws[WS_AMAX_W], pow2f(kw)), kMaxE4M3, L.margin, 0, kq);
+        if (C.wq_scale != nullptr)
+          ok &= scale_exponent(stored_value(ws[WS_AMAX_W], pow2f(kw)), kMaxE4M3, L.margin, 0, kq);
         if (!ok) atomicOr(&g_status, FP8_STATUS_NONFINITE);
         ws[WS_NEW_W] = pow2f(kw);
         ws[WS_NEW_WQ] = pow2f(kq);
@@ -371,7 +372,7 @@ __global__ void k_adam_finalize(const __grid_constant__ AdamLaunch L) {
       *C.m_scale = ws[WS_NEW_M];
       *C.v_scale = ws[WS_NEW_V];
       *C.w_scale = ws[WS_NEW_W];
-      if (C.wq != nullptr) {
+      if (C.wq_scale != nullptr) {  // a copy was asked for (its codes may be an empty slice)
         *C.wq_scale = ws[WS_NEW_WQ];
         *C.wq_inv = 1.0f / ws[WS_NEW_WQ];
       }

@@ -9,9 +9,11 @@
 // Every rank's payload was cast with one shared scale, so the codes of the
 // ranks can be added as they are.  Each FP8 value is an integer multiple of
 // the format's smallest subnormal (2^-16 for E5M2, 2^-9 for E4M3), so the sum
-// is formed exactly in integers (int64 / int32) and rounded once: to binary32
-// with round-to-odd (24 bits >= the 3- or 4-bit significand + 2, so the
-// following round-to-nearest-even is correct), then by the saturating cvt.
+// can be formed exactly and rounded once: to binary32 with round-to-odd (24
+// bits >= the 3- or 4-bit significand + 2, so the following
+// round-to-nearest-even is correct), then by the saturating cvt.  Two exact
+// summations: split binary32 accumulators (k_sum_codes_fast, the usual path)
+// and integer unit counts (k_sum_codes, E5M2 beyond 128 ranks).
 #pragma once
 
 #include "common.cuh"
@@ -122,6 +124,83 @@ __global__ void __launch_bounds__(kSumThreads)
       uint32_t special = 0;
       for (int r = 0; r < nranks; r++) acc += code_units<FMT>(in[(size_t)r * ld + i], special);
       out[i] = (uint8_t)encode_sum<FMT>(acc, special, under, over);
+    }
+    if (threadIdx.x == 0 && g_inv != nullptr) *g_inv = __fmul_rn(*inv_scale, 1.0f / (float)nranks);
+  }
+  if (counts != nullptr) {
+    __shared__ uint32_t red[64];
+    block_add_counts(under, over, red, counts);
+  }
+}
+
+// Faster exact sum for up to kSumFastMaxRanks ranks (E5M2; E4M3 up to
+// kSumMaxRanks).  The codes are decoded by the hardware cvt (fp8x2 -> f16x2,
+// exact) and summed in two binary32 accumulators split at |x| = 2: values
+// below are multiples of the smallest subnormal and stay below 2, values from
+// 2 up are multiples of 2^-1 (E5M2) or 2^-2 (E4M3), so neither partial sum
+// ever needs more than 24 significant bits and both are exact.  Their sum is
+// formed in binary64 (exact), rounded to binary32 by round-to-odd and then by
+// the saturating cvt.  inf and NaN propagate through the float adds (NaN ->
+// 0x7F, inf -> saturated and counted as an overflow), as in the integer path.
+constexpr int kSumFastMaxRanks = 128;
+
+template <int FMT>
+__device__ __forceinline__ uint32_t encode_split_sum(float hi, float lo, float fmax, uint32_t &under,
+                                                     uint32_t &over) {
+  if (!(fabsf(hi) <= 3.402823466e38f && fabsf(lo) <= 3.402823466e38f)) {  // inf or NaN involved
+    const float t = hi + lo;
+    if (t != t) return 0x7Fu;
+    over++;
+    return t > 0.0f ? top_code(FMT) : (0x80u | top_code(FMT));
+  }
+  const double d = (double)hi + (double)lo;
+  float f = __double2float_rz(d);
+  if ((double)f != d) f = __uint_as_float(__float_as_uint(f) | 1u);
+  const uint32_t c = enc2<FMT>(f, 0.0f) & 0xffu;
+  over += fabs(d) > (double)fmax ? 1u : 0u;
+  under += (d != 0.0 && (c & 0x7fu) == 0u) ? 1u : 0u;
+  return c;
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kSumThreads)
+    k_sum_codes_fast(const uint8_t *__restrict__ in, int nranks, size_t ld, size_t n, uint8_t *__restrict__ out,
+                     const float *__restrict__ inv_scale, float *__restrict__ g_inv,
+                     unsigned long long *__restrict__ counts) {
+  const float fmax = FMT == FP8_E5M2 ? 57344.0f : 448.0f;
+  const size_t groups = n / 16;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  uint32_t under = 0, over = 0;
+  for (size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x; g < groups; g += stride) {
+    float hi[16], lo[16];
+#pragma unroll
+    for (int j = 0; j < 16; j++) hi[j] = lo[j] = 0.0f;
+    for (int r = 0; r < nranks; r++) {
+      const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(in + (size_t)r * ld) + g);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int p = 0; p < 8; p++) {
+        const float2 x = dec2<FMT>(w[p >> 1] >> ((p & 1) * 16));
+        const bool ba = fabsf(x.x) >= 2.0f, bb = fabsf(x.y) >= 2.0f;
+        hi[2 * p] += ba ? x.x : 0.0f;
+        lo[2 * p] += ba ? 0.0f : x.x;
+        hi[2 * p + 1] += bb ? x.y : 0.0f;
+        lo[2 * p + 1] += bb ? 0.0f : x.y;
+      }
+    }
+    uint32_t o[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 16; j++) o[j >> 2] |= encode_split_sum<FMT>(hi[j], lo[j], fmax, under, over) << (8 * (j & 3));
+    __stcs(reinterpret_cast<uint4 *>(out) + g, make_uint4(o[0], o[1], o[2], o[3]));
+  }
+  if (blockIdx.x == 0) {
+    for (size_t i = groups * 16 + threadIdx.x; i < n; i += blockDim.x) {
+      float hi = 0.0f, lo = 0.0f;
+      for (int r = 0; r < nranks; r++) {
+        const float x = dec2<FMT>(in[(size_t)r * ld + i]).x;
+        if (fabsf(x) >= 2.0f) hi += x; else lo += x;
+      }
+      out[i] = (uint8_t)encode_split_sum<FMT>(hi, lo, fmax, under, over);
     }
     if (threadIdx.x == 0 && g_inv != nullptr) *g_inv = __fmul_rn(*inv_scale, 1.0f / (float)nranks);
   }

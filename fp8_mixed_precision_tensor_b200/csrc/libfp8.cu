@@ -352,10 +352,14 @@ int fp8_sum_codes(const uint8_t *in, int nranks, size_t ld, size_t n, int fmt, u
   if (rc) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const unsigned grid = grid_for(n / 16, kSumThreads, d->sms * 8);
-  if (fmt == FP8_E5M2)
+  if (fmt == FP8_E5M2 && nranks <= kSumFastMaxRanks)
+    k_sum_codes_fast<FP8_E5M2><<<grid, kSumThreads, 0, s>>>(in, nranks, ld, n, out, inv_scale_dev, g_inv_dev,
+                                                            counts_dev);
+  else if (fmt == FP8_E5M2)
     k_sum_codes<FP8_E5M2><<<grid, kSumThreads, 0, s>>>(in, nranks, ld, n, out, inv_scale_dev, g_inv_dev, counts_dev);
   else
-    k_sum_codes<FP8_E4M3><<<grid, kSumThreads, 0, s>>>(in, nranks, ld, n, out, inv_scale_dev, g_inv_dev, counts_dev);
+    k_sum_codes_fast<FP8_E4M3><<<grid, kSumThreads, 0, s>>>(in, nranks, ld, n, out, inv_scale_dev, g_inv_dev,
+                                                            counts_dev);
   return launch_rc();
 }
 
@@ -432,7 +436,9 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
   for (int i = 0; i < nchunks; i++) {
     const fp8_adam_chunk &c = chunks[i];
     if (!c.g_inv || !c.m_scale || !c.v_scale || !c.w_scale) return FP8_ERR_INVALID_ARG;
-    if (c.wq && (!c.wq_scale || !c.wq_inv)) return FP8_ERR_INVALID_ARG;
+    // the E4M3 copy is asked for by wq_scale; its codes may be NULL only for an empty chunk
+    if ((c.wq || c.wq_scale || c.wq_inv) && (!c.wq_scale || !c.wq_inv)) return FP8_ERR_INVALID_ARG;
+    if (c.wq_scale && c.n > 0 && !c.wq) return FP8_ERR_INVALID_ARG;
     if (phases != PH_ALL && c.w_amax) return FP8_ERR_INVALID_ARG;  // tracking needs the whole step
     if (c.n > 0 && (!c.g || !c.m || !c.v || !c.w)) return FP8_ERR_INVALID_ARG;
     if (c.n > 0 && (!aligned16(c.g) || !aligned16(c.m) || !aligned16(c.v) || !aligned16(c.w) ||

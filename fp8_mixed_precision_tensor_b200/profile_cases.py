@@ -3,11 +3,17 @@
     python -m fp8_mixed_precision_tensor_b200.profile_cases linear --M 4096 --N 16384 --K 4096
     python -m fp8_mixed_precision_tensor_b200.profile_cases cast --n 268435456
     python -m fp8_mixed_precision_tensor_b200.profile_cases adam --n 67108864 [--track]
+    python -m fp8_mixed_precision_tensor_b200.profile_cases allreduce --n 268435456 --world 8
+    python -m fp8_mixed_precision_tensor_b200.profile_cases castcount --n 268435456
 
 Each case runs `--iters` passes after one warm-up pass on seeded synthetic
 inputs and prints the CUDA-event time per pass.  Launch order per pass:
 linear: amax and fused scale+cast of X, W, dY (6 launches), then fwd, dgrad,
-wgrad; cast: amax, fused scale+cast; adam: stats pass, finalize, update pass.
+wgrad; cast: amax, fused scale+cast; adam: stats pass, finalize, update pass;
+allreduce: `world` emulated ranks' payload casts of an fp32 gradient, then
+the `world` per-slice code sums (no collective: one GPU); castcount: the cast
+with under/overflow counters, then the plain cast.  The two last cases also
+print each kernel's own time and algorithmic GB/s.
 """
 from __future__ import annotations
 
@@ -87,17 +93,81 @@ def case_adam(a):
     return one
 
 
+def _timed(fn, iters):
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    fn()
+    s.record()
+    for _ in range(iters):
+        fn()
+    e.record()
+    e.synchronize()
+    return s.elapsed_time(e) / iters
+
+
+def case_allreduce(a):
+    n, world = a.n, a.world
+    L = -(-(-(-n // 16)) // world) * 16
+    g = synth.device_normal((n,), 1e-4, 7, torch.float32, "cuda")
+    amax, mu, sc = _scalars(1), torch.full((1,), 1.0 / world, device="cuda"), _scalars(3)
+    fp8.fp8_amax(g, amax)
+    sends = torch.zeros(world, world * L, dtype=torch.uint8, device="cuda")
+    out = torch.zeros(world * L, dtype=torch.uint8, device="cuda")
+    counts = torch.zeros(2, dtype=torch.int64, device="cuda")
+    rows = torch.zeros(world, L, dtype=torch.uint8, device="cuda")
+
+    def casts():
+        for r in range(world):
+            fp8.fp8_grad_cast(g, fp8.FP8_E5M2, amax, 0, mu, sc[0:1], sc[1:2], sends[r], counts)
+
+    def sums():
+        for j in range(world):
+            fp8.fp8_sum_codes(rows, L, fp8.FP8_E5M2, out[j * L:(j + 1) * L], sc[1:2], sc[2:3], counts)
+
+    casts()
+    rows.copy_(sends[:, :L])
+    t_cast = _timed(casts, a.iters) / world
+    t_sum = _timed(sums, a.iters) / world
+    print(f"grad_cast: {t_cast:.4f} ms per rank, {5 * n / t_cast / 1e6:.0f} GB/s (4 B read + 1 B write per elem)")
+    print(f"sum_codes: {t_sum:.4f} ms per slice, {(world + 1) * L / t_sum / 1e6:.0f} GB/s "
+          f"({world} B read + 1 B write per slice elem)")
+
+    def one():
+        casts()
+        sums()
+
+    return one
+
+
+def case_castcount(a):
+    x = synth.device_normal((a.n,), 1.0, 8, torch.bfloat16, "cuda")
+    q = torch.empty(a.n, dtype=torch.uint8, device="cuda")
+    s = torch.full((1,), 2.0 ** 6, device="cuda")
+    counts = torch.zeros(2, dtype=torch.int64, device="cuda")
+    t_count = _timed(lambda: fp8.fp8_cast_count(x, fp8.FP8_E4M3, s, q, counts), a.iters)
+    t_plain = _timed(lambda: fp8.fp8_cast(x, fp8.FP8_E4M3, s, q), a.iters)
+    print(f"cast_count: {t_count:.4f} ms, {3 * a.n / t_count / 1e6:.0f} GB/s; plain cast: {t_plain:.4f} ms, "
+          f"{3 * a.n / t_plain / 1e6:.0f} GB/s (2 B read + 1 B write per elem)")
+
+    def one():
+        fp8.fp8_cast_count(x, fp8.FP8_E4M3, s, q, counts)
+        fp8.fp8_cast(x, fp8.FP8_E4M3, s, q)
+
+    return one
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["linear", "cast", "adam"])
+    ap.add_argument("case", choices=["linear", "cast", "adam", "allreduce", "castcount"])
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--N", type=int, default=16384)
     ap.add_argument("--K", type=int, default=4096)
     ap.add_argument("--n", type=int, default=1 << 26)
     ap.add_argument("--iters", type=int, default=2)
+    ap.add_argument("--world", type=int, default=8, help="allreduce: emulated ranks")
     ap.add_argument("--track", action="store_true", help="adam: track the master amax across steps")
     a = ap.parse_args()
-    one = {"linear": case_linear, "cast": case_cast, "adam": case_adam}[a.case](a)
+    one = {"linear": case_linear, "cast": case_cast, "adam": case_adam, "allreduce": case_allreduce,
+           "castcount": case_castcount}[a.case](a)
     one()
     torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -267,9 +267,10 @@ int fp8_linear_wgrad(const uint8_t *dyq, const float *dy_inv, const uint8_t *xq,
  * negative value means "unknown" (the step re-reads the master).  After
  * changing w or w_scale by other means, set *w_amax to -1.
  * E4M3 master copy (optional; the next forward pass's weight cast fused into
- * the update): when wq is not NULL the step also writes
+ * the update): when wq_scale is not NULL the step also writes
  * wq = E4M3(stored master * s_q), s_q from the amax of the stored master with
- * fmt_max 448 and the same margin, and s_q, 1/s_q to *wq_scale, *wq_inv.
+ * fmt_max 448 and the same margin, and s_q, 1/s_q to *wq_scale, *wq_inv
+ * (wq may be NULL only when n == 0, e.g. an empty slice of a sharded step).
  * Pointers g, m, v, w, wq are dev and 16-byte aligned; the scale pointers are
  * dev floats.  Chunks must not overlap.  `chunks` is a HOST array of nchunks.
  */
@@ -284,9 +285,9 @@ typedef struct {
   float *w_scale;      /* dev float (in/out) */
   size_t n;            /* parameters in this chunk (0 allowed) */
   float *w_amax;       /* dev float or NULL: tracked amax of the stored master (in/out) */
-  uint8_t *wq;         /* dev [n] or NULL: E4M3 copy of the new stored master (out) */
-  float *wq_scale;     /* dev float, required with wq (out) */
-  float *wq_inv;       /* dev float, required with wq (out) */
+  uint8_t *wq;         /* dev [n]: E4M3 copy of the new stored master (out), or NULL */
+  float *wq_scale;     /* dev float or NULL: asks for the copy (out) */
+  float *wq_inv;       /* dev float, required with wq_scale (out) */
 } fp8_adam_chunk;
 
 typedef struct {

@@ -130,6 +130,21 @@ def test_sum_codes_vs_oracle(fmt, nranks, n):
     assert g_inv.item() == float(np.float32(2.0 ** -13) * np.float32(1.0 / nranks))
 
 
+@pytest.mark.parametrize("fmt", [fp8.FP8_E4M3, fp8.FP8_E5M2])
+def test_sum_codes_many_ranks(fmt):
+    """160 ranks: E5M2 beyond the split-accumulator path's 128 ranks takes the
+    integer path; E4M3 stays on the split path."""
+    nranks, n = 160, 4099
+    ld = -(-n // 16) * 16
+    rows = _codes_with_specials(nranks, ld, fmt, ("many", fmt))
+    out = torch.zeros(ld, dtype=torch.uint8, device="cuda")
+    counts = torch.zeros(2, **I64)
+    fp8.fp8_sum_codes(to_dev(rows), n, fmt, out, counts=counts)
+    ref, c = oracle.sum_codes(rows[:, :n], OFMT[fmt])
+    assert_codes_equal(out.cpu().numpy()[:n], ref, None, "sum_codes many ranks")
+    assert tuple(counts.tolist()) == c
+
+
 def test_sum_codes_rejects_bad_layout():
     d = torch.zeros(2, 40, dtype=torch.uint8, device="cuda")
     out = torch.zeros(48, dtype=torch.uint8, device="cuda")

@@ -68,3 +68,27 @@ def test_gpt7b_linears_full_size(name, K, N):
 @pytest.mark.parametrize("name,K,N", synth.GPT175B_LINEARS)
 def test_gpt175b_linears_full_size(name, K, N):
     _check_linear(synth.GPT175B_TOKENS, K, N, synth.GPT175B_W_STD, 200)
+
+
+def test_bench_step_three_streams_equals_one_stream():
+    """The benchmark step's overlapped schedule (casts, fwd/dgrad and wgrad on
+    three streams) computes exactly what the one-stream order computes: the
+    same scalars, gradient codes and Adam state after two steps."""
+    import importlib.util
+    import os
+
+    spec = importlib.util.spec_from_file_location(
+        "bench_mod", os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    dev = torch.device("cuda", 0)
+    a, b = bench.Block7BStep(dev, seed=3), bench.Block7BStep(dev, seed=3)
+    for _ in range(2):
+        a.step()
+        b.step_overlapped()
+    torch.cuda.synchronize()
+    assert fp8.fp8_get_status() == 0
+    assert torch.equal(a.result_scalars(), b.result_scalars())
+    for da, db in zip(a.L, b.L):
+        for k in ("gq", "m", "v", "wh", "y", "dx", "dw"):
+            assert torch.equal(da[k], db[k]), (da["name"], k)

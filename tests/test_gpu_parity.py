@@ -264,6 +264,37 @@ def test_linear_gemms_pair_kernel_sampled(shape):
         assert amax.item() == float(np.max(np.abs(got))), name
 
 
+def test_linear_wide_kernel_16bit_outputs_and_bias():
+    """The 256x512 two-CTA kernel with every 16-bit output path: fwd with a
+    bias into fp16, dgrad into fp16, wgrad into bf16 (ragged edges)."""
+    M, N, K = 2320, 4624, 528
+    q = quantised_linear(M, N, K, ("gemm-wide16",))
+    (xq, xi), (wq, wi), (dyq, dyi) = q["x"], q["w"], q["dy"]
+    bias = synth.normal_f32((N,), 0.5, "wide16", "b")
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    dx = torch.empty((M, K), dtype=torch.float16, device="cuda")
+    dw = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+    ya, dxa, dwa = scalar(), scalar(), scalar()
+    fp8.fp8_linear_fwd(xq, xi, wq, wi, y, ya, bias=to_dev(bias))
+    fp8.fp8_linear_dgrad(dyq, dyi, wq, wi, dx, dxa)
+    fp8.fp8_linear_wgrad(dyq, dyi, xq, xi, dw, dwa)
+    assert fp8.fp8_get_status() == 0
+    h = {k: (v[0].cpu().numpy(), float(v[1].item())) for k, v in q.items()}
+    for name, out, amax, (rows, cols), fn in (
+            ("fwd", y, ya, (M, N), lambda smp: oracle.linear_fwd(h["x"][0], h["x"][1], h["w"][0], h["w"][1],
+                                                                 M, N, K, bias=bias.astype(np.float64),
+                                                                 samples=smp)),
+            ("dgrad", dx, dxa, (M, K), lambda smp: oracle.linear_dgrad(h["dy"][0], h["dy"][1], h["w"][0],
+                                                                       h["w"][1], M, N, K, samples=smp)),
+            ("wgrad", dw, dwa, (N, K), lambda smp: oracle.linear_wgrad(h["dy"][0], h["dy"][1], h["x"][0],
+                                                                       h["x"][1], M, N, K, samples=smp))):
+        r, c = boundary_samples(rows, cols, 3000, (name, "wide16"), tile_c=(256, 512))
+        ref, rabs = fn((r, c))
+        got = tensor_to_np(out) if out.dtype != torch.float16 else out.double().cpu().numpy()
+        assert_gemm_close(got[r, c], ref, rabs, out.dtype, f"{name} wide16")
+        assert amax.item() == float(np.max(np.abs(got))), name
+
+
 def test_linear_fwd_bias_f16_out():
     M, N, K = 256, 272, 128
     q = quantised_linear(M, N, K, ("bias",))
