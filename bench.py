@@ -19,9 +19,10 @@ Inputs are seeded synthetic tensors (bf16 activations ~N(0,1), weights
 more than the 126 MB L2, so no explicit L2 flush is needed between steps.
 
 The step's launches run on three streams by default (--schedule overlap):
-the casts of all four linears run ahead beside the GEMMs, wgrad and the
-gradient cast run beside fwd/dgrad, Adam joins them.  --schedule serial runs
-the same launches in order on one stream.  The per-kernel breakdown
+the casts of all four linears run ahead beside the GEMMs; wgrad, the
+gradient cast and that tensor's Adam step run beside the next fwd/dgrad (one
+Adam call per tensor instead of one over all four).  --schedule serial runs
+the work in order on one stream.  The per-kernel breakdown
 (`kernels`, `roofline`) always comes from a serial pass with CUDA events
 around each phase.
 
@@ -180,11 +181,19 @@ class Block7BStep:
             fp8.AdamChunk(d["gq"], d["sc"][11:12], d["m"], d["st"][0:1], d["v"], d["st"][1:2], d["wh"],
                           d["st"][2:3]) for d in self.L])
         self.ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(self.L)) // 4 + 64, **f32)
+        # one Adam call per tensor (overlapped schedule): own chunk array and a
+        # 256-byte-aligned workspace slice each
+        self.chunks_each = [fp8.pack_adam_chunks([
+            fp8.AdamChunk(d["gq"], d["sc"][11:12], d["m"], d["st"][0:1], d["v"], d["st"][1:2], d["wh"],
+                          d["st"][2:3])]) for d in self.L]
+        self.ws_each = torch.zeros(64 * len(self.L), **f32)
         self.t = 0
         self.flops = sum(3 * 2 * d["M"] * d["N"] * d["K"] for d in self.L)
         self.cast_elems = sum(d["M"] * d["K"] + d["N"] * d["K"] + d["M"] * d["N"] for d in self.L)
         self.params = sum(d["N"] * d["K"] for d in self.L)
-        self.launches_per_step = 4 * (3 * 2 + 3 + 1) + 3  # (amax, scale+cast) x3, GEMMs, grad scale+cast; Adam
+        # (amax, scale+cast) x3, GEMMs, grad scale+cast per linear; Adam (3 launches per call)
+        self.launches_per_step = 4 * (3 * 2 + 3 + 1) + 3
+        self.launches_per_step_overlapped = 4 * (3 * 2 + 3 + 1 + 3)
 
     def quantise(self, x, fmt, sc, i, mu=1.0, out=None):
         fp8 = self.fp8
@@ -225,15 +234,18 @@ class Block7BStep:
         if e: e[1].record()
 
     def step_overlapped(self):
-        """The same launches as step(), on three streams: the casts of every
+        """The same work as step(), on three streams: the casts of every
         linear run ahead on a cast stream (HBM-bound work beside the
-        tensor-bound GEMMs, whose CTAs leave room for one cast block per SM),
-        forward and dgrad run on the current stream, wgrad and the gradient
-        cast on an auxiliary stream (one GEMM's last wave overlaps the next
-        GEMM); Adam joins them on the current stream.  Every buffer of a
-        step is written once, and the next step's casts start only after this
-        step's Adam (the cast stream waits for an event recorded at the start
-        of the next step on the current stream)."""
+        tensor-bound GEMMs, whose CTAs leave room for a cast or Adam block per
+        SM), forward and dgrad run on the current stream, wgrad, the gradient
+        cast and that tensor's Adam step on an auxiliary stream (one GEMM's
+        last wave overlaps the next GEMM; each tensor's optimizer step
+        overlaps the following linears' GEMMs -- Adam is per tensor, so one
+        call per tensor computes exactly what one call over all does).  Every
+        buffer of a step is written once, and the next step's casts start
+        only after this step's last Adam (the cast stream waits for an event
+        recorded at the start of the next step on the current stream, which
+        has joined the auxiliary stream)."""
         fp8 = self.fp8
         main = torch.cuda.current_stream()
         if not hasattr(self, "s_cast"):
@@ -251,7 +263,7 @@ class Block7BStep:
                 self.quantise(d["W"], fp8.FP8_E4M3, sc, 3, out=d["wq"])
                 self.quantise(d["dY"], fp8.FP8_E5M2, sc, 6, mu=MU, out=d["dyq"])
                 e.record(self.s_cast)
-        for d, e in zip(self.L, self.ev_cast):
+        for i, (d, e) in enumerate(zip(self.L, self.ev_cast)):
             sc = d["sc"]
             main.wait_event(e)
             fp8.fp8_linear_fwd(d["xq"], sc[2:3], d["wq"], sc[5:6], d["y"], sc[12:13])
@@ -260,10 +272,11 @@ class Block7BStep:
             with torch.cuda.stream(self.s_aux):
                 fp8.fp8_linear_wgrad(d["dyq"], sc[8:9], d["xq"], sc[2:3], d["dw"], sc[14:15])
                 fp8.fp8_scale_cast(d["dw"], fp8.FP8_E5M2, sc[14:15], 0, MU, sc[10:11], sc[11:12], d["gq"])
+                fp8.fp8_adam_step(self.chunks_each[i], step=self.t + 1, margin=0,
+                                  workspace=self.ws_each[64 * i:64 * (i + 1)], **HP)
         self.ev_grad.record(self.s_aux)
         main.wait_event(self.ev_grad)
         self.t += 1
-        fp8.fp8_adam_step(self.chunks, step=self.t, margin=0, workspace=self.ws, **HP)
 
     def result_scalars(self):
         return torch.cat([d["sc"] for d in self.L] + [d["st"] for d in self.L])
@@ -462,7 +475,7 @@ def run_gpu(args):
         },
         "e2e": {"value": runner.flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": runner.launches_per_step * args.steps,
+        "gpu_launches": (runner.launches_per_step_overlapped if overlap else runner.launches_per_step) * args.steps,
         "clocks": sampler.summary(),
         "device_status": status,
     }

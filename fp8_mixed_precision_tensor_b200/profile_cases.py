@@ -5,6 +5,7 @@
     python -m fp8_mixed_precision_tensor_b200.profile_cases adam --n 67108864 [--track]
     python -m fp8_mixed_precision_tensor_b200.profile_cases allreduce --n 268435456 --world 8
     python -m fp8_mixed_precision_tensor_b200.profile_cases castcount --n 268435456
+    python -m fp8_mixed_precision_tensor_b200.profile_cases adam7b --iters 10
 
 Each case runs `--iters` passes after one warm-up pass on seeded synthetic
 inputs and prints the CUDA-event time per pass.  Launch order per pass:
@@ -12,8 +13,10 @@ linear: amax and fused scale+cast of X, W, dY (6 launches), then fwd, dgrad,
 wgrad; cast: amax, fused scale+cast; adam: stats pass, finalize, update pass;
 allreduce: `world` emulated ranks' payload casts of an fp32 gradient, then
 the `world` per-slice code sums (no collective: one GPU); castcount: the cast
-with under/overflow counters, then the plain cast.  The two last cases also
-print each kernel's own time and algorithmic GB/s.
+with under/overflow counters, then the plain cast; adam7b: one Adam step
+over all 129 per-tensor chunks of GPT-7B (6,648,496,128 parameters, 40 GB
+of FP8/FP16 state).  allreduce, castcount and adam7b also print each
+kernel's own time and algorithmic GB/s.
 """
 from __future__ import annotations
 
@@ -155,9 +158,49 @@ def case_castcount(a):
     return one
 
 
+def build_adam_state(chunks, device="cuda", seed=11, mu=2.0 ** 10):
+    """Device-resident decoupled-Adam state for (name, n) chunks: E5M2
+    gradients ~N(0, 1e-3) scaled by mu, FP16 master ~N(0, 0.02) with its
+    scale, zero moments with scale 1.  Returns a list of fp8.AdamChunk."""
+    out = []
+    for ci, (_, n) in enumerate(chunks):
+        sc = _scalars(6)
+        g = synth.device_normal((n,), 1e-3, seed * 100000 + 2 * ci, torch.float32, device)
+        gq = torch.empty(n, dtype=torch.uint8, device=device)
+        fp8.fp8_amax(g, sc[0:1])
+        fp8.fp8_scale_cast(g, fp8.FP8_E5M2, sc[0:1], 0, mu, sc[1:2], sc[2:3], gq)
+        del g
+        w = synth.device_normal((n,), 0.02, seed * 100000 + 2 * ci + 1, torch.float32, device)
+        wh = torch.empty(n, dtype=torch.int16, device=device)
+        st = torch.ones(3, dtype=torch.float32, device=device)
+        fp8.fp8_amax(w, sc[3:4])
+        fp8.fp8_scale_cast(w, fp8.FP8_F16S, sc[3:4], 0, 1.0, st[2:3], sc[5:6], wh)
+        del w
+        out.append(fp8.AdamChunk(gq, sc[2:3], torch.zeros(n, dtype=torch.uint8, device=device), st[0:1],
+                                 torch.zeros(n, dtype=torch.int16, device=device), st[1:2], wh, st[2:3]))
+    return out
+
+
+def case_adam7b(a):
+    chunks_list = build_adam_state(synth.gpt7b_adam_chunks())
+    params = sum(c.g.numel() for c in chunks_list)
+    chunks = fp8.pack_adam_chunks(chunks_list)
+    ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(chunks_list)) // 4, dtype=torch.float32, device="cuda")
+    state = {"t": 0}
+
+    def one():
+        state["t"] += 1
+        fp8.fp8_adam_step(chunks, 1e-4, 0.9, 0.95, 1e-8, state["t"], 0, ws)
+
+    t = _timed(one, a.iters)
+    print(f"adam7b: {len(chunks_list)} chunks, {params} params, {t:.3f} ms per step, "
+          f"{11 * params / t / 1e6:.0f} GB/s algorithmic (11 B/param), {17 * params / t / 1e6:.0f} GB/s moved")
+    return one
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["linear", "cast", "adam", "allreduce", "castcount"])
+    ap.add_argument("case", choices=["linear", "cast", "adam", "allreduce", "castcount", "adam7b"])
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--N", type=int, default=16384)
     ap.add_argument("--K", type=int, default=4096)
@@ -167,7 +210,7 @@ def main():
     ap.add_argument("--track", action="store_true", help="adam: track the master amax across steps")
     a = ap.parse_args()
     one = {"linear": case_linear, "cast": case_cast, "adam": case_adam, "allreduce": case_allreduce,
-           "castcount": case_castcount}[a.case](a)
+           "castcount": case_castcount, "adam7b": case_adam7b}[a.case](a)
     one()
     torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -92,3 +92,28 @@ def test_bench_step_three_streams_equals_one_stream():
     for da, db in zip(a.L, b.L):
         for k in ("gq", "m", "v", "wh", "y", "dx", "dw"):
             assert torch.equal(da[k], db[k]), (da["name"], k)
+
+
+def test_gpt7b_adam_full_model_two_steps():
+    """The decoupled Adam over all 129 per-tensor chunks of GPT-7B
+    (6,648,496,128 parameters, one call per step): the step-2 state of two
+    whole chunks (the first QKV and the last fc2) against the oracle, from the
+    GPU's own step-1 state; every chunk's scales stay finite powers of two."""
+    from fp8_mixed_precision_tensor_b200.profile_cases import build_adam_state
+    from test_gpu_parity import HP, check_adam_chunk, snapshot
+
+    specs = synth.gpt7b_adam_chunks()
+    assert sum(n for _, n in specs) == 6648496128
+    chunks = build_adam_state(specs)
+    arr = fp8.pack_adam_chunks(chunks)
+    ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(chunks)) // 4, dtype=torch.float32, device="cuda")
+    fp8.fp8_adam_step(arr, step=1, margin=0, workspace=ws, **HP)
+    picks = [0, len(specs) - 2]  # l0.qkv, l31.fc2
+    before = {i: snapshot(chunks[i]) for i in picks}
+    fp8.fp8_adam_step(arr, step=2, margin=0, workspace=ws, **HP)
+    assert fp8.fp8_get_status() == 0
+    for i in picks:
+        check_adam_chunk(before[i], chunks[i], 2)
+    scales = torch.stack([torch.cat([c.m_scale, c.v_scale, c.w_scale]) for c in chunks]).cpu().numpy()
+    mant, _ = np.frexp(scales)
+    assert np.all(np.isfinite(scales)) and np.all(mant == 0.5)
