@@ -255,22 +255,25 @@ class Block7BStep:
         if not hasattr(self, "s_cast"):
             self.s_cast, self.s_aux = torch.cuda.Stream(self.dev), torch.cuda.Stream(self.dev)
             self.ev_start = torch.cuda.Event()
-            self.ev_cast = [torch.cuda.Event() for _ in self.L]
+            self.ev_cast = [torch.cuda.Event() for _ in self.L]     # X, W and dY cast
+            self.ev_cast_xw = [torch.cuda.Event() for _ in self.L]  # X and W cast (enough for fwd)
             self.ev_grad = torch.cuda.Event()
         self.ev_start.record(main)
         self.s_cast.wait_event(self.ev_start)
         self.s_aux.wait_event(self.ev_start)
         with torch.cuda.stream(self.s_cast):
-            for d, e in zip(self.L, self.ev_cast):
+            for d, e, exw in zip(self.L, self.ev_cast, self.ev_cast_xw):
                 sc = d["sc"]
                 self.quantise(d["X"], fp8.FP8_E4M3, sc, 0, out=d["xq"])
                 self.quantise(d["W"], fp8.FP8_E4M3, sc, 3, out=d["wq"])
+                exw.record(self.s_cast)
                 self.quantise(d["dY"], fp8.FP8_E5M2, sc, 6, mu=MU, out=d["dyq"])
                 e.record(self.s_cast)
         for i, (d, e) in enumerate(zip(self.L, self.ev_cast)):
             sc = d["sc"]
-            main.wait_event(e)
+            main.wait_event(self.ev_cast_xw[i])
             fp8.fp8_linear_fwd(d["xq"], sc[2:3], d["wq"], sc[5:6], d["y"], sc[12:13])
+            main.wait_event(e)
             fp8.fp8_linear_dgrad(d["dyq"], sc[8:9], d["wq"], sc[5:6], d["dx"], sc[13:14])
             self.s_aux.wait_event(e)
             with torch.cuda.stream(self.s_aux):

@@ -922,6 +922,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       const int row0 = mb * (2 * kPairHalf) + (int)rank * kPairHalf + q * 32;
       const bool rows_in = row0 < args.rows;
       uint32_t amax_bits = 0;
+      uint32_t amax16 = 0;  // 16-bit outputs: two packed magnitude maxima
       // accumulator column c of half h holds output column
       //   nb*512 + (c < 128 ? 0 : 256) + h*128 + (c mod 128)
       const int cols_per_box = f32out ? 32 : 64;
@@ -951,15 +952,13 @@ __global__ void __launch_bounds__(kWideThreads, 1)
               __nv_bfloat162 x = __floats2bfloat162_rn(a0, a1), y = __floats2bfloat162_rn(b0, b1);
               pa = *reinterpret_cast<uint32_t *>(&x);
               pb = *reinterpret_cast<uint32_t *>(&y);
-              amax_bits = max(amax_bits, max(max((pa & 0x7fffu) << 16, pa & 0x7fff0000u),
-                                             max((pb & 0x7fffu) << 16, pb & 0x7fff0000u)));
             } else {
               pa = f16x2(a0, a1);
               pb = f16x2(b0, b1);
-              const float2 ba = h2f2(pa), bb = h2f2(pb);
-              amax_bits = max(amax_bits, max(max(absbits_f32(ba.x), absbits_f32(ba.y)),
-                                             max(absbits_f32(bb.x), absbits_f32(bb.y))));
             }
+            // running max of the stored 16-bit magnitudes, two per word (for
+            // both types the magnitude bits order like the values, NaN on top)
+            amax16 = __vmaxu2(amax16, __vmaxu2(pa & 0x7fff7fffu, pb & 0x7fff7fffu));
             w[j] = pa;
             w[16 + j] = pb;
           }
@@ -982,6 +981,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(map_to_rank(tempty_bar, 0));
+      if (!f32out) {
+        const uint32_t h16 = max(amax16 & 0xffffu, amax16 >> 16);
+        amax_bits = bfout ? (h16 << 16) : absbits_f32(__half2float(__ushort_as_half((unsigned short)h16)));
+      }
       if (row0 + lane >= args.rows) amax_bits = 0;  // a row past the output (holds only the bias)
       if (args.out_amax != nullptr) {
         amax_bits = warp_max_u32(amax_bits);
