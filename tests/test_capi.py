@@ -91,3 +91,39 @@ def test_product_never_touches_the_oracle():
             if fn.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, fn)).read()
                 assert not re.search(r"\boracle\b", text), f"{fn} mentions the oracle"
+
+
+def test_host_side_validation_of_the_next_rows(lib):
+    """Scaling variants, FP8 all-reduce, mu rule and sharded Adam entry points
+    reject bad arguments on the host, before any device work."""
+    p, i, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    fake = 0x10000
+    lib.fp8_cast_count.argtypes = [p, i, sz, i, p, p, p, p]
+    assert lib.fp8_cast_count(fake, 1, 32, 0, fake, fake, None, None) == 1       # no counters
+    lib.fp8_grad_cast.argtypes = [p, i, sz, i, p, i, p, p, p, p, p, p]
+    assert lib.fp8_grad_cast(fake, 0, 32, 2, fake, 0, fake, fake, fake, fake, None, None) == 1  # FP16 payload
+    assert lib.fp8_grad_cast(fake, 0, 32, 1, fake, 0, None, fake, fake, fake, None, None) == 1  # no mu
+    lib.fp8_sum_codes.argtypes = [p, i, sz, sz, i, p, p, p, p, p]
+    assert lib.fp8_sum_codes(fake, 0, 32, 32, 1, fake, None, None, None, None) == 1      # no ranks
+    assert lib.fp8_sum_codes(fake, 2, 40, 32, 1, fake, None, None, None, None) == 2      # ld % 16
+    assert lib.fp8_sum_codes(fake, 2, 32, 48, 1, fake, None, None, None, None) == 1      # n > ld
+    assert lib.fp8_sum_codes(fake, 5000, 32, 32, 1, fake, None, None, None, None) == 1   # too many ranks
+
+    from fp8_mixed_precision_tensor_b200 import fp8
+
+    lib.fp8_mu_update.argtypes = [p, p, p, ctypes.c_ulonglong, ctypes.POINTER(fp8._MuRule), p]
+    bad = fp8._MuRule(1e-3, 10, 3.0, 4.0)   # mu_min not a power of two
+    assert lib.fp8_mu_update(fake, fake, fake, 100, ctypes.byref(bad), None) == 1
+    bad = fp8._MuRule(1e-3, 0, 0.5, 1.0)    # interval 0
+    assert lib.fp8_mu_update(fake, fake, fake, 100, ctypes.byref(bad), None) == 1
+
+    arr = (fp8._Chunk * 1)()
+    arr[0] = fp8._Chunk(fake, fake, fake, fake, fake, fake, fake, fake, 64, fake, None, None, None)
+    hp = fp8._HParams(1e-4, 0.9, 0.95, 1e-8, 1, 0)
+    for name in ("fp8_adam_stats", "fp8_adam_apply"):
+        fn = getattr(lib, name)
+        fn.argtypes = [ctypes.POINTER(fp8._Chunk), i, ctypes.POINTER(fp8._HParams), p, sz, p]
+        assert fn(arr, 1, ctypes.byref(hp), fake, 64, None) == 1   # tracked amax in a sharded half
+    arr[0] = fp8._Chunk(fake, fake, fake, fake, fake, fake, fake, fake, 64, None, None, fake, fake)
+    lib.fp8_adam_step.argtypes = [ctypes.POINTER(fp8._Chunk), i, ctypes.POINTER(fp8._HParams), p, sz, p]
+    assert lib.fp8_adam_step(arr, 1, ctypes.byref(hp), fake, 64, None) == 1  # copy asked for, no codes
