@@ -347,6 +347,23 @@ __device__ __forceinline__ void descale_chunk(const Args &args, uint32_t (&r)[32
   }
 }
 
+// descale_chunk with the two descales folded into one factor inv_ab =
+// inv_a * inv_b (both powers of two, so the product is exact whenever it is a
+// normal float, and x * inv_ab rounds no worse than two multiplications).
+__device__ __forceinline__ void descale1_chunk(const Args &args, uint32_t (&r)[32], int col0, float inv_ab) {
+  if (args.bias == nullptr) {
+#pragma unroll
+    for (int j = 0; j < 32; j++) r[j] = __float_as_uint(__fmul_rn(__uint_as_float(r[j]), inv_ab));
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < 32; j++) {
+    float y = __fmul_rn(__uint_as_float(r[j]), inv_ab);
+    if (col0 + j < args.cols) y = __fadd_rn(y, load_bias(args.bias, args.bias_dtype, col0 + j));
+    r[j] = __float_as_uint(y);
+  }
+}
+
 // Epilogue of one 32-column chunk: descale, bias, round, store, amax.
 __device__ __forceinline__ uint32_t store_chunk(const Args &args, const uint32_t (&r)[32], int row, int col0,
                                                 float inv_a, float inv_b) {
@@ -908,6 +925,9 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     const int q = warp & 3;         // TMEM lane quarter
     const int h = (warp - 2) >> 2;  // accumulator half: 0 or 1
     const float inv_a = *args.inv_a, inv_b = *args.inv_b;
+    const float inv_ab = __fmul_rn(inv_a, inv_b);
+    // one multiplication when the folded factor is a normal float
+    const bool fold = fabsf(inv_ab) >= 1.17549435e-38f && fabsf(inv_ab) <= 3.402823466e38f;
     const uint32_t stg = out_stage0 + (warp - 2) * kWideStageOutBytes;
     const bool f32out = args.out_dtype == FP8_DT_F32;
     const bool bfout = args.out_dtype == FP8_DT_BF16;
@@ -931,7 +951,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         const int col0 = nb * kWideBN + (c < 128 ? 0 : 256) + h * kPairHalf + (c & 127);
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + h * 256 + c, r);
-        descale_chunk(args, r, col0, inv_a, inv_b);
+        if (fold) descale1_chunk(args, r, col0, inv_ab); else descale_chunk(args, r, col0, inv_a, inv_b);
         uint32_t w[32];  // the row's 128 bytes as 32 words
         if (f32out) {
 #pragma unroll
@@ -942,7 +962,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         } else {
           uint32_t r2[32];
           tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + h * 256 + c + 32, r2);
-          descale_chunk(args, r2, col0 + 32, inv_a, inv_b);
+          if (fold) descale1_chunk(args, r2, col0 + 32, inv_ab); else descale_chunk(args, r2, col0 + 32, inv_a, inv_b);
 #pragma unroll
           for (int j = 0; j < 16; j++) {
             const float a0 = __uint_as_float(r[2 * j]), a1 = __uint_as_float(r[2 * j + 1]);
