@@ -37,9 +37,11 @@ SCALINGS = ("auto", "pre", "post")
 
 
 def _group_info(group):
+    """(world, rank, collectives): collectives run whenever a process group
+    exists, a group of one rank included (so its code path is the same)."""
     if dist.is_available() and dist.is_initialized():
-        return dist.get_world_size(group), dist.get_rank(group)
-    return 1, 0
+        return dist.get_world_size(group), dist.get_rank(group), True
+    return 1, 0, False
 
 
 class FP8GradAllReduce:
@@ -57,7 +59,7 @@ class FP8GradAllReduce:
         if scaling not in SCALINGS:
             raise ValueError(f"scaling must be one of {SCALINGS}")
         self.n, self.fmt, self.margin, self.scaling, self.group = n, fmt, margin, scaling, group
-        self.world, self.rank = _group_info(group)
+        self.world, self.rank, self.collectives = _group_info(group)
         self.lo, self.hi = shard_bounds(n, self.world, self.rank)
         groups = -(-n // SHARD_ALIGN)
         self.L = -(-groups // self.world) * SHARD_ALIGN  # slice stride (the last slice may be shorter)
@@ -93,12 +95,12 @@ class FP8GradAllReduce:
             fp8.fp8_amax(g, self.amax)
         else:
             self.amax.copy_(g_amax.reshape(1))
-        if self.world > 1:
+        if self.collectives:
             # amaxes are floats >= 0 (or +NaN): their bit patterns order as int32
             dist.all_reduce(self.amax.view(torch.int32), op=dist.ReduceOp.MAX, group=self.group)
         fp8.fp8_grad_cast(g, self.fmt, self.amax, self.margin, self.mu, self.scalars[1:2], self.scalars[2:3],
                           self.send, self.cast_counts)
-        if self.world > 1:
+        if self.collectives:
             dist.all_to_all_single(self.recv.view(-1), self.send, group=self.group)
             rows = self.recv
         else:
@@ -106,14 +108,14 @@ class FP8GradAllReduce:
         fp8.fp8_sum_codes(rows, self.hi - self.lo, self.fmt, self.out, self.scalars[2:3], self.g_inv,
                           self.sum_counts)
         if self.scaling == "auto":
-            if self.world > 1:
+            if self.collectives:
                 dist.all_reduce(self.sum_counts, op=dist.ReduceOp.SUM, group=self.group)
             fp8.fp8_mu_update(self.mu, self.clean, self.sum_counts, self.n, **self.rule)
         return self.out[:self.hi - self.lo]
 
     def all_gather(self) -> torch.Tensor:
         """The whole summed gradient (n codes at scale S) on every rank."""
-        if self.world == 1:
+        if not self.collectives:
             return self.out[:self.n]
         full = torch.empty(self.world * self.L, dtype=torch.uint8, device=self.out.device)
         dist.all_gather_into_tensor(full, self.out, group=self.group)
@@ -123,7 +125,7 @@ class FP8GradAllReduce:
         """Underflow and overflow counts so far (summed over ranks; a host
         read, for monitoring).  Under "auto" the sum counts restart every step."""
         c = torch.cat([self.cast_counts, self.sum_counts])
-        if self.world > 1:
+        if self.collectives:
             c = c.clone()
             dist.all_reduce(c, op=dist.ReduceOp.SUM, group=self.group)
         c = c.tolist()

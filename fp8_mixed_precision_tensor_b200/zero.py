@@ -81,7 +81,7 @@ class ShardedAdam:
         collective also uses."""
         args = (lr, beta1, beta2, eps, t, margin, self.workspace)
         fp8.fp8_adam_stats(self.chunks, *args, stream=stream)
-        if dist.is_initialized() and dist.get_world_size(self.group) > 1:
+        if dist.is_available() and dist.is_initialized():  # a group of one rank too
             if stream is None:
                 reduce_workspace(self.workspace, self.group)
             else:
