@@ -2,6 +2,7 @@
 
     python -m fp8_mixed_precision_tensor_b200.profile_cases linear --M 4096 --N 16384 --K 4096
     python -m fp8_mixed_precision_tensor_b200.profile_cases cast --n 268435456
+    python -m fp8_mixed_precision_tensor_b200.profile_cases castsweep
     python -m fp8_mixed_precision_tensor_b200.profile_cases adam --n 67108864 [--track]
     python -m fp8_mixed_precision_tensor_b200.profile_cases allreduce --n 268435456 --world 8
     python -m fp8_mixed_precision_tensor_b200.profile_cases castcount --n 268435456
@@ -51,6 +52,13 @@ def case_linear(a):
         fp8.fp8_linear_dgrad(dyq, sc[8:9], wq, sc[5:6], dx, sc[13:14])
         fp8.fp8_linear_wgrad(dyq, sc[8:9], xq, sc[2:3], dw, sc[14:15])
 
+    one()
+    flops = 2.0 * M * N * K
+    for name, fn in (("fwd", lambda: fp8.fp8_linear_fwd(xq, sc[2:3], wq, sc[5:6], y, sc[12:13])),
+                     ("dgrad", lambda: fp8.fp8_linear_dgrad(dyq, sc[8:9], wq, sc[5:6], dx, sc[13:14])),
+                     ("wgrad", lambda: fp8.fp8_linear_wgrad(dyq, sc[8:9], xq, sc[2:3], dw, sc[14:15]))):
+        t = _timed(fn, max(a.iters, 3))
+        print(f"  {name:5s} M{M} N{N} K{K}: {t:.4f} ms, {flops / t / 1e9:.1f} TFLOP/s")
     return one
 
 
@@ -62,6 +70,42 @@ def case_cast(a):
     def one():
         fp8.fp8_amax(x, sc[0:1])
         fp8.fp8_scale_cast(x, fp8.FP8_E4M3, sc[0:1], 0, 1.0, sc[1:2], sc[2:3], q)
+
+    return one
+
+
+def case_castsweep(a):
+    """amax + fused scale/cast of bf16 tensors of 2^20..2^28 elements to E4M3
+    and E5M2, margin 0 and 1: device time per pass from a CUDA-graph replay,
+    GB/s (2 B amax read + 2 B read + 1 B write per element), and the time when
+    the two calls are issued one by one from Python."""
+    big = synth.device_normal((1 << 28,), 1.0, 4, torch.bfloat16, "cuda")
+    qbuf = torch.empty(1 << 28, dtype=torch.uint8, device="cuda")
+    sc = _scalars(3)
+    for e in range(20, 29, 2):
+        n = 1 << e
+        x, q = big[:n], qbuf[:n]
+        for fmt in (fp8.FP8_E4M3, fp8.FP8_E5M2):
+            for margin in (0, 1):
+                def f():
+                    fp8.fp8_amax(x, sc[0:1])
+                    fp8.fp8_scale_cast(x, fmt, sc[0:1], margin, 1.0, sc[1:2], sc[2:3], q)
+                # replay 20 passes captured in a CUDA graph: device time without
+                # the per-call host cost that dominates the small sizes
+                f()
+                torch.cuda.synchronize()
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph):
+                    for _ in range(20):
+                        f()
+                t = _timed(graph.replay, 3) / 20
+                t_host = _timed(f, 20)
+                print(f"  2^{e} fmt {fmt} margin {margin}: {t * 1e3:8.1f} us, {5 * n / t / 1e6:7.0f} GB/s "
+                      f"(graph replay; issued call by call: {t_host * 1e3:.1f} us)")
+
+    def one():
+        fp8.fp8_amax(big, sc[0:1])
+        fp8.fp8_scale_cast(big, fp8.FP8_E4M3, sc[0:1], 0, 1.0, sc[1:2], sc[2:3], qbuf)
 
     return one
 
@@ -200,7 +244,7 @@ def case_adam7b(a):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["linear", "cast", "adam", "allreduce", "castcount", "adam7b"])
+    ap.add_argument("case", choices=["linear", "cast", "castsweep", "adam", "allreduce", "castcount", "adam7b"])
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--N", type=int, default=16384)
     ap.add_argument("--K", type=int, default=4096)
@@ -209,7 +253,8 @@ def main():
     ap.add_argument("--world", type=int, default=8, help="allreduce: emulated ranks")
     ap.add_argument("--track", action="store_true", help="adam: track the master amax across steps")
     a = ap.parse_args()
-    one = {"linear": case_linear, "cast": case_cast, "adam": case_adam, "allreduce": case_allreduce,
+    one = {"linear": case_linear, "cast": case_cast, "castsweep": case_castsweep, "adam": case_adam,
+           "allreduce": case_allreduce,
            "castcount": case_castcount, "adam7b": case_adam7b}[a.case](a)
     one()
     torch.cuda.synchronize()
