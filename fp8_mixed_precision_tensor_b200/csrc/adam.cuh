@@ -78,51 +78,76 @@ struct AdamLaunch {
 // Per-chunk constants of the update: the descales are folded into the Adam
 // coefficients, m = (b1/s_m) m~ + ((1-b1)/(mu s_g)) g~ and
 // v = (b2/s_v) v~ + ((1-b2)/(mu s_g)^2) g~^2, where ~ marks a decoded code.
+// Every factor is held in both lanes of a float2: parameters are updated in
+// pairs with the packed binary32 instructions of sm_100 (two independent
+// round-to-nearest operations per instruction, the same results as the
+// scalar ones at half the issue slots).
 struct AdamScalars {
-  float cm, cgm;  // b1 / s_m,  (1 - b1) g_inv
-  float cv, cgv;  // b2 / s_v,  (1 - b2) g_inv^2
-  float w_inv;    // 1 / s_w
+  float2 cm, cgm;  // b1 / s_m,  (1 - b1) g_inv
+  float2 cv, cgv;  // b2 / s_v,  (1 - b2) g_inv^2
+  float2 w_inv;    // 1 / s_w
 };
 
 __device__ __forceinline__ AdamScalars adam_scalars(const AdamLaunch &L, float g_inv, float m_inv,
                                                     float v_inv, float w_inv) {
   AdamScalars s;
-  s.cm = __fmul_rn(L.beta1, m_inv);
-  s.cgm = __fmul_rn(__fsub_rn(1.0f, L.beta1), g_inv);
-  s.cv = __fmul_rn(L.beta2, v_inv);
-  s.cgv = __fmul_rn(__fmul_rn(__fsub_rn(1.0f, L.beta2), g_inv), g_inv);
-  s.w_inv = w_inv;
+  s.cm = both(__fmul_rn(L.beta1, m_inv));
+  s.cgm = both(__fmul_rn(__fsub_rn(1.0f, L.beta1), g_inv));
+  s.cv = both(__fmul_rn(L.beta2, v_inv));
+  s.cgv = both(__fmul_rn(__fmul_rn(__fsub_rn(1.0f, L.beta2), g_inv), g_inv));
+  s.w_inv = both(w_inv);
   return s;
 }
 
-// Approximate (MUFU) square root and reciprocal: relative error ~1e-7 on the
-// step direction m_hat / (sqrt(v_hat) + eps), which moves the master weight by
-// lr * O(1) -- far below an FP16 ULP of the stored master.
+// Approximate (MUFU) square root and reciprocal, subnormal inputs flushed:
+// relative error ~1e-7 on the step direction m_hat / (sqrt(v_hat) + eps),
+// which moves the master weight by lr * O(1) -- far below an FP16 ULP of the
+// stored master.  The flush changes nothing for eps >= 2^-39: the square root
+// of a subnormal is below 2^-63, under half an ULP of such an eps, and the
+// reciprocal's argument is at least eps.
 __device__ __forceinline__ float sqrt_approx(float x) {
   float r;
-  asm("sqrt.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
   return r;
 }
 __device__ __forceinline__ float rcp_approx(float x) {
   float r;
-  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
   return r;
 }
 
 // The new moments and the master step dw = -lr m_hat / (sqrt(v_hat) + eps)
-// of one parameter, float32, from decoded codes.  Explicit round-to-nearest
-// intrinsics keep every pass on exactly the same operations.
-__device__ __forceinline__ void adam_moments(const AdamLaunch &L, float gd, float md, float vd,
-                                             const AdamScalars &s, float &m, float &v, float &dw) {
-  m = __fmaf_rn(s.cm, md, __fmul_rn(s.cgm, gd));
-  v = __fmaf_rn(s.cv, vd, __fmul_rn(s.cgv, __fmul_rn(gd, gd)));
-  const float denom = __fadd_rn(sqrt_approx(__fmul_rn(v, L.inv_bc2)), L.eps);
-  dw = __fmul_rn(L.neg_lr_bc1, __fmul_rn(m, rcp_approx(denom)));
+// of two parameters, binary32, from decoded codes.  Explicit round-to-nearest
+// operations keep every pass (and the element-wise tail, which runs the same
+// function with one lane unused) on exactly the same arithmetic.
+__device__ __forceinline__ void adam_moments(const AdamLaunch &L, float2 gd, float2 md, float2 vd,
+                                             const AdamScalars &s, float2 &m, float2 &v, float2 &dw) {
+  m = __ffma2_rn(s.cm, md, __fmul2_rn(s.cgm, gd));
+  v = __ffma2_rn(s.cv, vd, __fmul2_rn(s.cgv, __fmul2_rn(gd, gd)));
+  const float2 vh = __fmul2_rn(v, both(L.inv_bc2));
+  const float2 den = __fadd2_rn(make_float2(sqrt_approx(vh.x), sqrt_approx(vh.y)), both(L.eps));
+  dw = __fmul2_rn(both(L.neg_lr_bc1), __fmul2_rn(m, make_float2(rcp_approx(den.x), rcp_approx(den.y))));
 }
 
-// w = w0 + dw as one rounding (the master's new value).
-__device__ __forceinline__ float adam_master(float wd, float dw, const AdamScalars &s) {
-  return __fadd_rn(__fmul_rn(wd, s.w_inv), dw);
+// w = w0 + dw as one rounding per parameter (the master's new value).
+__device__ __forceinline__ float2 adam_master(float2 wd, float2 dw, const AdamScalars &s) {
+  return __fadd2_rn(__fmul2_rn(wd, s.w_inv), dw);
+}
+
+// Running maxima of magnitudes as floats, NaN-propagating: a NaN anywhere
+// leaves the canonical NaN 0x7FFFFFFF, whose bits order above inf, so the
+// finalize stage sees it as a non-finite amax.  acc is >= +0 or that NaN.
+__device__ __forceinline__ float max_abs2(float acc, float2 x) {
+  float r;
+  asm("{\n\t.reg .f32 t0, t1;\n\tabs.f32 t0, %2;\n\tabs.f32 t1, %3;\n\t"
+      "max.NaN.f32 %0, %1, t0, t1;\n\t}"
+      : "=f"(r) : "f"(acc), "f"(x.x), "f"(x.y));
+  return r;
+}
+__device__ __forceinline__ float max_abs1(float acc, float x) {
+  float r;
+  asm("{\n\t.reg .f32 t0;\n\tabs.f32 t0, %2;\n\tmax.NaN.f32 %0, %1, t0;\n\t}" : "=f"(r) : "f"(acc), "f"(x));
+  return r;
 }
 
 __device__ __forceinline__ int find_chunk(const AdamLaunch &L, unsigned long long tile) {
@@ -142,11 +167,11 @@ __device__ __forceinline__ uint32_t ws_flags(const AdamLaunch &L, int ci) {
 }
 
 // Warp-reduce three running maxima and fold them into a chunk's slots.
-__device__ __forceinline__ void flush_max3(const AdamLaunch &L, int ci, int s0, uint32_t a0, int s1,
-                                           uint32_t a1, int s2, uint32_t a2) {
-  a0 = warp_max_u32(a0);
-  a1 = warp_max_u32(a1);
-  a2 = warp_max_u32(a2);
+__device__ __forceinline__ void flush_max3(const AdamLaunch &L, int ci, int s0, float m0, int s1, float m1,
+                                           int s2, float m2) {
+  const uint32_t a0 = warp_max_u32(__float_as_uint(m0));
+  const uint32_t a1 = warp_max_u32(__float_as_uint(m1));
+  const uint32_t a2 = warp_max_u32(__float_as_uint(m2));
   if ((threadIdx.x & 31) == 0) {
     float *ws = L.ws + ci * kAdamWsFloatsPerChunk;
     atomic_max_bits(ws + s0, a0);
@@ -155,14 +180,88 @@ __device__ __forceinline__ void flush_max3(const AdamLaunch &L, int ci, int s0, 
   }
 }
 
+// Per-chunk values of the update pass.
+struct AdamNewScales {
+  float2 m, v, w, wq, inv_w;  // new scales of m, v, w and the E4M3 copy; 1 / new s_w
+};
+
+// One thread's full group of 16 parameters: 16 B of g, 16 B of m, 32 B of v,
+// 32 B of w.  Whether the chunk tracks its master amax and whether the E4M3
+// copy is written are per chunk: the stats passes take them as template
+// arguments (no per-parameter test in the element loop); the update pass,
+// whose extra live values would cost a resident block per SM as separate
+// instantiations, takes them at run time (TRACK = WQ = true, track_rt and
+// wq_rt the chunk's flags).
+template <int PASS, bool TRACK, bool WQ>
+__device__ __forceinline__ void adam_group(const AdamLaunch &L, const AdamChunkDev &C, size_t grp,
+                                           const AdamScalars &sc, const AdamNewScales &ns, float &am, float &av,
+                                           float &aw, bool track_rt = TRACK, bool wq_rt = WQ) {
+  constexpr bool kReadW = PASS != 1 || !TRACK;
+  const bool track = TRACK && track_rt, wq = WQ && wq_rt;
+  const uint4 gq = __ldcs(reinterpret_cast<const uint4 *>(C.g) + grp);
+  const uint4 mq = __ldcs(reinterpret_cast<const uint4 *>(C.m) + grp);
+  const uint4 vq0 = __ldcs(reinterpret_cast<const uint4 *>(C.v) + 2 * grp);
+  const uint4 vq1 = __ldcs(reinterpret_cast<const uint4 *>(C.v) + 2 * grp + 1);
+  uint4 wq0 = make_uint4(0, 0, 0, 0), wq1 = make_uint4(0, 0, 0, 0);
+  if constexpr (kReadW) {
+    wq0 = __ldcs(reinterpret_cast<const uint4 *>(C.w) + 2 * grp);
+    wq1 = __ldcs(reinterpret_cast<const uint4 *>(C.w) + 2 * grp + 1);
+  }
+  const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
+  const uint32_t mw[4] = {mq.x, mq.y, mq.z, mq.w};
+  const uint32_t vw[8] = {vq0.x, vq0.y, vq0.z, vq0.w, vq1.x, vq1.y, vq1.z, vq1.w};
+  const uint32_t ww[8] = {wq0.x, wq0.y, wq0.z, wq0.w, wq1.x, wq1.y, wq1.z, wq1.w};
+  uint32_t mo[4], vo[8], wo[8], qo[4];
+#pragma unroll
+  for (int p = 0; p < 8; p++) {  // pairs of parameters
+    const uint32_t g2 = (gw[p >> 1] >> ((p & 1) * 16)) & 0xffffu;
+    const uint32_t m2 = (mw[p >> 1] >> ((p & 1) * 16)) & 0xffffu;
+    float2 m, v, d;
+    adam_moments(L, dec2<FP8_E5M2>(g2), dec2<FP8_E4M3>(m2), h2f2(vw[p]), sc, m, v, d);
+    if constexpr (PASS == 1) {
+      am = max_abs2(am, m);
+      av = max_abs2(av, v);
+      aw = max_abs2(aw, TRACK ? d : adam_master(h2f2(ww[p]), d, sc));
+    } else if constexpr (PASS == 3) {
+      aw = max_abs2(aw, adam_master(h2f2(ww[p]), d, sc));
+    } else {
+      const float2 w = adam_master(h2f2(ww[p]), d, sc);
+      if (track) aw = max_abs2(aw, w);
+      const float2 ms = __fmul2_rn(m, ns.m), vs = __fmul2_rn(v, ns.v), ws = __fmul2_rn(w, ns.w);
+      const uint32_t mc = enc2<FP8_E4M3>(ms.x, ms.y);
+      if (p & 1) mo[p >> 1] |= mc << 16; else mo[p >> 1] = mc;
+      vo[p] = f16x2(vs.x, vs.y);
+      wo[p] = f16x2(ws.x, ws.y);
+      if (track || wq) {
+        const float2 st = h2f2(wo[p]);  // the stored master (scaled)
+        if (track) am = max_abs2(am, st);
+        if (wq) {
+          // E4M3 copy of the stored master: (h / s_w) * s_q, exact in f32
+          const float2 qs = __fmul2_rn(__fmul2_rn(st, ns.inv_w), ns.wq);
+          const uint32_t qc = enc2<FP8_E4M3>(qs.x, qs.y);
+          if (p & 1) qo[p >> 1] |= qc << 16; else qo[p >> 1] = qc;
+        }
+      }
+    }
+  }
+  if constexpr (PASS == 2) {
+    __stcs(reinterpret_cast<uint4 *>(C.m) + grp, make_uint4(mo[0], mo[1], mo[2], mo[3]));
+    __stcs(reinterpret_cast<uint4 *>(C.v) + 2 * grp, make_uint4(vo[0], vo[1], vo[2], vo[3]));
+    __stcs(reinterpret_cast<uint4 *>(C.v) + 2 * grp + 1, make_uint4(vo[4], vo[5], vo[6], vo[7]));
+    __stcs(reinterpret_cast<uint4 *>(C.w) + 2 * grp, make_uint4(wo[0], wo[1], wo[2], wo[3]));
+    __stcs(reinterpret_cast<uint4 *>(C.w) + 2 * grp + 1, make_uint4(wo[4], wo[5], wo[6], wo[7]));
+    if (wq) __stcs(reinterpret_cast<uint4 *>(C.wq) + grp, make_uint4(qo[0], qo[1], qo[2], qo[3]));
+  }
+}
+
 // PASS 1: stats.  PASS 3: exact master amax of flagged chunks.  PASS 2: update.
 template <int PASS>
 __global__ void __launch_bounds__(kAdamThreads) k_adam(const __grid_constant__ AdamLaunch L) {
-  uint32_t am = 0, av = 0, aw = 0;  // running maxima of the current chunk
+  float am = 0.f, av = 0.f, aw = 0.f;  // running maxima of the current chunk
   int cur = -1;
   bool tracked = false, active = true, want_wq = false;
   AdamScalars sc{};
-  float new_m = 1.f, new_v = 1.f, new_w = 1.f, new_wq = 1.f, inv_new_w = 1.f;
+  AdamNewScales ns{both(1.f), both(1.f), both(1.f), both(1.f), both(1.f)};
 
   for (unsigned long long tile = blockIdx.x; tile < L.total_tiles; tile += gridDim.x) {
     const int ci = find_chunk(L, tile);  // uniform across the block
@@ -174,7 +273,7 @@ __global__ void __launch_bounds__(kAdamThreads) k_adam(const __grid_constant__ A
         if constexpr (PASS == 3)
           if (active) flush_max3(L, cur, WS_AMAX_W, aw, WS_AMAX_W, aw, WS_AMAX_W, aw);
         if constexpr (PASS == 2) flush_max3(L, cur, WS_STORED_W, am, WS_CHECK_W, aw, WS_CHECK_W, aw);
-        am = av = aw = 0;
+        am = av = aw = 0.f;
       }
       cur = ci;
       if constexpr (PASS == 1) {
@@ -188,108 +287,54 @@ __global__ void __launch_bounds__(kAdamThreads) k_adam(const __grid_constant__ A
         active = PASS == 2 || (fl & 1u) != 0;
         sc = adam_scalars(L, *C.g_inv, ws_get(L, ci, WS_OLDINV_M), ws_get(L, ci, WS_OLDINV_V),
                           ws_get(L, ci, WS_OLDINV_W));
-        new_m = ws_get(L, ci, WS_NEW_M);
-        new_v = ws_get(L, ci, WS_NEW_V);
-        new_w = ws_get(L, ci, WS_NEW_W);
-        inv_new_w = 1.0f / new_w;
+        ns.m = both(ws_get(L, ci, WS_NEW_M));
+        ns.v = both(ws_get(L, ci, WS_NEW_V));
+        ns.w = both(ws_get(L, ci, WS_NEW_W));
+        ns.inv_w = both(1.0f / ns.w.x);
         want_wq = C.wq != nullptr;
-        new_wq = want_wq ? ws_get(L, ci, WS_NEW_WQ) : 1.0f;
+        ns.wq = both(want_wq ? ws_get(L, ci, WS_NEW_WQ) : 1.0f);
       }
     }
     if (!active) continue;  // pass 1b: chunk not flagged
-    const bool read_w = PASS != 1 || !tracked;
     const unsigned long long base =
         (tile - C.tile_begin) * kAdamTile + (unsigned long long)threadIdx.x * kAdamPerThread;
     if (base >= C.n) continue;
     if (base + kAdamPerThread <= C.n) {
-      // Full group of 16: 16 B of g, 16 B of m, 32 B of v, 32 B of w.
       const size_t grp = base / kAdamPerThread;
-      uint4 gq = __ldcs(reinterpret_cast<const uint4 *>(C.g) + grp);
-      uint4 mq = __ldcs(reinterpret_cast<const uint4 *>(C.m) + grp);
-      uint4 vq0 = __ldcs(reinterpret_cast<const uint4 *>(C.v) + 2 * grp);
-      uint4 vq1 = __ldcs(reinterpret_cast<const uint4 *>(C.v) + 2 * grp + 1);
-      uint4 wq0 = make_uint4(0, 0, 0, 0), wq1 = make_uint4(0, 0, 0, 0);
-      if (read_w) {
-        wq0 = __ldcs(reinterpret_cast<const uint4 *>(C.w) + 2 * grp);
-        wq1 = __ldcs(reinterpret_cast<const uint4 *>(C.w) + 2 * grp + 1);
-      }
-      const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
-      const uint32_t mw[4] = {mq.x, mq.y, mq.z, mq.w};
-      const uint32_t vw[8] = {vq0.x, vq0.y, vq0.z, vq0.w, vq1.x, vq1.y, vq1.z, vq1.w};
-      const uint32_t ww[8] = {wq0.x, wq0.y, wq0.z, wq0.w, wq1.x, wq1.y, wq1.z, wq1.w};
-      uint32_t mo[4], vo[8], wo[8], qo[4];
-#pragma unroll
-      for (int p = 0; p < 8; p++) {  // pairs of parameters
-        const uint32_t g2 = (gw[p >> 1] >> ((p & 1) * 16)) & 0xffffu;
-        const uint32_t m2 = (mw[p >> 1] >> ((p & 1) * 16)) & 0xffffu;
-        const float2 gd = dec2<FP8_E5M2>(g2), md = dec2<FP8_E4M3>(m2);
-        const float2 vd = h2f2(vw[p]), wd = h2f2(ww[p]);
-        float m_a, v_a, d_a, m_b, v_b, d_b;
-        adam_moments(L, gd.x, md.x, vd.x, sc, m_a, v_a, d_a);
-        adam_moments(L, gd.y, md.y, vd.y, sc, m_b, v_b, d_b);
-        if constexpr (PASS == 1) {
-          am = max(am, max(absbits_f32(m_a), absbits_f32(m_b)));
-          av = max(av, max(absbits_f32(v_a), absbits_f32(v_b)));
-          if (tracked) {
-            aw = max(aw, max(absbits_f32(d_a), absbits_f32(d_b)));
-          } else {
-            aw = max(aw, max(absbits_f32(adam_master(wd.x, d_a, sc)), absbits_f32(adam_master(wd.y, d_b, sc))));
-          }
-        } else if constexpr (PASS == 3) {
-          aw = max(aw, max(absbits_f32(adam_master(wd.x, d_a, sc)), absbits_f32(adam_master(wd.y, d_b, sc))));
-        } else {
-          const float w_a = adam_master(wd.x, d_a, sc), w_b = adam_master(wd.y, d_b, sc);
-          if (tracked) aw = max(aw, max(absbits_f32(w_a), absbits_f32(w_b)));
-          const uint32_t mc = enc2<FP8_E4M3>(__fmul_rn(m_a, new_m), __fmul_rn(m_b, new_m));
-          if (p & 1) mo[p >> 1] |= mc << 16; else mo[p >> 1] = mc;
-          vo[p] = f16x2(__fmul_rn(v_a, new_v), __fmul_rn(v_b, new_v));
-          wo[p] = f16x2(__fmul_rn(w_a, new_w), __fmul_rn(w_b, new_w));
-          if (tracked) {  // amax of the stored master (scaled), for the tracked value
-            const uint32_t h = __vmaxu2(wo[p] & 0x7fff7fffu, 0u);
-            am = max(am, absbits_f32(__half2float(__ushort_as_half((unsigned short)max(h & 0xffffu, h >> 16)))));
-          }
-          if (want_wq) {
-            const float2 st = h2f2(wo[p]);  // the stored master (scaled)
-            // E4M3 copy of the stored master: (h / s_w) * s_q, exact in f32
-            const uint32_t qc = enc2<FP8_E4M3>(__fmul_rn(__fmul_rn(st.x, inv_new_w), new_wq),
-                                               __fmul_rn(__fmul_rn(st.y, inv_new_w), new_wq));
-            if (p & 1) qo[p >> 1] |= qc << 16; else qo[p >> 1] = qc;
-          }
-        }
-      }
-      if constexpr (PASS == 2) {
-        __stcs(reinterpret_cast<uint4 *>(C.m) + grp, make_uint4(mo[0], mo[1], mo[2], mo[3]));
-        __stcs(reinterpret_cast<uint4 *>(C.v) + 2 * grp, make_uint4(vo[0], vo[1], vo[2], vo[3]));
-        __stcs(reinterpret_cast<uint4 *>(C.v) + 2 * grp + 1, make_uint4(vo[4], vo[5], vo[6], vo[7]));
-        __stcs(reinterpret_cast<uint4 *>(C.w) + 2 * grp, make_uint4(wo[0], wo[1], wo[2], wo[3]));
-        __stcs(reinterpret_cast<uint4 *>(C.w) + 2 * grp + 1, make_uint4(wo[4], wo[5], wo[6], wo[7]));
-        if (want_wq) __stcs(reinterpret_cast<uint4 *>(C.wq) + grp, make_uint4(qo[0], qo[1], qo[2], qo[3]));
+      if constexpr (PASS == 1) {
+        if (tracked) adam_group<1, true, false>(L, C, grp, sc, ns, am, av, aw);
+        else adam_group<1, false, false>(L, C, grp, sc, ns, am, av, aw);
+      } else if constexpr (PASS == 3) {
+        adam_group<3, false, false>(L, C, grp, sc, ns, am, av, aw);
+      } else {
+        adam_group<2, true, true>(L, C, grp, sc, ns, am, av, aw, tracked, want_wq);
       }
     } else {
-      // Ragged end of a chunk: element by element.
+      // Ragged end of a chunk: element by element (lane y unused).
+      const bool read_w = PASS != 1 || !tracked;
       for (unsigned long long i = base; i < C.n; i++) {
-        const float gd = dec2<FP8_E5M2>(C.g[i]).x, md = dec2<FP8_E4M3>(C.m[i]).x;
-        const float vd = __half2float(__ushort_as_half(C.v[i]));
-        const float wd = read_w ? __half2float(__ushort_as_half(C.w[i])) : 0.0f;
-        float m, v, d;
-        adam_moments(L, gd, md, vd, sc, m, v, d);
+        const float2 gd = dec2<FP8_E5M2>(C.g[i]), md = dec2<FP8_E4M3>(C.m[i]);
+        const float2 vd = make_float2(__half2float(__ushort_as_half(C.v[i])), 0.0f);
+        const float2 wd = make_float2(read_w ? __half2float(__ushort_as_half(C.w[i])) : 0.0f, 0.0f);
+        float2 m, v, d;
+        adam_moments(L, make_float2(gd.x, 0.0f), make_float2(md.x, 0.0f), vd, sc, m, v, d);
         if constexpr (PASS == 1) {
-          am = max(am, absbits_f32(m));
-          av = max(av, absbits_f32(v));
-          aw = max(aw, tracked ? absbits_f32(d) : absbits_f32(adam_master(wd, d, sc)));
+          am = max_abs1(am, m.x);
+          av = max_abs1(av, v.x);
+          aw = max_abs1(aw, tracked ? d.x : adam_master(wd, d, sc).x);
         } else if constexpr (PASS == 3) {
-          aw = max(aw, absbits_f32(adam_master(wd, d, sc)));
+          aw = max_abs1(aw, adam_master(wd, d, sc).x);
         } else {
-          const float w = adam_master(wd, d, sc);
-          if (tracked) aw = max(aw, absbits_f32(w));
-          C.m[i] = (uint8_t)(enc2<FP8_E4M3>(__fmul_rn(m, new_m), 0.0f) & 0xffu);
-          C.v[i] = __half_as_ushort(__float2half_rn(__fmul_rn(v, new_v)));
-          const __half h = __float2half_rn(__fmul_rn(w, new_w));
+          const float w = adam_master(wd, d, sc).x;
+          if (tracked) aw = max_abs1(aw, w);
+          C.m[i] = (uint8_t)(enc2<FP8_E4M3>(__fmul_rn(m.x, ns.m.x), 0.0f) & 0xffu);
+          C.v[i] = __half_as_ushort(__float2half_rn(__fmul_rn(v.x, ns.v.x)));
+          const __half h = __float2half_rn(__fmul_rn(w, ns.w.x));
           C.w[i] = __half_as_ushort(h);
           const float st = __half2float(h);
-          if (tracked) am = max(am, absbits_f32(st));
+          if (tracked) am = max_abs1(am, st);
           if (want_wq)
-            C.wq[i] = (uint8_t)(enc2<FP8_E4M3>(__fmul_rn(__fmul_rn(st, inv_new_w), new_wq), 0.0f) & 0xffu);
+            C.wq[i] = (uint8_t)(enc2<FP8_E4M3>(__fmul_rn(__fmul_rn(st, ns.inv_w.x), ns.wq.x), 0.0f) & 0xffu);
         }
       }
     }

@@ -131,6 +131,11 @@ __device__ __forceinline__ float2 h2f2(uint32_t two_halves) {
   return __half22float2(*reinterpret_cast<__half2 *>(&two_halves));
 }
 
+// A factor in both lanes of a float2, for the packed binary32 instructions
+// of sm_100 (__fmul2_rn and friends: two round-to-nearest results per
+// instruction, each the same as the scalar operation's).
+__device__ __forceinline__ float2 both(float a) { return make_float2(a, a); }
+
 // ---------------------------------------------------------------------------
 // Magnitude of an element as the bit pattern of a binary32 (order-preserving
 // for non-negative values, NaN above inf), so maxima can use integer max.

@@ -27,7 +27,8 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   bool ready = false;
   int sms = 0;
-  int adam_blocks_per_sm = 1;
+  int adam_blocks_per_sm = 1;        // resident blocks of the update pass
+  int adam_stats_blocks_per_sm = 1;  // of the stats passes (fewer registers)
   int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair GEMM
   int wide_clusters = 0;  // co-resident 2-CTA clusters of the wide pair GEMM
 };
@@ -63,6 +64,9 @@ int device_info(DeviceInfo **out) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k_adam<2>, kAdamThreads, 0) != cudaSuccess)
       return FP8_ERR_CUDA;
     d.adam_blocks_per_sm = bps > 0 ? bps : 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k_adam<1>, kAdamThreads, 0) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    d.adam_stats_blocks_per_sm = bps > 0 ? bps : 1;
     int rc = FP8_OK;
     rc |= set_smem(gemm::k_gemm<256, false, false>, gemm::Cfg<256>::SMEM_BYTES);
     rc |= set_smem(gemm::k_gemm<256, false, true>, gemm::Cfg<256>::SMEM_BYTES);
@@ -461,6 +465,7 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
   L.neg_lr_bc1 = (float)(-(double)hp->lr / (1.0 - pow((double)hp->beta1, (double)hp->step)));
   L.inv_bc2 = (float)(1.0 / (1.0 - pow((double)hp->beta2, (double)hp->step)));
   const unsigned cap = (unsigned)(d->sms * d->adam_blocks_per_sm);
+  const unsigned cap1 = (unsigned)(d->sms * d->adam_stats_blocks_per_sm);
   for (int first = 0; first < nchunks; first += kAdamMaxChunksPerLaunch) {
     const int cnt = nchunks - first < kAdamMaxChunksPerLaunch ? nchunks - first : kAdamMaxChunksPerLaunch;
     unsigned long long tiles = 0;
@@ -478,13 +483,14 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
     L.total_tiles = tiles;
     L.ws = reinterpret_cast<float *>(workspace) + (size_t)first * kAdamWsFloatsPerChunk;
     const unsigned grid = tiles == 0 ? 1u : (unsigned)(tiles < cap ? tiles : cap);
+    const unsigned grid1 = tiles == 0 ? 1u : (unsigned)(tiles < cap1 ? tiles : cap1);
     bool tracked = false;
     for (int i = 0; i < cnt; i++) tracked |= L.c[i].w_amax != nullptr;
-    if (phases & PH_STATS) k_adam<1><<<grid, kAdamThreads, 0, s>>>(L);  // stats
+    if (phases & PH_STATS) k_adam<1><<<grid1, kAdamThreads, 0, s>>>(L);  // stats
     if (phases & PH_APPLY) {
       if (tracked) {
         k_adam_finalize<1><<<1, 256, 0, s>>>(L);
-        k_adam<3><<<grid, kAdamThreads, 0, s>>>(L);  // exact master amax, flagged chunks only
+        k_adam<3><<<grid1, kAdamThreads, 0, s>>>(L);  // exact master amax, flagged chunks only
         k_adam_finalize<2><<<1, 256, 0, s>>>(L);
       } else {
         k_adam_finalize<12><<<1, 256, 0, s>>>(L);
