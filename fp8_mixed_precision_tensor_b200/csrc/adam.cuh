@@ -77,14 +77,19 @@ struct AdamLaunch {
 
 // Per-chunk constants of the update: the descales are folded into the Adam
 // coefficients, m = (b1/s_m) m~ + ((1-b1)/(mu s_g)) g~ and
-// v = (b2/s_v) v~ + ((1-b2)/(mu s_g)^2) g~^2, where ~ marks a decoded code.
+// v = (b2/s_v) v~ + ((1-b2)/(mu s_g)) g~ * (1/(mu s_g)) g~, where ~ marks a
+// decoded code.  The gradient descale enters v once per factor, never
+// squared: (1-b2)/(mu s_g)^2 underflows binary32 once the gradient's amax is
+// below ~1e-17 (mu s_g above 2^72), while each factor stays a normal number
+// and only the product, the new v itself, can be subnormal.
 // Every factor is held in both lanes of a float2: parameters are updated in
 // pairs with the packed binary32 instructions of sm_100 (two independent
 // round-to-nearest operations per instruction, the same results as the
 // scalar ones at half the issue slots).
 struct AdamScalars {
   float2 cm, cgm;  // b1 / s_m,  (1 - b1) g_inv
-  float2 cv, cgv;  // b2 / s_v,  (1 - b2) g_inv^2
+  float2 cv, cgv;  // b2 / s_v,  (1 - b2) g_inv
+  float2 g_inv;    // 1 / (mu s_g)
   float2 w_inv;    // 1 / s_w
 };
 
@@ -94,7 +99,8 @@ __device__ __forceinline__ AdamScalars adam_scalars(const AdamLaunch &L, float g
   s.cm = both(__fmul_rn(L.beta1, m_inv));
   s.cgm = both(__fmul_rn(__fsub_rn(1.0f, L.beta1), g_inv));
   s.cv = both(__fmul_rn(L.beta2, v_inv));
-  s.cgv = both(__fmul_rn(__fmul_rn(__fsub_rn(1.0f, L.beta2), g_inv), g_inv));
+  s.cgv = both(__fmul_rn(__fsub_rn(1.0f, L.beta2), g_inv));
+  s.g_inv = both(g_inv);
   s.w_inv = both(w_inv);
   return s;
 }
@@ -123,7 +129,7 @@ __device__ __forceinline__ float rcp_approx(float x) {
 __device__ __forceinline__ void adam_moments(const AdamLaunch &L, float2 gd, float2 md, float2 vd,
                                              const AdamScalars &s, float2 &m, float2 &v, float2 &dw) {
   m = __ffma2_rn(s.cm, md, __fmul2_rn(s.cgm, gd));
-  v = __ffma2_rn(s.cv, vd, __fmul2_rn(s.cgv, __fmul2_rn(gd, gd)));
+  v = __ffma2_rn(s.cv, vd, __fmul2_rn(__fmul2_rn(s.cgv, gd), __fmul2_rn(s.g_inv, gd)));
   const float2 vh = __fmul2_rn(v, both(L.inv_bc2));
   const float2 den = __fadd2_rn(make_float2(sqrt_approx(vh.x), sqrt_approx(vh.y)), both(L.eps));
   dw = __fmul2_rn(both(L.neg_lr_bc1), __fmul2_rn(m, make_float2(rcp_approx(den.x), rcp_approx(den.y))));
@@ -254,9 +260,10 @@ __device__ __forceinline__ void adam_group(const AdamLaunch &L, const AdamChunkD
   }
 }
 
-// PASS 1: stats.  PASS 3: exact master amax of flagged chunks.  PASS 2: update.
+// One pass over all tiles of a launch.  PASS 1: stats.  PASS 3: exact master
+// amax of flagged chunks.  PASS 2: update.
 template <int PASS>
-__global__ void __launch_bounds__(kAdamThreads) k_adam(const __grid_constant__ AdamLaunch L) {
+__device__ __forceinline__ void adam_pass(const AdamLaunch &L) {
   float am = 0.f, av = 0.f, aw = 0.f;  // running maxima of the current chunk
   int cur = -1;
   bool tracked = false, active = true, want_wq = false;
@@ -347,6 +354,17 @@ __global__ void __launch_bounds__(kAdamThreads) k_adam(const __grid_constant__ A
       if (active) flush_max3(L, cur, WS_AMAX_W, aw, WS_AMAX_W, aw, WS_AMAX_W, aw);
     if constexpr (PASS == 2) flush_max3(L, cur, WS_STORED_W, am, WS_CHECK_W, aw, WS_CHECK_W, aw);
   }
+}
+
+template <int PASS>
+__global__ void __launch_bounds__(kAdamThreads) k_adam(const __grid_constant__ AdamLaunch L) {
+  adam_pass<PASS>(L);
+}
+// The update pass, latency-bound on its loads, is held to 48 registers: five
+// resident blocks per SM instead of four keep more loads in flight.
+template <>
+__global__ void __launch_bounds__(kAdamThreads, 5) k_adam<2>(const __grid_constant__ AdamLaunch L) {
+  adam_pass<2>(L);
 }
 
 // Exponent of the E4M3 copy's scale from an amax of the stored master: the

@@ -351,12 +351,13 @@ def test_gemm_empty_rows_writes_zero_amax():
 HP = dict(lr=1e-4, beta1=0.9, beta2=0.95, eps=1e-8)
 
 
-def make_adam_state(sizes, key, steps_done=0):
+def make_adam_state(sizes, key, steps_done=0, g_host=None):
     """Per chunk: E5M2 grads (mu = 2^10) and a stored state built by the GPU
-    cast chain from seeded fp32 tensors (zero moments when steps_done == 0)."""
+    cast chain from seeded fp32 tensors (zero moments when steps_done == 0).
+    The fp32 gradients are ~N(0, 1e-3), or g_host[ci] when given."""
     chunks, host = [], []
     for ci, n in enumerate(sizes):
-        gf = synth.adam_grad_f32(n, 1e-3, *key, ci, "g")
+        gf = synth.adam_grad_f32(n, 1e-3, *key, ci, "g") if g_host is None else g_host[ci]
         wf = synth.normal_f32((n,), 0.02, *key, ci, "w")
         st = {}
         for name, arr, fmt, mu in (("g", gf, fp8.FP8_E5M2, 2.0 ** 10), ("w", wf, fp8.FP8_F16S, 1.0)):
@@ -436,6 +437,28 @@ def test_adam_step_vs_oracle(sizes, steps_done):
     for b, c in zip(before, chunks):
         if b["g"].size:
             check_adam_chunk(b, c, step)
+
+
+def test_adam_subnormal_second_moment():
+    """Gradients of magnitude in [2^-66, 2^-65): the new second moment
+    (1 - beta2) g^2 lies in [2^-136.3, 2^-134.3), a binary32 subnormal, and
+    its scale is the clamped 2^126.  The codes and scales match the oracle, so
+    the packed multiply-adds keep subnormals (flushed, v would be 0 with scale
+    1); the step matches, so the flush-to-zero square root changes nothing
+    (sqrt(v_hat) ~ 2^-66 is far below half an ULP of eps = 1e-8).  The stored
+    v * 2^126 lies in [2^-10.3, 2^-8.3), where binary32's subnormal spacing
+    (2^-149, i.e. 2^-23 after scaling) is far below an FP16 ULP."""
+    n = 65536 + 3
+    g = synth.rng("adam-subnormal", "g")
+    gf = (np.where(g.random(n) < 0.5, -1.0, 1.0) * 2.0 ** -66 * (1.0 + g.random(n))).astype(np.float32)
+    chunks = make_adam_state([n], ("adam-subnormal",), g_host=[gf])
+    ws = torch.zeros(fp8.fp8_adam_workspace_bytes(1) // 4, **F32)
+    before = snapshot(chunks[0])
+    fp8.fp8_adam_step(chunks, step=1, margin=0, workspace=ws, **HP)
+    assert fp8.fp8_get_status() == 0
+    out = check_adam_chunk(before, chunks[0], 1)
+    assert 0.0 < out["amax"][1] < 2.0 ** -126  # the oracle's new amax(v) is subnormal
+    assert snapshot(chunks[0])["s_v"] == 2.0 ** 126  # its scale, clamped
 
 
 def test_adam_three_steps_stage_parity():
