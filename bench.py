@@ -1,22 +1,28 @@
 """Benchmark of the FP8 mixed-precision training hot path on B200.
 
-One step = one pass of the whole path over one batch of the GPT-7B
-transformer block's four linears (tokens 4096 = batch 2 x seq 2048, hidden
-4096: QKV 4096->12288, out-proj 4096->4096, FFN 4096->16384->4096):
+One step = one pass of the whole path over one batch of a transformer
+block's four linears.  The default workload is the GPT-175B block (tokens
+8192 = batch 4 x seq 2048, hidden 12288: QKV 12288->36864, out-proj
+12288->12288, FFN 12288->49152->12288); `--workload gpt7b_block` runs the
+GPT-7B block (tokens 4096, hidden 4096).  Per step:
 
-  for each linear:  amax/scale/cast X (E4M3), W (E4M3), dY (E5M2, mu-scaled)
-                    fwd   Y  = Xq Wq^T     (bf16 out, fused amax)
-                    dgrad dX = dYq Wq      (bf16 out, fused amax)
+  for each linear:  amax + fused scale/cast of X (E4M3) and dY (E5M2, mu-scaled)
+                    fwd   Y  = Xq Wq^T     (bf16 out, fused next-amax)
+                    dgrad dX = dYq Wq      (bf16 out, fused next-amax)
                     wgrad dW = dYq^T Xq    (fp32 out, fused amax)
                     grad  gq = E5M2(mu s_g dW)
-  then one precision-decoupled FP8 Adam step over the 4 weight tensors
-  (201,326,592 parameters: E5M2 grad, E4M3 m1, FP16 m2, FP16 master).
+  then the precision-decoupled FP8 Adam step over the 4 weight tensors
+  (E5M2 grad, E4M3 m1, FP16 m2, FP16 master; 1,811,939,328 parameters for
+  GPT-175B), which also writes the E4M3 copy of each new master: the next
+  step's forward and dgrad read the weight from that copy, so no weight cast
+  runs in the step.  The master's amax is tracked between steps.
 
-`value` is the step's algorithmic GEMM work (3 x 2MNK per linear, 4.948
-TFLOP) divided by the device time of the whole step, inputs resident in HBM.
-Inputs are seeded synthetic tensors (bf16 activations ~N(0,1), weights
-~N(0,0.02), output gradients ~N(0,1e-4)); every step touches several GB, far
-more than the 126 MB L2, so no explicit L2 flush is needed between steps.
+`value` is the step's algorithmic GEMM work (3 x 2MNK per linear; 89.06 TFLOP
+for GPT-175B) divided by the device time of the whole step, inputs resident
+in HBM.  Inputs are seeded synthetic tensors (bf16 activations ~N(0,1),
+weights ~N(0,0.006) for GPT-175B / N(0,0.02) for GPT-7B, output gradients
+~N(0,1e-4)); every step touches tens of GB, far more than the 126 MB L2, so no
+explicit L2 flush is needed between steps.
 
 End to end (`e2e`), each step's X and dY come from pinned host memory and
 its result scalars go back; with the overlapped schedule the next step's
@@ -30,7 +36,8 @@ the work in order on one stream.  The per-kernel breakdown
 (`kernels`, `roofline`) always comes from a serial pass with CUDA events
 around each phase.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--schedule serial]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload gpt175b_block|gpt7b_block] [--schedule serial]
 """
 from __future__ import annotations
 
@@ -51,7 +58,12 @@ import torch  # noqa: E402
 from fp8_mixed_precision_tensor_b200 import synth  # noqa: E402
 
 METRIC = "FP8 linear fwd+bwd TFLOP/s (% FP8 peak); cast & Adam GB/s (% HBM peak)"
-WORKLOAD = "gpt7b_block_linears_fp8_train_step"
+WORKLOADS = {
+    "gpt175b_block": dict(workload="gpt175b_block_linears_fp8_train_step", linears=synth.GPT175B_LINEARS,
+                          tokens=synth.GPT175B_TOKENS, hidden=12288, w_std=synth.GPT175B_W_STD),
+    "gpt7b_block": dict(workload="gpt7b_block_linears_fp8_train_step", linears=synth.GPT7B_LINEARS,
+                        tokens=synth.GPT7B_TOKENS, hidden=4096, w_std=synth.GPT7B_W_STD),
+}
 MU = 2.0 ** 10
 HP = dict(lr=1e-4, beta1=0.9, beta2=0.95, eps=1e-8)
 # Algorithmic bytes per element / parameter (reads + writes of the definition).
@@ -60,15 +72,26 @@ GRAD_CAST_BYTES = 4 + 1       # fp32 dW read (amax fused in the GEMM) + code wri
 ADAM_BYTES = 11               # read g1 m1 v2 w2, write m1 v2 w2
 
 
-def gemm_traffic():
+def config_of(wl: dict, schedule: str, world: int) -> dict:
+    """The `config` object of the JSON line (the same for both arms)."""
+    flops = sum(3 * 2 * wl["tokens"] * N * K for _, K, N in wl["linears"])
+    return {"workload": wl["workload"], "tokens": wl["tokens"], "hidden": wl["hidden"],
+            "linears": [l[0] for l in wl["linears"]], "adam_params": sum(N * K for _, K, N in wl["linears"]),
+            "gemm_flops_per_step": flops, "l2": "inputs larger than L2 (no flush)", "schedule": schedule,
+            "weight_operand": "E4M3 copy written by the previous Adam step", "master_amax": "tracked",
+            "parallelism": f"replicas{world}" if world > 1 else "single"}
+
+
+def gemm_traffic(workload: str):
     """Mean DRAM bytes per GEMM launch of this step from the committed ncu
-    capture, valid while the GEMM kernel source is the one that was measured."""
+    capture, valid while the GEMM kernel source is the one that was measured
+    and the capture is of this workload."""
     import hashlib
 
     try:
         rec = json.load(open(os.path.join(ROOT, "profiles", "gemm_step_traffic.json")))
         src = open(os.path.join(ROOT, "fp8_mixed_precision_tensor_b200", "csrc", "gemm.cuh"), "rb").read()
-        if hashlib.sha256(src).hexdigest() == rec["gemm_source_sha256"]:
+        if hashlib.sha256(src).hexdigest() == rec["gemm_source_sha256"] and rec.get("workload") == workload:
             return rec["dram_bytes_per_launch_mean"]
     except Exception:
         pass
@@ -83,6 +106,19 @@ def load_peaks():
                     src="measured")
     except Exception:
         return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def fp8_peak(peaks: dict, clocks: dict):
+    """Dense FP8 peak = 2 x the bf16 peak (the nominal 4.5 / 2.25 ratio).  The
+    burst figure when the timed region ran at the maximum SM clock (within
+    3 %), else the sustained one (measured under the power cap at a lower
+    clock).  Returns (peak TFLOP/s, source text)."""
+    mhz, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    if mhz is not None and mx and mhz < 0.97 * mx:
+        return 2.0 * peaks["bf16_sus"], (f"2 x bf16_tflops_sustained ({peaks['src']}): median SM clock "
+                                         f"{mhz} MHz below the {mx} MHz maximum")
+    return 2.0 * peaks["bf16"], (f"2 x bf16_tflops, burst ({peaks['src']}): median SM clock {mhz} MHz "
+                                 f"of {mx} MHz maximum")
 
 
 # ---------------------------------------------------------------- clocks
@@ -144,17 +180,21 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- the step
-class Block7BStep:
-    """Device buffers and the launch sequence of one training step."""
+class BlockStep:
+    """Device buffers and the launch sequence of one training step over a
+    block's linears.  The weights exist in bf16 only at set-up: they seed the
+    FP16 masters (the Adam state) and the first E4M3 weight operands; from
+    then on each step's Adam writes the next step's E4M3 weights."""
 
-    def __init__(self, device, seed: int = 0, linears=None, tokens=None, w_std=None):
+    def __init__(self, device, seed: int = 0, workload: str = "gpt175b_block"):
         from fp8_mixed_precision_tensor_b200 import fp8
 
+        wl = WORKLOADS[workload]
         self.fp8 = fp8
         self.dev = device
-        self.linears = linears or synth.GPT7B_LINEARS
-        self.M = tokens or synth.GPT7B_TOKENS
-        w_std = w_std or synth.GPT7B_W_STD
+        self.wl = wl
+        self.linears = wl["linears"]
+        self.M = wl["tokens"]
         f32 = dict(dtype=torch.float32, device=device)
         u8 = dict(dtype=torch.uint8, device=device)
         self.L = []
@@ -162,42 +202,45 @@ class Block7BStep:
             M = self.M
             d = dict(name=name, M=M, N=N, K=K)
             d["X"] = synth.device_normal((M, K), synth.ACT_STD, seed * 1000 + 10 * li + 1, torch.bfloat16, device)
-            d["W"] = synth.device_normal((N, K), w_std, seed * 1000 + 10 * li + 2, torch.bfloat16, device)
             d["dY"] = synth.device_normal((M, N), synth.GRAD_STD, seed * 1000 + 10 * li + 3, torch.bfloat16, device)
             d["xq"], d["wq"], d["dyq"] = (torch.empty(s, **u8) for s in ((M, K), (N, K), (M, N)))
             d["y"] = torch.empty((M, N), dtype=torch.bfloat16, device=device)
             d["dx"] = torch.empty((M, K), dtype=torch.bfloat16, device=device)
             d["dw"] = torch.empty((N, K), **f32)
             d["gq"] = torch.empty((N, K), **u8)
-            # scalars: amax, scale, inv for x, w, dy, g; fused amaxes of y, dx, dw
+            # scalars: amax/scale/inv of x (0-2), w (3-5: the E4M3 weight's, rewritten by
+            # Adam), dy (6-8); g scale and inverse (10, 11); fused amaxes of y, dx, dw (12-14)
             d["sc"] = torch.zeros(16, **f32)
-            # Adam state: master from W (tensor-scaled FP16), zero moments
+            # Adam state: master from W (tensor-scaled FP16), zero moments, tracked master amax
             d["m"] = torch.zeros((N, K), **u8)
             d["v"] = torch.zeros((N, K), dtype=torch.int16, device=device)
             d["wh"] = torch.empty((N, K), dtype=torch.int16, device=device)
-            d["st"] = torch.ones(4, **f32)  # m_scale, v_scale, w_scale, spare
-            tmp = torch.zeros(3, **f32)
-            fp8.fp8_amax(d["W"], tmp[0:1])
-            fp8.fp8_compute_scale(tmp[0:1], fp8.FP8_F16S, 0, 1.0, d["st"][2:3], tmp[1:2])
-            fp8.fp8_cast(d["W"], fp8.FP8_F16S, d["st"][2:3], d["wh"])
+            d["st"] = torch.ones(4, **f32)  # m_scale, v_scale, w_scale, tracked master amax
+            d["st"][3] = -1.0
+            W = synth.device_normal((N, K), wl["w_std"], seed * 1000 + 10 * li + 2, torch.bfloat16, device)
+            tmp = torch.zeros(2, **f32)
+            fp8.fp8_amax(W, tmp[0:1])
+            fp8.fp8_scale_cast(W, fp8.FP8_F16S, tmp[0:1], 0, 1.0, d["st"][2:3], tmp[1:2], d["wh"])
+            self.quantise(W, fp8.FP8_E4M3, d["sc"], 3, out=d["wq"])
+            del W
             self.L.append(d)
-        self.chunks = fp8.pack_adam_chunks([
-            fp8.AdamChunk(d["gq"], d["sc"][11:12], d["m"], d["st"][0:1], d["v"], d["st"][1:2], d["wh"],
-                          d["st"][2:3]) for d in self.L])
+        self.chunk_list = [fp8.AdamChunk(d["gq"], d["sc"][11:12], d["m"], d["st"][0:1], d["v"], d["st"][1:2],
+                                         d["wh"], d["st"][2:3], d["st"][3:4], d["wq"], d["sc"][4:5], d["sc"][5:6])
+                           for d in self.L]
+        self.chunks = fp8.pack_adam_chunks(self.chunk_list)
         self.ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(self.L)) // 4 + 64, **f32)
         # one Adam call per tensor (overlapped schedule): own chunk array and a
         # 256-byte-aligned workspace slice each
-        self.chunks_each = [fp8.pack_adam_chunks([
-            fp8.AdamChunk(d["gq"], d["sc"][11:12], d["m"], d["st"][0:1], d["v"], d["st"][1:2], d["wh"],
-                          d["st"][2:3])]) for d in self.L]
+        self.chunks_each = [fp8.pack_adam_chunks([c]) for c in self.chunk_list]
         self.ws_each = torch.zeros(64 * len(self.L), **f32)
         self.t = 0
         self.flops = sum(3 * 2 * d["M"] * d["N"] * d["K"] for d in self.L)
-        self.cast_elems = sum(d["M"] * d["K"] + d["N"] * d["K"] + d["M"] * d["N"] for d in self.L)
+        self.cast_elems = sum(d["M"] * d["K"] + d["M"] * d["N"] for d in self.L)
         self.params = sum(d["N"] * d["K"] for d in self.L)
-        # (amax, scale+cast) x3, GEMMs, grad scale+cast per linear; Adam (3 launches per call)
-        self.launches_per_step = 4 * (3 * 2 + 3 + 1) + 3
-        self.launches_per_step_overlapped = 4 * (3 * 2 + 3 + 1 + 3)
+        # per linear: (amax, scale+cast) x2, 3 GEMMs, grad scale+cast; Adam with a tracked
+        # master: stats, finalize 1, exact-master pass, finalize 2, update, finalize 3
+        self.launches_per_step = 4 * (2 * 2 + 3 + 1) + 6
+        self.launches_per_step_overlapped = 4 * (2 * 2 + 3 + 1 + 6)
 
     def quantise(self, x, fmt, sc, i, mu=1.0, out=None):
         fp8 = self.fp8
@@ -205,8 +248,9 @@ class Block7BStep:
         fp8.fp8_scale_cast(x, fmt, sc[i:i + 1], 0, mu, sc[i + 1:i + 2], sc[i + 2:i + 3], out)
 
     def step(self, ev=None):
-        """Enqueue one step.  ev: optional dict name -> list of (start, end)
-        events recorded around the GEMM / cast / Adam launches."""
+        """Enqueue one step on the current stream.  ev: optional dict name ->
+        list of (start, end) events recorded around the GEMM / cast / Adam
+        launches."""
         fp8 = self.fp8
 
         def mark(kind):
@@ -221,7 +265,6 @@ class Block7BStep:
             sc = d["sc"]
             e = mark("cast")
             self.quantise(d["X"], fp8.FP8_E4M3, sc, 0, out=d["xq"])
-            self.quantise(d["W"], fp8.FP8_E4M3, sc, 3, out=d["wq"])
             self.quantise(d["dY"], fp8.FP8_E5M2, sc, 6, mu=MU, out=d["dyq"])
             if e: e[1].record()
             e = mark("gemm")
@@ -245,40 +288,44 @@ class Block7BStep:
         cast and that tensor's Adam step on an auxiliary stream (one GEMM's
         last wave overlaps the next GEMM; each tensor's optimizer step
         overlaps the following linears' GEMMs -- Adam is per tensor, so one
-        call per tensor computes exactly what one call over all does).  Every
-        buffer of a step is written once, and the next step's casts start
-        only after this step's last Adam (the cast stream waits for an event
-        recorded at the start of the next step on the current stream, which
-        has joined the auxiliary stream)."""
+        call per tensor computes exactly what one call over all does).  A
+        tensor's Adam rewrites its E4M3 weight, so it also waits for that
+        linear's dgrad, the weight's last reader in the step.  Every buffer of
+        a step is written once, and the next step's casts start only after
+        this step's last Adam (the cast stream waits for an event recorded at
+        the start of the next step on the current stream, which has joined the
+        auxiliary stream)."""
         fp8 = self.fp8
         main = torch.cuda.current_stream()
         if not hasattr(self, "s_cast"):
             self.s_cast, self.s_aux = torch.cuda.Stream(self.dev), torch.cuda.Stream(self.dev)
             self.ev_start = torch.cuda.Event()
-            self.ev_cast = [torch.cuda.Event() for _ in self.L]     # X, W and dY cast
-            self.ev_cast_xw = [torch.cuda.Event() for _ in self.L]  # X and W cast (enough for fwd)
+            self.ev_cast = [torch.cuda.Event() for _ in self.L]    # X and dY cast
+            self.ev_cast_x = [torch.cuda.Event() for _ in self.L]  # X cast (enough for fwd)
+            self.ev_dgrad = [torch.cuda.Event() for _ in self.L]   # the weight's last reader done
             self.ev_grad = torch.cuda.Event()
         self.ev_start.record(main)
         self.s_cast.wait_event(self.ev_start)
         self.s_aux.wait_event(self.ev_start)
         with torch.cuda.stream(self.s_cast):
-            for d, e, exw in zip(self.L, self.ev_cast, self.ev_cast_xw):
+            for d, e, ex in zip(self.L, self.ev_cast, self.ev_cast_x):
                 sc = d["sc"]
                 self.quantise(d["X"], fp8.FP8_E4M3, sc, 0, out=d["xq"])
-                self.quantise(d["W"], fp8.FP8_E4M3, sc, 3, out=d["wq"])
-                exw.record(self.s_cast)
+                ex.record(self.s_cast)
                 self.quantise(d["dY"], fp8.FP8_E5M2, sc, 6, mu=MU, out=d["dyq"])
                 e.record(self.s_cast)
         for i, (d, e) in enumerate(zip(self.L, self.ev_cast)):
             sc = d["sc"]
-            main.wait_event(self.ev_cast_xw[i])
+            main.wait_event(self.ev_cast_x[i])
             fp8.fp8_linear_fwd(d["xq"], sc[2:3], d["wq"], sc[5:6], d["y"], sc[12:13])
             main.wait_event(e)
             fp8.fp8_linear_dgrad(d["dyq"], sc[8:9], d["wq"], sc[5:6], d["dx"], sc[13:14])
+            self.ev_dgrad[i].record(main)
             self.s_aux.wait_event(e)
             with torch.cuda.stream(self.s_aux):
                 fp8.fp8_linear_wgrad(d["dyq"], sc[8:9], d["xq"], sc[2:3], d["dw"], sc[14:15])
                 fp8.fp8_scale_cast(d["dw"], fp8.FP8_E5M2, sc[14:15], 0, MU, sc[10:11], sc[11:12], d["gq"])
+                self.s_aux.wait_event(self.ev_dgrad[i])
                 fp8.fp8_adam_step(self.chunks_each[i], step=self.t + 1, margin=0,
                                   workspace=self.ws_each[64 * i:64 * (i + 1)], **HP)
         self.ev_grad.record(self.s_aux)
@@ -307,70 +354,96 @@ def sum_events(ev, kind):
 
 
 # ---------------------------------------------------------------- CPU oracle timing
-def oracle_step_estimate(budget_s: float = 12.0):
-    """Times the CPU oracle on bounded samples of one step's work and
-    extrapolates to a full step (seconds).  Returns (seconds, cores, sample text)."""
-    import oracle
+class OracleSample:
+    """A bounded sample of one step's work for the CPU oracle: per linear the
+    forward GEMM of one token row against the whole weight (dgrad and wgrad
+    have the same multiply-add count, so the row's time counts three
+    times), an amax + scale + cast of 2^21 bf16 elements and an Adam step on
+    2^20 parameters.  Inputs are drawn once; run() times one sample and
+    returns (seconds of the sample, seconds extrapolated to the whole step by
+    units)."""
 
-    cores = oracle.num_threads()
-    t_total = 0.0
-    parts = []
-    rows = 4
-    for name, K, N in synth.GPT7B_LINEARS:
-        M = synth.GPT7B_TOKENS
-        g = synth.rng("bench-oracle", name)
-        # codes for a row block: fwd uses rows of X, dgrad rows of dY, wgrad rows of dW (cols of dY)
-        xq = g.integers(0, 0x7E, (rows, K), dtype=np.uint8)
-        wq = g.integers(0, 0x7E, (N, K), dtype=np.uint8)
+    ROWS = 1
+
+    def __init__(self, wl: dict):
+        import oracle
+
+        self.oracle = oracle
+        self.wl = wl
+        self.ops = []
+        for name, K, N in wl["linears"]:
+            g = synth.rng("bench-oracle", name)
+            # finite positive E4M3 codes (bit 3 clear: never 0x7F)
+            wq = (np.frombuffer(g.bytes(N * K), dtype=np.uint8) & 0x77).reshape(N, K)
+            xq = (np.frombuffer(g.bytes(self.ROWS * K), dtype=np.uint8) & 0x77).reshape(self.ROWS, K)
+            self.ops.append((name, K, N, xq, wq))
+        self.n_cast = 1 << 21
+        self.xb = synth.normal_bf16((self.n_cast,), 1.0, "bench-oracle", "cast")
+        self.n_adam = 1 << 20
+        self.gq = np.random.default_rng(0).integers(0, 0x7B, self.n_adam, dtype=np.uint8)
+        M = wl["tokens"]
+        self.elems = sum(M * K + M * N for _, K, N in wl["linears"])  # X and dY casts
+        self.params = sum(N * K for _, K, N in wl["linears"])
+        self.cores = oracle.num_threads()
+        self.text = (f"oracle timed on: per linear a {self.ROWS}-row forward GEMM block "
+                     f"({'; '.join(f'{n}: {self.ROWS}x{N}x{K}' for n, K, N, _, _ in self.ops)}), counted "
+                     f"x3 for dgrad/wgrad; amax+scale+cast of 2^21 bf16; Adam on 2^20 params; "
+                     f"extrapolated to the full step by units")
+
+    def run(self):
+        o = self.oracle
+        M = self.wl["tokens"]
+        t_sample = 0.0
+        t_full = 0.0
+        for name, K, N, xq, wq in self.ops:
+            t0 = time.perf_counter()
+            o.linear_fwd(xq, 1.0, wq, 1.0, self.ROWS, N, K)
+            dt = time.perf_counter() - t0
+            t_sample += dt
+            t_full += 3 * dt * M / self.ROWS
         t0 = time.perf_counter()
-        oracle.linear_fwd(xq, 1.0, wq, 1.0, rows, N, K)
-        t_fwd = (time.perf_counter() - t0) * M / rows
-        # dgrad and wgrad have the same MNK product: scale the fwd row-block rate
-        t_total += 3 * t_fwd
-        parts.append(f"{name}: {rows}x{N}x{K} fwd row block")
-    n = 1 << 21
-    xb = synth.normal_bf16((n,), 1.0, "bench-oracle", "cast")
-    t0 = time.perf_counter()
-    a = oracle.amax(xb, oracle.DT_BF16, parallel=True)
-    _, s = oracle.compute_scale(a, oracle.E4M3, 0)
-    oracle.cast(xb, oracle.E4M3, s, oracle.DT_BF16)
-    t_cast = (time.perf_counter() - t0) / n
-    elems = sum(synth.GPT7B_TOKENS * K + N * K + synth.GPT7B_TOKENS * N for _, K, N in synth.GPT7B_LINEARS)
-    params = sum(N * K for _, K, N in synth.GPT7B_LINEARS)
-    t_total += t_cast * (elems + params)  # activation/weight/grad casts + gradient cast
-    na = 1 << 20
-    gq = np.random.default_rng(0).integers(0, 0x7B, na, dtype=np.uint8)
-    w = np.full(na, 0x2C00, np.uint16)
-    t0 = time.perf_counter()
-    oracle.adam_step(gq, 1e-6, np.zeros(na, np.uint8), 1.0, np.zeros(na, np.uint16), 1.0, w, 1.0,
-                     t=1, margin=0, **HP)
-    t_adam = (time.perf_counter() - t0) / na
-    t_total += t_adam * params
-    sample = (f"oracle timed on: {'; '.join(parts)}; amax+scale+cast of 2^21 bf16; Adam on 2^20 params; "
-              f"extrapolated to the full step by units")
-    return t_total, cores, sample
+        a = o.amax(self.xb, o.DT_BF16, parallel=True)
+        _, s = o.compute_scale(a, o.E4M3, 0)
+        o.cast(self.xb, o.E4M3, s, o.DT_BF16)
+        dt = time.perf_counter() - t0
+        t_sample += dt
+        t_full += dt / self.n_cast * (self.elems + self.params)  # X/dY casts + gradient cast
+        n = self.n_adam
+        t0 = time.perf_counter()
+        o.adam_step(self.gq, 1e-6, np.zeros(n, np.uint8), 1.0, np.zeros(n, np.uint16), 1.0,
+                    np.full(n, 0x2C00, np.uint16), 1.0, t=1, margin=0, **HP)
+        dt = time.perf_counter() - t0
+        t_sample += dt
+        t_full += dt / n * self.params
+        return t_sample, t_full
 
 
 # ---------------------------------------------------------------- arms
 def run_reference(args):
+    """The CPU oracle as it stands, on the host cores: each step is one
+    bounded sample of the step's work (OracleSample); `ms_per_step` is the
+    measured time of one such sample, `value` the GEMM work of the whole
+    step over the time extrapolated from the sample by units."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    vals = []
-    t_all = []
+    wl = WORKLOADS[args.workload]
+    cfg = config_of(wl, args.schedule, args.gpus)
+    sample = OracleSample(wl)
+    t_s, t_f = [], []
     for i in range(args.warmup + args.steps):
-        t, cores, sample = oracle_step_estimate()
+        a, b = sample.run()
         if i >= args.warmup:
-            t_all.append(t)
-    t = statistics.median(t_all)
-    flops = sum(3 * 2 * synth.GPT7B_TOKENS * N * K for _, K, N in synth.GPT7B_LINEARS)
-    v = flops / t / 1e12
+            t_s.append(a)
+            t_f.append(b)
+    ts, tf = statistics.median(t_s), statistics.median(t_f)
+    v = cfg["gemm_flops_per_step"] / tf / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "tokens": synth.GPT7B_TOKENS, "hidden": 4096,
-                       "linears": [l[0] for l in synth.GPT7B_LINEARS], "adam_params": 201326592},
-            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ts * 1e3,
+            "ms_per_full_step_extrapolated": tf * 1e3, "extrapolated": True, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": sample.cores, "kind": "oracle",
+                             "sample": sample.text},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -398,7 +471,8 @@ def run_gpu(args):
     from fp8_mixed_precision_tensor_b200 import fp8
 
     peaks = load_peaks()
-    runner = Block7BStep(dev, seed=rank)
+    wl = WORKLOADS[args.workload]
+    runner = BlockStep(dev, seed=rank, workload=args.workload)
     overlap = args.schedule == "overlap"
     for _ in range(args.warmup):
         runner.step_overlapped() if overlap else runner.step()
@@ -416,6 +490,7 @@ def run_gpu(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_step = t.item()
     status = fp8.fp8_get_status()
+    clocks = sampler.summary()
 
     # ---- per-kernel breakdown (separate pass with events between phases)
     ev = {}
@@ -435,14 +510,14 @@ def run_gpu(args):
         for d, (x, y) in zip(runner.L, host_in):
             d["X"].copy_(x, non_blocking=True)
             d["dY"].copy_(y, non_blocking=True)
-        runner.step_overlapped() if overlap else runner.step()
+        runner.step()
         res.copy_(runner.result_scalars(), non_blocking=True)
 
     # Overlapped schedule: the inputs of step t+1 are copied on a copy stream
     # into a second set of device buffers while step t computes (prefetching
     # input pipeline); every step's copy is still inside the timed region.
-    sets = [[(d["X"], d["dY"]) for d in runner.L],
-            [(torch.empty_like(d["X"]), torch.empty_like(d["dY"])) for d in runner.L]]
+    sets = ([[(d["X"], d["dY"]) for d in runner.L],
+             [(torch.empty_like(d["X"]), torch.empty_like(d["dY"])) for d in runner.L]] if overlap else None)
     copy_stream = torch.cuda.Stream(dev)
     ev_copied = [torch.cuda.Event(), torch.cuda.Event()]
     ev_used = [torch.cuda.Event(), torch.cuda.Event()]
@@ -488,15 +563,17 @@ def run_gpu(args):
     s1.record()
     s1.synchronize()
     e2e_ms = s0.elapsed_time(s1) / args.steps
-    for d, (xd, yd) in zip(runner.L, sets[0]):
-        d["X"], d["dY"] = xd, yd
+    if overlap:
+        for d, (xd, yd) in zip(runner.L, sets[0]):
+            d["X"], d["dY"] = xd, yd
     if dist is not None:
         t = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = t.item()
+    status |= fp8.fp8_get_status()
 
     value = runner.flops * world / (ms_step * 1e-3) / 1e12
-    fp8_peak = 2.0 * peaks["bf16_sus"]  # FP8 dense = 2 x bf16 dense (nominal ratio), sustained
+    peak, peak_src = fp8_peak(peaks, clocks)
     gemm_tflops = runner.flops / (t_gemm * 1e-3) / 1e12
     cast_gbs = runner.cast_elems * CAST_BYTES_BF16 / (t_cast * 1e-3) / 1e9
     gcast_gbs = runner.params * GRAD_CAST_BYTES / (t_gcast * 1e-3) / 1e9
@@ -505,33 +582,36 @@ def run_gpu(args):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp8(e4m3/e5m2)->f32 accum; f32 elementwise", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "tokens": runner.M, "hidden": 4096,
-                   "linears": [d["name"] for d in runner.L], "adam_params": runner.params,
-                   "gemm_flops_per_step": runner.flops, "l2": "inputs larger than L2 (no flush)",
-                   "schedule": args.schedule,
-                   "parallelism": f"replicas{world}" if world > 1 else "single"},
-        "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
-                     "frac": gemm_tflops / fp8_peak, "traffic": gemm_traffic(),
+        "config": config_of(wl, args.schedule, world),
+        "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": gemm_tflops / peak, "traffic": gemm_traffic(wl["workload"]),
                      "kernel": "k_gemm3 (fwd+dgrad+wgrad; achieved = GEMM flops per step / summed GEMM "
                                "time; traffic = mean DRAM bytes per launch)",
-                     "peak_src": f"2 x bf16_tflops_sustained ({peaks['src']})"},
+                     "peak_src": peak_src},
         "kernels": {
-            "gemm": {"ms": t_gemm, "TFLOP/s": gemm_tflops, "frac_fp8_peak": gemm_tflops / fp8_peak},
-            "amax_scale_cast": {"ms": t_cast, "GB/s": cast_gbs, "frac_hbm": cast_gbs / peaks["hbm"]},
+            "gemm": {"ms": t_gemm, "TFLOP/s": gemm_tflops, "frac_fp8_peak": gemm_tflops / peak},
+            "amax_scale_cast": {"ms": t_cast, "GB/s": cast_gbs, "frac_hbm": cast_gbs / peaks["hbm"],
+                                "tensors": "X and dY of every linear (the weight operand comes from Adam)"},
             "grad_cast": {"ms": t_gcast, "GB/s": gcast_gbs, "frac_hbm": gcast_gbs / peaks["hbm"]},
             "adam": {"ms": t_adam, "GB/s": adam_gbs, "frac_hbm": adam_gbs / peaks["hbm"],
-                     "bytes_per_param_algorithmic": ADAM_BYTES},
+                     "bytes_per_param_algorithmic": ADAM_BYTES,
+                     "bytes_per_param_moved": "15 (stats pass 4 with the tracked master + update 11) "
+                                              "+ 1 for the E4M3 weight copy"},
+            "hbm_peak_gbs": peaks["hbm"],
         },
         "e2e": {"value": runner.flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": (runner.launches_per_step_overlapped if overlap else runner.launches_per_step) * args.steps,
-        "clocks": sampler.summary(),
+        "clocks": clocks,
         "device_status": status,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t_cpu, cores, sample = oracle_step_estimate()
-        line["cpu_baseline"] = {"value": runner.flops / t_cpu / 1e12, "unit": "TFLOP/s", "cores": cores,
-                                "kind": "oracle", "sample": sample}
+        sample = OracleSample(wl)
+        runs = [sample.run() for _ in range(2)]
+        t_cpu = statistics.median(r[1] for r in runs)
+        line["cpu_baseline"] = {"value": runner.flops / t_cpu / 1e12, "unit": "TFLOP/s", "cores": sample.cores,
+                                "kind": "oracle", "sample": sample.text,
+                                "sample_seconds": statistics.median(r[0] for r in runs)}
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -543,9 +623,10 @@ def run_gpu(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="gpt175b_block", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--schedule", default="overlap", choices=["overlap", "serial"],
                     help="overlap: casts / GEMMs / wgrad on three streams; serial: one stream")

@@ -71,6 +71,9 @@ class FP8GradAllReduce:
         self.scalars = torch.zeros(4, **f32)  # shared amax, S, 1/S, g_inv
         self.cast_counts = torch.zeros(2, dtype=torch.int64, device=device)
         self.sum_counts = torch.zeros(2, dtype=torch.int64, device=device)
+        # "auto": running total of the summed counts over the ranks (fp8_mu_update
+        # clears sum_counts every step once it has read them)
+        self.sum_total = torch.zeros(2, dtype=torch.int64, device=device)
         self.send = torch.zeros(self.world * self.L, dtype=torch.uint8, device=device)  # tail stays 0
         self.recv = torch.zeros(self.world, self.L, dtype=torch.uint8, device=device)
         self.out = torch.zeros(self.L, dtype=torch.uint8, device=device)
@@ -110,6 +113,7 @@ class FP8GradAllReduce:
         if self.scaling == "auto":
             if self.collectives:
                 dist.all_reduce(self.sum_counts, op=dist.ReduceOp.SUM, group=self.group)
+            self.sum_total += self.sum_counts
             fp8.fp8_mu_update(self.mu, self.clean, self.sum_counts, self.n, **self.rule)
         return self.out[:self.hi - self.lo]
 
@@ -122,12 +126,14 @@ class FP8GradAllReduce:
         return full[:self.n]
 
     def rates(self) -> dict:
-        """Underflow and overflow counts so far (summed over ranks; a host
-        read, for monitoring).  Under "auto" the sum counts restart every step."""
-        c = torch.cat([self.cast_counts, self.sum_counts])
+        """Underflow and overflow counts of all steps so far, summed over the
+        ranks (a host read, for monitoring; every rank must call it, it runs a
+        collective).  Under "auto" the sum counts are the running total that
+        was already summed over the ranks step by step."""
+        auto = self.scaling == "auto"
+        c = self.cast_counts.clone() if auto else torch.cat([self.cast_counts, self.sum_counts])
         if self.collectives:
-            c = c.clone()
             dist.all_reduce(c, op=dist.ReduceOp.SUM, group=self.group)
-        c = c.tolist()
+        c = (torch.cat([c, self.sum_total]) if auto else c).tolist()
         return dict(cast_underflow=c[0], cast_overflow=c[1], sum_underflow=c[2], sum_overflow=c[3],
                     mu=self.mu.item())

@@ -105,34 +105,23 @@ __device__ __forceinline__ AdamScalars adam_scalars(const AdamLaunch &L, float g
   return s;
 }
 
-// Approximate (MUFU) square root and reciprocal, subnormal inputs flushed:
-// relative error ~1e-7 on the step direction m_hat / (sqrt(v_hat) + eps),
-// which moves the master weight by lr * O(1) -- far below an FP16 ULP of the
-// stored master.  The flush changes nothing for eps >= 2^-39: the square root
-// of a subnormal is below 2^-63, under half an ULP of such an eps, and the
-// reciprocal's argument is at least eps.
-__device__ __forceinline__ float sqrt_approx(float x) {
-  float r;
-  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-  return r;
-}
-__device__ __forceinline__ float rcp_approx(float x) {
-  float r;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-  return r;
-}
-
 // The new moments and the master step dw = -lr m_hat / (sqrt(v_hat) + eps)
-// of two parameters, binary32, from decoded codes.  Explicit round-to-nearest
-// operations keep every pass (and the element-wise tail, which runs the same
-// function with one lane unused) on exactly the same arithmetic.
+// of two parameters, binary32, from decoded codes.  Every operation rounds to
+// nearest (the square root and the quotient are CUDA's correctly rounded
+// __fsqrt_rn / __fdiv_rn, subnormals kept), so the step's error is a fixed
+// number of binary32 roundings: |dw - dw_exact| <= 24 * 2^-24 * dw_abs, where
+// dw_abs is the step with |m| replaced by b1 |m0| + (1 - b1) |g| (which also
+// covers the cancellation of m's two terms), counting the hyper-parameters'
+// own binary32 representation.  Explicit round-to-nearest operations keep
+// every pass (and the element-wise tail, which runs the same function with
+// one lane unused) on exactly the same arithmetic.
 __device__ __forceinline__ void adam_moments(const AdamLaunch &L, float2 gd, float2 md, float2 vd,
                                              const AdamScalars &s, float2 &m, float2 &v, float2 &dw) {
   m = __ffma2_rn(s.cm, md, __fmul2_rn(s.cgm, gd));
   v = __ffma2_rn(s.cv, vd, __fmul2_rn(__fmul2_rn(s.cgv, gd), __fmul2_rn(s.g_inv, gd)));
   const float2 vh = __fmul2_rn(v, both(L.inv_bc2));
-  const float2 den = __fadd2_rn(make_float2(sqrt_approx(vh.x), sqrt_approx(vh.y)), both(L.eps));
-  dw = __fmul2_rn(both(L.neg_lr_bc1), __fmul2_rn(m, make_float2(rcp_approx(den.x), rcp_approx(den.y))));
+  const float2 den = __fadd2_rn(make_float2(__fsqrt_rn(vh.x), __fsqrt_rn(vh.y)), both(L.eps));
+  dw = __fmul2_rn(both(L.neg_lr_bc1), make_float2(__fdiv_rn(m.x, den.x), __fdiv_rn(m.y, den.y)));
 }
 
 // w = w0 + dw as one rounding per parameter (the master's new value).

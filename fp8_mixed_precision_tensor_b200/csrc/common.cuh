@@ -19,6 +19,11 @@ namespace fp8lib {
 
 // Sticky device status word (FP8_STATUS_* bits), read back by fp8_get_status.
 __device__ unsigned int g_status;
+// The value fp8_get_status took out of g_status, for its copy to the host.
+__device__ unsigned int g_status_taken;
+
+// Read and clear the status word in one atomic operation.
+__global__ void k_take_status() { g_status_taken = atomicExch(&g_status, 0u); }
 
 constexpr float kMaxE4M3 = 448.0f;
 constexpr float kMaxE5M2 = 57344.0f;

@@ -433,9 +433,13 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
   if (!chunks || !hp || nchunks <= 0 || !workspace) return FP8_ERR_INVALID_ARG;
   if (ws_bytes < fp8_adam_workspace_bytes(nchunks)) return FP8_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FP8_ERR_UNALIGNED;
-  if (!(hp->lr >= 0.0f) || !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) ||
-      !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f) || !(hp->eps >= 0.0f) || hp->step < 1 ||
-      hp->margin < 0 || hp->margin > 64)
+  // eps >= 2^-39: the square root of a binary32-subnormal v_hat (< 2^-126)
+  // is below 2^-63, under half an ULP of such an eps, so sqrt(v_hat) + eps
+  // rounds to eps and the subnormal's lost precision never reaches the step;
+  // eps = 0 would also turn a zero gradient on a zero state into 0/0.
+  if (!(hp->lr >= 0.0f && hp->lr <= 3.402823466e38f) || !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) ||
+      !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f) || !(hp->eps >= 0x1p-39f && hp->eps <= 3.402823466e38f) ||
+      hp->step < 1 || hp->margin < 0 || hp->margin > 64)
     return FP8_ERR_INVALID_ARG;
   for (int i = 0; i < nchunks; i++) {
     const fp8_adam_chunk &c = chunks[i];
@@ -557,10 +561,10 @@ int fp8_adam_step_noalloc(const fp8_adam_chunk *chunks, int nchunks, const fp8_a
 int fp8_get_status(unsigned *host_out, void *stream) {
   if (!host_out) return FP8_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  unsigned v = 0, zero = 0;
-  if (cudaMemcpyFromSymbolAsync(&v, g_status, sizeof(v), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return FP8_ERR_CUDA;
-  if (cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
+  unsigned v = 0;
+  k_take_status<<<1, 1, 0, s>>>();
+  if (cudaGetLastError() != cudaSuccess) return FP8_ERR_CUDA;
+  if (cudaMemcpyFromSymbolAsync(&v, g_status_taken, sizeof(v), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return FP8_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return FP8_ERR_CUDA;
   *host_out = v;

@@ -257,8 +257,9 @@ int fp8_linear_wgrad(const uint8_t *dyq, const float *dy_inv, const uint8_t *xq,
  * then new per-chunk scales from the amax of the new m, v, w (same rule as
  * fp8_compute_scale with `margin`, fmt_max 448 / 65504 / 65504) and the state
  * is re-encoded with them; the new scales replace m_scale, v_scale, w_scale.
- * Arithmetic is float32.  A non-finite new amax sets FP8_STATUS_NONFINITE and
- * that scale to 1.
+ * Arithmetic is float32 with every operation rounded to nearest (square root
+ * and quotient correctly rounded); a non-finite new amax sets
+ * FP8_STATUS_NONFINITE and that scale to 1.
  * Tracked master amax (optional; the first pass then moves 4 instead of 6
  * bytes per parameter): when w_amax points to the exact amax of the
  * dequantised stored master (a value >= 0), the new master amax is bounded by
@@ -291,7 +292,10 @@ typedef struct {
 } fp8_adam_chunk;
 
 typedef struct {
-  float lr, beta1, beta2, eps; /* lr > 0, 0 <= beta < 1, eps >= 0 */
+  float lr, beta1, beta2, eps; /* 0 <= lr finite, 0 <= beta < 1, 2^-39 <= eps finite
+                                  (a smaller eps returns FP8_ERR_INVALID_ARG: eps = 0
+                                  makes a zero gradient on a zero state 0/0, and below
+                                  2^-39 a binary32-subnormal v_hat would reach the step) */
   int step;                    /* t >= 1 (bias correction) */
   int margin;                  /* scale margin, >= 0 */
 } fp8_adam_hparams;
@@ -353,6 +357,10 @@ int fp8_adam_apply(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hpa
  * any stream capture.  Every call on a device shares the one array: the step
  * clears the part it needs before use, and two calls whose work overlaps on
  * the GPU (different streams, no ordering between them) race on it.
+ * The looked-up address is kept per device ordinal for the life of the
+ * process: do not use this entry point across a cudaDeviceReset (or any
+ * other teardown of the device's primary context), after which the kept
+ * address no longer belongs to the device.
  * Arguments, results and errors are otherwise those of fp8_adam_step.
  */
 #define FP8_ADAM_NOALLOC_MAX_CHUNKS 1024
@@ -360,9 +368,13 @@ int fp8_adam_step_noalloc(const fp8_adam_chunk *chunks, int nchunks, const fp8_a
                           void *stream);
 
 /*
- * fp8_get_status -- waits for `stream`, then reads the device status word
- * (OR of FP8_STATUS_* bits raised since the last read) into *host_out and
- * clears it.  Returns FP8_ERR_CUDA if the stream reported an error.
+ * fp8_get_status -- enqueues on `stream` one atomic exchange that reads the
+ * device status word (OR of FP8_STATUS_* bits raised since the last read) and
+ * clears it in the same operation, so a bit raised by a kernel on another
+ * stream is either in this read or left for the next one; then waits for
+ * `stream` and writes the value to *host_out.  Calls on different streams
+ * must not overlap (they share the one readback word).  Returns FP8_ERR_CUDA
+ * if the stream reported an error.
  */
 int fp8_get_status(unsigned *host_out, void *stream);
 

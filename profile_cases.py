@@ -1,12 +1,12 @@
 """Run one kernel family of the hot path on a chosen case (for profilers).
 
-    python -m fp8_mixed_precision_tensor_b200.profile_cases linear --M 4096 --N 16384 --K 4096
-    python -m fp8_mixed_precision_tensor_b200.profile_cases cast --n 268435456
-    python -m fp8_mixed_precision_tensor_b200.profile_cases castsweep
-    python -m fp8_mixed_precision_tensor_b200.profile_cases adam --n 67108864 [--track]
-    python -m fp8_mixed_precision_tensor_b200.profile_cases allreduce --n 268435456 --world 8
-    python -m fp8_mixed_precision_tensor_b200.profile_cases castcount --n 268435456
-    python -m fp8_mixed_precision_tensor_b200.profile_cases adam7b --iters 10
+    python profile_cases.py linear --M 4096 --N 16384 --K 4096
+    python profile_cases.py cast --n 268435456
+    python profile_cases.py castsweep
+    python profile_cases.py adam --n 67108864 [--track]
+    python profile_cases.py allreduce --n 268435456 --world 8
+    python profile_cases.py castcount --n 268435456
+    python profile_cases.py adam7b --iters 10
 
 Each case runs `--iters` passes after one warm-up pass on seeded synthetic
 inputs and prints the CUDA-event time per pass.  Launch order per pass:
@@ -22,10 +22,15 @@ kernel's own time and algorithmic GB/s.
 from __future__ import annotations
 
 import argparse
+import os
+import sys
 
 import torch
 
-from fp8_mixed_precision_tensor_b200 import fp8, synth
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+
+from fp8_mixed_precision_tensor_b200 import fp8, synth  # noqa: E402
+from fp8_mixed_precision_tensor_b200.adam_state import AdamTensorState  # noqa: E402
 
 
 def _scalars(n):
@@ -202,31 +207,24 @@ def case_castcount(a):
     return one
 
 
-def build_adam_state(chunks, device="cuda", seed=11, mu=2.0 ** 10):
-    """Device-resident decoupled-Adam state for (name, n) chunks: E5M2
-    gradients ~N(0, 1e-3) scaled by mu, FP16 master ~N(0, 0.02) with its
-    scale, zero moments with scale 1.  Returns a list of fp8.AdamChunk."""
+def build_adam_state(chunks, device="cuda", seed=11, mu=2.0 ** 10, track=False):
+    """Decoupled-Adam state for (name, n) chunks: FP16 master from weights
+    ~N(0, 0.02), zero moments, E5M2 gradients ~N(0, 1e-3) scaled by mu.
+    Returns the AdamTensorState list."""
     out = []
     for ci, (_, n) in enumerate(chunks):
-        sc = _scalars(6)
-        g = synth.device_normal((n,), 1e-3, seed * 100000 + 2 * ci, torch.float32, device)
-        gq = torch.empty(n, dtype=torch.uint8, device=device)
-        fp8.fp8_amax(g, sc[0:1])
-        fp8.fp8_scale_cast(g, fp8.FP8_E5M2, sc[0:1], 0, mu, sc[1:2], sc[2:3], gq)
-        del g
         w = synth.device_normal((n,), 0.02, seed * 100000 + 2 * ci + 1, torch.float32, device)
-        wh = torch.empty(n, dtype=torch.int16, device=device)
-        st = torch.ones(3, dtype=torch.float32, device=device)
-        fp8.fp8_amax(w, sc[3:4])
-        fp8.fp8_scale_cast(w, fp8.FP8_F16S, sc[3:4], 0, 1.0, st[2:3], sc[5:6], wh)
+        st = AdamTensorState(w, track_master_amax=track)
         del w
-        out.append(fp8.AdamChunk(gq, sc[2:3], torch.zeros(n, dtype=torch.uint8, device=device), st[0:1],
-                                 torch.zeros(n, dtype=torch.int16, device=device), st[1:2], wh, st[2:3]))
+        g = synth.device_normal((n,), 1e-3, seed * 100000 + 2 * ci, torch.float32, device)
+        st.set_gradient(g, mu)
+        del g
+        out.append(st)
     return out
 
 
 def case_adam7b(a):
-    chunks_list = build_adam_state(synth.gpt7b_adam_chunks())
+    chunks_list = [st.chunk for st in build_adam_state(synth.gpt7b_adam_chunks(), track=a.track)]
     params = sum(c.g.numel() for c in chunks_list)
     chunks = fp8.pack_adam_chunks(chunks_list)
     ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(chunks_list)) // 4, dtype=torch.float32, device="cuda")

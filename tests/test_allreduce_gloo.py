@@ -82,6 +82,7 @@ def _worker(rank, world, port, scaling, n):
         lo, hi = zero.shard_bounds(n, world, rank)
         mu = {"auto": 1.0, "post": 1.0, "pre": 2.0 ** -int(np.ceil(np.log2(world)))}[scaling]
         clean = 0
+        auto_sums = np.zeros(2, dtype=np.int64)
         for step in range(4):
             grads = _grads(world, n, step)
             want = oracle.fp8_allreduce(grads, oracle.E5M2, 0, mu)
@@ -91,8 +92,14 @@ def _worker(rank, world, port, scaling, n):
             assert np.array_equal(ar.all_gather().numpy(), want["codes"])
             assert ar.g_inv.item() == float(np.float32(1.0 / want["S"]) * np.float32(1.0 / world))
             if scaling == "auto":
+                auto_sums += np.asarray(want["sum_counts"], dtype=np.int64)
                 mu, clean = oracle.mu_update(mu, clean, want["sum_counts"][1], n, 0.0, 2, 2.0 ** -16, 1.0)
             assert ar.mu.item() == mu, (step, ar.mu.item(), mu)
+        if scaling == "auto":
+            # the running totals of the rank-summed counts, not re-summed over the ranks
+            r = ar.rates()
+            assert (r["sum_underflow"], r["sum_overflow"]) == tuple(auto_sums.tolist()), (r, auto_sums)
+            assert auto_sums[1] > 0  # the first step, at mu = 1, saturates elements 0..3
         if scaling == "post":
             assert ar.rates()["sum_overflow"] == 4 * 4  # four steps, elements 0..3 saturate
         if scaling == "pre" and world > 1:

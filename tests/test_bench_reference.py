@@ -19,4 +19,10 @@ def test_reference_arm_prints_the_contract_line():
         assert k in line, k
     assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
-    assert line["config"]["workload"] == "gpt7b_block_linears_fp8_train_step"
+    assert line["config"]["workload"] == "gpt175b_block_linears_fp8_train_step"
+    assert line["extrapolated"] is True and line["ms_per_full_step_extrapolated"] > line["ms_per_step"]
+    # the reference arm's config is the GPU arm's (one function builds both)
+    sys.path.insert(0, ROOT)
+    import bench
+
+    assert line["config"] == bench.config_of(bench.WORKLOADS["gpt175b_block"], "overlap", 1)

@@ -394,35 +394,87 @@ def snapshot(c):
                 w=c.w.cpu().numpy().view(np.uint16), s_w=c.w_scale.item())
 
 
-def check_adam_chunk(before, c, step, margin=0):
-    out = oracle.adam_step(before["g"], before["g_inv"], before["m"], before["s_m"], before["v"],
-                           before["s_v"], before["w"], before["s_w"], t=step, margin=margin, **HP)
+# The kernel evaluates the update in binary32 with every operation rounded to
+# nearest; counting those roundings (and the binary32 representation of lr,
+# beta1, beta2, eps and the bias corrections) bounds its step's error by
+# STEP_ROUNDINGS * 2^-24 * dw_abs, where dw_abs is the step computed from the
+# magnitudes of m's two terms, lr (b1 |m0| + (1 - b1) |g|) / (1 - b1^t) /
+# (sqrt(v_hat) + eps).  The master is compared at 1 FP16 ULP plus that term
+# (which only matters where the step cancels most of the weight).
+STEP_ROUNDINGS = 24
+MAX_TIES = 1  # scale ties tolerated per test (each is still checked element by element)
+FMAX_ADAM = (("s_m", 448.0), ("s_v", 65504.0), ("s_w", 65504.0))
+
+
+def adam_step_magnitude(before, step, hp=HP):
+    """dw_abs of every element, float64, from the decoded stored state."""
+    g = oracle.decode_table(oracle.E5M2)[before["g"]] * before["g_inv"]
+    m0 = oracle.decode_table(oracle.E4M3)[before["m"]] / before["s_m"]
+    v0 = f16_vals(before["v"]) / before["s_v"]
+    b1, b2 = hp["beta1"], hp["beta2"]
+    v = b2 * v0 + (1 - b2) * g * g
+    den = np.sqrt(v / (1 - b2 ** step)) + hp["eps"]
+    return hp["lr"] * (b1 * np.abs(m0) + (1 - b1) * np.abs(g)) / (1 - b1 ** step) / den
+
+
+def _slice(state, lo, hi):
+    return {k: (v[lo:hi] if isinstance(v, np.ndarray) else v) for k, v in state.items()}
+
+
+def check_adam_chunk(before, c, step, margin=0, ties=None, slices=1):
+    """Oracle step from `before` against the chunk's state now.  Scales must be
+    bit-equal; a mismatch is allowed only where the oracle's float64 amax lies
+    within 4 binary32 ULPs of a scale threshold (a tie).  A tie is appended to
+    `ties` (a failure when `ties` is None) and the elements are still compared,
+    against the oracle re-run at the GPU's scale for the tied tensor.
+    slices > 1 bounds the oracle's memory for large chunks: the tensor's new
+    amaxes are the maximum of its slices' (the element-sharded oracle step),
+    then every slice is requantised with them and compared on its own."""
     after = snapshot(c)
-    # scales bit-equal unless the oracle amax sits on a power-of-two threshold
-    for key, amax, fmax in (("s_m", out["amax"][0], 448.0), ("s_v", out["amax"][1], 65504.0),
-                            ("s_w", out["amax"][2], 65504.0)):
-        if after[key] != out[key]:
-            e = oracle.floor_log2_ratio(amax, fmax)
+    n = before["g"].size
+    bounds = [(n * k // slices, n * (k + 1) // slices) for k in range(slices)]
+
+    def run(b, amax_in=None):
+        return oracle.adam_step(b["g"], b["g_inv"], b["m"], b["s_m"], b["v"], b["s_v"], b["w"], b["s_w"],
+                                t=step, margin=margin, amax_in=amax_in, **HP)
+
+    first = run(before) if slices == 1 else None
+    amax = first["amax"] if slices == 1 else tuple(
+        max(x) if not any(np.isnan(x)) else float("nan")
+        for x in zip(*(run(_slice(before, lo, hi))["amax"] for lo, hi in bounds)))
+    ref_scales = first if slices == 1 else run(_slice(before, 0, bounds[0][1] if n else 0), amax_in=amax)
+    tied = []
+    for j, (key, fmax) in enumerate(FMAX_ADAM):
+        if after[key] != ref_scales[key]:
+            e = oracle.floor_log2_ratio(amax[j], fmax)
             thresh = fmax * 2.0 ** (-e)
-            assert abs(amax - thresh) <= 4 * np.spacing(np.float32(thresh)), (key, after[key], out[key])
-            pytest.skip(f"tie: oracle amax {amax} on a scale threshold")
-    # master and second moment within 1 FP16 ULP of the dequantised oracle value;
-    # for the master add the float32 evaluation's own rounding bound (the step
-    # dw = -lr m/(sqrt(v)+eps) carries a few float32 ULPs, the add one more):
-    # 2^-24 (|w0| + 16 |dw|).  It exceeds an FP16 ULP of the result only where
-    # the step cancels the weight to near zero.
-    w0 = f16_vals(before["w"]) / before["s_w"]
-    for key, okey, skey in (("w", "wh", "s_w"), ("v", "vh", "s_v")):
-        ref = f16_vals(out[okey]) / out[skey]
-        got = f16_vals(after[key]) / after[skey]
-        ulp = f16_ulp(f16_vals(out[okey])) / out[skey]
-        if key == "w":
-            ulp = ulp + 2.0 ** -24 * (np.abs(w0) + 16 * np.abs(ref - w0))
-        bad = np.abs(got - ref) > ulp
-        assert not np.any(bad), (key, np.count_nonzero(bad), got[bad][:4], ref[bad][:4])
-    # first moment within 1 code (scales equal)
-    assert np.all(np.abs(code_rank(after["m"]) - code_rank(out["mq"])) <= 1)
-    return out
+            assert abs(amax[j] - thresh) <= 4 * np.spacing(np.float32(thresh)), (key, after[key], ref_scales[key])
+            tied.append(j)
+    amax_in = None if slices == 1 else amax
+    if tied:
+        assert ties is not None, f"scale tie at an oracle amax on a threshold: {tied}"
+        ties.append((step, tied))
+        amax_in = list(amax)
+        for j in tied:
+            amax_in[j] = FMAX_ADAM[j][1] / (after[FMAX_ADAM[j][0]] * 2.0 ** margin)
+        amax_in = tuple(amax_in)
+    for lo, hi in bounds:
+        b, a = _slice(before, lo, hi), _slice(after, lo, hi)
+        out = first if (slices == 1 and amax_in is None) else run(b, amax_in)
+        assert (a["s_m"], a["s_v"], a["s_w"]) == (out["s_m"], out["s_v"], out["s_w"])
+        # master within 1 FP16 ULP (+ the binary32 step term); second moment within 1 FP16 ULP
+        slack = STEP_ROUNDINGS * 2.0 ** -24 * adam_step_magnitude(b, step)
+        for key, okey, skey in (("w", "wh", "s_w"), ("v", "vh", "s_v")):
+            ref = f16_vals(out[okey]) / out[skey]
+            got = f16_vals(a[key]) / a[skey]
+            ulp = f16_ulp(f16_vals(out[okey])) / out[skey]
+            if key == "w":
+                ulp = ulp * (1.0 + 2.0 ** -12) + slack
+            bad = np.abs(got - ref) > ulp
+            assert not np.any(bad), (key, lo, np.count_nonzero(bad), got[bad][:4], ref[bad][:4])
+        # first moment within 1 code (scales equal)
+        assert np.all(np.abs(code_rank(a["m"]) - code_rank(out["mq"])) <= 1), lo
+    return first if slices == 1 and amax_in is None else out
 
 
 @pytest.mark.parametrize("sizes", [[65536], [1, 7, 16, 4099, 65536 + 5, 0], [300000, 4096 * 3]])
@@ -434,9 +486,11 @@ def test_adam_step_vs_oracle(sizes, steps_done):
     before = [snapshot(c) for c in chunks]
     fp8.fp8_adam_step(chunks, step=step, margin=0, workspace=ws, **HP)
     assert fp8.fp8_get_status() == 0
+    ties = []
     for b, c in zip(before, chunks):
         if b["g"].size:
-            check_adam_chunk(b, c, step)
+            check_adam_chunk(b, c, step, ties=ties)
+    assert len(ties) <= MAX_TIES, ties
 
 
 def test_adam_subnormal_second_moment():
@@ -444,7 +498,7 @@ def test_adam_subnormal_second_moment():
     (1 - beta2) g^2 lies in [2^-136.3, 2^-134.3), a binary32 subnormal, and
     its scale is the clamped 2^126.  The codes and scales match the oracle, so
     the packed multiply-adds keep subnormals (flushed, v would be 0 with scale
-    1); the step matches, so the flush-to-zero square root changes nothing
+    1), and so does the correctly rounded square root; the step matches
     (sqrt(v_hat) ~ 2^-66 is far below half an ULP of eps = 1e-8).  The stored
     v * 2^126 lies in [2^-10.3, 2^-8.3), where binary32's subnormal spacing
     (2^-149, i.e. 2^-23 after scaling) is far below an FP16 ULP."""
@@ -481,8 +535,10 @@ def test_adam_many_chunks_multiple_launches():
     ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(chunks)) // 4, **F32)
     before = [snapshot(c) for c in chunks]
     fp8.fp8_adam_step(chunks, step=1, margin=0, workspace=ws, **HP)
+    ties = []
     for i in (0, 1, 255, 256, 299):
-        check_adam_chunk(before[i], chunks[i], 1)
+        check_adam_chunk(before[i], chunks[i], 1, ties=ties)
+    assert len(ties) <= MAX_TIES, ties
 
 
 def test_adam_rejects_bad_args():
@@ -518,6 +574,7 @@ def test_adam_tracked_master_amax_matches_untracked(sizes):
     ref = make_adam_state(sizes, ("adam-track",))
     trk = _with_tracking(make_adam_state(sizes, ("adam-track",)), wq=True)
     ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(ref)) // 4, **F32)
+    ties = []
     for step in (1, 2, 3):
         before = [snapshot(c) for c in trk]
         fp8.fp8_adam_step(ref, step=step, margin=0, workspace=ws, **HP)
@@ -532,7 +589,8 @@ def test_adam_tracked_master_amax_matches_untracked(sizes):
             assert t.wq_scale.item() == s_q and t.wq_inv.item() == 1.0 / s_q
             assert np.array_equal(t.wq.cpu().numpy(), q)
             if b["g"].size:
-                check_adam_chunk(b, t, step)
+                check_adam_chunk(b, t, step, ties=ties)
+    assert len(ties) <= MAX_TIES, ties
 
 
 def test_adam_mixed_tracked_and_untracked_chunks_in_one_launch():
@@ -646,6 +704,7 @@ def test_adam_sharded_ranks_equal_whole_tensor_step(world, wq):
     ranks = [[zero.shard_chunk(c, lo, hi) for c, (lo, hi) in zip(full, bounds[r])] for r in range(world)]
     ws_ref = torch.zeros(fp8.fp8_adam_workspace_bytes(len(sizes)) // 4, **F32)
     ws = [torch.zeros_like(ws_ref) for _ in range(world)]
+    ties = []
     for step in (1, 2):
         before = [snapshot(c) for c in ref]
         fp8.fp8_adam_step(ref, step=step, margin=0, workspace=ws_ref, **HP)
@@ -671,7 +730,8 @@ def test_adam_sharded_ranks_equal_whole_tensor_step(world, wq):
             if wq:
                 assert torch.equal(full[k].wq, c.wq)
             if before[k]["g"].size:
-                check_adam_chunk(before[k], c, step)
+                check_adam_chunk(before[k], c, step, ties=ties)
+    assert len(ties) <= MAX_TIES, ties
 
 
 def test_adam_sharded_halves_reject_tracking_and_bad_workspace():
