@@ -99,26 +99,34 @@ def gemm_traffic(workload: str):
 
 
 def load_peaks():
+    """Measured peaks of this machine's B200s (generated file), else the
+    profiling recipe's fallback.  `sus_mhz`: the median SM clock of the
+    sustained measurement, when the file records one."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         p = json.load(open(path))
+        sus_mhz = None
+        for k, v in p.items():
+            kl = k.lower()
+            if "sustained" in kl and ("mhz" in kl or "clock" in kl) and isinstance(v, (int, float)):
+                sus_mhz = float(v)
         return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sus=p["bf16_tflops_sustained"],
-                    src="measured")
+                    sus_mhz=sus_mhz, src="measured")
     except Exception:
-        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, sus_mhz=1300.0, src="fallback")
 
 
 def fp8_peak(peaks: dict, clocks: dict):
     """Dense FP8 peak = 2 x the bf16 peak (the nominal 4.5 / 2.25 ratio).  The
-    burst figure when the timed region ran at the maximum SM clock (within
-    3 %), else the sustained one (measured under the power cap at a lower
-    clock).  Returns (peak TFLOP/s, source text)."""
-    mhz, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
-    if mhz is not None and mx and mhz < 0.97 * mx:
-        return 2.0 * peaks["bf16_sus"], (f"2 x bf16_tflops_sustained ({peaks['src']}): median SM clock "
-                                         f"{mhz} MHz below the {mx} MHz maximum")
+    sustained figure only when the timed region's median SM clock matches the
+    clock of the sustained measurement (within 5 %); otherwise the burst
+    figure, the larger one.  Returns (peak TFLOP/s, source text)."""
+    mhz, mx, sus = clocks.get("sm_mhz"), clocks.get("sm_max_mhz"), peaks.get("sus_mhz")
+    if mhz is not None and sus and mhz <= 1.05 * sus:
+        return 2.0 * peaks["bf16_sus"], (f"2 x bf16_tflops_sustained ({peaks['src']}): median SM clock {mhz} MHz "
+                                         f"matches the sustained measurement's {sus} MHz")
     return 2.0 * peaks["bf16"], (f"2 x bf16_tflops, burst ({peaks['src']}): median SM clock {mhz} MHz "
-                                 f"of {mx} MHz maximum")
+                                 f"(max {mx} MHz; sustained measurement at {sus} MHz)")
 
 
 # ---------------------------------------------------------------- clocks

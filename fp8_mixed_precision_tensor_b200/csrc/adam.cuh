@@ -124,6 +124,34 @@ __device__ __forceinline__ void adam_moments(const AdamLaunch &L, float2 gd, flo
   dw = __fmul2_rn(both(L.neg_lr_bc1), make_float2(__fdiv_rn(m.x, den.x), __fdiv_rn(m.y, den.y)));
 }
 
+// The same moments and an upper-bound estimate of the step, with the MUFU
+// square root and reciprocal (flush-to-zero) in place of the correctly
+// rounded operations: for the tracked master's interval only, which needs a
+// bound U >= max |dw|, not the step itself.  The approximations' relative
+// errors (a few 2^-23) are covered by widening U by 2^-16 in the finalize
+// stage; the flush changes nothing because eps >= 2^-39 makes
+// sqrt(v_hat) + eps round to eps for every subnormal v_hat.  The update pass
+// checks the scale this bound selected against the exact new amax.
+__device__ __forceinline__ float sqrt_approx(float x) {
+  float r;
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void adam_moments_bound(const AdamLaunch &L, float2 gd, float2 md, float2 vd,
+                                                   const AdamScalars &s, float2 &m, float2 &v, float2 &dw) {
+  m = __ffma2_rn(s.cm, md, __fmul2_rn(s.cgm, gd));
+  v = __ffma2_rn(s.cv, vd, __fmul2_rn(__fmul2_rn(s.cgv, gd), __fmul2_rn(s.g_inv, gd)));
+  const float2 vh = __fmul2_rn(v, both(L.inv_bc2));
+  const float2 den = __fadd2_rn(make_float2(sqrt_approx(vh.x), sqrt_approx(vh.y)), both(L.eps));
+  dw = __fmul2_rn(both(L.neg_lr_bc1), __fmul2_rn(m, make_float2(rcp_approx(den.x), rcp_approx(den.y))));
+}
+constexpr float kStepBoundWiden = 1.0f + 0x1p-16f;
+
 // w = w0 + dw as one rounding per parameter (the master's new value).
 __device__ __forceinline__ float2 adam_master(float2 wd, float2 dw, const AdamScalars &s) {
   return __fadd2_rn(__fmul2_rn(wd, s.w_inv), dw);
@@ -212,7 +240,10 @@ __device__ __forceinline__ void adam_group(const AdamLaunch &L, const AdamChunkD
     const uint32_t g2 = (gw[p >> 1] >> ((p & 1) * 16)) & 0xffffu;
     const uint32_t m2 = (mw[p >> 1] >> ((p & 1) * 16)) & 0xffffu;
     float2 m, v, d;
-    adam_moments(L, dec2<FP8_E5M2>(g2), dec2<FP8_E4M3>(m2), h2f2(vw[p]), sc, m, v, d);
+    if constexpr (PASS == 1 && TRACK)  // only the bound U >= max |dw| is needed
+      adam_moments_bound(L, dec2<FP8_E5M2>(g2), dec2<FP8_E4M3>(m2), h2f2(vw[p]), sc, m, v, d);
+    else
+      adam_moments(L, dec2<FP8_E5M2>(g2), dec2<FP8_E4M3>(m2), h2f2(vw[p]), sc, m, v, d);
     if constexpr (PASS == 1) {
       am = max_abs2(am, m);
       av = max_abs2(av, v);
@@ -249,10 +280,15 @@ __device__ __forceinline__ void adam_group(const AdamLaunch &L, const AdamChunkD
   }
 }
 
-// One pass over all tiles of a launch.  PASS 1: stats.  PASS 3: exact master
-// amax of flagged chunks.  PASS 2: update.
+// One pass over all tiles of a launch.  PASS 1: stats of the chunks that do
+// not track their master amax (exact new amaxes).  PASS 4: stats of the
+// chunks that do (amax of m and v, the step bound U).  PASS 3: exact master
+// amax of flagged chunks.  PASS 2: update.  The two stats passes are separate
+// kernels so that the bound-only arithmetic of PASS 4 does not carry the
+// register count of the exact one.
 template <int PASS>
 __device__ __forceinline__ void adam_pass(const AdamLaunch &L) {
+  constexpr bool kStats = PASS == 1 || PASS == 4;
   float am = 0.f, av = 0.f, aw = 0.f;  // running maxima of the current chunk
   int cur = -1;
   bool tracked = false, active = true, want_wq = false;
@@ -264,16 +300,17 @@ __device__ __forceinline__ void adam_pass(const AdamLaunch &L) {
     const AdamChunkDev &C = L.c[ci];
     if (ci != cur) {
       if (cur >= 0) {
-        if constexpr (PASS == 1)
-          flush_max3(L, cur, WS_AMAX_M, am, WS_AMAX_V, av, tracked ? WS_STEP_MAX : WS_AMAX_W, aw);
+        if constexpr (kStats)
+          if (active) flush_max3(L, cur, WS_AMAX_M, am, WS_AMAX_V, av, tracked ? WS_STEP_MAX : WS_AMAX_W, aw);
         if constexpr (PASS == 3)
           if (active) flush_max3(L, cur, WS_AMAX_W, aw, WS_AMAX_W, aw, WS_AMAX_W, aw);
         if constexpr (PASS == 2) flush_max3(L, cur, WS_STORED_W, am, WS_CHECK_W, aw, WS_CHECK_W, aw);
         am = av = aw = 0.f;
       }
       cur = ci;
-      if constexpr (PASS == 1) {
+      if constexpr (kStats) {
         tracked = C.w_amax != nullptr && *C.w_amax >= 0.0f;
+        active = tracked == (PASS == 4);
         sc = adam_scalars(L, *C.g_inv, 1.0f / *C.m_scale, 1.0f / *C.v_scale, 1.0f / *C.w_scale);
       } else {
         const uint32_t fl = ws_flags(L, ci);
@@ -291,15 +328,21 @@ __device__ __forceinline__ void adam_pass(const AdamLaunch &L) {
         ns.wq = both(want_wq ? ws_get(L, ci, WS_NEW_WQ) : 1.0f);
       }
     }
-    if (!active) continue;  // pass 1b: chunk not flagged
+    if (!active) {  // pass 1b: chunk not flagged; stats: the other stats pass's chunk
+      // jump to this block's last tile inside the chunk; the loop step leaves it
+      const unsigned long long end = C.tile_begin + (C.n + kAdamTile - 1) / kAdamTile;
+      tile += ((end - tile - 1) / gridDim.x) * gridDim.x;
+      continue;
+    }
     const unsigned long long base =
         (tile - C.tile_begin) * kAdamTile + (unsigned long long)threadIdx.x * kAdamPerThread;
     if (base >= C.n) continue;
     if (base + kAdamPerThread <= C.n) {
       const size_t grp = base / kAdamPerThread;
-      if constexpr (PASS == 1) {
-        if (tracked) adam_group<1, true, false>(L, C, grp, sc, ns, am, av, aw);
-        else adam_group<1, false, false>(L, C, grp, sc, ns, am, av, aw);
+      if constexpr (PASS == 4) {
+        adam_group<1, true, false>(L, C, grp, sc, ns, am, av, aw);
+      } else if constexpr (PASS == 1) {
+        adam_group<1, false, false>(L, C, grp, sc, ns, am, av, aw);
       } else if constexpr (PASS == 3) {
         adam_group<3, false, false>(L, C, grp, sc, ns, am, av, aw);
       } else {
@@ -307,14 +350,17 @@ __device__ __forceinline__ void adam_pass(const AdamLaunch &L) {
       }
     } else {
       // Ragged end of a chunk: element by element (lane y unused).
-      const bool read_w = PASS != 1 || !tracked;
+      const bool read_w = PASS != 4;
       for (unsigned long long i = base; i < C.n; i++) {
         const float2 gd = dec2<FP8_E5M2>(C.g[i]), md = dec2<FP8_E4M3>(C.m[i]);
         const float2 vd = make_float2(__half2float(__ushort_as_half(C.v[i])), 0.0f);
         const float2 wd = make_float2(read_w ? __half2float(__ushort_as_half(C.w[i])) : 0.0f, 0.0f);
         float2 m, v, d;
-        adam_moments(L, make_float2(gd.x, 0.0f), make_float2(md.x, 0.0f), vd, sc, m, v, d);
-        if constexpr (PASS == 1) {
+        if constexpr (PASS == 4)
+          adam_moments_bound(L, make_float2(gd.x, 0.0f), make_float2(md.x, 0.0f), vd, sc, m, v, d);
+        else
+          adam_moments(L, make_float2(gd.x, 0.0f), make_float2(md.x, 0.0f), vd, sc, m, v, d);
+        if constexpr (kStats) {
           am = max_abs1(am, m.x);
           av = max_abs1(av, v.x);
           aw = max_abs1(aw, tracked ? d.x : adam_master(wd, d, sc).x);
@@ -337,8 +383,8 @@ __device__ __forceinline__ void adam_pass(const AdamLaunch &L) {
   }
   // cur is block-uniform, so whole warps take these branches together.
   if (cur >= 0) {
-    if constexpr (PASS == 1)
-      flush_max3(L, cur, WS_AMAX_M, am, WS_AMAX_V, av, tracked ? WS_STEP_MAX : WS_AMAX_W, aw);
+    if constexpr (kStats)
+      if (active) flush_max3(L, cur, WS_AMAX_M, am, WS_AMAX_V, av, tracked ? WS_STEP_MAX : WS_AMAX_W, aw);
     if constexpr (PASS == 3)
       if (active) flush_max3(L, cur, WS_AMAX_W, aw, WS_AMAX_W, aw, WS_AMAX_W, aw);
     if constexpr (PASS == 2) flush_max3(L, cur, WS_STORED_W, am, WS_CHECK_W, aw, WS_CHECK_W, aw);
@@ -354,6 +400,11 @@ __global__ void __launch_bounds__(kAdamThreads) k_adam(const __grid_constant__ A
 template <>
 __global__ void __launch_bounds__(kAdamThreads, 5) k_adam<2>(const __grid_constant__ AdamLaunch L) {
   adam_pass<2>(L);
+}
+// The bound-only stats pass of tracking chunks: six resident blocks per SM.
+template <>
+__global__ void __launch_bounds__(kAdamThreads, 6) k_adam<4>(const __grid_constant__ AdamLaunch L) {
+  adam_pass<4>(L);
 }
 
 // Exponent of the E4M3 copy's scale from an amax of the stored master: the
@@ -384,7 +435,7 @@ __global__ void k_adam_finalize(const __grid_constant__ AdamLaunch L) {
       bool exact = !tracked;
       if (tracked) {
         // amax|w_new| lies in [A0 - U, A0 + U], widened for the one rounding of w0 + dw
-        const float a0 = *C.w_amax, u = ws[WS_STEP_MAX];
+        const float a0 = *C.w_amax, u = __fmul_ru(ws[WS_STEP_MAX], kStepBoundWiden);
         const float hi = __fmul_rn(__fadd_ru(a0, u), 1.0f + 0x1p-20f);
         const float lo = __fmul_rn(__fsub_rd(a0, u), 1.0f - 0x1p-20f);
         int klo, khi;

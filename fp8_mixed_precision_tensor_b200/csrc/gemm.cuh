@@ -112,19 +112,36 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // Bounded wait on one phase of an mbarrier.  Returns false on timeout (after
 // raising the status bit and the CTA's abort flag) or when another role of
-// the CTA has already aborted.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+// the CTA has already aborted.  limit_ns: kTimeoutNs in the GEMMs.
+__device__ __noinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                           uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer_ns();
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > kTimeoutNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       atomicOr(&g_status, FP8_STATUS_TIMEOUT);
       *abort_flag = 1;
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+  return mbar_wait_for(bar, parity, abort_flag, kTimeoutNs);
+}
+
+// Self-test of the wait above: one thread waits on a barrier that nothing
+// arrives at, with a short limit, and must come back with the timeout status
+// raised (the GEMMs' abort path starts from exactly this return).
+__global__ void k_wait_selftest(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  abort_flag = 0;
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  mbar_wait_for(b, 0, &abort_flag, limit_ns);
 }
 
 // A wait used only while tearing down after an abort: bounded, no flag check.

@@ -28,7 +28,8 @@ struct DeviceInfo {
   bool ready = false;
   int sms = 0;
   int adam_blocks_per_sm = 1;        // resident blocks of the update pass
-  int adam_stats_blocks_per_sm = 1;  // of the stats passes (fewer registers)
+  int adam_stats_blocks_per_sm = 1;  // of the exact stats pass and the exact master pass
+  int adam_bound_blocks_per_sm = 1;  // of the bound-only stats pass of tracking chunks
   int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair GEMM
   int wide_clusters = 0;  // co-resident 2-CTA clusters of the wide pair GEMM
 };
@@ -67,6 +68,9 @@ int device_info(DeviceInfo **out) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k_adam<1>, kAdamThreads, 0) != cudaSuccess)
       return FP8_ERR_CUDA;
     d.adam_stats_blocks_per_sm = bps > 0 ? bps : 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k_adam<4>, kAdamThreads, 0) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    d.adam_bound_blocks_per_sm = bps > 0 ? bps : 1;
     int rc = FP8_OK;
     rc |= set_smem(gemm::k_gemm<256, false, false>, gemm::Cfg<256>::SMEM_BYTES);
     rc |= set_smem(gemm::k_gemm<256, false, true>, gemm::Cfg<256>::SMEM_BYTES);
@@ -470,6 +474,7 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
   L.inv_bc2 = (float)(1.0 / (1.0 - pow((double)hp->beta2, (double)hp->step)));
   const unsigned cap = (unsigned)(d->sms * d->adam_blocks_per_sm);
   const unsigned cap1 = (unsigned)(d->sms * d->adam_stats_blocks_per_sm);
+  const unsigned cap4 = (unsigned)(d->sms * d->adam_bound_blocks_per_sm);
   for (int first = 0; first < nchunks; first += kAdamMaxChunksPerLaunch) {
     const int cnt = nchunks - first < kAdamMaxChunksPerLaunch ? nchunks - first : kAdamMaxChunksPerLaunch;
     unsigned long long tiles = 0;
@@ -488,9 +493,16 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
     L.ws = reinterpret_cast<float *>(workspace) + (size_t)first * kAdamWsFloatsPerChunk;
     const unsigned grid = tiles == 0 ? 1u : (unsigned)(tiles < cap ? tiles : cap);
     const unsigned grid1 = tiles == 0 ? 1u : (unsigned)(tiles < cap1 ? tiles : cap1);
+    const unsigned grid4 = tiles == 0 ? 1u : (unsigned)(tiles < cap4 ? tiles : cap4);
     bool tracked = false;
     for (int i = 0; i < cnt; i++) tracked |= L.c[i].w_amax != nullptr;
-    if (phases & PH_STATS) k_adam<1><<<grid1, kAdamThreads, 0, s>>>(L);  // stats
+    if (phases & PH_STATS) {
+      // exact stats of the chunks without a known tracked amax (whether a
+      // tracking chunk's amax is known yet is only visible on the device);
+      // the bound-only stats of those with one
+      k_adam<1><<<grid1, kAdamThreads, 0, s>>>(L);
+      if (tracked) k_adam<4><<<grid4, kAdamThreads, 0, s>>>(L);
+    }
     if (phases & PH_APPLY) {
       if (tracked) {
         k_adam_finalize<1><<<1, 256, 0, s>>>(L);
@@ -556,6 +568,12 @@ int fp8_adam_step_noalloc(const fp8_adam_chunk *chunks, int nchunks, const fp8_a
   if (rc) return rc;
   return fp8_adam_step(chunks, nchunks, hp, scratch,
                        (size_t)FP8_ADAM_NOALLOC_MAX_CHUNKS * kAdamWsFloatsPerChunk * sizeof(float), stream);
+}
+
+int fp8_selftest_wait_timeout(unsigned limit_us, void *stream) {
+  if (limit_us == 0 || limit_us > 1000000u) return FP8_ERR_INVALID_ARG;
+  gemm::k_wait_selftest<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>((uint64_t)limit_us * 1000ull);
+  return launch_rc();
 }
 
 int fp8_get_status(unsigned *host_out, void *stream) {

@@ -31,7 +31,7 @@ SYMBOLS = ("fp8_amax", "fp8_compute_scale", "fp8_cast", "fp8_scale_cast", "fp8_c
            "fp8_sum_codes", "fp8_mu_update", "fp8_linear_fwd", "fp8_linear_dgrad",
            "fp8_linear_wgrad", "fp8_adam_workspace_bytes", "fp8_adam_step", "fp8_adam_stats",
            "fp8_adam_apply", "fp8_adam_step_noalloc",
-           "fp8_get_status", "fp8_strerror")
+           "fp8_selftest_wait_timeout", "fp8_get_status", "fp8_strerror")
 
 
 class FP8Error(RuntimeError):
@@ -85,6 +85,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     for name in ("fp8_adam_step", "fp8_adam_stats", "fp8_adam_apply"):
         getattr(lib, name).argtypes = [ctypes.POINTER(_Chunk), i, ctypes.POINTER(_HParams), p, sz, p]
     lib.fp8_adam_step_noalloc.argtypes = [ctypes.POINTER(_Chunk), i, ctypes.POINTER(_HParams), p]
+    lib.fp8_selftest_wait_timeout.argtypes = [ctypes.c_uint, p]
     lib.fp8_get_status.argtypes = [ctypes.POINTER(ctypes.c_uint), p]
     lib.fp8_strerror.argtypes, lib.fp8_strerror.restype = [i], ctypes.c_char_p
     for name in SYMBOLS:
@@ -286,6 +287,13 @@ def fp8_adam_step_noalloc(chunks, lr: float, beta1: float, beta2: float, eps: fl
     hp = _HParams(lr, beta1, beta2, eps, step, margin)
     _check(load_library().fp8_adam_step_noalloc(arr, len(arr), ctypes.byref(hp), _stream(stream)),
            "fp8_adam_step_noalloc")
+
+
+def fp8_selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    """Run the GEMM pipeline's bounded wait on a barrier nothing arrives at
+    (limit in microseconds); it must end and raise FP8_STATUS_TIMEOUT."""
+    _check(load_library().fp8_selftest_wait_timeout(ctypes.c_uint(limit_us), _stream(stream)),
+           "fp8_selftest_wait_timeout")
 
 
 def fp8_get_status(stream=None) -> int:

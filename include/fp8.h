@@ -378,6 +378,18 @@ int fp8_adam_step_noalloc(const fp8_adam_chunk *chunks, int nchunks, const fp8_a
  */
 int fp8_get_status(unsigned *host_out, void *stream);
 
+/*
+ * fp8_selftest_wait_timeout -- failure-detection self-test.  Enqueues one
+ * thread that runs the GEMM pipeline's bounded barrier wait on a barrier
+ * that nothing ever arrives at, with a limit of limit_us microseconds
+ * (1 .. 1,000,000) instead of the GEMMs' 2 s.  The wait must end by itself
+ * and raise FP8_STATUS_TIMEOUT in the status word (read it with
+ * fp8_get_status); the context stays usable.  Returns FP8_ERR_INVALID_ARG
+ * for a limit outside the range, nothing enqueued.  The pages have no
+ * counterpart; it checks the library's own hang protection.
+ */
+int fp8_selftest_wait_timeout(unsigned limit_us, void *stream);
+
 /* Human-readable message of a status code (static string). */
 const char *fp8_strerror(int code);
 

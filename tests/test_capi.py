@@ -146,3 +146,9 @@ def test_adam_rejects_hyper_parameters_outside_the_argued_range(lib):
         hp = fp8._HParams(lr, b1, b2, eps, t, 0)
         assert lib.fp8_adam_step(arr, 1, ctypes.byref(hp), fake, 64, None) == fp8.FP8_ERR_INVALID_ARG, \
             (lr, b1, b2, eps, t)
+
+
+def test_wait_selftest_rejects_limits_outside_its_range(lib):
+    lib.fp8_selftest_wait_timeout.argtypes = [ctypes.c_uint, ctypes.c_void_p]
+    assert lib.fp8_selftest_wait_timeout(0, None) == 1
+    assert lib.fp8_selftest_wait_timeout(1000001, None) == 1

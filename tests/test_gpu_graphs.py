@@ -77,3 +77,4 @@ def test_adam_step_in_a_cuda_graph_equals_eager():
         sa, sb = snapshot(a), snapshot(b)
         for k in ("m", "v", "w", "s_m", "s_v", "s_w"):
             assert np.array_equal(np.asarray(sa[k]), np.asarray(sb[k])), k
+
