@@ -266,8 +266,14 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Arrive on a barrier of the peer CTA.  Relaxed: every use hands over a
+// resource (a TMEM accumulator whose tcgen05.ld have completed, a ring slot
+// whose MMAs have completed) that the arriving thread did not write through
+// generic memory, so no release ordering is needed; a release.cluster arrive
+// measured about 1.2 us per hand-over on B200, a relaxed one the same as a
+// local arrive.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // TMA load whose completion is counted on a barrier that may live in the
@@ -793,20 +799,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Per k-slice the leader issues two tcgen05.mma.cta_group::2 (M = 256,
 // N = 256), one into each of two accumulators that together fill all 512
 // TMEM columns.  Each CTA loads its 128 rows of A (16 KB) and 256 rows of B
-// (32 KB) per stage: the same A tile now feeds twice the tensor-core work,
-// so each SM streams 48 KB per 2 x 128x256x128 MACs instead of 32 KB per one.
-// Column bookkeeping: CTA r holds B rows (output columns) [r*256, r*256+256)
-// of the tile; the MMA reading B rows [0,128) of both CTAs produces tile
-// columns {0..127, 256..383} in accumulator 0, and rows [128,256) produce
-// {128..255, 384..511} in accumulator 1.  There is no room left in TMEM for a
-// second tile, so the epilogue (eight warps, one accumulator half each)
-// runs between tiles while the producer already refills the ring.
+// (32 KB) per stage into a 3-stage ring: the same A tile feeds twice the
+// tensor-core work, so each SM streams 48 KB per 2 x 128x256x128 MACs
+// instead of 32 KB per one.  Column bookkeeping: CTA r holds B rows (output
+// columns) [r*256, r*256+256) of the tile; the MMA reading B rows [0,128) of
+// both CTAs produces tile columns {0..127, 256..383} in accumulator 0, and
+// rows [128,256) produce {128..255, 384..511} in accumulator 1.  There is no
+// room left in TMEM for a second tile, so the epilogue runs between tiles
+// while the producer already refills the ring; it hands the accumulator back
+// right after its last TMEM read and drains its staged output with pipelined
+// bulk stores (two staging boxes per epilogue warp).  The MMAs' commits free
+// the leader's ring slots; a relay warp frees the follower's copy of each
+// slot with a remote arrive once the leader's slot is free.  Warps: 0
+// producer (both CTAs), 1 TMEM allocation and MMA issue (leader), 2-9
+// epilogue (both CTAs), 10 release relay (leader).
 constexpr int kWideBN = 512;
-constexpr int kWideStages = 4;
+constexpr int kWideStages = 3;
 constexpr int kWideStageBytes = kPairHalf * BK + 2 * kPairHalf * BK;  // A 16 KB + B 32 KB
-constexpr int kWideThreads = 320;                                     // 10 warps
+constexpr int kWideThreads = 352;                                     // 11 warps
 constexpr int kWideStageOutBytes = 32 * 128;                             // per epilogue warp: 32 rows x 128 B
-constexpr int kWideSmemBytes = kWideStages * kWideStageBytes + 8 * kWideStageOutBytes + 256 + 1024;
+constexpr int kWideOutBoxes = 2;  // staging boxes per epilogue warp (stores pipelined)
+constexpr int kWideSmemBytes = kWideStages * kWideStageBytes + 8 * kWideOutBoxes * kWideStageOutBytes + 256 + 1024;
 
 template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(kWideThreads, 1)
@@ -816,8 +829,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t *base_ptr = smem_raw + (base - raw);
-  const uint32_t out_stage0 = base + kWideStages * kWideStageBytes;  // 8 x 4 KB, 1024-aligned
-  const uint32_t bar0 = out_stage0 + 8 * kWideStageOutBytes;
+  const uint32_t out_stage0 = base + kWideStages * kWideStageBytes;  // 8 x 2 x 4 KB, 1024-aligned
+  const uint32_t bar0 = out_stage0 + 8 * kWideOutBoxes * kWideStageOutBytes;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (kWideStages + s); };
   const uint32_t tfull_bar = bar0 + 8u * (2 * kWideStages);
@@ -916,7 +929,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
               tc_mma_pair_lastuse_a(tmem_base + 256, ad, operand_desc<B_MN>(sb + kPairHalf * BK, ks), args.idesc,
                                     accum);
             }
-            tc_commit_pair(empty_bar(stage));
+            // the leader's own ring slot; the relay warp frees the follower's
+            asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                             empty_bar(stage))
+                         : "memory");
             issued_any = true;
           }
           __syncwarp();
@@ -933,6 +949,23 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         mbar_wait_drain(drain_bar, 0);
       }
     }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ release relay (leader only)
+    // Once the MMAs that read a ring slot have completed (the leader's empty
+    // barrier), free the follower's copy of that slot with a relaxed remote
+    // arrive: the reads are over before the arrive is issued.
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < args.num_tiles && ok; tile += num_pairs) {
+        for (int kb = 0; kb < args.num_k_blocks; kb++) {
+          if (!mbar_wait(empty_bar(stage), phase, abort_flag)) { ok = false; break; }
+          mbar_arrive_remote(map_to_rank(empty_bar(stage), 1));
+          if (++stage == kWideStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue (8 warps, both CTAs)
     // Each warp drains 32 rows x 256 columns of one accumulator half in
@@ -945,7 +978,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     const float inv_ab = __fmul_rn(inv_a, inv_b);
     // one multiplication when the folded factor is a normal float
     const bool fold = fabsf(inv_ab) >= 1.17549435e-38f && fabsf(inv_ab) <= 3.402823466e38f;
-    const uint32_t stg = out_stage0 + (warp - 2) * kWideStageOutBytes;
+    const uint32_t stg0 = out_stage0 + (warp - 2) * kWideOutBoxes * kWideStageOutBytes;
+    uint32_t box = 0;
     const bool f32out = args.out_dtype == FP8_DT_F32;
     const bool bfout = args.out_dtype == FP8_DT_BF16;
     uint32_t acc_phase = 0;
@@ -966,11 +1000,17 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < 256; c += cols_per_box) {
         const int col0 = nb * kWideBN + (c < 128 ? 0 : 256) + h * kPairHalf + (c & 127);
+        const bool last = c + cols_per_box >= 256;
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + h * 256 + c, r);
         if (fold) descale1_chunk(args, r, col0, inv_ab); else descale_chunk(args, r, col0, inv_a, inv_b);
         uint32_t w[32];  // the row's 128 bytes as 32 words
         if (f32out) {
+          if (last) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(map_to_rank(tempty_bar, 0));
+          }
 #pragma unroll
           for (int j = 0; j < 32; j++) {
             w[j] = r[j];
@@ -979,6 +1019,11 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         } else {
           uint32_t r2[32];
           tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + h * 256 + c + 32, r2);
+          if (last) {  // the tile's last TMEM read: hand the accumulator back now
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(map_to_rank(tempty_bar, 0));
+          }
           if (fold) descale1_chunk(args, r2, col0 + 32, inv_ab); else descale_chunk(args, r2, col0 + 32, inv_a, inv_b);
 #pragma unroll
           for (int j = 0; j < 16; j++) {
@@ -1000,8 +1045,12 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             w[16 + j] = pb;
           }
         }
-        // the staging box must be free: the previous bulk store has read it
-        if (lane == 0) bulk_wait_read0();
+        // this staging box must be free: the store that used it two boxes ago
+        // has read it (every box commits one bulk group, empty when it stores
+        // nothing, so "at most one group pending" means exactly that)
+        const uint32_t stg = stg0 + box * kWideStageOutBytes;
+        box ^= 1u;
+        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
         __syncwarp();
 #pragma unroll
         for (int ch = 0; ch < 8; ch++) {  // 16-byte chunk ch of this row, 128B swizzle
@@ -1010,14 +1059,11 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         }
         fence_async_shared();
         __syncwarp();
-        if (lane == 0 && rows_in && col0 < args.cols) {
-          tma_store_2d(&tmOut, stg, col0, row0);
+        if (lane == 0) {
+          if (rows_in && col0 < args.cols) tma_store_2d(&tmOut, stg, col0, row0);
           bulk_commit();
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(map_to_rank(tempty_bar, 0));
       if (!f32out) {
         const uint32_t h16 = max(amax16 & 0xffffu, amax16 >> 16);
         amax_bits = bfout ? (h16 << 16) : absbits_f32(__half2float(__ushort_as_half((unsigned short)h16)));
