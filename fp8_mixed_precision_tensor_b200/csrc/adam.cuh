@@ -280,6 +280,93 @@ __device__ __forceinline__ void adam_group(const AdamLaunch &L, const AdamChunkD
   }
 }
 
+// Per-chunk state of a pass: what a block sets up when its tile walk enters a
+// new chunk, and the running maxima it folds into the chunk's workspace slots
+// when it leaves.
+struct AdamChunkState {
+  float am = 0.f, av = 0.f, aw = 0.f;  // running maxima of the current chunk
+  int cur = -1;
+  bool tracked = false, active = true, want_wq = false;
+  AdamScalars sc{};
+  AdamNewScales ns{both(1.f), both(1.f), both(1.f), both(1.f), both(1.f)};
+};
+
+template <int PASS>
+__device__ __forceinline__ void adam_chunk_flush(const AdamLaunch &L, AdamChunkState &S) {
+  constexpr bool kStats = PASS == 1 || PASS == 4;
+  if constexpr (kStats)
+    if (S.active) flush_max3(L, S.cur, WS_AMAX_M, S.am, WS_AMAX_V, S.av, S.tracked ? WS_STEP_MAX : WS_AMAX_W, S.aw);
+  if constexpr (PASS == 3)
+    if (S.active) flush_max3(L, S.cur, WS_AMAX_W, S.aw, WS_AMAX_W, S.aw, WS_AMAX_W, S.aw);
+  if constexpr (PASS == 2) flush_max3(L, S.cur, WS_STORED_W, S.am, WS_CHECK_W, S.aw, WS_CHECK_W, S.aw);
+  S.am = S.av = S.aw = 0.f;
+}
+
+template <int PASS>
+__device__ __forceinline__ void adam_chunk_enter(const AdamLaunch &L, int ci, AdamChunkState &S) {
+  constexpr bool kStats = PASS == 1 || PASS == 4;
+  const AdamChunkDev &C = L.c[ci];
+  S.cur = ci;
+  if constexpr (kStats) {
+    S.tracked = C.w_amax != nullptr && *C.w_amax >= 0.0f;
+    S.active = S.tracked == (PASS == 4);
+    S.sc = adam_scalars(L, *C.g_inv, 1.0f / *C.m_scale, 1.0f / *C.v_scale, 1.0f / *C.w_scale);
+  } else {
+    const uint32_t fl = ws_flags(L, ci);
+    // pass 2: keep the stored-master amax (and its check) for every chunk
+    // that tracks it, including the step that first establishes it
+    S.tracked = PASS == 2 ? C.w_amax != nullptr : (fl & 2u) != 0;
+    S.active = PASS == 2 || (fl & 1u) != 0;
+    S.sc = adam_scalars(L, *C.g_inv, ws_get(L, ci, WS_OLDINV_M), ws_get(L, ci, WS_OLDINV_V),
+                        ws_get(L, ci, WS_OLDINV_W));
+    S.ns.m = both(ws_get(L, ci, WS_NEW_M));
+    S.ns.v = both(ws_get(L, ci, WS_NEW_V));
+    S.ns.w = both(ws_get(L, ci, WS_NEW_W));
+    S.ns.inv_w = both(1.0f / S.ns.w.x);
+    S.want_wq = C.wq != nullptr;
+    S.ns.wq = both(S.want_wq ? ws_get(L, ci, WS_NEW_WQ) : 1.0f);
+  }
+}
+
+// The ragged end of a chunk, [base, n) with n - base < 16: element by element
+// from global memory (lane y of the packed arithmetic unused).
+template <int PASS>
+__device__ __forceinline__ void adam_tail(const AdamLaunch &L, const AdamChunkDev &C, unsigned long long base,
+                                       AdamChunkState &S) {
+  constexpr bool kStats = PASS == 1 || PASS == 4;
+  const bool read_w = PASS != 4;
+  const AdamScalars &sc = S.sc;
+  const AdamNewScales &ns = S.ns;
+  for (unsigned long long i = base; i < C.n; i++) {
+    const float2 gd = dec2<FP8_E5M2>(C.g[i]), md = dec2<FP8_E4M3>(C.m[i]);
+    const float2 vd = make_float2(__half2float(__ushort_as_half(C.v[i])), 0.0f);
+    const float2 wd = make_float2(read_w ? __half2float(__ushort_as_half(C.w[i])) : 0.0f, 0.0f);
+    float2 m, v, d;
+    if constexpr (PASS == 4)
+      adam_moments_bound(L, make_float2(gd.x, 0.0f), make_float2(md.x, 0.0f), vd, sc, m, v, d);
+    else
+      adam_moments(L, make_float2(gd.x, 0.0f), make_float2(md.x, 0.0f), vd, sc, m, v, d);
+    if constexpr (kStats) {
+      S.am = max_abs1(S.am, m.x);
+      S.av = max_abs1(S.av, v.x);
+      S.aw = max_abs1(S.aw, S.tracked ? d.x : adam_master(wd, d, sc).x);
+    } else if constexpr (PASS == 3) {
+      S.aw = max_abs1(S.aw, adam_master(wd, d, sc).x);
+    } else {
+      const float w = adam_master(wd, d, sc).x;
+      if (S.tracked) S.aw = max_abs1(S.aw, w);
+      C.m[i] = (uint8_t)(enc2<FP8_E4M3>(__fmul_rn(m.x, ns.m.x), 0.0f) & 0xffu);
+      C.v[i] = __half_as_ushort(__float2half_rn(__fmul_rn(v.x, ns.v.x)));
+      const __half h = __float2half_rn(__fmul_rn(w, ns.w.x));
+      C.w[i] = __half_as_ushort(h);
+      const float st = __half2float(h);
+      if (S.tracked) S.am = max_abs1(S.am, st);
+      if (S.want_wq)
+        C.wq[i] = (uint8_t)(enc2<FP8_E4M3>(__fmul_rn(__fmul_rn(st, ns.inv_w.x), ns.wq.x), 0.0f) & 0xffu);
+    }
+  }
+}
+
 // One pass over all tiles of a launch.  PASS 1: stats of the chunks that do
 // not track their master amax (exact new amaxes).  PASS 4: stats of the
 // chunks that do (amax of m and v, the step bound U).  PASS 3: exact master
@@ -288,47 +375,15 @@ __device__ __forceinline__ void adam_group(const AdamLaunch &L, const AdamChunkD
 // register count of the exact one.
 template <int PASS>
 __device__ __forceinline__ void adam_pass(const AdamLaunch &L) {
-  constexpr bool kStats = PASS == 1 || PASS == 4;
-  float am = 0.f, av = 0.f, aw = 0.f;  // running maxima of the current chunk
-  int cur = -1;
-  bool tracked = false, active = true, want_wq = false;
-  AdamScalars sc{};
-  AdamNewScales ns{both(1.f), both(1.f), both(1.f), both(1.f), both(1.f)};
-
+  AdamChunkState S;
   for (unsigned long long tile = blockIdx.x; tile < L.total_tiles; tile += gridDim.x) {
     const int ci = find_chunk(L, tile);  // uniform across the block
     const AdamChunkDev &C = L.c[ci];
-    if (ci != cur) {
-      if (cur >= 0) {
-        if constexpr (kStats)
-          if (active) flush_max3(L, cur, WS_AMAX_M, am, WS_AMAX_V, av, tracked ? WS_STEP_MAX : WS_AMAX_W, aw);
-        if constexpr (PASS == 3)
-          if (active) flush_max3(L, cur, WS_AMAX_W, aw, WS_AMAX_W, aw, WS_AMAX_W, aw);
-        if constexpr (PASS == 2) flush_max3(L, cur, WS_STORED_W, am, WS_CHECK_W, aw, WS_CHECK_W, aw);
-        am = av = aw = 0.f;
-      }
-      cur = ci;
-      if constexpr (kStats) {
-        tracked = C.w_amax != nullptr && *C.w_amax >= 0.0f;
-        active = tracked == (PASS == 4);
-        sc = adam_scalars(L, *C.g_inv, 1.0f / *C.m_scale, 1.0f / *C.v_scale, 1.0f / *C.w_scale);
-      } else {
-        const uint32_t fl = ws_flags(L, ci);
-        // pass 2: keep the stored-master amax (and its check) for every chunk
-        // that tracks it, including the step that first establishes it
-        tracked = PASS == 2 ? C.w_amax != nullptr : (fl & 2u) != 0;
-        active = PASS == 2 || (fl & 1u) != 0;
-        sc = adam_scalars(L, *C.g_inv, ws_get(L, ci, WS_OLDINV_M), ws_get(L, ci, WS_OLDINV_V),
-                          ws_get(L, ci, WS_OLDINV_W));
-        ns.m = both(ws_get(L, ci, WS_NEW_M));
-        ns.v = both(ws_get(L, ci, WS_NEW_V));
-        ns.w = both(ws_get(L, ci, WS_NEW_W));
-        ns.inv_w = both(1.0f / ns.w.x);
-        want_wq = C.wq != nullptr;
-        ns.wq = both(want_wq ? ws_get(L, ci, WS_NEW_WQ) : 1.0f);
-      }
+    if (ci != S.cur) {
+      if (S.cur >= 0) adam_chunk_flush<PASS>(L, S);
+      adam_chunk_enter<PASS>(L, ci, S);
     }
-    if (!active) {  // pass 1b: chunk not flagged; stats: the other stats pass's chunk
+    if (!S.active) {  // pass 1b: chunk not flagged; stats: the other stats pass's chunk
       // jump to this block's last tile inside the chunk; the loop step leaves it
       const unsigned long long end = C.tile_begin + (C.n + kAdamTile - 1) / kAdamTile;
       tile += ((end - tile - 1) / gridDim.x) * gridDim.x;
@@ -340,55 +395,20 @@ __device__ __forceinline__ void adam_pass(const AdamLaunch &L) {
     if (base + kAdamPerThread <= C.n) {
       const size_t grp = base / kAdamPerThread;
       if constexpr (PASS == 4) {
-        adam_group<1, true, false>(L, C, grp, sc, ns, am, av, aw);
+        adam_group<1, true, false>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw);
       } else if constexpr (PASS == 1) {
-        adam_group<1, false, false>(L, C, grp, sc, ns, am, av, aw);
+        adam_group<1, false, false>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw);
       } else if constexpr (PASS == 3) {
-        adam_group<3, false, false>(L, C, grp, sc, ns, am, av, aw);
+        adam_group<3, false, false>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw);
       } else {
-        adam_group<2, true, true>(L, C, grp, sc, ns, am, av, aw, tracked, want_wq);
+        adam_group<2, true, true>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw, S.tracked, S.want_wq);
       }
     } else {
-      // Ragged end of a chunk: element by element (lane y unused).
-      const bool read_w = PASS != 4;
-      for (unsigned long long i = base; i < C.n; i++) {
-        const float2 gd = dec2<FP8_E5M2>(C.g[i]), md = dec2<FP8_E4M3>(C.m[i]);
-        const float2 vd = make_float2(__half2float(__ushort_as_half(C.v[i])), 0.0f);
-        const float2 wd = make_float2(read_w ? __half2float(__ushort_as_half(C.w[i])) : 0.0f, 0.0f);
-        float2 m, v, d;
-        if constexpr (PASS == 4)
-          adam_moments_bound(L, make_float2(gd.x, 0.0f), make_float2(md.x, 0.0f), vd, sc, m, v, d);
-        else
-          adam_moments(L, make_float2(gd.x, 0.0f), make_float2(md.x, 0.0f), vd, sc, m, v, d);
-        if constexpr (kStats) {
-          am = max_abs1(am, m.x);
-          av = max_abs1(av, v.x);
-          aw = max_abs1(aw, tracked ? d.x : adam_master(wd, d, sc).x);
-        } else if constexpr (PASS == 3) {
-          aw = max_abs1(aw, adam_master(wd, d, sc).x);
-        } else {
-          const float w = adam_master(wd, d, sc).x;
-          if (tracked) aw = max_abs1(aw, w);
-          C.m[i] = (uint8_t)(enc2<FP8_E4M3>(__fmul_rn(m.x, ns.m.x), 0.0f) & 0xffu);
-          C.v[i] = __half_as_ushort(__float2half_rn(__fmul_rn(v.x, ns.v.x)));
-          const __half h = __float2half_rn(__fmul_rn(w, ns.w.x));
-          C.w[i] = __half_as_ushort(h);
-          const float st = __half2float(h);
-          if (tracked) am = max_abs1(am, st);
-          if (want_wq)
-            C.wq[i] = (uint8_t)(enc2<FP8_E4M3>(__fmul_rn(__fmul_rn(st, ns.inv_w.x), ns.wq.x), 0.0f) & 0xffu);
-        }
-      }
+      adam_tail<PASS>(L, C, base, S);
     }
   }
   // cur is block-uniform, so whole warps take these branches together.
-  if (cur >= 0) {
-    if constexpr (kStats)
-      if (active) flush_max3(L, cur, WS_AMAX_M, am, WS_AMAX_V, av, tracked ? WS_STEP_MAX : WS_AMAX_W, aw);
-    if constexpr (PASS == 3)
-      if (active) flush_max3(L, cur, WS_AMAX_W, aw, WS_AMAX_W, aw, WS_AMAX_W, aw);
-    if constexpr (PASS == 2) flush_max3(L, cur, WS_STORED_W, am, WS_CHECK_W, aw, WS_CHECK_W, aw);
-  }
+  if (S.cur >= 0) adam_chunk_flush<PASS>(L, S);
 }
 
 template <int PASS>
@@ -396,7 +416,11 @@ __global__ void __launch_bounds__(kAdamThreads) k_adam(const __grid_constant__ A
   adam_pass<PASS>(L);
 }
 // The update pass, latency-bound on its loads, is held to 48 registers: five
-// resident blocks per SM instead of four keep more loads in flight.
+// resident blocks per SM instead of four keep more loads in flight.  (A
+// variant fed through a shared-memory ring by bulk copies, one producer warp
+// and eight consumer warps per block, two blocks per SM, was correct but 12 %
+// slower at 64 M parameters: too few warps left to hide the update's
+// arithmetic.)
 template <>
 __global__ void __launch_bounds__(kAdamThreads, 5) k_adam<2>(const __grid_constant__ AdamLaunch L) {
   adam_pass<2>(L);
