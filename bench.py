@@ -34,7 +34,8 @@ gradient cast and that tensor's Adam step run beside the next fwd/dgrad (one
 Adam call per tensor instead of one over all four).  --schedule serial runs
 the work in order on one stream.  The per-kernel breakdown
 (`kernels`, `roofline`) always comes from a serial pass with CUDA events
-around each phase.
+around each phase.  NVTX ranges mark each linear, the Adam step and each
+overlapped step for timeline profilers.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--workload gpt175b_block|gpt7b_block] [--schedule serial]
@@ -269,8 +270,10 @@ class BlockStep:
             ev.setdefault(kind, []).append(e)
             return e
 
+        nvtx = torch.cuda.nvtx
         for d in self.L:
             sc = d["sc"]
+            nvtx.range_push(f"linear {d['name']}")
             e = mark("cast")
             self.quantise(d["X"], fp8.FP8_E4M3, sc, 0, out=d["xq"])
             self.quantise(d["dY"], fp8.FP8_E5M2, sc, 6, mu=MU, out=d["dyq"])
@@ -283,10 +286,13 @@ class BlockStep:
             e = mark("grad_cast")
             fp8.fp8_scale_cast(d["dw"], fp8.FP8_E5M2, sc[14:15], 0, MU, sc[10:11], sc[11:12], d["gq"])
             if e: e[1].record()
+            nvtx.range_pop()
         self.t += 1
+        nvtx.range_push("adam")
         e = mark("adam")
         fp8.fp8_adam_step(self.chunks, step=self.t, margin=0, workspace=self.ws, **HP)
         if e: e[1].record()
+        nvtx.range_pop()
 
     def step_overlapped(self):
         """The same work as step(), on three streams: the casts of every
@@ -312,6 +318,8 @@ class BlockStep:
             self.ev_cast_x = [torch.cuda.Event() for _ in self.L]  # X cast (enough for fwd)
             self.ev_dgrad = [torch.cuda.Event() for _ in self.L]   # the weight's last reader done
             self.ev_grad = torch.cuda.Event()
+        nvtx = torch.cuda.nvtx
+        nvtx.range_push("step (three streams)")
         self.ev_start.record(main)
         self.s_cast.wait_event(self.ev_start)
         self.s_aux.wait_event(self.ev_start)
@@ -339,6 +347,7 @@ class BlockStep:
         self.ev_grad.record(self.s_aux)
         main.wait_event(self.ev_grad)
         self.t += 1
+        nvtx.range_pop()
 
     def result_scalars(self):
         return torch.cat([d["sc"] for d in self.L] + [d["st"] for d in self.L])

@@ -843,51 +843,54 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     }
     if (!ok && issued && lane == 0) sleep_ns_bounded(50000);  // let copies in flight land
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (leader only)
-    if (leader) {
+    // ------------------------------------------------------------ MMA issuer (leader, one thread)
+    // The whole loop runs in one thread with no warp-wide step per k-block,
+    // and the 64-bit operand descriptors advance by constant adds: a k-slice
+    // moves the start-address field (address >> 4) by 2 (K-major, 32 B) or
+    // 256 (MN-major, 32 rows of 128 B), a stage by kWideStageBytes >> 4, and
+    // the field cannot carry (shared addresses stay below 2^18).
+    if (leader && lane == 0) {
+      const uint64_t a_d0 = operand_desc<A_MN>(base, 0);
+      const uint64_t b_d0 = operand_desc<B_MN>(base + kPairHalf * BK, 0);
+      const uint64_t b_d1 = operand_desc<B_MN>(base + 2 * kPairHalf * BK, 0);
+      constexpr uint64_t a_ks = A_MN ? (UMMA_K * 128) >> 4 : UMMA_K >> 4;
+      constexpr uint64_t b_ks = B_MN ? (UMMA_K * 128) >> 4 : UMMA_K >> 4;
+      constexpr uint64_t st_d = kWideStageBytes >> 4;
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true, issued_any = false;
       for (int tile = pair; tile < args.num_tiles && ok; tile += num_pairs) {
-        bool got = lane == 0 ? mbar_wait(tempty_bar, acc_phase ^ 1u, abort_flag) : true;
-        got = __shfl_sync(0xffffffffu, got, 0);
-        if (!got) { ok = false; break; }
+        if (!mbar_wait(tempty_bar, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         for (int kb = 0; kb < args.num_k_blocks; kb++) {
-          got = lane == 0 ? stage_ready(full_bar(stage), phase, abort_flag) : true;
-          got = __shfl_sync(0xffffffffu, got, 0);
-          if (!got) { ok = false; break; }
-          if (lane == 0) {
-            const uint32_t sa = base + stage * kWideStageBytes, sb = sa + kPairHalf * BK;
+          if (!stage_ready(full_bar(stage), phase, abort_flag)) { ok = false; break; }
+          const uint64_t so = (uint64_t)stage * st_d;
 #pragma unroll
-            for (int ks = 0; ks < BK / UMMA_K; ks++) {
-              const uint64_t ad = operand_desc<A_MN>(sa, ks);
-              const uint32_t accum = (kb | ks) != 0 ? 1u : 0u;
-              // the same A slice feeds both accumulators: read it from shared memory once
-              tc_mma_pair_fill_a(tmem_base, ad, operand_desc<B_MN>(sb, ks), args.idesc, accum);
-              tc_mma_pair_lastuse_a(tmem_base + 256, ad, operand_desc<B_MN>(sb + kPairHalf * BK, ks), args.idesc,
-                                    accum);
-            }
-            // the leader's own ring slot; the relay warp frees the follower's
-            asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                             empty_bar(stage))
-                         : "memory");
-            issued_any = true;
+          for (int ks = 0; ks < BK / UMMA_K; ks++) {
+            const uint64_t ad = a_d0 + so + ks * a_ks;
+            const uint32_t accum = (kb | ks) != 0 ? 1u : 0u;
+            // the same A slice feeds both accumulators: read it from shared memory once
+            tc_mma_pair_fill_a(tmem_base, ad, b_d0 + so + ks * b_ks, args.idesc, accum);
+            tc_mma_pair_lastuse_a(tmem_base + 256, ad, b_d1 + so + ks * b_ks, args.idesc, accum);
           }
-          __syncwarp();
+          // the leader's own ring slot; the relay warp frees the follower's
+          asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                           empty_bar(stage))
+                       : "memory");
+          issued_any = true;
           if (++stage == kWideStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        if (lane == 0) tc_commit_pair(tfull_bar);
-        __syncwarp();
+        tc_commit_pair(tfull_bar);
         acc_phase ^= 1u;
       }
-      if (!ok && lane == 0 && issued_any) {
+      if (!ok && issued_any) {
         asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(drain_bar)
                      : "memory");
         mbar_wait_drain(drain_bar, 0);
       }
     }
+    __syncwarp();
   } else if (warp == 10) {
     // ------------------------------------------------------------ release relay (leader only)
     // Once the MMAs that read a ring slot have completed (the leader's empty

@@ -744,3 +744,57 @@ def test_adam_sharded_halves_reject_tracking_and_bad_workspace():
     plain = make_adam_state([64], ("adam-shard-bad",))
     with pytest.raises(fp8.FP8Error):
         fp8.fp8_adam_stats(plain, step=1, margin=0, workspace=ws[:3], **HP)
+
+
+def test_two_step_linear_chain_reads_adam_weight_copy():
+    """f1 in a training chain: step 1 runs fwd/dgrad/wgrad on the E4M3 weight
+    cast from the initial weights, casts the gradient (mu-scaled E5M2) and
+    takes the Adam step, which also writes the E4M3 copy of the new master;
+    step 2's fwd and dgrad read that copy and its inverse scale.  The copy
+    equals the oracle's E4M3 cast of the stored master (codes and scale), and
+    step 2's outputs match the oracle's GEMMs on it."""
+    from fp8_mixed_precision_tensor_b200.adam_state import AdamTensorState, FP8Adam
+
+    M, N, K = 512, 768, 1024
+    W = to_dev(synth.normal_f32((N, K), 0.02, "chain", "W"))
+    st = AdamTensorState(W, track_master_amax=True, e4m3_copy=True)
+    opt = FP8Adam([st], **HP)
+    wq = torch.empty((N, K), dtype=torch.uint8, device="cuda")
+    w_sc = torch.zeros(3, **F32)  # amax, scale, inverse of the step-1 weight operand
+    fp8.fp8_amax(W, w_sc[0:1])
+    fp8.fp8_scale_cast(W, fp8.FP8_E4M3, w_sc[0:1], 0, 1.0, w_sc[1:2], w_sc[2:3], wq)
+    w_inv = w_sc[2:3]
+    for step in (1, 2):
+        X = to_dev(synth.normal_f32((M, K), 1.0, "chain", "X", step))
+        dY = to_dev(synth.normal_f32((M, N), 1e-4, "chain", "dY", step))
+        sc = torch.zeros(9, **F32)
+        xq = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+        dyq = torch.empty((M, N), dtype=torch.uint8, device="cuda")
+        fp8.fp8_amax(X, sc[0:1])
+        fp8.fp8_scale_cast(X, fp8.FP8_E4M3, sc[0:1], 0, 1.0, sc[1:2], sc[2:3], xq)
+        fp8.fp8_amax(dY, sc[3:4])
+        fp8.fp8_scale_cast(dY, fp8.FP8_E5M2, sc[3:4], 0, 2.0 ** 10, sc[4:5], sc[5:6], dyq)
+        y = torch.empty((M, N), **F32)
+        dx = torch.empty((M, K), **F32)
+        dw = torch.empty((N, K), **F32)
+        fp8.fp8_linear_fwd(xq, sc[2:3], wq if step == 1 else st.wq.view(N, K), w_inv, y)
+        fp8.fp8_linear_dgrad(dyq, sc[5:6], wq if step == 1 else st.wq.view(N, K), w_inv, dx)
+        fp8.fp8_linear_wgrad(dyq, sc[5:6], xq, sc[2:3], dw, sc[6:7])
+        if step == 2:
+            # the weight operand is the copy step 1's Adam wrote: check the GEMMs on it
+            w_codes = st.wq.cpu().numpy().reshape(N, K)
+            h_x, h_dy = xq.cpu().numpy(), dyq.cpu().numpy()
+            ref, rabs = oracle.linear_fwd(h_x, sc[2].item(), w_codes, w_inv.item(), M, N, K)
+            assert_gemm_close(tensor_to_np(y), ref, rabs, torch.float32, "step-2 fwd on the Adam copy")
+            ref, rabs = oracle.linear_dgrad(h_dy, sc[5].item(), w_codes, w_inv.item(), M, N, K)
+            assert_gemm_close(tensor_to_np(dx), ref, rabs, torch.float32, "step-2 dgrad on the Adam copy")
+            break
+        st.set_gradient(dw, 2.0 ** 10, grad_amax=sc[6:7])
+        opt.step()
+        assert fp8.fp8_get_status() == 0
+        # the copy is the oracle's E4M3 cast of the stored FP16 master
+        q_ref, s_q = oracle.adam_master_e4m3(st.w.cpu().numpy(), st.scalars[3].item(), 0)
+        assert st.wq_scale.item() == s_q and st.wq_inv.item() == 1.0 / s_q
+        assert np.array_equal(st.wq.cpu().numpy(), q_ref)
+        w_inv = st.wq_inv
+    assert fp8.fp8_get_status() == 0
