@@ -471,44 +471,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (issued_mask & (1u << s)) mbar_wait_drain(full_bar(s), (issued_par >> s) & 1u);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    int stage = 0;
-    uint32_t phase = 0;
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    bool ok = true, issued_any = false;
-    for (int tile = blockIdx.x; tile < args.num_tiles && ok; tile += gridDim.x) {
-      bool got = lane == 0 ? mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag) : true;
-      got = __shfl_sync(0xffffffffu, got, 0);
-      if (!got) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + acc * BN;
-      for (int kb = 0; kb < args.num_k_blocks; kb++) {
-        got = lane == 0 ? stage_ready(full_bar(stage), phase, abort_flag) : true;
-        got = __shfl_sync(0xffffffffu, got, 0);
-        if (!got) { ok = false; break; }
-        if (lane == 0) {
-          const uint32_t sa = base + stage * C::STAGE_BYTES, sb = sa + C::A_BYTES;
+    // ------------------------------------------------------------ MMA issuer (one thread)
+    // Descriptors advance by constant adds, as in k_gemm3's issuer.
+    if (lane == 0) {
+      const uint64_t a_d0 = operand_desc<A_MN>(base, 0);
+      const uint64_t b_d0 = operand_desc<B_MN>(base + C::A_BYTES, 0);
+      constexpr uint64_t a_ks = A_MN ? (UMMA_K * 128) >> 4 : UMMA_K >> 4;
+      constexpr uint64_t b_ks = B_MN ? (UMMA_K * 128) >> 4 : UMMA_K >> 4;
+      constexpr uint64_t st_d = C::STAGE_BYTES >> 4;
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true, issued_any = false;
+      for (int tile = blockIdx.x; tile < args.num_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < args.num_k_blocks; kb++) {
+          if (!stage_ready(full_bar(stage), phase, abort_flag)) { ok = false; break; }
+          const uint64_t so = (uint64_t)stage * st_d;
 #pragma unroll
-          for (int ks = 0; ks < BK / UMMA_K; ks++) {
-            tc_mma(d_tmem, operand_desc<A_MN>(sa, ks), operand_desc<B_MN>(sb, ks), args.idesc,
-                   (kb | ks) != 0 ? 1u : 0u);
-          }
+          for (int ks = 0; ks < BK / UMMA_K; ks++)
+            tc_mma(d_tmem, a_d0 + so + ks * a_ks, b_d0 + so + ks * b_ks, args.idesc, (kb | ks) != 0 ? 1u : 0u);
           tc_commit(empty_bar(stage));  // ring slot free once these MMAs have read it
           issued_any = true;
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
-        __syncwarp();
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        if (!ok) break;
+        tc_commit(tfull_bar(acc));  // accumulator complete
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
-      if (!ok) break;
-      if (lane == 0) tc_commit(tfull_bar(acc));  // accumulator complete
-      __syncwarp();
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      if (!ok && issued_any) {
+        tc_commit(drain_bar);  // arrives once every MMA issued so far has completed
+        mbar_wait_drain(drain_bar, 0);
+      }
     }
-    if (!ok && lane == 0 && issued_any) {
-      tc_commit(drain_bar);  // arrives once every MMA issued so far has completed
-      mbar_wait_drain(drain_bar, 0);
-    }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
@@ -649,47 +648,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!ok && issued && lane == 0) sleep_ns_bounded(50000);  // let copies in flight land
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (leader only)
-    if (leader) {
+    // ------------------------------------------------------------ MMA issuer (leader, one thread)
+    // Descriptors advance by constant adds, as in k_gemm3's issuer.
+    if (leader && lane == 0) {
+      const uint64_t a_d0 = operand_desc<A_MN>(base, 0);
+      const uint64_t b_d0 = operand_desc<B_MN>(base + kPairHalf * BK, 0);
+      constexpr uint64_t a_ks = A_MN ? (UMMA_K * 128) >> 4 : UMMA_K >> 4;
+      constexpr uint64_t b_ks = B_MN ? (UMMA_K * 128) >> 4 : UMMA_K >> 4;
+      constexpr uint64_t st_d = kPairStageBytes >> 4;
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true, issued_any = false;
       for (int tile = pair; tile < args.num_tiles && ok; tile += num_pairs) {
-        bool got = lane == 0 ? mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag) : true;
-        got = __shfl_sync(0xffffffffu, got, 0);
-        if (!got) { ok = false; break; }
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kPairBN;
         for (int kb = 0; kb < args.num_k_blocks; kb++) {
-          got = lane == 0 ? stage_ready(full_bar(stage), phase, abort_flag) : true;
-          got = __shfl_sync(0xffffffffu, got, 0);
-          if (!got) { ok = false; break; }
-          if (lane == 0) {
-            const uint32_t sa = base + stage * kPairStageBytes, sb = sa + kPairHalf * BK;
+          if (!stage_ready(full_bar(stage), phase, abort_flag)) { ok = false; break; }
+          const uint64_t so = (uint64_t)stage * st_d;
 #pragma unroll
-            for (int ks = 0; ks < BK / UMMA_K; ks++) {
-              tc_mma_pair(d_tmem, operand_desc<A_MN>(sa, ks), operand_desc<B_MN>(sb, ks), args.idesc,
-                          (kb | ks) != 0 ? 1u : 0u);
-            }
-            tc_commit_pair(empty_bar(stage));
-            issued_any = true;
-          }
-          __syncwarp();
+          for (int ks = 0; ks < BK / UMMA_K; ks++)
+            tc_mma_pair(d_tmem, a_d0 + so + ks * a_ks, b_d0 + so + ks * b_ks, args.idesc, (kb | ks) != 0 ? 1u : 0u);
+          tc_commit_pair(empty_bar(stage));
+          issued_any = true;
           if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        if (lane == 0) tc_commit_pair(tfull_bar(acc));
-        __syncwarp();
+        tc_commit_pair(tfull_bar(acc));
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
-      if (!ok && lane == 0 && issued_any) {
+      if (!ok && issued_any) {
         asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(drain_bar)
                      : "memory");
         mbar_wait_drain(drain_bar, 0);
       }
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;
