@@ -6,20 +6,29 @@
 // The new scales are just-in-time: each comes from the amax of the *new*
 // values (the same rule as the linear layer's casts).  A step is
 //   pass 1 (stats):   decode, update in registers, reduce per chunk amax|m|,
-//                     amax v and either amax|w| (reading the master) or, when
-//                     the caller tracks the master's amax A0, the largest
-//                     step |dw| (not reading the master: 4 instead of 6 B);
-//   finalize 1:       new scales; with a tracked A0 the new master amax lies
-//                     in [A0 - U, A0 + U] and the scale exponent is taken from
-//                     that interval when it contains no scale threshold,
-//                     otherwise the chunk is flagged;
+//                     amax v (both exact), the largest step U >= max |dw|
+//                     and, reading the master, an estimate A~ of the new
+//                     master's amax (|A~ - A| <= 2^-16 U + 2^-21 A~), or, when
+//                     the caller tracks the stored master's amax A0, U alone
+//                     (not reading the master: 4 instead of 6 B); the step is
+//                     estimated with the MUFU square root and reciprocal;
+//   finalize 1:       new scales of m and v; the new master amax lies in
+//                     [A~ - e, A~ + e] or, tracked, in [A0 - U, A0 + U], and
+//                     the master's scale exponent is taken from that interval
+//                     when it contains no scale threshold, otherwise the chunk
+//                     is flagged;
 //   pass 1b:          exact amax|w| for flagged chunks only (others skip);
 //   finalize 2:       remaining scales; publish all new scales;
 //   pass 2 (update):  decode, update again (bit-identical arithmetic), encode
 //                     m, v, w with the new scales, optionally write the E4M3
 //                     copy of the new stored master for the next forward GEMM,
 //                     and reduce the stored master's amax;
-//   finalize 3:       new tracked A0; consistency check of the inferred scale.
+//   finalize 3:       new tracked A0; every chunk's master scale checked
+//                     against the exact new amax the update pass reduced.
+// The phased form of the step (stats and update as separate calls, with the
+// workspace MAX-reduced over ranks in between) computes the exact new amaxes
+// in pass 1 instead: an interval decision there would need a second
+// reduction for the flagged chunks.
 // All chunks of one call share each launch: the chunk table travels in the
 // kernel parameters and tiles of 4096 parameters are mapped to chunks by a
 // binary search over the chunks' first-tile indices.
@@ -46,7 +55,11 @@ enum : int {
   WS_NEW_WQ = 11,      // scale of the E4M3 master copy
   WS_STORED_W = 12,    // max |stored FP16 master| (as f32 bits of the half)
   WS_CHECK_W = 13,     // exact amax|w| of the new f32 master (pass 2)
+  WS_APPROX_W = 14,    // estimate of amax|w| of the new master (pass 1, estimated step)
 };
+// WS_FLAGS bits: the exact master pass must run; the chunk tracks its master
+// amax; the master's scale was decided in finalize 1.
+enum : uint32_t { FLAG_EXACT = 1u, FLAG_TRACKED = 2u, FLAG_KNOWN = 4u };
 
 struct AdamChunkDev {
   const uint8_t *g;
@@ -72,6 +85,7 @@ struct AdamLaunch {
   float beta1, beta2, eps;
   float neg_lr_bc1;  // -lr / (1 - beta1^t)
   float inv_bc2;     // 1 / (1 - beta2^t)
+  int estimate;      // 1: untracked chunks take the estimated stats pass (PASS 5)
   float *ws;         // kAdamWsFloatsPerChunk floats per chunk of this launch
 };
 
@@ -124,14 +138,15 @@ __device__ __forceinline__ void adam_moments(const AdamLaunch &L, float2 gd, flo
   dw = __fmul2_rn(both(L.neg_lr_bc1), make_float2(__fdiv_rn(m.x, den.x), __fdiv_rn(m.y, den.y)));
 }
 
-// The same moments and an upper-bound estimate of the step, with the MUFU
-// square root and reciprocal (flush-to-zero) in place of the correctly
-// rounded operations: for the tracked master's interval only, which needs a
-// bound U >= max |dw|, not the step itself.  The approximations' relative
-// errors (a few 2^-23) are covered by widening U by 2^-16 in the finalize
-// stage; the flush changes nothing because eps >= 2^-39 makes
-// sqrt(v_hat) + eps round to eps for every subnormal v_hat.  The update pass
-// checks the scale this bound selected against the exact new amax.
+// The same moments and an estimate of the step, with the MUFU square root and
+// reciprocal (flush-to-zero) in place of the correctly rounded operations:
+// for the stats passes, which need the exact m and v (computed the same way
+// here) but only an interval for the master's new amax.  The approximations'
+// relative errors (a few 2^-23, so |dw~ - dw| < 2^-18 |dw|) are covered by
+// the 2^-16 U widening in the finalize stage; the flush changes nothing
+// because eps >= 2^-39 makes sqrt(v_hat) + eps round to eps for every
+// subnormal v_hat.  The update pass checks every scale decided this way
+// against the exact new amax.
 __device__ __forceinline__ float sqrt_approx(float x) {
   float r;
   asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
@@ -218,7 +233,7 @@ struct AdamNewScales {
 template <int PASS, bool TRACK, bool WQ>
 __device__ __forceinline__ void adam_group(const AdamLaunch &L, const AdamChunkDev &C, size_t grp,
                                            const AdamScalars &sc, const AdamNewScales &ns, float &am, float &av,
-                                           float &aw, bool track_rt = TRACK, bool wq_rt = WQ) {
+                                           float &aw, float &au, bool track_rt = TRACK, bool wq_rt = WQ) {
   constexpr bool kReadW = PASS != 1 || !TRACK;
   const bool track = TRACK && track_rt, wq = WQ && wq_rt;
   const uint4 gq = __ldcs(reinterpret_cast<const uint4 *>(C.g) + grp);
@@ -240,11 +255,16 @@ __device__ __forceinline__ void adam_group(const AdamLaunch &L, const AdamChunkD
     const uint32_t g2 = (gw[p >> 1] >> ((p & 1) * 16)) & 0xffffu;
     const uint32_t m2 = (mw[p >> 1] >> ((p & 1) * 16)) & 0xffffu;
     float2 m, v, d;
-    if constexpr (PASS == 1 && TRACK)  // only the bound U >= max |dw| is needed
+    if constexpr ((PASS == 1 && TRACK) || PASS == 5)  // the step is only estimated
       adam_moments_bound(L, dec2<FP8_E5M2>(g2), dec2<FP8_E4M3>(m2), h2f2(vw[p]), sc, m, v, d);
     else
       adam_moments(L, dec2<FP8_E5M2>(g2), dec2<FP8_E4M3>(m2), h2f2(vw[p]), sc, m, v, d);
-    if constexpr (PASS == 1) {
+    if constexpr (PASS == 5) {
+      am = max_abs2(am, m);
+      av = max_abs2(av, v);
+      aw = max_abs2(aw, adam_master(h2f2(ww[p]), d, sc));
+      au = max_abs2(au, d);
+    } else if constexpr (PASS == 1) {
       am = max_abs2(am, m);
       av = max_abs2(av, v);
       aw = max_abs2(aw, TRACK ? d : adam_master(h2f2(ww[p]), d, sc));
@@ -252,7 +272,7 @@ __device__ __forceinline__ void adam_group(const AdamLaunch &L, const AdamChunkD
       aw = max_abs2(aw, adam_master(h2f2(ww[p]), d, sc));
     } else {
       const float2 w = adam_master(h2f2(ww[p]), d, sc);
-      if (track) aw = max_abs2(aw, w);
+      aw = max_abs2(aw, w);  // the exact new amax: checks the scale finalize 1 decided
       const float2 ms = __fmul2_rn(m, ns.m), vs = __fmul2_rn(v, ns.v), ws = __fmul2_rn(w, ns.w);
       const uint32_t mc = enc2<FP8_E4M3>(ms.x, ms.y);
       if (p & 1) mo[p >> 1] |= mc << 16; else mo[p >> 1] = mc;
@@ -284,7 +304,7 @@ __device__ __forceinline__ void adam_group(const AdamLaunch &L, const AdamChunkD
 // new chunk, and the running maxima it folds into the chunk's workspace slots
 // when it leaves.
 struct AdamChunkState {
-  float am = 0.f, av = 0.f, aw = 0.f;  // running maxima of the current chunk
+  float am = 0.f, av = 0.f, aw = 0.f, au = 0.f;  // running maxima of the current chunk
   int cur = -1;
   bool tracked = false, active = true, want_wq = false;
   AdamScalars sc{};
@@ -296,15 +316,20 @@ __device__ __forceinline__ void adam_chunk_flush(const AdamLaunch &L, AdamChunkS
   constexpr bool kStats = PASS == 1 || PASS == 4;
   if constexpr (kStats)
     if (S.active) flush_max3(L, S.cur, WS_AMAX_M, S.am, WS_AMAX_V, S.av, S.tracked ? WS_STEP_MAX : WS_AMAX_W, S.aw);
+  if constexpr (PASS == 5)
+    if (S.active) {
+      flush_max3(L, S.cur, WS_AMAX_M, S.am, WS_AMAX_V, S.av, WS_APPROX_W, S.aw);
+      flush_max3(L, S.cur, WS_STEP_MAX, S.au, WS_STEP_MAX, S.au, WS_STEP_MAX, S.au);
+    }
   if constexpr (PASS == 3)
     if (S.active) flush_max3(L, S.cur, WS_AMAX_W, S.aw, WS_AMAX_W, S.aw, WS_AMAX_W, S.aw);
   if constexpr (PASS == 2) flush_max3(L, S.cur, WS_STORED_W, S.am, WS_CHECK_W, S.aw, WS_CHECK_W, S.aw);
-  S.am = S.av = S.aw = 0.f;
+  S.am = S.av = S.aw = S.au = 0.f;
 }
 
 template <int PASS>
 __device__ __forceinline__ void adam_chunk_enter(const AdamLaunch &L, int ci, AdamChunkState &S) {
-  constexpr bool kStats = PASS == 1 || PASS == 4;
+  constexpr bool kStats = PASS == 1 || PASS == 4 || PASS == 5;
   const AdamChunkDev &C = L.c[ci];
   S.cur = ci;
   if constexpr (kStats) {
@@ -315,8 +340,8 @@ __device__ __forceinline__ void adam_chunk_enter(const AdamLaunch &L, int ci, Ad
     const uint32_t fl = ws_flags(L, ci);
     // pass 2: keep the stored-master amax (and its check) for every chunk
     // that tracks it, including the step that first establishes it
-    S.tracked = PASS == 2 ? C.w_amax != nullptr : (fl & 2u) != 0;
-    S.active = PASS == 2 || (fl & 1u) != 0;
+    S.tracked = PASS == 2 ? C.w_amax != nullptr : (fl & FLAG_TRACKED) != 0;
+    S.active = PASS == 2 || (fl & FLAG_EXACT) != 0;
     S.sc = adam_scalars(L, *C.g_inv, ws_get(L, ci, WS_OLDINV_M), ws_get(L, ci, WS_OLDINV_V),
                         ws_get(L, ci, WS_OLDINV_W));
     S.ns.m = both(ws_get(L, ci, WS_NEW_M));
@@ -333,7 +358,7 @@ __device__ __forceinline__ void adam_chunk_enter(const AdamLaunch &L, int ci, Ad
 template <int PASS>
 __device__ __forceinline__ void adam_tail(const AdamLaunch &L, const AdamChunkDev &C, unsigned long long base,
                                        AdamChunkState &S) {
-  constexpr bool kStats = PASS == 1 || PASS == 4;
+  constexpr bool kStats = PASS == 1 || PASS == 4 || PASS == 5;
   const bool read_w = PASS != 4;
   const AdamScalars &sc = S.sc;
   const AdamNewScales &ns = S.ns;
@@ -342,7 +367,7 @@ __device__ __forceinline__ void adam_tail(const AdamLaunch &L, const AdamChunkDe
     const float2 vd = make_float2(__half2float(__ushort_as_half(C.v[i])), 0.0f);
     const float2 wd = make_float2(read_w ? __half2float(__ushort_as_half(C.w[i])) : 0.0f, 0.0f);
     float2 m, v, d;
-    if constexpr (PASS == 4)
+    if constexpr (PASS == 4 || PASS == 5)
       adam_moments_bound(L, make_float2(gd.x, 0.0f), make_float2(md.x, 0.0f), vd, sc, m, v, d);
     else
       adam_moments(L, make_float2(gd.x, 0.0f), make_float2(md.x, 0.0f), vd, sc, m, v, d);
@@ -350,11 +375,12 @@ __device__ __forceinline__ void adam_tail(const AdamLaunch &L, const AdamChunkDe
       S.am = max_abs1(S.am, m.x);
       S.av = max_abs1(S.av, v.x);
       S.aw = max_abs1(S.aw, S.tracked ? d.x : adam_master(wd, d, sc).x);
+      if constexpr (PASS == 5) S.au = max_abs1(S.au, d.x);
     } else if constexpr (PASS == 3) {
       S.aw = max_abs1(S.aw, adam_master(wd, d, sc).x);
     } else {
       const float w = adam_master(wd, d, sc).x;
-      if (S.tracked) S.aw = max_abs1(S.aw, w);
+      S.aw = max_abs1(S.aw, w);
       C.m[i] = (uint8_t)(enc2<FP8_E4M3>(__fmul_rn(m.x, ns.m.x), 0.0f) & 0xffu);
       C.v[i] = __half_as_ushort(__float2half_rn(__fmul_rn(v.x, ns.v.x)));
       const __half h = __float2half_rn(__fmul_rn(w, ns.w.x));
@@ -367,12 +393,13 @@ __device__ __forceinline__ void adam_tail(const AdamLaunch &L, const AdamChunkDe
   }
 }
 
-// One pass over all tiles of a launch.  PASS 1: stats of the chunks that do
-// not track their master amax (exact new amaxes).  PASS 4: stats of the
-// chunks that do (amax of m and v, the step bound U).  PASS 3: exact master
-// amax of flagged chunks.  PASS 2: update.  The two stats passes are separate
-// kernels so that the bound-only arithmetic of PASS 4 does not carry the
-// register count of the exact one.
+// One pass over all tiles of a launch.  PASS 5: stats of the chunks that do
+// not track their master amax (exact amaxes of m and v, the estimate A~ and
+// the step bound U).  PASS 1: the same chunks' exact new amaxes (the phased
+// step).  PASS 4: stats of the chunks that track it (amaxes of m and v, U).
+// PASS 3: exact master amax of flagged chunks.  PASS 2: update.  The stats
+// passes are separate kernels so that the estimated arithmetic does not
+// carry the register count of the exact one.
 template <int PASS>
 __device__ __forceinline__ void adam_pass(const AdamLaunch &L) {
   AdamChunkState S;
@@ -395,13 +422,15 @@ __device__ __forceinline__ void adam_pass(const AdamLaunch &L) {
     if (base + kAdamPerThread <= C.n) {
       const size_t grp = base / kAdamPerThread;
       if constexpr (PASS == 4) {
-        adam_group<1, true, false>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw);
+        adam_group<1, true, false>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw, S.au);
+      } else if constexpr (PASS == 5) {
+        adam_group<5, false, false>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw, S.au);
       } else if constexpr (PASS == 1) {
-        adam_group<1, false, false>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw);
+        adam_group<1, false, false>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw, S.au);
       } else if constexpr (PASS == 3) {
-        adam_group<3, false, false>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw);
+        adam_group<3, false, false>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw, S.au);
       } else {
-        adam_group<2, true, true>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw, S.tracked, S.want_wq);
+        adam_group<2, true, true>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw, S.au, S.tracked, S.want_wq);
       }
     } else {
       adam_tail<PASS>(L, C, base, S);
@@ -425,10 +454,14 @@ template <>
 __global__ void __launch_bounds__(kAdamThreads, 5) k_adam<2>(const __grid_constant__ AdamLaunch L) {
   adam_pass<2>(L);
 }
-// The bound-only stats pass of tracking chunks: six resident blocks per SM.
+// The estimated stats passes: six resident blocks per SM.
 template <>
 __global__ void __launch_bounds__(kAdamThreads, 6) k_adam<4>(const __grid_constant__ AdamLaunch L) {
   adam_pass<4>(L);
+}
+template <>
+__global__ void __launch_bounds__(kAdamThreads, 6) k_adam<5>(const __grid_constant__ AdamLaunch L) {
+  adam_pass<5>(L);
 }
 
 // Exponent of the E4M3 copy's scale from an amax of the stored master: the
@@ -437,9 +470,31 @@ __device__ __forceinline__ float stored_value(float x, float s_w) {
   return __fmul_rn(__half2float(__float2half_rn(__fmul_rn(x, s_w))), 1.0f / s_w);
 }
 
-// STAGE 1: after pass 1.  STAGE 2: after pass 1b.  STAGE 3: after pass 2.
-// STAGE 12: stages 1 and 2 in one launch (no chunk tracks its master amax,
-// so no chunk can be flagged and pass 1b has nothing to do).
+// Scale exponents of the master (FP16) and of its E4M3 copy when the new
+// master's amax is known to lie in [lo, hi] and that interval holds no scale
+// threshold of either; false otherwise (also for lo <= 0 or a non-finite hi).
+__device__ __forceinline__ bool interval_scales(const AdamLaunch &L, const AdamChunkDev &C, float lo, float hi,
+                                                int &kw, int &kq) {
+  int klo, khi;
+  if (!(lo > 0.0f && scale_exponent(lo, kMaxF16, L.margin, 0, klo) &&
+        scale_exponent(hi, kMaxF16, L.margin, 0, khi) && klo == khi))
+    return false;
+  kw = klo;
+  kq = 0;
+  if (C.wq_scale != nullptr) {
+    const float s = pow2f(kw);
+    int qlo, qhi;
+    if (!(scale_exponent(stored_value(lo, s), kMaxE4M3, L.margin, 0, qlo) &&
+          scale_exponent(stored_value(hi, s), kMaxE4M3, L.margin, 0, qhi) && qlo == qhi))
+      return false;
+    kq = qlo;
+  }
+  return true;
+}
+
+// STAGE 1: after the stats passes.  STAGE 2: after pass 1b.  STAGE 3: after
+// pass 2.  STAGE 12: stages 1 and 2 in one launch (the phased step: every
+// chunk's exact amaxes came from pass 1, so nothing is flagged).
 template <int STAGE>
 __global__ void k_adam_finalize(const __grid_constant__ AdamLaunch L) {
   for (int ci = threadIdx.x; ci < L.nchunks; ci += blockDim.x) {
@@ -447,7 +502,7 @@ __global__ void k_adam_finalize(const __grid_constant__ AdamLaunch L) {
     const AdamChunkDev &C = L.c[ci];
     uint32_t flags = __float_as_uint(ws[WS_FLAGS]);
     if constexpr (STAGE == 1 || STAGE == 12) {
-      int km, kv, kw = 0, kq = 0;
+      int km, kv;
       bool ok = scale_exponent(ws[WS_AMAX_M], kMaxE4M3, L.margin, 0, km);
       ok &= scale_exponent(ws[WS_AMAX_V], kMaxF16, L.margin, 0, kv);
       ws[WS_OLDINV_M] = 1.0f / *C.m_scale;
@@ -455,39 +510,39 @@ __global__ void k_adam_finalize(const __grid_constant__ AdamLaunch L) {
       ws[WS_OLDINV_W] = 1.0f / *C.w_scale;
       ws[WS_NEW_M] = pow2f(km);
       ws[WS_NEW_V] = pow2f(kv);
-      const bool tracked = C.w_amax != nullptr && *C.w_amax >= 0.0f;
-      bool exact = !tracked;
-      if (tracked) {
-        // amax|w_new| lies in [A0 - U, A0 + U], widened for the one rounding of w0 + dw
-        const float a0 = *C.w_amax, u = __fmul_ru(ws[WS_STEP_MAX], kStepBoundWiden);
-        const float hi = __fmul_rn(__fadd_ru(a0, u), 1.0f + 0x1p-20f);
-        const float lo = __fmul_rn(__fsub_rd(a0, u), 1.0f - 0x1p-20f);
-        int klo, khi;
-        bool known = lo > 0.0f && scale_exponent(lo, kMaxF16, L.margin, 0, klo) &&
-                     scale_exponent(hi, kMaxF16, L.margin, 0, khi) && klo == khi;
-        if (known) {
-          kw = klo;
-          if (C.wq_scale != nullptr) {
-            const float s = pow2f(kw);
-            int qlo, qhi;
-            known = scale_exponent(stored_value(lo, s), kMaxE4M3, L.margin, 0, qlo) &&
-                    scale_exponent(stored_value(hi, s), kMaxE4M3, L.margin, 0, qhi) && qlo == qhi;
-            kq = qlo;
-          }
-        }
-        flags = 2u | (known ? 0u : 1u);
-        exact = !known;
-      }
-      if (!exact) {
-        ws[WS_NEW_W] = pow2f(kw);
-        ws[WS_NEW_WQ] = pow2f(kq);
-      }
       if (!ok) atomicOr(&g_status, FP8_STATUS_NONFINITE);
+      const bool tracked = C.w_amax != nullptr && *C.w_amax >= 0.0f;
+      flags = tracked ? FLAG_TRACKED : 0u;
+      if (STAGE == 1 && (tracked || L.estimate)) {
+        float lo, hi;
+        if (tracked) {
+          // amax|w_new| lies in [A0 - U, A0 + U], widened for the estimated
+          // step and the one rounding of w0 + dw
+          const float a0 = *C.w_amax, u = __fmul_ru(ws[WS_STEP_MAX], kStepBoundWiden);
+          hi = __fmul_rn(__fadd_ru(a0, u), 1.0f + 0x1p-20f);
+          lo = __fmul_rn(__fsub_rd(a0, u), 1.0f - 0x1p-20f);
+        } else {
+          // the estimate A~ differs from the exact amax by at most the largest
+          // step error (< 2^-18 U) plus one rounding of the master (2^-23 A~)
+          const float a = ws[WS_APPROX_W];
+          const float e = __fadd_ru(__fmul_ru(ws[WS_STEP_MAX], 0x1p-16f), __fmul_ru(a, 0x1p-21f));
+          hi = __fmul_rn(__fadd_ru(a, e), 1.0f + 0x1p-20f);
+          lo = __fmul_rn(__fsub_rd(a, e), 1.0f - 0x1p-20f);
+        }
+        int kw, kq;
+        if (interval_scales(L, C, lo, hi, kw, kq)) {
+          ws[WS_NEW_W] = pow2f(kw);
+          ws[WS_NEW_WQ] = pow2f(kq);
+          flags |= FLAG_KNOWN;
+        } else {
+          flags |= FLAG_EXACT;
+        }
+      }
       ws[WS_FLAGS] = __uint_as_float(flags);
     }
     if constexpr (STAGE == 2 || STAGE == 12) {
-      // exact master amax: untracked chunks (pass 1) or flagged ones (pass 1b)
-      if (!(flags & 2u) || (flags & 1u)) {
+      // exact master amax: from pass 1 (phased step) or pass 1b (flagged chunks)
+      if (!(flags & FLAG_KNOWN)) {
         int kw, kq = 0;
         bool ok = scale_exponent(ws[WS_AMAX_W], kMaxF16, L.margin, 0, kw);
         if (C.wq_scale != nullptr)
@@ -505,13 +560,12 @@ __global__ void k_adam_finalize(const __grid_constant__ AdamLaunch L) {
       }
     }
     if constexpr (STAGE == 3) {
-      if (C.w_amax != nullptr) {
-        // the exact new amax must give the scale that was used
-        int kw;
-        if (scale_exponent(ws[WS_CHECK_W], kMaxF16, L.margin, 0, kw) && pow2f(kw) != ws[WS_NEW_W])
-          atomicOr(&g_status, FP8_STATUS_INTERNAL);
-        *C.w_amax = __fmul_rn(ws[WS_STORED_W], 1.0f / ws[WS_NEW_W]);
-      }
+      // a scale decided from an interval must be the one the exact new amax gives
+      int kw;
+      if ((flags & FLAG_KNOWN) && scale_exponent(ws[WS_CHECK_W], kMaxF16, L.margin, 0, kw) &&
+          pow2f(kw) != ws[WS_NEW_W])
+        atomicOr(&g_status, FP8_STATUS_INTERNAL);
+      if (C.w_amax != nullptr) *C.w_amax = __fmul_rn(ws[WS_STORED_W], 1.0f / ws[WS_NEW_W]);
     }
   }
 }

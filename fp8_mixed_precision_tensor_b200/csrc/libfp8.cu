@@ -29,7 +29,8 @@ struct DeviceInfo {
   int sms = 0;
   int adam_blocks_per_sm = 1;        // resident blocks of the update pass
   int adam_stats_blocks_per_sm = 1;  // of the exact stats pass and the exact master pass
-  int adam_bound_blocks_per_sm = 1;  // of the bound-only stats pass of tracking chunks
+  int adam_bound_blocks_per_sm = 1;  // of the estimated stats pass of tracking chunks
+  int adam_est_blocks_per_sm = 1;    // of the estimated stats pass of the other chunks
   int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair GEMM
   int wide_clusters = 0;  // co-resident 2-CTA clusters of the wide pair GEMM
 };
@@ -71,6 +72,9 @@ int device_info(DeviceInfo **out) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k_adam<4>, kAdamThreads, 0) != cudaSuccess)
       return FP8_ERR_CUDA;
     d.adam_bound_blocks_per_sm = bps > 0 ? bps : 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k_adam<5>, kAdamThreads, 0) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    d.adam_est_blocks_per_sm = bps > 0 ? bps : 1;
     int rc = FP8_OK;
     rc |= set_smem(gemm::k_gemm<256, false, false>, gemm::Cfg<256>::SMEM_BYTES);
     rc |= set_smem(gemm::k_gemm<256, false, true>, gemm::Cfg<256>::SMEM_BYTES);
@@ -472,9 +476,14 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
   L.eps = hp->eps;
   L.neg_lr_bc1 = (float)(-(double)hp->lr / (1.0 - pow((double)hp->beta1, (double)hp->step)));
   L.inv_bc2 = (float)(1.0 / (1.0 - pow((double)hp->beta2, (double)hp->step)));
+  // the whole step decides master scales from intervals (exact pass for the
+  // chunks whose interval is ambiguous); the phased step reduces the exact
+  // amaxes over ranks between its two calls
+  L.estimate = phases == PH_ALL ? 1 : 0;
   const unsigned cap = (unsigned)(d->sms * d->adam_blocks_per_sm);
   const unsigned cap1 = (unsigned)(d->sms * d->adam_stats_blocks_per_sm);
   const unsigned cap4 = (unsigned)(d->sms * d->adam_bound_blocks_per_sm);
+  const unsigned cap5 = (unsigned)(d->sms * d->adam_est_blocks_per_sm);
   for (int first = 0; first < nchunks; first += kAdamMaxChunksPerLaunch) {
     const int cnt = nchunks - first < kAdamMaxChunksPerLaunch ? nchunks - first : kAdamMaxChunksPerLaunch;
     unsigned long long tiles = 0;
@@ -494,25 +503,26 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
     const unsigned grid = tiles == 0 ? 1u : (unsigned)(tiles < cap ? tiles : cap);
     const unsigned grid1 = tiles == 0 ? 1u : (unsigned)(tiles < cap1 ? tiles : cap1);
     const unsigned grid4 = tiles == 0 ? 1u : (unsigned)(tiles < cap4 ? tiles : cap4);
+    const unsigned grid5 = tiles == 0 ? 1u : (unsigned)(tiles < cap5 ? tiles : cap5);
     bool tracked = false;
     for (int i = 0; i < cnt; i++) tracked |= L.c[i].w_amax != nullptr;
     if (phases & PH_STATS) {
-      // exact stats of the chunks without a known tracked amax (whether a
-      // tracking chunk's amax is known yet is only visible on the device);
-      // the bound-only stats of those with one
-      k_adam<1><<<grid1, kAdamThreads, 0, s>>>(L);
+      // stats of the chunks without a known tracked amax (whether a tracking
+      // chunk's amax is known yet is only visible on the device): estimated
+      // (whole step) or exact (phased step); those with one: estimated
+      if (L.estimate) k_adam<5><<<grid5, kAdamThreads, 0, s>>>(L);
+      else            k_adam<1><<<grid1, kAdamThreads, 0, s>>>(L);
       if (tracked) k_adam<4><<<grid4, kAdamThreads, 0, s>>>(L);
     }
-    if (phases & PH_APPLY) {
-      if (tracked) {
-        k_adam_finalize<1><<<1, 256, 0, s>>>(L);
-        k_adam<3><<<grid1, kAdamThreads, 0, s>>>(L);  // exact master amax, flagged chunks only
-        k_adam_finalize<2><<<1, 256, 0, s>>>(L);
-      } else {
-        k_adam_finalize<12><<<1, 256, 0, s>>>(L);
-      }
+    if (phases == PH_ALL) {
+      k_adam_finalize<1><<<1, 256, 0, s>>>(L);
+      k_adam<3><<<grid1, kAdamThreads, 0, s>>>(L);  // exact master amax, flagged chunks only
+      k_adam_finalize<2><<<1, 256, 0, s>>>(L);
       k_adam<2><<<grid, kAdamThreads, 0, s>>>(L);    // update
-      if (tracked) k_adam_finalize<3><<<1, 256, 0, s>>>(L);
+      k_adam_finalize<3><<<1, 256, 0, s>>>(L);       // check of the decided scales; tracked amax
+    } else if (phases & PH_APPLY) {
+      k_adam_finalize<12><<<1, 256, 0, s>>>(L);
+      k_adam<2><<<grid, kAdamThreads, 0, s>>>(L);    // update
     }
     if ((rc = launch_rc())) return rc;
   }

@@ -6,7 +6,7 @@
     python profile_cases.py adam --n 67108864 [--track]
     python profile_cases.py allreduce --n 268435456 --world 8
     python profile_cases.py castcount --n 268435456
-    python profile_cases.py adam7b --iters 10
+    python profile_cases.py adam7b --iters 10 [--track] [--copy]
 
 Each case runs `--iters` passes after one warm-up pass on seeded synthetic
 inputs and prints the CUDA-event time per pass.  Launch order per pass:
@@ -207,14 +207,15 @@ def case_castcount(a):
     return one
 
 
-def build_adam_state(chunks, device="cuda", seed=11, mu=2.0 ** 10, track=False):
+def build_adam_state(chunks, device="cuda", seed=11, mu=2.0 ** 10, track=False, copy=False):
     """Decoupled-Adam state for (name, n) chunks: FP16 master from weights
-    ~N(0, 0.02), zero moments, E5M2 gradients ~N(0, 1e-3) scaled by mu.
-    Returns the AdamTensorState list."""
+    ~N(0, 0.02), zero moments, E5M2 gradients ~N(0, 1e-3) scaled by mu; with
+    `copy` the step also writes each tensor's E4M3 weight copy.  Returns the
+    AdamTensorState list."""
     out = []
     for ci, (_, n) in enumerate(chunks):
         w = synth.device_normal((n,), 0.02, seed * 100000 + 2 * ci + 1, torch.float32, device)
-        st = AdamTensorState(w, track_master_amax=track)
+        st = AdamTensorState(w, track_master_amax=track, e4m3_copy=copy)
         del w
         g = synth.device_normal((n,), 1e-3, seed * 100000 + 2 * ci, torch.float32, device)
         st.set_gradient(g, mu)
@@ -224,7 +225,7 @@ def build_adam_state(chunks, device="cuda", seed=11, mu=2.0 ** 10, track=False):
 
 
 def case_adam7b(a):
-    chunks_list = [st.chunk for st in build_adam_state(synth.gpt7b_adam_chunks(), track=a.track)]
+    chunks_list = [st.chunk for st in build_adam_state(synth.gpt7b_adam_chunks(), track=a.track, copy=a.copy)]
     params = sum(c.g.numel() for c in chunks_list)
     chunks = fp8.pack_adam_chunks(chunks_list)
     ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(chunks_list)) // 4, dtype=torch.float32, device="cuda")
@@ -235,8 +236,13 @@ def case_adam7b(a):
         fp8.fp8_adam_step(chunks, 1e-4, 0.9, 0.95, 1e-8, state["t"], 0, ws)
 
     t = _timed(one, a.iters)
-    print(f"adam7b: {len(chunks_list)} chunks, {params} params, {t:.3f} ms per step, "
-          f"{11 * params / t / 1e6:.0f} GB/s algorithmic (11 B/param), {17 * params / t / 1e6:.0f} GB/s moved")
+    # bytes moved per parameter: the stats pass reads g, m, v (and the master
+    # unless its amax is tracked), the update pass reads g, m, v, w and writes
+    # m, v, w (and the E4M3 copy)
+    moved = (4 if a.track else 6) + 11 + (1 if a.copy else 0)
+    print(f"adam7b: {len(chunks_list)} chunks, {params} params, track={a.track} copy={a.copy}: "
+          f"{t:.3f} ms per step, {11 * params / t / 1e6:.0f} GB/s algorithmic (11 B/param), "
+          f"{moved * params / t / 1e6:.0f} GB/s moved ({moved} B/param)")
     return one
 
 
@@ -250,6 +256,7 @@ def main():
     ap.add_argument("--iters", type=int, default=2)
     ap.add_argument("--world", type=int, default=8, help="allreduce: emulated ranks")
     ap.add_argument("--track", action="store_true", help="adam: track the master amax across steps")
+    ap.add_argument("--copy", action="store_true", help="adam7b: write the E4M3 weight copy")
     a = ap.parse_args()
     one = {"linear": case_linear, "cast": case_cast, "castsweep": case_castsweep, "adam": case_adam,
            "allreduce": case_allreduce,

@@ -27,7 +27,13 @@ def f16_vals(bits: np.ndarray) -> np.ndarray:
 
 
 def f16_ulp(vals: np.ndarray) -> np.ndarray:
-    return np.spacing(np.abs(vals).astype(np.float16)).astype(np.float64)
+    """Unit in the last place of binary16 values: 2^(e - 10) in the binade
+    [2^e, 2^(e+1)), 2^-24 among subnormals, 32 at the largest finite 65504
+    (np.spacing would step past it to inf)."""
+    a = np.abs(np.asarray(vals)).astype(np.float16).astype(np.float64)
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.maximum(a, 2.0 ** -14)))
+    return 2.0 ** (e - 10)
 
 
 def half_ulp_out(ref: np.ndarray, out_dtype: torch.dtype) -> np.ndarray:

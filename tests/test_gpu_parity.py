@@ -421,7 +421,7 @@ def _slice(state, lo, hi):
     return {k: (v[lo:hi] if isinstance(v, np.ndarray) else v) for k, v in state.items()}
 
 
-def check_adam_chunk(before, c, step, margin=0, ties=None, slices=1):
+def check_adam_chunk(before, c, step, margin=0, ties=None, slices=1, hp=HP):
     """Oracle step from `before` against the chunk's state now.  Scales must be
     bit-equal; a mismatch is allowed only where the oracle's float64 amax lies
     within 4 binary32 ULPs of a scale threshold (a tie).  A tie is appended to
@@ -436,7 +436,7 @@ def check_adam_chunk(before, c, step, margin=0, ties=None, slices=1):
 
     def run(b, amax_in=None):
         return oracle.adam_step(b["g"], b["g_inv"], b["m"], b["s_m"], b["v"], b["s_v"], b["w"], b["s_w"],
-                                t=step, margin=margin, amax_in=amax_in, **HP)
+                                t=step, margin=margin, amax_in=amax_in, **hp)
 
     first = run(before) if slices == 1 else None
     amax = first["amax"] if slices == 1 else tuple(
@@ -463,7 +463,7 @@ def check_adam_chunk(before, c, step, margin=0, ties=None, slices=1):
         out = first if (slices == 1 and amax_in is None) else run(b, amax_in)
         assert (a["s_m"], a["s_v"], a["s_w"]) == (out["s_m"], out["s_v"], out["s_w"])
         # master within 1 FP16 ULP (+ the binary32 step term); second moment within 1 FP16 ULP
-        slack = STEP_ROUNDINGS * 2.0 ** -24 * adam_step_magnitude(b, step)
+        slack = STEP_ROUNDINGS * 2.0 ** -24 * adam_step_magnitude(b, step, hp)
         for key, okey, skey in (("w", "wh", "s_w"), ("v", "vh", "s_v")):
             ref = f16_vals(out[okey]) / out[skey]
             got = f16_vals(a[key]) / a[skey]
@@ -551,11 +551,11 @@ def test_adam_rejects_bad_args():
 
 
 # ---------------------------------------------------------------- Adam: tracked master amax, E4M3 copy
-def _with_tracking(chunks, wq=False):
+def _with_tracking(chunks, wq=False, track=True):
     out = []
     for c in chunks:
         n = c.g.numel()
-        extra = dict(w_amax=torch.full((1,), -1.0, **F32))
+        extra = dict(w_amax=torch.full((1,), -1.0, **F32)) if track else {}
         if wq:
             extra.update(wq=torch.empty(n, dtype=torch.uint8, device="cuda"), wq_scale=scalar(), wq_inv=scalar())
         out.append(fp8.AdamChunk(c.g, c.g_inv, c.m, c.m_scale, c.v, c.v_scale, c.w, c.w_scale, **extra))
@@ -643,6 +643,71 @@ def test_adam_tracked_amax_straddling_a_threshold_takes_the_exact_pass():
     got = f16_vals(after["w"]) / after["s_w"]
     assert np.all(np.abs(got - ref) <= f16_ulp(f16_vals(out["wh"])) / out["s_w"])
     assert trk[0].w_amax.item() == _stored_amax(after)
+
+
+def _set_master(c, w):
+    """Store host weights w as the chunk's FP16 master (scale from their amax)."""
+    d = to_dev(w)
+    a, inv = scalar(), scalar()
+    fp8.fp8_amax(d, a)
+    fp8.fp8_compute_scale(a, fp8.FP8_F16S, 0, 1.0, c.w_scale, inv)
+    fp8.fp8_cast(d, fp8.FP8_F16S, c.w_scale, c.w)
+
+
+@pytest.mark.parametrize("wq", [False, True])
+def test_adam_estimated_stats_equal_exact_stats(wq):
+    """The whole step decides each untracked chunk's master scale from an
+    estimated amax and its error interval; the phased step (stats, then
+    apply) computes the exact amax.  Both must leave the same state bit for
+    bit: for a chunk whose largest weight sits exactly on an FP16 scale
+    threshold and does not move (zero gradient and moment), one whose largest
+    weight steps from above the threshold onto it (within a few binary32
+    ULPs: the interval cannot decide either, so the exact pass runs), and
+    plain chunks."""
+    n = 8192
+    thresh = 65504.0 * 2.0 ** -17  # 0.499755859375: scale 2^17 at or below it, 2^16 above
+    sets = []
+    for _ in range(2):
+        chunks = make_adam_state([n] * 3, ("estimate",))
+        for k, c in enumerate(chunks):
+            w = synth.normal_f32((n,), 0.05, "estimate", k, "w")
+            if k < 2:
+                w[100 + k] = thresh if k == 0 else 0.5  # 0.5: the next FP16 value above it at scale 2^16
+            _set_master(c, w)
+        chunks[0].g[100] = 0      # does not move
+        chunks[1].g[101] = 0x3C   # E5M2 1.0: a positive gradient, the step goes down
+        if wq:
+            chunks = _with_tracking(chunks, wq=True, track=False)
+        sets.append(chunks)
+    whole, phased = sets
+    # step 1 from zero moments: dw = -lr g / (|g| + eps); this lr makes the
+    # second chunk's 0.5 land on the threshold (0.5 - 2^-12) up to roundings
+    g = float(whole[1].g_inv.item())
+    hp = dict(HP, lr=2.0 ** -12 * (g + HP["eps"]) / g)
+    ws = torch.zeros(fp8.fp8_adam_workspace_bytes(3) // 4, **F32)
+    ws2 = torch.zeros_like(ws)
+    ties = []
+    for step in (1, 2):
+        before = [snapshot(c) for c in whole]
+        fp8.fp8_adam_step(whole, step=step, margin=0, workspace=ws, **hp)
+        fp8.fp8_adam_stats(phased, step=step, margin=0, workspace=ws2, **hp)
+        fp8.fp8_adam_apply(phased, step=step, margin=0, workspace=ws2, **hp)
+        assert fp8.fp8_get_status() == 0
+        for b, x, y in zip(before, whole, phased):
+            sx, sy = snapshot(x), snapshot(y)
+            for k in ("m", "v", "w", "s_m", "s_v", "s_w"):
+                assert np.array_equal(np.asarray(sx[k]), np.asarray(sy[k])), (step, k)
+            if wq:
+                assert x.wq_scale.item() == y.wq_scale.item()
+                assert np.array_equal(x.wq.cpu().numpy(), y.wq.cpu().numpy())
+        if step == 1:
+            # both threshold chunks really ended at the threshold
+            for c in whole[:2]:
+                assert abs(_stored_amax(snapshot(c)) - thresh) <= thresh * 2.0 ** -10
+        # the oracle agrees (the threshold chunks may tie in float64)
+        for b, x in zip(before, whole):
+            check_adam_chunk(b, x, step, ties=ties, hp=hp)
+    assert len(ties) <= 2 + MAX_TIES, ties
 
 
 @pytest.mark.parametrize("dt", [fp8.FP8_DT_F32, fp8.FP8_DT_BF16])
