@@ -445,8 +445,11 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
   // is below 2^-63, under half an ULP of such an eps, so sqrt(v_hat) + eps
   // rounds to eps and the subnormal's lost precision never reaches the step;
   // eps = 0 would also turn a zero gradient on a zero state into 0/0.
+  // eps <= 2^64: sqrt(v_hat) + eps stays below 2^66 (v_hat is a finite
+  // float), so its reciprocal, by which the step multiplies, is a normal
+  // number with full precision.
   if (!(hp->lr >= 0.0f && hp->lr <= 3.402823466e38f) || !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) ||
-      !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f) || !(hp->eps >= 0x1p-39f && hp->eps <= 3.402823466e38f) ||
+      !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f) || !(hp->eps >= 0x1p-39f && hp->eps <= 0x1p64f) ||
       hp->step < 1 || hp->margin < 0 || hp->margin > 64)
     return FP8_ERR_INVALID_ARG;
   for (int i = 0; i < nchunks; i++) {

@@ -258,7 +258,8 @@ int fp8_linear_wgrad(const uint8_t *dyq, const float *dy_inv, const uint8_t *xq,
  * fp8_compute_scale with `margin`, fmt_max 448 / 65504 / 65504) and the state
  * is re-encoded with them; the new scales replace m_scale, v_scale, w_scale.
  * Arithmetic is float32 with every operation rounded to nearest (square root
- * and quotient correctly rounded); a non-finite new amax sets
+ * and reciprocal correctly rounded; the quotient multiplies by the
+ * reciprocal); a non-finite new amax sets
  * FP8_STATUS_NONFINITE and that scale to 1.
  * Tracked master amax (optional; the first pass then moves 4 instead of 6
  * bytes per parameter): when w_amax points to the exact amax of the
@@ -292,10 +293,12 @@ typedef struct {
 } fp8_adam_chunk;
 
 typedef struct {
-  float lr, beta1, beta2, eps; /* 0 <= lr finite, 0 <= beta < 1, 2^-39 <= eps finite
-                                  (a smaller eps returns FP8_ERR_INVALID_ARG: eps = 0
-                                  makes a zero gradient on a zero state 0/0, and below
-                                  2^-39 a binary32-subnormal v_hat would reach the step) */
+  float lr, beta1, beta2, eps; /* 0 <= lr finite, 0 <= beta < 1, 2^-39 <= eps <= 2^64
+                                  (else FP8_ERR_INVALID_ARG: eps = 0 makes a zero
+                                  gradient on a zero state 0/0, below 2^-39 a
+                                  binary32-subnormal v_hat would reach the step, above
+                                  2^64 the reciprocal of sqrt(v_hat) + eps could be
+                                  subnormal) */
   int step;                    /* t >= 1 (bias correction) */
   int margin;                  /* scale margin, >= 0 */
 } fp8_adam_hparams;

@@ -130,8 +130,9 @@ def test_host_side_validation_of_the_next_rows(lib):
 
 
 def test_adam_rejects_hyper_parameters_outside_the_argued_range(lib):
-    """eps below 2^-39 (eps = 0 included), a non-finite lr or eps, beta >= 1 and
-    step 0 are refused on the host with FP8_ERR_INVALID_ARG, nothing enqueued."""
+    """eps below 2^-39 (eps = 0 included) or above 2^64, a non-finite lr or eps,
+    beta >= 1 and step 0 are refused on the host with FP8_ERR_INVALID_ARG,
+    nothing enqueued."""
     from fp8_mixed_precision_tensor_b200 import fp8
 
     p, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
@@ -141,7 +142,8 @@ def test_adam_rejects_hyper_parameters_outside_the_argued_range(lib):
     lib.fp8_adam_step.argtypes = [ctypes.POINTER(fp8._Chunk), i, ctypes.POINTER(fp8._HParams), p, sz, p]
     inf = float("inf")
     for lr, b1, b2, eps, t in ((1e-4, 0.9, 0.95, 0.0, 1), (1e-4, 0.9, 0.95, 2.0 ** -40, 1),
-                               (1e-4, 0.9, 0.95, inf, 1), (inf, 0.9, 0.95, 1e-8, 1),
+                               (1e-4, 0.9, 0.95, inf, 1), (1e-4, 0.9, 0.95, 2.0 ** 65, 1),
+                               (inf, 0.9, 0.95, 1e-8, 1),
                                (1e-4, 1.0, 0.95, 1e-8, 1), (1e-4, 0.9, 0.95, 1e-8, 0)):
         hp = fp8._HParams(lr, b1, b2, eps, t, 0)
         assert lib.fp8_adam_step(arr, 1, ctypes.byref(hp), fake, 64, None) == fp8.FP8_ERR_INVALID_ARG, \
