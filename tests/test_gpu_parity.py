@@ -662,20 +662,23 @@ def test_adam_estimated_stats_equal_exact_stats(wq):
     bit: for a chunk whose largest weight sits exactly on an FP16 scale
     threshold and does not move (zero gradient and moment), one whose largest
     weight steps from above the threshold onto it (within a few binary32
-    ULPs: the interval cannot decide either, so the exact pass runs), and
-    plain chunks."""
+    ULPs: the interval cannot decide either, so the exact pass runs), one
+    whose largest weight sits on a threshold of the E4M3 copy's scale (448 *
+    2^-10: only the copy's interval is ambiguous), and a plain chunk."""
     n = 8192
     thresh = 65504.0 * 2.0 ** -17  # 0.499755859375: scale 2^17 at or below it, 2^16 above
     sets = []
     for _ in range(2):
-        chunks = make_adam_state([n] * 3, ("estimate",))
+        chunks = make_adam_state([n] * 4, ("estimate",))
         for k, c in enumerate(chunks):
             w = synth.normal_f32((n,), 0.05, "estimate", k, "w")
-            if k < 2:
-                w[100 + k] = thresh if k == 0 else 0.5  # 0.5: the next FP16 value above it at scale 2^16
+            if k < 3:
+                # 0.5: the next FP16 value above the threshold at scale 2^16
+                w[100 + k] = (thresh, 0.5, 448.0 * 2.0 ** -10)[k]
             _set_master(c, w)
         chunks[0].g[100] = 0      # does not move
         chunks[1].g[101] = 0x3C   # E5M2 1.0: a positive gradient, the step goes down
+        chunks[2].g[102] = 0      # does not move
         if wq:
             chunks = _with_tracking(chunks, wq=True, track=False)
         sets.append(chunks)
@@ -684,7 +687,7 @@ def test_adam_estimated_stats_equal_exact_stats(wq):
     # second chunk's 0.5 land on the threshold (0.5 - 2^-12) up to roundings
     g = float(whole[1].g_inv.item())
     hp = dict(HP, lr=2.0 ** -12 * (g + HP["eps"]) / g)
-    ws = torch.zeros(fp8.fp8_adam_workspace_bytes(3) // 4, **F32)
+    ws = torch.zeros(fp8.fp8_adam_workspace_bytes(4) // 4, **F32)
     ws2 = torch.zeros_like(ws)
     ties = []
     for step in (1, 2):
@@ -704,6 +707,7 @@ def test_adam_estimated_stats_equal_exact_stats(wq):
             # both threshold chunks really ended at the threshold
             for c in whole[:2]:
                 assert abs(_stored_amax(snapshot(c)) - thresh) <= thresh * 2.0 ** -10
+            assert _stored_amax(snapshot(whole[2])) == 448.0 * 2.0 ** -10
         # the oracle agrees (the threshold chunks may tie in float64)
         for b, x in zip(before, whole):
             check_adam_chunk(b, x, step, ties=ties, hp=hp)
