@@ -433,20 +433,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    int stage = 0;
-    uint32_t phase = 0;
-    // parity of the last load issued into each stage (for the abort drain)
-    uint32_t issued_mask = 0, issued_par = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < args.num_tiles && ok; tile += gridDim.x) {
-      int mb, nb;
-      tile_coords(tile, args, mb, nb);
-      for (int kb = 0; kb < args.num_k_blocks; kb++) {
-        bool got = lane == 0 ? mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag) : true;
-        got = __shfl_sync(0xffffffffu, got, 0);
-        if (!got) { ok = false; break; }
-        if (lane == 0) {
+    // ------------------------------------------------------------ producer (one thread)
+    // The loop runs in one thread with no warp-wide step per k-block, as the
+    // MMA issuer's does: a warp-synchronous loop (lane 0 waits, the warp
+    // re-converges on a shuffle) held the wide kernel's operand feed to about
+    // 60 % of what this loop streams.
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      // parity of the last load issued into each stage (for the abort drain)
+      uint32_t issued_mask = 0, issued_par = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < args.num_tiles && ok; tile += gridDim.x) {
+        int mb, nb;
+        tile_coords(tile, args, mb, nb);
+        for (int kb = 0; kb < args.num_k_blocks; kb++) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) { ok = false; break; }
           const uint32_t sa = base + stage * C::STAGE_BYTES, sb = sa + C::A_BYTES;
           mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
           if (A_MN) tma_load_2d(sa, &tmA, mb * BM, kb * BK, full_bar(stage));
@@ -460,16 +462,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           issued_mask |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
-        __syncwarp();
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) {
+        // let every issued copy land before the CTA can exit
+        for (int s = 0; s < C::STAGES; s++)
+          if (issued_mask & (1u << s)) mbar_wait_drain(full_bar(s), (issued_par >> s) & 1u);
       }
     }
-    if (!ok && lane == 0) {
-      // let every issued copy land before the CTA can exit
-      for (int s = 0; s < C::STAGES; s++)
-        if (issued_mask & (1u << s)) mbar_wait_drain(full_bar(s), (issued_par >> s) & 1u);
-    }
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (one thread)
     // Descriptors advance by constant adds, as in k_gemm3's issuer.
@@ -619,20 +621,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producers (both CTAs)
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true, issued = false;
-    for (int tile = pair; tile < args.num_tiles && ok; tile += num_pairs) {
-      int mb, nb;
-      tile_coords(tile, args, mb, nb);
-      const int arow = mb * (2 * kPairHalf) + (int)rank * kPairHalf;
-      const int bcol = nb * kPairBN + (int)rank * kPairHalf;
-      for (int kb = 0; kb < args.num_k_blocks; kb++) {
-        bool got = lane == 0 ? mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag) : true;
-        got = __shfl_sync(0xffffffffu, got, 0);
-        if (!got) { ok = false; break; }
-        if (lane == 0) {
+    // ------------------------------------------------------------ producers (both CTAs, one thread)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, issued = false;
+      for (int tile = pair; tile < args.num_tiles && ok; tile += num_pairs) {
+        int mb, nb;
+        tile_coords(tile, args, mb, nb);
+        const int arow = mb * (2 * kPairHalf) + (int)rank * kPairHalf;
+        const int bcol = nb * kPairBN + (int)rank * kPairHalf;
+        for (int kb = 0; kb < args.num_k_blocks; kb++) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) { ok = false; break; }
           const uint32_t sa = base + stage * kPairStageBytes, sb = sa + kPairHalf * BK;
           const uint32_t fb = map_to_rank(full_bar(stage), 0);
           if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * kPairStageBytes);
@@ -641,12 +641,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (B_MN) tma_load_2d_pair(sb, &tmB, bcol, kb * BK, fb);
           else      tma_load_2d_pair(sb, &tmB, kb * BK, bcol, fb);
           issued = true;
+          if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
         }
-        __syncwarp();
-        if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
       }
+      if (!ok && issued) sleep_ns_bounded(50000);  // let copies in flight land
     }
-    if (!ok && issued && lane == 0) sleep_ns_bounded(50000);  // let copies in flight land
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader, one thread)
     // Descriptors advance by constant adds, as in k_gemm3's issuer.
@@ -806,20 +806,21 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producers (both CTAs)
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true, issued = false;
-    for (int tile = pair; tile < args.num_tiles && ok; tile += num_pairs) {
-      int mb, nb;
-      tile_coords(tile, args, mb, nb);
-      const int arow = mb * (2 * kPairHalf) + (int)rank * kPairHalf;
-      const int bcol = nb * kWideBN + (int)rank * (2 * kPairHalf);
-      for (int kb = 0; kb < args.num_k_blocks; kb++) {
-        bool got = lane == 0 ? mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag) : true;
-        got = __shfl_sync(0xffffffffu, got, 0);
-        if (!got) { ok = false; break; }
-        if (lane == 0) {
+    // ------------------------------------------------------------ producers (both CTAs, one thread)
+    // One thread runs the loop (no warp-wide step per k-block): the
+    // warp-synchronous form streamed a stage every ~1260 SM cycles, this one
+    // every ~810, ahead of the tensor core's ~1030.
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, issued = false;
+      for (int tile = pair; tile < args.num_tiles && ok; tile += num_pairs) {
+        int mb, nb;
+        tile_coords(tile, args, mb, nb);
+        const int arow = mb * (2 * kPairHalf) + (int)rank * kPairHalf;
+        const int bcol = nb * kWideBN + (int)rank * (2 * kPairHalf);
+        for (int kb = 0; kb < args.num_k_blocks; kb++) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) { ok = false; break; }
           const uint32_t sa = base + stage * kWideStageBytes, sb = sa + kPairHalf * BK;
           const uint32_t fb = map_to_rank(full_bar(stage), 0);
           if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * kWideStageBytes);
@@ -832,12 +833,12 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             tma_load_2d_pair(sb, &tmB, kb * BK, bcol, fb);  // one box of 256 rows
           }
           issued = true;
+          if (++stage == kWideStages) { stage = 0; phase ^= 1u; }
         }
-        __syncwarp();
-        if (++stage == kWideStages) { stage = 0; phase ^= 1u; }
       }
+      if (!ok && issued) sleep_ns_bounded(50000);  // let copies in flight land
     }
-    if (!ok && issued && lane == 0) sleep_ns_bounded(50000);  // let copies in flight land
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader, one thread)
     // The whole loop runs in one thread with no warp-wide step per k-block,
