@@ -135,23 +135,28 @@ __global__ void __launch_bounds__(kSumThreads)
 
 // Faster exact sum for up to kSumFastMaxRanks ranks (E5M2; E4M3 up to
 // kSumMaxRanks).  The codes are decoded by the hardware cvt (fp8x2 -> f16x2,
-// exact) and summed in two binary32 accumulators split at |x| = 2: values
-// below are multiples of the smallest subnormal and stay below 2, values from
-// 2 up are multiples of 2^-1 (E5M2) or 2^-2 (E4M3), so neither partial sum
-// ever needs more than 24 significant bits and both are exact.  Their sum is
-// formed in binary64 (exact), rounded to binary32 by round-to-odd and then by
-// the saturating cvt.  inf and NaN propagate through the float adds (NaN ->
-// 0x7F, inf -> saturated and counted as an overflow), as in the integer path.
+// exact) and each value x is split as x = t + (x - t), t = x rounded to a
+// multiple of 1/2 by adding and subtracting 1.5 * 2^22 (whose binary32 ULP is
+// 1/2; |x| <= 57344 keeps x + 1.5 * 2^22 in that binade).  The t are
+// multiples of 1/2 below 57344 and the x - t multiples of the smallest
+// subnormal (2^-16 E5M2, 2^-9 E4M3) of magnitude at most 1/4, so for up to 128
+// E5M2 or 4096 E4M3 ranks neither running sum needs more than 24 significant
+// bits: both are exact, and the split costs packed adds only (no compare,
+// no select).  Their sum is formed in binary64 (exact), rounded to binary32
+// by round-to-odd and then by the saturating cvt.  An inf or NaN code makes
+// t, and so the t-sum, non-finite (the other sum then holds a NaN): a NaN
+// t-sum (a NaN code, or +inf with -inf) encodes as 0x7F, an infinite one
+// saturates and counts as an overflow, as in the integer path.
 constexpr int kSumFastMaxRanks = 128;
+constexpr float kSplitC = 0x1.8p22f;  // 1.5 * 2^22: binary32 ULP 1/2
 
 template <int FMT>
 __device__ __forceinline__ uint32_t encode_split_sum(float hi, float lo, float fmax, uint32_t &under,
                                                      uint32_t &over) {
-  if (!(fabsf(hi) <= 3.402823466e38f && fabsf(lo) <= 3.402823466e38f)) {  // inf or NaN involved
-    const float t = hi + lo;
-    if (t != t) return 0x7Fu;
+  if (!(fabsf(hi) <= 3.402823466e38f)) {  // an inf or NaN code was summed
+    if (hi != hi) return 0x7Fu;
     over++;
-    return t > 0.0f ? top_code(FMT) : (0x80u | top_code(FMT));
+    return hi > 0.0f ? top_code(FMT) : (0x80u | top_code(FMT));
   }
   const double d = (double)hi + (double)lo;
   float f = __double2float_rz(d);
@@ -171,26 +176,28 @@ __global__ void __launch_bounds__(kSumThreads)
   const size_t groups = n / 16;
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   uint32_t under = 0, over = 0;
+  const float2 c = both(kSplitC), neg_c = both(-kSplitC), minus1 = both(-1.0f);
   for (size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x; g < groups; g += stride) {
-    float hi[16], lo[16];
+    float2 hi[8], lo[8];  // pairs of elements
 #pragma unroll
-    for (int j = 0; j < 16; j++) hi[j] = lo[j] = 0.0f;
+    for (int p = 0; p < 8; p++) hi[p] = lo[p] = both(0.0f);
     for (int r = 0; r < nranks; r++) {
       const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(in + (size_t)r * ld) + g);
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int p = 0; p < 8; p++) {
         const float2 x = dec2<FMT>(w[p >> 1] >> ((p & 1) * 16));
-        const bool ba = fabsf(x.x) >= 2.0f, bb = fabsf(x.y) >= 2.0f;
-        hi[2 * p] += ba ? x.x : 0.0f;
-        lo[2 * p] += ba ? 0.0f : x.x;
-        hi[2 * p + 1] += bb ? x.y : 0.0f;
-        lo[2 * p + 1] += bb ? 0.0f : x.y;
+        const float2 t = __fadd2_rn(__fadd2_rn(x, c), neg_c);  // x to a multiple of 1/2
+        hi[p] = __fadd2_rn(hi[p], t);
+        lo[p] = __fadd2_rn(lo[p], __ffma2_rn(t, minus1, x));   // x - t, exact
       }
     }
     uint32_t o[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int j = 0; j < 16; j++) o[j >> 2] |= encode_split_sum<FMT>(hi[j], lo[j], fmax, under, over) << (8 * (j & 3));
+    for (int j = 0; j < 16; j++) {
+      const float h = (j & 1) ? hi[j >> 1].y : hi[j >> 1].x, l = (j & 1) ? lo[j >> 1].y : lo[j >> 1].x;
+      o[j >> 2] |= encode_split_sum<FMT>(h, l, fmax, under, over) << (8 * (j & 3));
+    }
     __stcs(reinterpret_cast<uint4 *>(out) + g, make_uint4(o[0], o[1], o[2], o[3]));
   }
   if (blockIdx.x == 0) {
@@ -198,7 +205,9 @@ __global__ void __launch_bounds__(kSumThreads)
       float hi = 0.0f, lo = 0.0f;
       for (int r = 0; r < nranks; r++) {
         const float x = dec2<FMT>(in[(size_t)r * ld + i]).x;
-        if (fabsf(x) >= 2.0f) hi += x; else lo += x;
+        const float t = __fadd_rn(__fadd_rn(x, kSplitC), -kSplitC);
+        hi = __fadd_rn(hi, t);
+        lo = __fadd_rn(lo, __fmaf_rn(t, -1.0f, x));
       }
       out[i] = (uint8_t)encode_split_sum<FMT>(hi, lo, fmax, under, over);
     }
