@@ -85,13 +85,15 @@ def config_of(wl: dict, schedule: str, world: int) -> dict:
 
 def gemm_traffic(workload: str):
     """Mean DRAM bytes per GEMM launch of this step from the committed ncu
-    capture, valid while the GEMM kernel source is the one that was measured
-    and the capture is of this workload."""
+    capture, valid while the GEMM kernel source and its launch set-up (tile
+    order) are the ones that were measured and the capture is of this
+    workload."""
     import hashlib
 
     try:
         rec = json.load(open(os.path.join(ROOT, "profiles", "gemm_step_traffic.json")))
-        src = open(os.path.join(ROOT, "fp8_mixed_precision_tensor_b200", "csrc", "gemm.cuh"), "rb").read()
+        csrc = os.path.join(ROOT, "fp8_mixed_precision_tensor_b200", "csrc")
+        src = b"".join(open(os.path.join(csrc, f), "rb").read() for f in ("gemm.cuh", "libfp8.cu"))
         if hashlib.sha256(src).hexdigest() == rec["gemm_source_sha256"] and rec.get("workload") == workload:
             return rec["dram_bytes_per_launch_mean"]
     except Exception:
