@@ -69,7 +69,7 @@ MU = 2.0 ** 10
 HP = dict(lr=1e-4, beta1=0.9, beta2=0.95, eps=1e-8)
 # Algorithmic bytes per element / parameter (reads + writes of the definition).
 CAST_BYTES_BF16 = 2 + 2 + 1   # amax read + cast read + code write
-GRAD_CAST_BYTES = 4 + 1       # fp32 dW read (amax fused in the GEMM) + code write
+GRAD_CAST_BYTES = 2 + 1       # round-to-odd bf16 dW read (amax fused in the GEMM) + code write
 ADAM_BYTES = 11               # read g1 m1 v2 w2, write m1 v2 w2
 
 
@@ -80,6 +80,7 @@ def config_of(wl: dict, schedule: str, world: int) -> dict:
             "linears": [l[0] for l in wl["linears"]], "adam_params": sum(N * K for _, K, N in wl["linears"]),
             "gemm_flops_per_step": flops, "l2": "inputs larger than L2 (no flush)", "schedule": schedule,
             "weight_operand": "E4M3 copy written by the previous Adam step", "master_amax": "tracked",
+            "weight_gradient": "bf16 rounded to odd (its E5M2 cast equals the float32 dW's)",
             "parallelism": f"replicas{world}" if world > 1 else "single"}
 
 
@@ -217,7 +218,9 @@ class BlockStep:
             d["xq"], d["wq"], d["dyq"] = (torch.empty(s, **u8) for s in ((M, K), (N, K), (M, N)))
             d["y"] = torch.empty((M, N), dtype=torch.bfloat16, device=device)
             d["dx"] = torch.empty((M, K), dtype=torch.bfloat16, device=device)
-            d["dw"] = torch.empty((N, K), **f32)
+            # the wgrad's output, bfloat16 rounded to odd: its E5M2 cast gives the
+            # codes and scale of the float32 dW's at half the bytes
+            d["dw"] = torch.empty((N, K), dtype=torch.bfloat16, device=device)
             d["gq"] = torch.empty((N, K), **u8)
             # scalars: amax/scale/inv of x (0-2), w (3-5: the E4M3 weight's, rewritten by
             # Adam), dy (6-8); g scale and inverse (10, 11); fused amaxes of y, dx, dw (12-14)
@@ -283,7 +286,7 @@ class BlockStep:
             e = mark("gemm")
             fp8.fp8_linear_fwd(d["xq"], sc[2:3], d["wq"], sc[5:6], d["y"], sc[12:13])
             fp8.fp8_linear_dgrad(d["dyq"], sc[8:9], d["wq"], sc[5:6], d["dx"], sc[13:14])
-            fp8.fp8_linear_wgrad(d["dyq"], sc[8:9], d["xq"], sc[2:3], d["dw"], sc[14:15])
+            fp8.fp8_linear_wgrad(d["dyq"], sc[8:9], d["xq"], sc[2:3], d["dw"], sc[14:15], rto=True)
             if e: e[1].record()
             e = mark("grad_cast")
             fp8.fp8_scale_cast(d["dw"], fp8.FP8_E5M2, sc[14:15], 0, MU, sc[10:11], sc[11:12], d["gq"])
@@ -341,7 +344,7 @@ class BlockStep:
             self.ev_dgrad[i].record(main)
             self.s_aux.wait_event(e)
             with torch.cuda.stream(self.s_aux):
-                fp8.fp8_linear_wgrad(d["dyq"], sc[8:9], d["xq"], sc[2:3], d["dw"], sc[14:15])
+                fp8.fp8_linear_wgrad(d["dyq"], sc[8:9], d["xq"], sc[2:3], d["dw"], sc[14:15], rto=True)
                 fp8.fp8_scale_cast(d["dw"], fp8.FP8_E5M2, sc[14:15], 0, MU, sc[10:11], sc[11:12], d["gq"])
                 self.s_aux.wait_event(self.ev_dgrad[i])
                 fp8.fp8_adam_step(self.chunks_each[i], step=self.t + 1, margin=0,

@@ -329,6 +329,15 @@ __device__ __forceinline__ void descale1_chunk(const Args &args, uint32_t (&r)[3
   }
 }
 
+// Two floats as bfloat16 rounded to odd: truncate, then set the last bit when
+// any of the 16 discarded bits was set (a NaN whose payload sits in the low
+// bits stays a NaN; +-0 and +-inf are exact).
+__device__ __forceinline__ uint32_t bf16x2_rto(float a, float b) {
+  const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
+  const uint32_t sticky = ((ua & 0xffffu) != 0u ? 1u : 0u) | ((ub & 0xffffu) != 0u ? 0x10000u : 0u);
+  return __byte_perm(ua, ub, 0x7632) | sticky;
+}
+
 // Epilogue of one 32-column chunk: descale, bias, round, store, amax.
 __device__ __forceinline__ uint32_t store_chunk(const Args &args, const uint32_t (&r)[32], int row, int col0,
                                                 float inv_a, float inv_b) {
@@ -354,7 +363,8 @@ __device__ __forceinline__ uint32_t store_chunk(const Args &args, const uint32_t
     }
   } else {
     uint16_t *orow = reinterpret_cast<uint16_t *>(args.out) + (size_t)row * args.cols;
-    const bool bf = args.out_dtype == FP8_DT_BF16;
+    const bool rto = args.out_dtype == FP8_DT_BF16_RTO;
+    const bool bf = args.out_dtype == FP8_DT_BF16 || rto;
 #pragma unroll
     for (int j = 0; j < 32; j += 8) {
       uint32_t p[4];
@@ -363,8 +373,12 @@ __device__ __forceinline__ uint32_t store_chunk(const Args &args, const uint32_t
       for (int t = 0; t < 4; t++) {
         uint32_t lo, hi;
         if (bf) {
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(y[j + 2 * t], y[j + 2 * t + 1]);
-          p[t] = *reinterpret_cast<uint32_t *>(&h2);
+          if (rto) {
+            p[t] = bf16x2_rto(y[j + 2 * t], y[j + 2 * t + 1]);
+          } else {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(y[j + 2 * t], y[j + 2 * t + 1]);
+            p[t] = *reinterpret_cast<uint32_t *>(&h2);
+          }
           lo = (p[t] & 0x7fffu) << 16;
           hi = p[t] & 0x7fff0000u;
         } else {
@@ -757,7 +771,9 @@ constexpr int kWideStageOutBytes = 32 * 128;                             // per 
 constexpr int kWideOutBoxes = 2;  // staging boxes per epilogue warp (stores pipelined)
 constexpr int kWideSmemBytes = kWideStages * kWideStageBytes + 8 * kWideOutBoxes * kWideStageOutBytes + 256 + 1024;
 
-template <bool A_MN, bool B_MN>
+// OUT: the output type (FP8_DT_*), a template argument so that the
+// epilogue's element loop carries no type test.
+template <bool A_MN, bool B_MN, int OUT>
 __global__ void __launch_bounds__(kWideThreads, 1)
     k_gemm3(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmOut, const Args args) {
@@ -919,8 +935,9 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     const bool fold = fabsf(inv_ab) >= 1.17549435e-38f && fabsf(inv_ab) <= 3.402823466e38f;
     const uint32_t stg0 = out_stage0 + (warp - 2) * kWideOutBoxes * kWideStageOutBytes;
     uint32_t box = 0;
-    const bool f32out = args.out_dtype == FP8_DT_F32;
-    const bool bfout = args.out_dtype == FP8_DT_BF16;
+    constexpr bool f32out = OUT == FP8_DT_F32;
+    constexpr bool rtoout = OUT == FP8_DT_BF16_RTO;
+    constexpr bool bfout = OUT == FP8_DT_BF16 || rtoout;
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < args.num_tiles; tile += num_pairs) {
       int mb, nb;
@@ -937,7 +954,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       uint32_t amax16 = 0;  // 16-bit outputs: two packed magnitude maxima
       // accumulator column c of half h holds output column
       //   nb*512 + (c < 128 ? 0 : 256) + h*128 + (c mod 128)
-      const int cols_per_box = f32out ? 32 : 64;
+      constexpr int cols_per_box = f32out ? 32 : 64;
 #pragma unroll 1
       for (int c = 0; c < 256; c += cols_per_box) {
         const int col0 = nb * kWideBN + (c < 128 ? 0 : 256) + h * kPairHalf + (c & 127);
@@ -946,7 +963,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + h * 256 + c, r);
         if (fold) descale1_chunk(args, r, col0, inv_ab); else descale_chunk(args, r, col0, inv_a, inv_b);
         uint32_t w[32];  // the row's 128 bytes as 32 words
-        if (f32out) {
+        if constexpr (f32out) {
           if (last) {
             tc_fence_before();
             __syncwarp();
@@ -971,7 +988,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             const float a0 = __uint_as_float(r[2 * j]), a1 = __uint_as_float(r[2 * j + 1]);
             const float b0 = __uint_as_float(r2[2 * j]), b1 = __uint_as_float(r2[2 * j + 1]);
             uint32_t pa, pb;
-            if (bfout) {
+            if constexpr (rtoout) {
+              pa = bf16x2_rto(a0, a1);
+              pb = bf16x2_rto(b0, b1);
+            } else if constexpr (bfout) {
               __nv_bfloat162 x = __floats2bfloat162_rn(a0, a1), y = __floats2bfloat162_rn(b0, b1);
               pa = *reinterpret_cast<uint32_t *>(&x);
               pb = *reinterpret_cast<uint32_t *>(&y);
@@ -1005,7 +1025,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           bulk_commit();
         }
       }
-      if (!f32out) {
+      if constexpr (!f32out) {
         const uint32_t h16 = max(amax16 & 0xffffu, amax16 >> 16);
         amax_bits = bfout ? (h16 << 16) : absbits_f32(__half2float(__ushort_as_half((unsigned short)h16)));
       }

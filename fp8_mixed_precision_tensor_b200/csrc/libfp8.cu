@@ -52,6 +52,14 @@ template <typename K>
 int set_smem(K kernel, int bytes) {
   return cuda_rc(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
 }
+// The wide kernel is instantiated per output type.
+template <bool A_MN, bool B_MN>
+int set_wide_smem() {
+  return set_smem(gemm::k_gemm3<A_MN, B_MN, FP8_DT_F32>, gemm::kWideSmemBytes) |
+         set_smem(gemm::k_gemm3<A_MN, B_MN, FP8_DT_BF16>, gemm::kWideSmemBytes) |
+         set_smem(gemm::k_gemm3<A_MN, B_MN, FP8_DT_F16>, gemm::kWideSmemBytes) |
+         set_smem(gemm::k_gemm3<A_MN, B_MN, FP8_DT_BF16_RTO>, gemm::kWideSmemBytes);
+}
 
 // One-time per-device set-up: SM count, occupancy, kernel attributes.
 int device_info(DeviceInfo **out) {
@@ -82,9 +90,9 @@ int device_info(DeviceInfo **out) {
     rc |= set_smem(gemm::k_gemm2<false, false>, gemm::kPairSmemBytes);
     rc |= set_smem(gemm::k_gemm2<false, true>, gemm::kPairSmemBytes);
     rc |= set_smem(gemm::k_gemm2<true, true>, gemm::kPairSmemBytes);
-    rc |= set_smem(gemm::k_gemm3<false, false>, gemm::kWideSmemBytes);
-    rc |= set_smem(gemm::k_gemm3<false, true>, gemm::kWideSmemBytes);
-    rc |= set_smem(gemm::k_gemm3<true, true>, gemm::kWideSmemBytes);
+    rc |= set_wide_smem<false, false>();
+    rc |= set_wide_smem<false, true>();
+    rc |= set_wide_smem<true, true>();
     if (rc) return FP8_ERR_CUDA;
     {
       cudaLaunchConfig_t cfg = {};
@@ -104,7 +112,7 @@ int device_info(DeviceInfo **out) {
       d.pair_clusters = clusters;
       cfg.blockDim = dim3(gemm::kWideThreads);
       cfg.dynamicSmemBytes = gemm::kWideSmemBytes;
-      if (cudaOccupancyMaxActiveClusters(&clusters, gemm::k_gemm3<false, false>, &cfg) != cudaSuccess)
+      if (cudaOccupancyMaxActiveClusters(&clusters, gemm::k_gemm3<false, false, FP8_DT_BF16>, &cfg) != cudaSuccess)
         return FP8_ERR_CUDA;
       d.wide_clusters = clusters;
     }
@@ -125,6 +133,7 @@ int device_info(DeviceInfo **out) {
 int launch_rc() { return cuda_rc(cudaGetLastError()); }
 
 bool valid_dtype(int dt) { return dt == FP8_DT_F32 || dt == FP8_DT_BF16 || dt == FP8_DT_F16; }
+bool valid_out_dtype(int dt) { return valid_dtype(dt) || dt == FP8_DT_BF16_RTO; }
 bool valid_fmt(int f) { return f == FP8_E4M3 || f == FP8_E5M2 || f == FP8_F16S; }
 
 unsigned grid_for(size_t work_items, int per_block, int cap) {
@@ -151,7 +160,7 @@ int make_map(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer, ui
 // (32 fp32 or 64 16-bit columns) with the 128-byte swizzle (bulk stores).
 int make_out_map(CUtensorMap *m, void *out, int dtype, uint64_t rows, uint64_t cols) {
   const CUtensorMapDataType t = dtype == FP8_DT_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
-                                : dtype == FP8_DT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                : (dtype == FP8_DT_BF16 || dtype == FP8_DT_BF16_RTO) ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   const uint64_t esz = dtype == FP8_DT_F32 ? 4 : 2;
   cuuint64_t dims[2] = {cols, rows};
@@ -171,7 +180,7 @@ int run_gemm(const uint8_t *A, int fmt_a, const float *inv_a, const uint8_t *B, 
              const float *inv_b, const void *bias, int bias_dtype, void *out, int out_dtype,
              float *out_amax, int rows, int cols, int K, cudaStream_t stream) {
   if (rows < 0 || cols < 0 || K < 0) return FP8_ERR_INVALID_ARG;
-  if (!valid_dtype(out_dtype) || (bias && !valid_dtype(bias_dtype))) return FP8_ERR_INVALID_ARG;
+  if (!valid_out_dtype(out_dtype) || (bias && !valid_dtype(bias_dtype))) return FP8_ERR_INVALID_ARG;
   if (rows == 0 || cols == 0) {  // empty output: operands may be null
     if (out_amax) return cuda_rc(cudaMemsetAsync(out_amax, 0, sizeof(float), stream));
     return FP8_OK;
@@ -244,7 +253,12 @@ int run_gemm(const uint8_t *A, int fmt_a, const float *inv_a, const uint8_t *B, 
     if (variant == 3) {
       CUtensorMap mo;
       if ((rc = make_out_map(&mo, out, out_dtype, (uint64_t)rows, (uint64_t)cols))) return rc;
-      return cuda_rc(cudaLaunchKernelEx(&cfg, gemm::k_gemm3<A_MN, B_MN>, ma, mb, mo, a));
+      switch (out_dtype) {
+        case FP8_DT_F32: return cuda_rc(cudaLaunchKernelEx(&cfg, gemm::k_gemm3<A_MN, B_MN, FP8_DT_F32>, ma, mb, mo, a));
+        case FP8_DT_BF16: return cuda_rc(cudaLaunchKernelEx(&cfg, gemm::k_gemm3<A_MN, B_MN, FP8_DT_BF16>, ma, mb, mo, a));
+        case FP8_DT_F16: return cuda_rc(cudaLaunchKernelEx(&cfg, gemm::k_gemm3<A_MN, B_MN, FP8_DT_F16>, ma, mb, mo, a));
+        default: return cuda_rc(cudaLaunchKernelEx(&cfg, gemm::k_gemm3<A_MN, B_MN, FP8_DT_BF16_RTO>, ma, mb, mo, a));
+      }
     }
     return cuda_rc(cudaLaunchKernelEx(&cfg, gemm::k_gemm2<A_MN, B_MN>, ma, mb, a));
   }

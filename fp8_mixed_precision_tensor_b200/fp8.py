@@ -23,6 +23,7 @@ FP8_OK, FP8_ERR_INVALID_ARG, FP8_ERR_UNALIGNED, FP8_ERR_UNSUPPORTED = 0, 1, 2, 3
 FP8_ERR_CUDA, FP8_ERR_TIMEOUT, FP8_ERR_NONFINITE = 4, 5, 6
 FP8_STATUS_NONFINITE, FP8_STATUS_TIMEOUT, FP8_STATUS_INTERNAL, FP8_STATUS_BAD_MU = 1, 2, 4, 8
 FP8_DT_F32, FP8_DT_BF16, FP8_DT_F16 = 0, 1, 2
+FP8_DT_BF16_RTO = 3  # GEMM outputs only: bfloat16 rounded to odd, for a following FP8 cast
 FP8_E4M3, FP8_E5M2, FP8_F16S = 0, 1, 2
 
 _DT = {torch.float32: FP8_DT_F32, torch.bfloat16: FP8_DT_BF16, torch.float16: FP8_DT_F16}
@@ -181,30 +182,41 @@ def fp8_mu_update(mu: torch.Tensor, clean: torch.Tensor, counts: torch.Tensor, n
 
 
 # ---------------------------------------------------------------- GEMMs
-def fp8_linear_fwd(xq, x_inv, wq, w_inv, y, y_amax=None, bias=None, stream=None) -> None:
+def _out_dt(t, rto: bool) -> int:
+    """Output type code; rto asks a bfloat16 output to be rounded to odd."""
+    if rto:
+        if t.dtype != torch.bfloat16:
+            raise TypeError("a round-to-odd output is bfloat16")
+        return FP8_DT_BF16_RTO
+    return _DT[t.dtype]
+
+
+def fp8_linear_fwd(xq, x_inv, wq, w_inv, y, y_amax=None, bias=None, stream=None, rto=False) -> None:
     """y[M,N] = (xq[M,K] . wq[N,K]^T) * x_inv * w_inv (+ bias)."""
     M, K = xq.shape
     N = wq.shape[0]
     _check(load_library().fp8_linear_fwd(_ptr(xq), _ptr(x_inv), _ptr(wq), _ptr(w_inv), _ptr(bias),
-                                         _DT[bias.dtype] if bias is not None else 0, _ptr(y), _DT[y.dtype],
+                                         _DT[bias.dtype] if bias is not None else 0, _ptr(y), _out_dt(y, rto),
                                          _ptr(y_amax), M, N, K, _stream(stream)), "fp8_linear_fwd")
 
 
-def fp8_linear_dgrad(dyq, dy_inv, wq, w_inv, dx, dx_amax=None, stream=None) -> None:
+def fp8_linear_dgrad(dyq, dy_inv, wq, w_inv, dx, dx_amax=None, stream=None, rto=False) -> None:
     """dx[M,K] = (dyq[M,N] . wq[N,K]) * dy_inv * w_inv."""
     M, N = dyq.shape
     K = wq.shape[1]
     _check(load_library().fp8_linear_dgrad(_ptr(dyq), _ptr(dy_inv), _ptr(wq), _ptr(w_inv), _ptr(dx),
-                                           _DT[dx.dtype], _ptr(dx_amax), M, N, K, _stream(stream)),
+                                           _out_dt(dx, rto), _ptr(dx_amax), M, N, K, _stream(stream)),
            "fp8_linear_dgrad")
 
 
-def fp8_linear_wgrad(dyq, dy_inv, xq, x_inv, dw, dw_amax=None, stream=None) -> None:
-    """dw[N,K] = (dyq[M,N]^T . xq[M,K]) * dy_inv * x_inv."""
+def fp8_linear_wgrad(dyq, dy_inv, xq, x_inv, dw, dw_amax=None, stream=None, rto=False) -> None:
+    """dw[N,K] = (dyq[M,N]^T . xq[M,K]) * dy_inv * x_inv.  rto: a bfloat16 dw
+    rounded to odd, the form whose FP8 gradient cast gives exactly the codes
+    and scale of the float32 dw's (half the bytes written and read)."""
     M, N = dyq.shape
     K = xq.shape[1]
     _check(load_library().fp8_linear_wgrad(_ptr(dyq), _ptr(dy_inv), _ptr(xq), _ptr(x_inv), _ptr(dw),
-                                           _DT[dw.dtype], _ptr(dw_amax), M, N, K, _stream(stream)),
+                                           _out_dt(dw, rto), _ptr(dw_amax), M, N, K, _stream(stream)),
            "fp8_linear_wgrad")
 
 

@@ -59,6 +59,17 @@ extern "C" {
 #define FP8_DT_F32 0
 #define FP8_DT_BF16 1
 #define FP8_DT_F16 2
+/* GEMM outputs only: bfloat16 rounded to odd (truncated, the last bit set
+ * when any discarded bit was set).  An intermediate for a following FP8 cast:
+ * bfloat16 keeps 8 significant bits, at least 2 more than E4M3 (4) or E5M2
+ * (3) at any scaled magnitude, so rounding to nearest even from the
+ * round-to-odd value gives the code the cast of the float32 result would
+ * give (round-to-odd is innocuous before a rounding that keeps 2 or more
+ * fewer bits), and every power-of-two scale threshold is a bfloat16 value
+ * that round-to-odd never crosses, so the amax of the stored values yields
+ * the scale of the float32 amax.  Read back as FP8_DT_BF16 (the gradient
+ * cast reads 2 instead of 4 bytes per element). */
+#define FP8_DT_BF16_RTO 3
 
 /* ---- storage formats ---------------------------------------------------
  * FP8_E4M3: OCP E4M3, max 448, no infinities (weights, activations, Adam m1).
@@ -221,7 +232,8 @@ int fp8_mu_update(float *mu_dev, int *clean_dev, unsigned long long *counts_dev,
  * of the output *as stored* (overwritten, not accumulated).
  * Shape rule: M, N, K must each be a multiple of 16 (TMA row pitch);
  * otherwise FP8_ERR_UNSUPPORTED.  M == 0 or N == 0 is a no-op that writes an
- * amax of 0.  Output types: FP8_DT_F32, FP8_DT_BF16, FP8_DT_F16.
+ * amax of 0.  Output types: FP8_DT_F32, FP8_DT_BF16, FP8_DT_F16 and
+ * FP8_DT_BF16_RTO (bias types: the first three).
  * A mis-tiled pipeline cannot hang: every wait is bounded, and a wait that
  * runs out sets FP8_STATUS_TIMEOUT and the kernel returns.
  */

@@ -1,6 +1,6 @@
 """Run one kernel family of the hot path on a chosen case (for profilers).
 
-    python profile_cases.py linear --M 4096 --N 16384 --K 4096
+    python profile_cases.py linear --M 4096 --N 16384 --K 4096 [--rto]
     python profile_cases.py cast --n 268435456
     python profile_cases.py castsweep
     python profile_cases.py adam --n 67108864 [--track]
@@ -46,7 +46,8 @@ def case_linear(a):
     xq, wq, dyq = torch.empty((M, K), **u8), torch.empty((N, K), **u8), torch.empty((M, N), **u8)
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     dx = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
-    dw = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    # --rto: dW as bfloat16 rounded to odd (the bench step's form), else float32
+    dw = torch.empty((N, K), dtype=torch.bfloat16 if a.rto else torch.float32, device="cuda")
     sc = _scalars(16)
 
     def one():
@@ -55,13 +56,13 @@ def case_linear(a):
             fp8.fp8_scale_cast(t, fmt, sc[i:i + 1], 0, 1.0, sc[i + 1:i + 2], sc[i + 2:i + 3], q)
         fp8.fp8_linear_fwd(xq, sc[2:3], wq, sc[5:6], y, sc[12:13])
         fp8.fp8_linear_dgrad(dyq, sc[8:9], wq, sc[5:6], dx, sc[13:14])
-        fp8.fp8_linear_wgrad(dyq, sc[8:9], xq, sc[2:3], dw, sc[14:15])
+        fp8.fp8_linear_wgrad(dyq, sc[8:9], xq, sc[2:3], dw, sc[14:15], rto=a.rto)
 
     one()
     flops = 2.0 * M * N * K
     for name, fn in (("fwd", lambda: fp8.fp8_linear_fwd(xq, sc[2:3], wq, sc[5:6], y, sc[12:13])),
                      ("dgrad", lambda: fp8.fp8_linear_dgrad(dyq, sc[8:9], wq, sc[5:6], dx, sc[13:14])),
-                     ("wgrad", lambda: fp8.fp8_linear_wgrad(dyq, sc[8:9], xq, sc[2:3], dw, sc[14:15]))):
+                     ("wgrad", lambda: fp8.fp8_linear_wgrad(dyq, sc[8:9], xq, sc[2:3], dw, sc[14:15], rto=a.rto))):
         t = _timed(fn, max(a.iters, 3))
         print(f"  {name:5s} M{M} N{N} K{K}: {t:.4f} ms, {flops / t / 1e9:.1f} TFLOP/s")
     return one
@@ -257,6 +258,7 @@ def main():
     ap.add_argument("--world", type=int, default=8, help="allreduce: emulated ranks")
     ap.add_argument("--track", action="store_true", help="adam: track the master amax across steps")
     ap.add_argument("--copy", action="store_true", help="adam7b: write the E4M3 weight copy")
+    ap.add_argument("--rto", action="store_true", help="linear: dW as bfloat16 rounded to odd")
     a = ap.parse_args()
     one = {"linear": case_linear, "cast": case_cast, "castsweep": case_castsweep, "adam": case_adam,
            "allreduce": case_allreduce,

@@ -312,6 +312,40 @@ def test_linear_fwd_bias_f16_out():
         assert ya.item() == float(np.max(np.abs(got)))
 
 
+@pytest.mark.parametrize("shape", [(256, 256, 256), (272, 400, 208), (1024, 768, 4096), (1024, 16384, 2048)])
+def test_wgrad_round_to_odd_output_feeds_the_same_gradient_codes(shape):
+    """The bfloat16 round-to-odd wgrad output (FP8_DT_BF16_RTO) is, bit for
+    bit, the round-to-odd image of the same kernel's float32 output (the
+    accumulation does not change with the output type), its fused amax is the
+    amax of the stored values, and the E5M2 gradient cast of it -- scale,
+    codes and under/overflow counts -- equals the cast of the float32 output.
+    The shapes run the one-CTA, pair and wide kernels."""
+    M, N, K = shape
+    q = quantised_linear(M, N, K, ("rto", M, N, K))
+    (dyq, dy_inv), (xq, x_inv) = q["dy"], q["x"]
+    dw32, a32 = torch.empty((N, K), **F32), scalar()
+    fp8.fp8_linear_wgrad(dyq, dy_inv, xq, x_inv, dw32, a32)
+    dwb, ab = torch.empty((N, K), dtype=torch.bfloat16, device="cuda"), scalar()
+    fp8.fp8_linear_wgrad(dyq, dy_inv, xq, x_inv, dwb, ab, rto=True)
+    u = dw32.cpu().numpy().view(np.uint32)
+    want = (u >> 16).astype(np.uint16) | ((u & 0xFFFF) != 0).astype(np.uint16)
+    got = dwb.cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, want)
+    stored = (got.astype(np.uint32) << 16).view(np.float32)
+    assert ab.item() == float(np.max(np.abs(stored)))
+    mu = torch.full((1,), 2.0 ** 10, **F32)
+    res = []
+    for g, a in ((dw32, a32), (dwb, ab)):
+        S, inv, counts = scalar(), scalar(), torch.zeros(2, dtype=torch.int64, device="cuda")
+        codes = torch.empty((N, K), dtype=torch.uint8, device="cuda")
+        fp8.fp8_grad_cast(g, fp8.FP8_E5M2, a, 0, mu, S, inv, codes, counts)
+        res.append((S.item(), codes.cpu().numpy(), tuple(counts.tolist())))
+    assert res[0][0] == res[1][0] and res[0][2] == res[1][2]
+    assert np.array_equal(res[0][1], res[1][1])
+    with pytest.raises(TypeError):  # a round-to-odd output is bfloat16
+        fp8.fp8_linear_wgrad(dyq, dy_inv, xq, x_inv, dw32, a32, rto=True)
+
+
 def test_gemm_exact_integer_operands():
     """Codes for +-1, +-2 only: every partial sum is an exact integer, so the
     FP32 accumulation must equal the oracle exactly."""
