@@ -73,7 +73,14 @@ GRAD_CAST_BYTES = 2 + 1       # round-to-odd bf16 dW read (amax fused in the GEM
 ADAM_BYTES = 11               # read g1 m1 v2 w2, write m1 v2 w2
 
 
-def config_of(wl: dict, schedule: str, world: int) -> dict:
+ADAM_MODES = {
+    "into": "out of place into a second set of state buffers (one pass over the state while the scales "
+            "hold, a second for the chunks whose scales change)",
+    "in_place": "in place (a stats pass, then the update pass)",
+}
+
+
+def config_of(wl: dict, schedule: str, world: int, adam: str = "into") -> dict:
     """The `config` object of the JSON line (the same for both arms)."""
     flops = sum(3 * 2 * wl["tokens"] * N * K for _, K, N in wl["linears"])
     return {"workload": wl["workload"], "tokens": wl["tokens"], "hidden": wl["hidden"],
@@ -81,6 +88,7 @@ def config_of(wl: dict, schedule: str, world: int) -> dict:
             "gemm_flops_per_step": flops, "l2": "inputs larger than L2 (no flush)", "schedule": schedule,
             "weight_operand": "E4M3 copy written by the previous Adam step", "master_amax": "tracked",
             "weight_gradient": "bf16 rounded to odd (its E5M2 cast equals the float32 dW's)",
+            "adam_step": ADAM_MODES[adam],
             "parallelism": f"replicas{world}" if world > 1 else "single"}
 
 
@@ -198,7 +206,7 @@ class BlockStep:
     FP16 masters (the Adam state) and the first E4M3 weight operands; from
     then on each step's Adam writes the next step's E4M3 weights."""
 
-    def __init__(self, device, seed: int = 0, workload: str = "gpt175b_block"):
+    def __init__(self, device, seed: int = 0, workload: str = "gpt175b_block", adam: str = "into"):
         from fp8_mixed_precision_tensor_b200 import fp8
 
         wl = WORKLOADS[workload]
@@ -229,6 +237,8 @@ class BlockStep:
             d["m"] = torch.zeros((N, K), **u8)
             d["v"] = torch.zeros((N, K), dtype=torch.int16, device=device)
             d["wh"] = torch.empty((N, K), dtype=torch.int16, device=device)
+            if adam == "into":  # the out-of-place step's second state buffers
+                d["m2"], d["v2"], d["wh2"] = (torch.empty_like(d[k]) for k in ("m", "v", "wh"))
             d["st"] = torch.ones(4, **f32)  # m_scale, v_scale, w_scale, tracked master amax
             d["st"][3] = -1.0
             W = synth.device_normal((N, K), wl["w_std"], seed * 1000 + 10 * li + 2, torch.bfloat16, device)
@@ -238,23 +248,49 @@ class BlockStep:
             self.quantise(W, fp8.FP8_E4M3, d["sc"], 3, out=d["wq"])
             del W
             self.L.append(d)
-        self.chunk_list = [fp8.AdamChunk(d["gq"], d["sc"][11:12], d["m"], d["st"][0:1], d["v"], d["st"][1:2],
-                                         d["wh"], d["st"][2:3], d["st"][3:4], d["wq"], d["sc"][4:5], d["sc"][5:6])
-                           for d in self.L]
-        self.chunks = fp8.pack_adam_chunks(self.chunk_list)
+        # Adam's chunk arrays: in place one set; out of place, step t reads the
+        # state buffers of parity t % 2 (0: m, v, wh; 1: m2, v2, wh2) and writes
+        # the other set
+        self.adam = adam
+        sets = (("m", "v", "wh"), ("m2", "v2", "wh2")) if adam == "into" else (("m", "v", "wh"),)
+
+        def chunk(d, k):
+            m, v, w = (d[x] for x in sets[k])
+            return fp8.AdamChunk(d["gq"], d["sc"][11:12], m, d["st"][0:1], v, d["st"][1:2], w, d["st"][2:3],
+                                 d["st"][3:4], d["wq"], d["sc"][4:5], d["sc"][5:6])
+
+        def dest(d, k):
+            return tuple(d[x] for x in sets[1 - k])
+
+        self.packs, self.packs_each = [], []
+        for k in range(len(sets)):
+            self.packs.append((fp8.pack_adam_chunks([chunk(d, k) for d in self.L]),
+                               fp8.pack_adam_dests([dest(d, k) for d in self.L]) if adam == "into" else None))
+            # one Adam call per tensor (overlapped schedule)
+            self.packs_each.append([(fp8.pack_adam_chunks([chunk(d, k)]),
+                                     fp8.pack_adam_dests([dest(d, k)]) if adam == "into" else None)
+                                    for d in self.L])
         self.ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(self.L)) // 4 + 64, **f32)
-        # one Adam call per tensor (overlapped schedule): own chunk array and a
-        # 256-byte-aligned workspace slice each
-        self.chunks_each = [fp8.pack_adam_chunks([c]) for c in self.chunk_list]
+        # a 256-byte-aligned workspace slice per tensor for the per-tensor calls
         self.ws_each = torch.zeros(64 * len(self.L), **f32)
         self.t = 0
         self.flops = sum(3 * 2 * d["M"] * d["N"] * d["K"] for d in self.L)
         self.cast_elems = sum(d["M"] * d["K"] + d["M"] * d["N"] for d in self.L)
         self.params = sum(d["N"] * d["K"] for d in self.L)
-        # per linear: (amax, scale+cast) x2, 3 GEMMs, grad scale+cast; Adam with a tracked
-        # master: stats, finalize 1, exact-master pass, finalize 2, update, finalize 3
-        self.launches_per_step = 4 * (2 * 2 + 3 + 1) + 6
-        self.launches_per_step_overlapped = 4 * (2 * 2 + 3 + 1 + 6)
+        # per linear: (amax, scale+cast) x2, 3 GEMMs, grad scale+cast; Adam out of
+        # place: update, finalize, redo, finalize; in place with a tracked master:
+        # stats, finalize 1, exact-master pass, finalize 2, update, finalize 3
+        na = 4 if adam == "into" else 6
+        self.launches_per_step = 4 * (2 * 2 + 3 + 1) + na
+        self.launches_per_step_overlapped = 4 * (2 * 2 + 3 + 1 + na)
+
+    def adam_step(self, pack, t, ws):
+        """Adam step t over the tensors of one packed (chunks, dests) pair."""
+        chunks, dests = pack
+        if self.adam == "into":
+            self.fp8.fp8_adam_step_into(chunks, dests, step=t, margin=0, workspace=ws, **HP)
+        else:
+            self.fp8.fp8_adam_step(chunks, step=t, margin=0, workspace=ws, **HP)
 
     def quantise(self, x, fmt, sc, i, mu=1.0, out=None):
         fp8 = self.fp8
@@ -295,7 +331,7 @@ class BlockStep:
         self.t += 1
         nvtx.range_push("adam")
         e = mark("adam")
-        fp8.fp8_adam_step(self.chunks, step=self.t, margin=0, workspace=self.ws, **HP)
+        self.adam_step(self.packs[(self.t - 1) % len(self.packs)], self.t, self.ws)
         if e: e[1].record()
         nvtx.range_pop()
 
@@ -347,8 +383,8 @@ class BlockStep:
                 fp8.fp8_linear_wgrad(d["dyq"], sc[8:9], d["xq"], sc[2:3], d["dw"], sc[14:15], rto=True)
                 fp8.fp8_scale_cast(d["dw"], fp8.FP8_E5M2, sc[14:15], 0, MU, sc[10:11], sc[11:12], d["gq"])
                 self.s_aux.wait_event(self.ev_dgrad[i])
-                fp8.fp8_adam_step(self.chunks_each[i], step=self.t + 1, margin=0,
-                                  workspace=self.ws_each[64 * i:64 * (i + 1)], **HP)
+                self.adam_step(self.packs_each[self.t % len(self.packs_each)][i], self.t + 1,
+                               self.ws_each[64 * i:64 * (i + 1)])
         self.ev_grad.record(self.s_aux)
         main.wait_event(self.ev_grad)
         self.t += 1
@@ -450,7 +486,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     wl = WORKLOADS[args.workload]
-    cfg = config_of(wl, args.schedule, args.gpus)
+    cfg = config_of(wl, args.schedule, args.gpus, args.adam)
     sample = OracleSample(wl)
     t_s, t_f = [], []
     for i in range(args.warmup + args.steps):
@@ -494,7 +530,7 @@ def run_gpu(args):
 
     peaks = load_peaks()
     wl = WORKLOADS[args.workload]
-    runner = BlockStep(dev, seed=rank, workload=args.workload)
+    runner = BlockStep(dev, seed=rank, workload=args.workload, adam=args.adam)
     overlap = args.schedule == "overlap"
     for _ in range(args.warmup):
         runner.step_overlapped() if overlap else runner.step()
@@ -604,7 +640,7 @@ def run_gpu(args):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp8(e4m3/e5m2)->f32 accum; f32 elementwise", "data": "synthetic",
-        "config": config_of(wl, args.schedule, world),
+        "config": config_of(wl, args.schedule, world, args.adam),
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": gemm_tflops / peak, "traffic": gemm_traffic(wl["workload"]),
                      "kernel": "k_gemm3 (fwd+dgrad+wgrad; achieved = GEMM flops per step / summed GEMM "
@@ -617,8 +653,11 @@ def run_gpu(args):
             "grad_cast": {"ms": t_gcast, "GB/s": gcast_gbs, "frac_hbm": gcast_gbs / peaks["hbm"]},
             "adam": {"ms": t_adam, "GB/s": adam_gbs, "frac_hbm": adam_gbs / peaks["hbm"],
                      "bytes_per_param_algorithmic": ADAM_BYTES,
-                     "bytes_per_param_moved": "15 (stats pass 4 with the tracked master + update 11) "
-                                              "+ 1 for the E4M3 weight copy"},
+                     "bytes_per_param_moved": ("11 (one pass while the scales hold; 22 for a chunk whose "
+                                               "scales change) + 1 for the E4M3 weight copy"
+                                               if args.adam == "into" else
+                                               "15 (stats pass 4 with the tracked master + update 11) "
+                                               "+ 1 for the E4M3 weight copy")},
             "hbm_peak_gbs": peaks["hbm"],
         },
         "e2e": {"value": runner.flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
@@ -652,6 +691,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--schedule", default="overlap", choices=["overlap", "serial"],
                     help="overlap: casts / GEMMs / wgrad on three streams; serial: one stream")
+    ap.add_argument("--adam", default="into", choices=sorted(ADAM_MODES),
+                    help="into: out-of-place Adam step (two state buffers); in_place: stats + update passes")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

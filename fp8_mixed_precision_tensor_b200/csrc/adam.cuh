@@ -29,6 +29,19 @@
 // workspace MAX-reduced over ranks in between) computes the exact new amaxes
 // in pass 1 instead: an interval decision there would need a second
 // reduction for the flagged chunks.
+// The out-of-place step (new state into separate buffers, the inputs left
+// as they were) needs no stats pass: it predicts that every new scale equals
+// the old one and
+//   pass 6 (update):  decodes, updates and encodes with the predicted scales
+//                     into the new buffers while reducing the exact amax|m|,
+//                     amax v and amax|w| of the new values;
+//   finalize 6:       the scales those amaxes give; a chunk whose prediction
+//                     was wrong is flagged;
+//   pass 7 (redo):    the update again, flagged chunks only, from the
+//                     unchanged inputs with the right scales;
+//   finalize 7:       tracked amax of the redone chunks.
+// One pass of 6 B read and 5-6 B written per parameter when the scales hold,
+// the same results as the in-place step in every case.
 // All chunks of one call share each launch: the chunk table travels in the
 // kernel parameters and tiles of 4096 parameters are mapped to chunks by a
 // binary search over the chunks' first-tile indices.
@@ -41,7 +54,8 @@ namespace fp8lib {
 constexpr int kAdamThreads = 256;
 constexpr int kAdamPerThread = 16;
 constexpr int kAdamTile = kAdamThreads * kAdamPerThread;  // parameters per tile
-constexpr int kAdamMaxChunksPerLaunch = 256;
+// the chunk table travels in the kernel parameters (at most 32,764 bytes)
+constexpr int kAdamMaxChunksPerLaunch = 224;
 constexpr int kAdamWsFloatsPerChunk = 16;  // workspace slots per chunk (64 bytes)
 
 // Workspace slots of one chunk (float bits; amax slots are max-reduced as
@@ -58,8 +72,9 @@ enum : int {
   WS_APPROX_W = 14,    // estimate of amax|w| of the new master (pass 1, estimated step)
 };
 // WS_FLAGS bits: the exact master pass must run; the chunk tracks its master
-// amax; the master's scale was decided in finalize 1.
-enum : uint32_t { FLAG_EXACT = 1u, FLAG_TRACKED = 2u, FLAG_KNOWN = 4u };
+// amax; the master's scale was decided in finalize 1; the out-of-place
+// step's predicted scales were wrong and the chunk is updated again.
+enum : uint32_t { FLAG_EXACT = 1u, FLAG_TRACKED = 2u, FLAG_KNOWN = 4u, FLAG_REDO = 8u };
 
 struct AdamChunkDev {
   const uint8_t *g;
@@ -73,6 +88,9 @@ struct AdamChunkDev {
   float *w_amax;  // optional tracked amax of the stored master
   uint8_t *wq;    // optional E4M3 copy of the new master
   float *wq_scale, *wq_inv;
+  uint8_t *m_out;    // where the update writes the new state: m, v, w
+  uint16_t *v_out;   // themselves (in place) or the out-of-place step's
+  uint16_t *w_out;   // new buffers
   unsigned long long n;
   unsigned long long tile_begin;
 };
@@ -88,6 +106,7 @@ struct AdamLaunch {
   int estimate;      // 1: untracked chunks take the estimated stats pass (PASS 5)
   float *ws;         // kAdamWsFloatsPerChunk floats per chunk of this launch
 };
+static_assert(sizeof(AdamLaunch) <= 32764, "kernel parameters are limited to 32,764 bytes");
 
 // Per-chunk constants of the update: the descales are folded into the Adam
 // coefficients, m = (b1/s_m) m~ + ((1-b1)/(mu s_g)) g~ and
@@ -233,7 +252,9 @@ struct AdamNewScales {
 // arguments (no per-parameter test in the element loop); the update pass,
 // whose extra live values would cost a resident block per SM as separate
 // instantiations, takes them at run time (TRACK = WQ = true, track_rt and
-// wq_rt the chunk's flags).
+// wq_rt the chunk's flags).  The update passes (2 in place; 6 and 7 out of
+// place, which also reduce the exact amaxes of the new m and v) write the
+// new state through m_out, v_out, w_out.
 template <int PASS, bool TRACK, bool WQ>
 __device__ __forceinline__ void adam_group(const AdamLaunch &L, const AdamChunkDev &C, size_t grp,
                                            const AdamScalars &sc, const AdamNewScales &ns, float &am, float &av,
@@ -276,7 +297,11 @@ __device__ __forceinline__ void adam_group(const AdamLaunch &L, const AdamChunkD
       aw = max_abs2(aw, adam_master(h2f2(ww[p]), d, sc));
     } else {
       const float2 w = adam_master(h2f2(ww[p]), d, sc);
-      aw = max_abs2(aw, w);  // the exact new amax: checks the scale finalize 1 decided
+      aw = max_abs2(aw, w);  // the exact new amax: checks the decided or the predicted scale
+      if constexpr (PASS != 2) {
+        am = max_abs2(am, m);
+        av = max_abs2(av, v);
+      }
       const float2 ms = __fmul2_rn(m, ns.m), vs = __fmul2_rn(v, ns.v), ws = __fmul2_rn(w, ns.w);
       const uint32_t mc = enc2<FP8_E4M3>(ms.x, ms.y);
       if (p & 1) mo[p >> 1] |= mc << 16; else mo[p >> 1] = mc;
@@ -284,7 +309,9 @@ __device__ __forceinline__ void adam_group(const AdamLaunch &L, const AdamChunkD
       wo[p] = f16x2(ws.x, ws.y);
       if (track || wq) {
         const float2 st = h2f2(wo[p]);  // the stored master (scaled)
-        if (track) am = max_abs2(am, st);
+        if (track) {
+          if constexpr (PASS == 2) am = max_abs2(am, st); else au = max_abs2(au, st);
+        }
         if (wq) {
           // E4M3 copy of the stored master: h * (s_q / s_w), exact in f32
           const float2 qs = __fmul2_rn(st, ns.q);
@@ -294,12 +321,12 @@ __device__ __forceinline__ void adam_group(const AdamLaunch &L, const AdamChunkD
       }
     }
   }
-  if constexpr (PASS == 2) {
-    __stcs(reinterpret_cast<uint4 *>(C.m) + grp, make_uint4(mo[0], mo[1], mo[2], mo[3]));
-    __stcs(reinterpret_cast<uint4 *>(C.v) + 2 * grp, make_uint4(vo[0], vo[1], vo[2], vo[3]));
-    __stcs(reinterpret_cast<uint4 *>(C.v) + 2 * grp + 1, make_uint4(vo[4], vo[5], vo[6], vo[7]));
-    __stcs(reinterpret_cast<uint4 *>(C.w) + 2 * grp, make_uint4(wo[0], wo[1], wo[2], wo[3]));
-    __stcs(reinterpret_cast<uint4 *>(C.w) + 2 * grp + 1, make_uint4(wo[4], wo[5], wo[6], wo[7]));
+  if constexpr (PASS == 2 || PASS == 6 || PASS == 7) {
+    __stcs(reinterpret_cast<uint4 *>(C.m_out) + grp, make_uint4(mo[0], mo[1], mo[2], mo[3]));
+    __stcs(reinterpret_cast<uint4 *>(C.v_out) + 2 * grp, make_uint4(vo[0], vo[1], vo[2], vo[3]));
+    __stcs(reinterpret_cast<uint4 *>(C.v_out) + 2 * grp + 1, make_uint4(vo[4], vo[5], vo[6], vo[7]));
+    __stcs(reinterpret_cast<uint4 *>(C.w_out) + 2 * grp, make_uint4(wo[0], wo[1], wo[2], wo[3]));
+    __stcs(reinterpret_cast<uint4 *>(C.w_out) + 2 * grp + 1, make_uint4(wo[4], wo[5], wo[6], wo[7]));
     if (wq) __stcs(reinterpret_cast<uint4 *>(C.wq) + grp, make_uint4(qo[0], qo[1], qo[2], qo[3]));
   }
 }
@@ -328,6 +355,11 @@ __device__ __forceinline__ void adam_chunk_flush(const AdamLaunch &L, AdamChunkS
   if constexpr (PASS == 3)
     if (S.active) flush_max3(L, S.cur, WS_AMAX_W, S.aw, WS_AMAX_W, S.aw, WS_AMAX_W, S.aw);
   if constexpr (PASS == 2) flush_max3(L, S.cur, WS_STORED_W, S.am, WS_CHECK_W, S.aw, WS_CHECK_W, S.aw);
+  if constexpr (PASS == 6 || PASS == 7)
+    if (S.active) {
+      flush_max3(L, S.cur, WS_AMAX_M, S.am, WS_AMAX_V, S.av, WS_CHECK_W, S.aw);
+      if (S.tracked) flush_max3(L, S.cur, WS_STORED_W, S.au, WS_STORED_W, S.au, WS_STORED_W, S.au);
+    }
   S.am = S.av = S.aw = S.au = 0.f;
 }
 
@@ -340,12 +372,24 @@ __device__ __forceinline__ void adam_chunk_enter(const AdamLaunch &L, int ci, Ad
     S.tracked = C.w_amax != nullptr && *C.w_amax >= 0.0f;
     S.active = S.tracked == (PASS == 4);
     S.sc = adam_scalars(L, *C.g_inv, 1.0f / *C.m_scale, 1.0f / *C.v_scale, 1.0f / *C.w_scale);
+  } else if constexpr (PASS == 6) {
+    // the predicted new scales are the old ones (the same expressions as the
+    // in-place step's, so a prediction that holds gives its exact results)
+    S.tracked = C.w_amax != nullptr;
+    S.active = true;
+    const float sm = *C.m_scale, sv = *C.v_scale, sw = *C.w_scale;
+    S.sc = adam_scalars(L, *C.g_inv, 1.0f / sm, 1.0f / sv, 1.0f / sw);
+    S.ns.m = both(sm);
+    S.ns.v = both(sv);
+    S.ns.w = both(sw);
+    S.want_wq = C.wq != nullptr;
+    S.ns.q = both(S.want_wq ? __fmul_rn(*C.wq_scale, 1.0f / sw) : 1.0f);
   } else {
     const uint32_t fl = ws_flags(L, ci);
-    // pass 2: keep the stored-master amax (and its check) for every chunk
-    // that tracks it, including the step that first establishes it
-    S.tracked = PASS == 2 ? C.w_amax != nullptr : (fl & FLAG_TRACKED) != 0;
-    S.active = PASS == 2 || (fl & FLAG_EXACT) != 0;
+    // passes 2 and 7: keep the stored-master amax (and its check) for every
+    // chunk that tracks it, including the step that first establishes it
+    S.tracked = PASS == 3 ? (fl & FLAG_TRACKED) != 0 : C.w_amax != nullptr;
+    S.active = PASS == 2 || (fl & (PASS == 7 ? FLAG_REDO : FLAG_EXACT)) != 0;
     S.sc = adam_scalars(L, *C.g_inv, ws_get(L, ci, WS_OLDINV_M), ws_get(L, ci, WS_OLDINV_V),
                         ws_get(L, ci, WS_OLDINV_W));
     S.ns.m = both(ws_get(L, ci, WS_NEW_M));
@@ -387,12 +431,18 @@ __device__ __forceinline__ void adam_tail(const AdamLaunch &L, const AdamChunkDe
     } else {
       const float w = adam_master(wd, d, sc).x;
       S.aw = max_abs1(S.aw, w);
-      C.m[i] = (uint8_t)(enc2<FP8_E4M3>(__fmul_rn(m.x, ns.m.x), 0.0f) & 0xffu);
-      C.v[i] = __half_as_ushort(__float2half_rn(__fmul_rn(v.x, ns.v.x)));
+      if constexpr (PASS != 2) {
+        S.am = max_abs1(S.am, m.x);
+        S.av = max_abs1(S.av, v.x);
+      }
+      C.m_out[i] = (uint8_t)(enc2<FP8_E4M3>(__fmul_rn(m.x, ns.m.x), 0.0f) & 0xffu);
+      C.v_out[i] = __half_as_ushort(__float2half_rn(__fmul_rn(v.x, ns.v.x)));
       const __half h = __float2half_rn(__fmul_rn(w, ns.w.x));
-      C.w[i] = __half_as_ushort(h);
+      C.w_out[i] = __half_as_ushort(h);
       const float st = __half2float(h);
-      if (S.tracked) S.am = max_abs1(S.am, st);
+      if (S.tracked) {
+        if constexpr (PASS == 2) S.am = max_abs1(S.am, st); else S.au = max_abs1(S.au, st);
+      }
       if (S.want_wq)
         C.wq[i] = (uint8_t)(enc2<FP8_E4M3>(__fmul_rn(st, ns.q.x), 0.0f) & 0xffu);
     }
@@ -403,7 +453,9 @@ __device__ __forceinline__ void adam_tail(const AdamLaunch &L, const AdamChunkDe
 // not track their master amax (exact amaxes of m and v, the estimate A~ and
 // the step bound U).  PASS 1: the same chunks' exact new amaxes (the phased
 // step).  PASS 4: stats of the chunks that track it (amaxes of m and v, U).
-// PASS 3: exact master amax of flagged chunks.  PASS 2: update.  The stats
+// PASS 3: exact master amax of flagged chunks.  PASS 2: update.  PASS 6:
+// out-of-place update with the predicted scales.  PASS 7: its redo of the
+// flagged chunks.  The stats
 // passes are separate kernels so that the estimated arithmetic does not
 // carry the register count of the exact one.
 template <int PASS>
@@ -416,7 +468,7 @@ __device__ __forceinline__ void adam_pass(const AdamLaunch &L) {
       if (S.cur >= 0) adam_chunk_flush<PASS>(L, S);
       adam_chunk_enter<PASS>(L, ci, S);
     }
-    if (!S.active) {  // pass 1b: chunk not flagged; stats: the other stats pass's chunk
+    if (!S.active) {  // passes 1b and 7: chunk not flagged; stats: the other stats pass's chunk
       // jump to this block's last tile inside the chunk; the loop step leaves it
       const unsigned long long end = C.tile_begin + (C.n + kAdamTile - 1) / kAdamTile;
       tile += ((end - tile - 1) / gridDim.x) * gridDim.x;
@@ -435,8 +487,8 @@ __device__ __forceinline__ void adam_pass(const AdamLaunch &L) {
         adam_group<1, false, false>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw, S.au);
       } else if constexpr (PASS == 3) {
         adam_group<3, false, false>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw, S.au);
-      } else {
-        adam_group<2, true, true>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw, S.au, S.tracked, S.want_wq);
+      } else {  // an update pass: 2, 6 or 7
+        adam_group<PASS, true, true>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw, S.au, S.tracked, S.want_wq);
       }
     } else {
       adam_tail<PASS>(L, C, base, S);
@@ -459,6 +511,18 @@ __global__ void __launch_bounds__(kAdamThreads) k_adam(const __grid_constant__ A
 template <>
 __global__ void __launch_bounds__(kAdamThreads, 5) k_adam<2>(const __grid_constant__ AdamLaunch L) {
   adam_pass<2>(L);
+}
+// The out-of-place update and its redo: 64 registers and four resident
+// blocks per SM.  (Held to five blocks' 48 registers they spilled ~100 bytes
+// per thread and moved 4.2-4.4 TB/s at 2^26-2^28 parameters instead of
+// 4.8-5.1.)
+template <>
+__global__ void __launch_bounds__(kAdamThreads, 4) k_adam<6>(const __grid_constant__ AdamLaunch L) {
+  adam_pass<6>(L);
+}
+template <>
+__global__ void __launch_bounds__(kAdamThreads, 4) k_adam<7>(const __grid_constant__ AdamLaunch L) {
+  adam_pass<7>(L);
 }
 // The estimated stats passes: six resident blocks per SM.
 template <>
@@ -500,7 +564,8 @@ __device__ __forceinline__ bool interval_scales(const AdamLaunch &L, const AdamC
 
 // STAGE 1: after the stats passes.  STAGE 2: after pass 1b.  STAGE 3: after
 // pass 2.  STAGE 12: stages 1 and 2 in one launch (the phased step: every
-// chunk's exact amaxes came from pass 1, so nothing is flagged).
+// chunk's exact amaxes came from pass 1, so nothing is flagged).  STAGE 6:
+// after the out-of-place pass 6.  STAGE 7: after its redo pass 7.
 template <int STAGE>
 __global__ void k_adam_finalize(const __grid_constant__ AdamLaunch L) {
   for (int ci = threadIdx.x; ci < L.nchunks; ci += blockDim.x) {
@@ -564,6 +629,41 @@ __global__ void k_adam_finalize(const __grid_constant__ AdamLaunch L) {
         *C.wq_scale = ws[WS_NEW_WQ];
         *C.wq_inv = 1.0f / ws[WS_NEW_WQ];
       }
+    }
+    if constexpr (STAGE == 6) {
+      // the scales of the exact new amaxes pass 6 reduced (the rule of
+      // stages 1 and 2), compared with the predicted old scales
+      int km, kv, kw, kq = 0;
+      bool ok = scale_exponent(ws[WS_AMAX_M], kMaxE4M3, L.margin, 0, km);
+      ok &= scale_exponent(ws[WS_AMAX_V], kMaxF16, L.margin, 0, kv);
+      ok &= scale_exponent(ws[WS_CHECK_W], kMaxF16, L.margin, 0, kw);
+      if (C.wq_scale != nullptr)
+        ok &= scale_exponent(stored_value(ws[WS_CHECK_W], pow2f(kw)), kMaxE4M3, L.margin, 0, kq);
+      if (!ok) atomicOr(&g_status, FP8_STATUS_NONFINITE);
+      const float sm = *C.m_scale, sv = *C.v_scale, sw = *C.w_scale;
+      const float nm = pow2f(km), nv = pow2f(kv), nw = pow2f(kw), nq = pow2f(kq);
+      const bool held = nm == sm && nv == sv && nw == sw && (C.wq_scale == nullptr || nq == *C.wq_scale);
+      ws[WS_OLDINV_M] = 1.0f / sm;
+      ws[WS_OLDINV_V] = 1.0f / sv;
+      ws[WS_OLDINV_W] = 1.0f / sw;
+      ws[WS_NEW_M] = nm;
+      ws[WS_NEW_V] = nv;
+      ws[WS_NEW_W] = nw;
+      ws[WS_NEW_WQ] = nq;
+      if (!held) ws[WS_STORED_W] = 0.0f;  // the redo reduces it again with the right scale
+      ws[WS_FLAGS] = __uint_as_float(held ? 0u : FLAG_REDO);
+      *C.m_scale = nm;
+      *C.v_scale = nv;
+      *C.w_scale = nw;
+      if (C.wq_scale != nullptr) {
+        *C.wq_scale = nq;
+        *C.wq_inv = 1.0f / nq;
+      }
+      if (held && C.w_amax != nullptr) *C.w_amax = __fmul_rn(ws[WS_STORED_W], 1.0f / nw);
+    }
+    if constexpr (STAGE == 7) {
+      if ((flags & FLAG_REDO) && C.w_amax != nullptr)
+        *C.w_amax = __fmul_rn(ws[WS_STORED_W], 1.0f / ws[WS_NEW_W]);
     }
     if constexpr (STAGE == 3) {
       // a scale decided from an interval must be the one the exact new amax gives

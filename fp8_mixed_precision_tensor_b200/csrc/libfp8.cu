@@ -31,6 +31,7 @@ struct DeviceInfo {
   int adam_stats_blocks_per_sm = 1;  // of the exact stats pass and the exact master pass
   int adam_bound_blocks_per_sm = 1;  // of the estimated stats pass of tracking chunks
   int adam_est_blocks_per_sm = 1;    // of the estimated stats pass of the other chunks
+  int adam_into_blocks_per_sm = 1;   // of the out-of-place update (and its redo)
   int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair GEMM
   int wide_clusters = 0;  // co-resident 2-CTA clusters of the wide pair GEMM
 };
@@ -83,6 +84,9 @@ int device_info(DeviceInfo **out) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k_adam<5>, kAdamThreads, 0) != cudaSuccess)
       return FP8_ERR_CUDA;
     d.adam_est_blocks_per_sm = bps > 0 ? bps : 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k_adam<6>, kAdamThreads, 0) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    d.adam_into_blocks_per_sm = bps > 0 ? bps : 1;
     int rc = FP8_OK;
     rc |= set_smem(gemm::k_gemm<256, false, false>, gemm::Cfg<256>::SMEM_BYTES);
     rc |= set_smem(gemm::k_gemm<256, false, true>, gemm::Cfg<256>::SMEM_BYTES);
@@ -451,11 +455,15 @@ size_t fp8_adam_workspace_bytes(int nchunks) {
 namespace {
 
 // The Adam step in phases: PH_STATS runs the stats pass into the workspace,
-// PH_APPLY finalizes the scales from it and runs the update, PH_ALL both.
-enum { PH_STATS = 1, PH_APPLY = 2, PH_ALL = 3 };
+// PH_APPLY finalizes the scales from it and runs the update, PH_ALL both;
+// PH_INTO is the out-of-place step (dest holds the new buffers).
+enum { PH_STATS = 1, PH_APPLY = 2, PH_ALL = 3, PH_INTO = 4 };
+
+bool same_buffer(const void *a, const void *b) { return a != nullptr && a == b; }
 
 int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp, void *workspace,
-             size_t ws_bytes, void *stream, int phases) {
+             size_t ws_bytes, void *stream, int phases, const fp8_adam_dest *dest = nullptr) {
+  if ((phases == PH_INTO) != (dest != nullptr)) return FP8_ERR_INVALID_ARG;
   if (!chunks || !hp || nchunks <= 0 || !workspace) return FP8_ERR_INVALID_ARG;
   if (ws_bytes < fp8_adam_workspace_bytes(nchunks)) return FP8_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FP8_ERR_UNALIGNED;
@@ -476,21 +484,31 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
     // the E4M3 copy is asked for by wq_scale; its codes may be NULL only for an empty chunk
     if ((c.wq || c.wq_scale || c.wq_inv) && (!c.wq_scale || !c.wq_inv)) return FP8_ERR_INVALID_ARG;
     if (c.wq_scale && c.n > 0 && !c.wq) return FP8_ERR_INVALID_ARG;
-    if (phases != PH_ALL && c.w_amax) return FP8_ERR_INVALID_ARG;  // tracking needs the whole step
+    if ((phases == PH_STATS || phases == PH_APPLY) && c.w_amax)
+      return FP8_ERR_INVALID_ARG;  // tracking needs the whole step
     if (c.n > 0 && (!c.g || !c.m || !c.v || !c.w)) return FP8_ERR_INVALID_ARG;
     if (c.n > 0 && (!aligned16(c.g) || !aligned16(c.m) || !aligned16(c.v) || !aligned16(c.w) ||
                     (c.wq && !aligned16(c.wq))))
       return FP8_ERR_UNALIGNED;
+    if (dest && c.n > 0) {
+      const fp8_adam_dest &o = dest[i];
+      if (!o.m || !o.v || !o.w) return FP8_ERR_INVALID_ARG;
+      // the inputs must survive the first pass: no new buffer may be an old one
+      if (same_buffer(o.m, c.m) || same_buffer(o.v, c.v) || same_buffer(o.w, c.w) ||
+          same_buffer(o.m, c.g) || same_buffer(o.m, c.wq))
+        return FP8_ERR_INVALID_ARG;
+      if (!aligned16(o.m) || !aligned16(o.v) || !aligned16(o.w)) return FP8_ERR_UNALIGNED;
+    }
   }
   DeviceInfo *d;
   int rc = device_info(&d);
   if (rc) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if ((phases & PH_STATS) &&
+  if ((phases & (PH_STATS | PH_INTO)) &&
       (rc = cuda_rc(cudaMemsetAsync(workspace, 0, fp8_adam_workspace_bytes(nchunks), s))))
     return rc;
 
-  static thread_local AdamLaunch L;  // ~29 KB: kept off the stack
+  static thread_local AdamLaunch L;  // ~30 KB: kept off the stack
   L.margin = hp->margin;
   L.beta1 = hp->beta1;
   L.beta2 = hp->beta2;
@@ -505,6 +523,7 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
   const unsigned cap1 = (unsigned)(d->sms * d->adam_stats_blocks_per_sm);
   const unsigned cap4 = (unsigned)(d->sms * d->adam_bound_blocks_per_sm);
   const unsigned cap5 = (unsigned)(d->sms * d->adam_est_blocks_per_sm);
+  const unsigned cap6 = (unsigned)(d->sms * d->adam_into_blocks_per_sm);
   for (int first = 0; first < nchunks; first += kAdamMaxChunksPerLaunch) {
     const int cnt = nchunks - first < kAdamMaxChunksPerLaunch ? nchunks - first : kAdamMaxChunksPerLaunch;
     unsigned long long tiles = 0;
@@ -514,6 +533,11 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
       e.g = c.g; e.g_inv = c.g_inv; e.m = c.m; e.m_scale = c.m_scale;
       e.v = c.v; e.v_scale = c.v_scale; e.w = c.w; e.w_scale = c.w_scale;
       e.w_amax = c.w_amax; e.wq = c.wq; e.wq_scale = c.wq_scale; e.wq_inv = c.wq_inv;
+      if (dest) {
+        e.m_out = dest[first + i].m; e.v_out = dest[first + i].v; e.w_out = dest[first + i].w;
+      } else {
+        e.m_out = c.m; e.v_out = c.v; e.w_out = c.w;
+      }
       e.n = c.n;
       e.tile_begin = tiles;
       tiles += (c.n + kAdamTile - 1) / kAdamTile;
@@ -525,6 +549,7 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
     const unsigned grid1 = tiles == 0 ? 1u : (unsigned)(tiles < cap1 ? tiles : cap1);
     const unsigned grid4 = tiles == 0 ? 1u : (unsigned)(tiles < cap4 ? tiles : cap4);
     const unsigned grid5 = tiles == 0 ? 1u : (unsigned)(tiles < cap5 ? tiles : cap5);
+    const unsigned grid6 = tiles == 0 ? 1u : (unsigned)(tiles < cap6 ? tiles : cap6);
     bool tracked = false;
     for (int i = 0; i < cnt; i++) tracked |= L.c[i].w_amax != nullptr;
     if (phases & PH_STATS) {
@@ -544,6 +569,11 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
     } else if (phases & PH_APPLY) {
       k_adam_finalize<12><<<1, 256, 0, s>>>(L);
       k_adam<2><<<grid, kAdamThreads, 0, s>>>(L);    // update
+    } else if (phases == PH_INTO) {
+      k_adam<6><<<grid6, kAdamThreads, 0, s>>>(L);   // update with the predicted scales
+      k_adam_finalize<6><<<1, 256, 0, s>>>(L);       // the right scales; wrong predictions flagged
+      k_adam<7><<<grid6, kAdamThreads, 0, s>>>(L);   // flagged chunks again, from the inputs
+      k_adam_finalize<7><<<1, 256, 0, s>>>(L);
     }
     if ((rc = launch_rc())) return rc;
   }
@@ -557,6 +587,12 @@ extern "C" {
 int fp8_adam_step(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp,
                   void *workspace, size_t ws_bytes, void *stream) {
   return adam_run(chunks, nchunks, hp, workspace, ws_bytes, stream, PH_ALL);
+}
+
+int fp8_adam_step_into(const fp8_adam_chunk *chunks, const fp8_adam_dest *dest, int nchunks,
+                       const fp8_adam_hparams *hp, void *workspace, size_t ws_bytes, void *stream) {
+  if (!dest) return FP8_ERR_INVALID_ARG;
+  return adam_run(chunks, nchunks, hp, workspace, ws_bytes, stream, PH_INTO, dest);
 }
 
 int fp8_adam_stats(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp,

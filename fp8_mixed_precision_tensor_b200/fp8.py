@@ -31,7 +31,7 @@ _DT = {torch.float32: FP8_DT_F32, torch.bfloat16: FP8_DT_BF16, torch.float16: FP
 SYMBOLS = ("fp8_amax", "fp8_compute_scale", "fp8_cast", "fp8_scale_cast", "fp8_cast_count", "fp8_grad_cast",
            "fp8_sum_codes", "fp8_mu_update", "fp8_linear_fwd", "fp8_linear_dgrad",
            "fp8_linear_wgrad", "fp8_adam_workspace_bytes", "fp8_adam_step", "fp8_adam_stats",
-           "fp8_adam_apply", "fp8_adam_step_noalloc",
+           "fp8_adam_apply", "fp8_adam_step_noalloc", "fp8_adam_step_into",
            "fp8_selftest_wait_timeout", "fp8_get_status", "fp8_strerror")
 
 
@@ -47,6 +47,10 @@ class _Chunk(ctypes.Structure):
                 ("w", ctypes.c_void_p), ("w_scale", ctypes.c_void_p), ("n", ctypes.c_size_t),
                 ("w_amax", ctypes.c_void_p), ("wq", ctypes.c_void_p), ("wq_scale", ctypes.c_void_p),
                 ("wq_inv", ctypes.c_void_p)]
+
+
+class _Dest(ctypes.Structure):
+    _fields_ = [("m", ctypes.c_void_p), ("v", ctypes.c_void_p), ("w", ctypes.c_void_p)]
 
 
 class _MuRule(ctypes.Structure):
@@ -86,6 +90,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     for name in ("fp8_adam_step", "fp8_adam_stats", "fp8_adam_apply"):
         getattr(lib, name).argtypes = [ctypes.POINTER(_Chunk), i, ctypes.POINTER(_HParams), p, sz, p]
     lib.fp8_adam_step_noalloc.argtypes = [ctypes.POINTER(_Chunk), i, ctypes.POINTER(_HParams), p]
+    lib.fp8_adam_step_into.argtypes = [ctypes.POINTER(_Chunk), ctypes.POINTER(_Dest), i,
+                                       ctypes.POINTER(_HParams), p, sz, p]
     lib.fp8_selftest_wait_timeout.argtypes = [ctypes.c_uint, p]
     lib.fp8_get_status.argtypes = [ctypes.POINTER(ctypes.c_uint), p]
     lib.fp8_strerror.argtypes, lib.fp8_strerror.restype = [i], ctypes.c_char_p
@@ -264,6 +270,30 @@ def fp8_adam_step(chunks, lr: float, beta1: float, beta2: float, eps: float, ste
     _check(load_library().fp8_adam_step(arr, len(arr), ctypes.byref(hp), _ptr(workspace),
                                         workspace.numel() * workspace.element_size(), _stream(stream)),
            "fp8_adam_step")
+
+
+def pack_adam_dests(dests) -> ctypes.Array:
+    """Host array of fp8_adam_dest from (m, v, w) device tensors per chunk."""
+    arr = (_Dest * len(dests))()
+    for i, (m, v, w) in enumerate(dests):
+        arr[i] = _Dest(_ptr(m), _ptr(v), _ptr(w))
+    return arr
+
+
+def fp8_adam_step_into(chunks, dests, lr: float, beta1: float, beta2: float, eps: float, step: int,
+                       margin: int, workspace: torch.Tensor, stream=None) -> None:
+    """The step of fp8_adam_step with the new m, v, w written into `dests`
+    (a list of (m, v, w) tensors per chunk, or pack_adam_dests' array); the
+    chunks' own m, v, w are only read.  Bit for bit the in-place step's
+    results, in one pass over the state when the scales do not change."""
+    arr = chunks if isinstance(chunks, ctypes.Array) else pack_adam_chunks(chunks)
+    darr = dests if isinstance(dests, ctypes.Array) else pack_adam_dests(dests)
+    if len(darr) != len(arr):
+        raise ValueError("one dest per chunk")
+    hp = _HParams(lr, beta1, beta2, eps, step, margin)
+    _check(load_library().fp8_adam_step_into(arr, darr, len(arr), ctypes.byref(hp), _ptr(workspace),
+                                             workspace.numel() * workspace.element_size(), _stream(stream)),
+           "fp8_adam_step_into")
 
 
 def _adam_half(name, chunks, lr, beta1, beta2, eps, step, margin, workspace, stream):

@@ -327,6 +327,36 @@ size_t fp8_adam_workspace_bytes(int nchunks);
 int fp8_adam_step(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp,
                   void *workspace, size_t ws_bytes, void *stream);
 
+/* New state buffers of one chunk for fp8_adam_step_into. */
+typedef struct {
+  uint8_t *m;   /* dev [n] E4M3 first-moment codes (out) */
+  uint16_t *v;  /* dev [n] FP16 second moment, scaled (out) */
+  uint16_t *w;  /* dev [n] FP16 master weight, scaled (out) */
+} fp8_adam_dest;
+
+/*
+ * fp8_adam_step_into -- the step of fp8_adam_step with the new m, v, w
+ * written to dest[i] instead of over chunks[i].m, .v, .w, which are only
+ * read (a caller alternates two sets of buffers).  Every result -- codes,
+ * FP16 values, scales, tracked amax, E4M3 copy -- is bit for bit the one
+ * fp8_adam_step gives on the same inputs.  The step predicts that each new
+ * scale equals the old one: one pass reads the old state (6 B/param) and
+ * writes the new one with the predicted scales (5 B/param, +1 B for the
+ * E4M3 copy) while reducing the exact new amaxes; a chunk whose prediction
+ * was wrong (some new scale differs) is updated a second time from its
+ * unchanged inputs with the right scales.  When the scales hold, the state
+ * is read once instead of twice.
+ *   dest: HOST array of nchunks; for a chunk with n > 0 its three pointers
+ *   are dev, 16-byte aligned (else FP8_ERR_UNALIGNED) and must not overlap
+ *   any chunk's g, m, v, w, wq or another dest (a dest pointer equal to the
+ *   same chunk's m, v, w, g or wq is rejected with FP8_ERR_INVALID_ARG; other
+ *   overlaps are not detected).  Scales, w_amax, wq, wq_scale, wq_inv are
+ *   updated in place as by fp8_adam_step.  Workspace and errors as for
+ *   fp8_adam_step; nchunks with any n.
+ */
+int fp8_adam_step_into(const fp8_adam_chunk *chunks, const fp8_adam_dest *dest, int nchunks,
+                       const fp8_adam_hparams *hp, void *workspace, size_t ws_bytes, void *stream);
+
 /*
  * Element-sharded step ([FP8-LM] 提案手法 O3: FP8 optimizer state under a
  * ZeRO-style partition).  fp8_adam_step in two halves so that ranks which

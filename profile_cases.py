@@ -3,15 +3,17 @@
     python profile_cases.py linear --M 4096 --N 16384 --K 4096 [--rto]
     python profile_cases.py cast --n 268435456
     python profile_cases.py castsweep
-    python profile_cases.py adam --n 67108864 [--track]
+    python profile_cases.py adam --n 67108864 [--track] [--into]
     python profile_cases.py allreduce --n 268435456 --world 8
     python profile_cases.py castcount --n 268435456
-    python profile_cases.py adam7b --iters 10 [--track] [--copy]
+    python profile_cases.py adam7b --iters 10 [--track] [--copy] [--into]
 
 Each case runs `--iters` passes after one warm-up pass on seeded synthetic
 inputs and prints the CUDA-event time per pass.  Launch order per pass:
 linear: amax and fused scale+cast of X, W, dY (6 launches), then fwd, dgrad,
-wgrad; cast: amax, fused scale+cast; adam: stats pass, finalize, update pass;
+wgrad; cast: amax, fused scale+cast; adam: stats pass, finalize, update pass
+(with --into the out-of-place step: update with the predicted scales,
+finalize, redo pass, finalize);
 allreduce: `world` emulated ranks' payload casts of an fp32 gradient, then
 the `world` per-slice code sums (no collective: one GPU); castcount: the cast
 with under/overflow counters, then the plain cast; adam7b: one Adam step
@@ -30,7 +32,7 @@ import torch
 sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
 
 from fp8_mixed_precision_tensor_b200 import fp8, synth  # noqa: E402
-from fp8_mixed_precision_tensor_b200.adam_state import AdamTensorState  # noqa: E402
+from fp8_mixed_precision_tensor_b200.adam_state import AdamTensorState, FP8Adam  # noqa: E402
 
 
 def _scalars(n):
@@ -134,14 +136,23 @@ def case_adam(a):
     v = torch.zeros(n, dtype=torch.int16, device="cuda")
     st = torch.ones(3, dtype=torch.float32, device="cuda")
     st[2] = -1.0  # tracked master amax: unknown until the first step
-    chunks = fp8.pack_adam_chunks([fp8.AdamChunk(gq, sc[2:3], m, st[0:1], v, st[1:2], wh, sc[4:5],
-                                                 w_amax=st[2:3] if a.track else None)])
+    bufs = [(m, v, wh)]
+    if a.into:
+        bufs.append((torch.empty_like(m), torch.empty_like(v), torch.empty_like(wh)))
+    packs = [(fp8.pack_adam_chunks([fp8.AdamChunk(gq, sc[2:3], mm, st[0:1], vv, st[1:2], ww, sc[4:5],
+                                                  w_amax=st[2:3] if a.track else None)]),
+              fp8.pack_adam_dests([bufs[1 - k]]) if a.into else None)
+             for k, (mm, vv, ww) in enumerate(bufs)]
     ws = torch.zeros(64, dtype=torch.float32, device="cuda")
     state = {"t": 0}
 
     def one():
         state["t"] += 1
-        fp8.fp8_adam_step(chunks, 1e-4, 0.9, 0.95, 1e-8, state["t"], 0, ws)
+        chunks, dests = packs[(state["t"] - 1) % len(packs)]
+        if a.into:
+            fp8.fp8_adam_step_into(chunks, dests, 1e-4, 0.9, 0.95, 1e-8, state["t"], 0, ws)
+        else:
+            fp8.fp8_adam_step(chunks, 1e-4, 0.9, 0.95, 1e-8, state["t"], 0, ws)
 
     return one
 
@@ -208,15 +219,16 @@ def case_castcount(a):
     return one
 
 
-def build_adam_state(chunks, device="cuda", seed=11, mu=2.0 ** 10, track=False, copy=False):
+def build_adam_state(chunks, device="cuda", seed=11, mu=2.0 ** 10, track=False, copy=False, spare=False):
     """Decoupled-Adam state for (name, n) chunks: FP16 master from weights
     ~N(0, 0.02), zero moments, E5M2 gradients ~N(0, 1e-3) scaled by mu; with
-    `copy` the step also writes each tensor's E4M3 weight copy.  Returns the
+    `copy` the step also writes each tensor's E4M3 weight copy, with `spare`
+    each state gets the out-of-place step's second buffers.  Returns the
     AdamTensorState list."""
     out = []
     for ci, (_, n) in enumerate(chunks):
         w = synth.device_normal((n,), 0.02, seed * 100000 + 2 * ci + 1, torch.float32, device)
-        st = AdamTensorState(w, track_master_amax=track, e4m3_copy=copy)
+        st = AdamTensorState(w, track_master_amax=track, e4m3_copy=copy, spare_buffers=spare)
         del w
         g = synth.device_normal((n,), 1e-3, seed * 100000 + 2 * ci, torch.float32, device)
         st.set_gradient(g, mu)
@@ -226,22 +238,20 @@ def build_adam_state(chunks, device="cuda", seed=11, mu=2.0 ** 10, track=False, 
 
 
 def case_adam7b(a):
-    chunks_list = [st.chunk for st in build_adam_state(synth.gpt7b_adam_chunks(), track=a.track, copy=a.copy)]
-    params = sum(c.g.numel() for c in chunks_list)
-    chunks = fp8.pack_adam_chunks(chunks_list)
-    ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(chunks_list)) // 4, dtype=torch.float32, device="cuda")
-    state = {"t": 0}
+    states = build_adam_state(synth.gpt7b_adam_chunks(), track=a.track, copy=a.copy, spare=a.into)
+    opt = FP8Adam(states, lr=1e-4, out_of_place=a.into)
+    params = sum(st.n for st in states)
 
     def one():
-        state["t"] += 1
-        fp8.fp8_adam_step(chunks, 1e-4, 0.9, 0.95, 1e-8, state["t"], 0, ws)
+        opt.step()
 
     t = _timed(one, a.iters)
     # bytes moved per parameter: the stats pass reads g, m, v (and the master
     # unless its amax is tracked), the update pass reads g, m, v, w and writes
-    # m, v, w (and the E4M3 copy)
-    moved = (4 if a.track else 6) + 11 + (1 if a.copy else 0)
-    print(f"adam7b: {len(chunks_list)} chunks, {params} params, track={a.track} copy={a.copy}: "
+    # m, v, w (and the E4M3 copy); out of place, the update pass alone (while
+    # the scales hold)
+    moved = (0 if a.into else (4 if a.track else 6)) + 11 + (1 if a.copy else 0)
+    print(f"adam7b: {len(states)} chunks, {params} params, track={a.track} copy={a.copy} into={a.into}: "
           f"{t:.3f} ms per step, {11 * params / t / 1e6:.0f} GB/s algorithmic (11 B/param), "
           f"{moved * params / t / 1e6:.0f} GB/s moved ({moved} B/param)")
     return one
@@ -258,6 +268,7 @@ def main():
     ap.add_argument("--world", type=int, default=8, help="allreduce: emulated ranks")
     ap.add_argument("--track", action="store_true", help="adam: track the master amax across steps")
     ap.add_argument("--copy", action="store_true", help="adam7b: write the E4M3 weight copy")
+    ap.add_argument("--into", action="store_true", help="adam, adam7b: the out-of-place step")
     ap.add_argument("--rto", action="store_true", help="linear: dW as bfloat16 rounded to odd")
     a = ap.parse_args()
     one = {"linear": case_linear, "cast": case_cast, "castsweep": case_castsweep, "adam": case_adam,

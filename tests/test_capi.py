@@ -150,6 +150,31 @@ def test_adam_rejects_hyper_parameters_outside_the_argued_range(lib):
             (lr, b1, b2, eps, t)
 
 
+def test_adam_step_into_rejects_missing_or_aliased_destinations(lib):
+    """The out-of-place step refuses, on the host and before any launch, a
+    NULL dest array, a dest with a NULL buffer, a dest buffer that is the
+    chunk's own m, v, w or gradient (the inputs must survive the first pass),
+    and an unaligned dest."""
+    from fp8_mixed_precision_tensor_b200 import fp8
+
+    p, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    G, M, V, W, S = 0x10000, 0x20000, 0x30000, 0x40000, 0x50000
+    arr = (fp8._Chunk * 1)()
+    arr[0] = fp8._Chunk(G, S, M, S, V, S, W, S, 64, None, None, None, None)
+    hp = fp8._HParams(1e-4, 0.9, 0.95, 1e-8, 1, 0)
+    fn = lib.fp8_adam_step_into
+    fn.argtypes = [ctypes.POINTER(fp8._Chunk), ctypes.POINTER(fp8._Dest), i, ctypes.POINTER(fp8._HParams), p,
+                   sz, p]
+    assert fn(arr, None, 1, ctypes.byref(hp), S, 64, None) == fp8.FP8_ERR_INVALID_ARG
+    dst = (fp8._Dest * 1)()
+    for d in ((0x60000, None, 0x80000), (M, 0x70000, 0x80000), (0x60000, V, 0x80000), (0x60000, 0x70000, W),
+              (G, 0x70000, 0x80000)):
+        dst[0] = fp8._Dest(*d)
+        assert fn(arr, dst, 1, ctypes.byref(hp), S, 64, None) == fp8.FP8_ERR_INVALID_ARG, d
+    dst[0] = fp8._Dest(0x60008, 0x70000, 0x80000)
+    assert fn(arr, dst, 1, ctypes.byref(hp), S, 64, None) == fp8.FP8_ERR_UNALIGNED
+
+
 def test_wait_selftest_rejects_limits_outside_its_range(lib):
     lib.fp8_selftest_wait_timeout.argtypes = [ctypes.c_uint, ctypes.c_void_p]
     assert lib.fp8_selftest_wait_timeout(0, None) == 1

@@ -1,0 +1,165 @@
+"""The out-of-place Adam step (fp8_adam_step_into) against the in-place step.
+
+Both run the same arithmetic ("FP8-LM: Training FP8 Large Language Models",
+提案手法 O2: FP8 gradient and first moment, FP16 second moment and master,
+just-in-time per-tensor scales), so the new state must agree bit for bit:
+codes, FP16 values, scales, the tracked master amax and the E4M3 copy.  The
+out-of-place step predicts that each new scale equals the old one and updates
+a chunk a second time when that was wrong; the cases here take both branches
+(read back from the workspace's per-chunk flag word, bit 3) and cross the
+launch-group boundary of the chunk table.  The in-place step is held to the
+oracle by test_gpu_parity.py; one case here also checks the out-of-place
+result against the oracle directly.
+"""
+import numpy as np
+import pytest
+import torch
+
+from fp8_mixed_precision_tensor_b200 import fp8
+
+from test_gpu_parity import (F32, HP, MAX_TIES, _stored_amax, _with_tracking, check_adam_chunk, make_adam_state,
+                             scalar, snapshot)
+
+pytestmark = pytest.mark.gpu
+
+WS_FLAGS, FLAG_REDO, WS_FLOATS = 10, 8, 16
+
+
+def _clone(chunks):
+    """An independent copy of every buffer and scalar of the chunks."""
+    out = []
+    for c in chunks:
+        kw = {k: (getattr(c, k).clone() if getattr(c, k) is not None else None)
+              for k in ("w_amax", "wq", "wq_scale", "wq_inv")}
+        out.append(fp8.AdamChunk(c.g, c.g_inv.clone(), c.m.clone(), c.m_scale.clone(), c.v.clone(),
+                                 c.v_scale.clone(), c.w.clone(), c.w_scale.clone(), **kw))
+    return out
+
+
+class IntoRunner:
+    """Chunks stepped out of place: each step writes the spare buffers, which
+    then become the chunk's state (the old ones become the spares)."""
+
+    def __init__(self, chunks):
+        self.chunks = chunks
+        self.spare = [(torch.empty_like(c.m), torch.empty_like(c.v), torch.empty_like(c.w)) for c in chunks]
+        self.ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(chunks)) // 4, **F32)
+
+    def step(self, step, hp=HP, margin=0):
+        fp8.fp8_adam_step_into(self.chunks, self.spare, step=step, margin=margin, workspace=self.ws, **hp)
+        new = []
+        for c, (m, v, w) in zip(self.chunks, self.spare):
+            new.append(fp8.AdamChunk(c.g, c.g_inv, m, c.m_scale, v, c.v_scale, w, c.w_scale, c.w_amax, c.wq,
+                                     c.wq_scale, c.wq_inv))
+        self.spare = [(c.m, c.v, c.w) for c in self.chunks]
+        self.chunks = new
+
+    def redone(self):
+        """Per chunk: True where the last step updated it a second time."""
+        flags = self.ws.view(-1, WS_FLOATS)[:, WS_FLAGS].view(torch.int32).cpu().numpy()
+        return (flags & FLAG_REDO) != 0
+
+
+def assert_same_state(ref, got, where):
+    for r, g in zip(ref, got):
+        sr, sg = snapshot(r), snapshot(g)
+        for k in ("m", "v", "w", "s_m", "s_v", "s_w"):
+            assert np.array_equal(np.asarray(sr[k]), np.asarray(sg[k])), (where, k)
+        if r.w_amax is not None:
+            assert r.w_amax.item() == g.w_amax.item(), where
+            if sg["w"].size:
+                assert g.w_amax.item() == _stored_amax(sg), where
+        if r.wq_scale is not None:
+            assert r.wq_scale.item() == g.wq_scale.item() and r.wq_inv.item() == g.wq_inv.item(), where
+            assert torch.equal(r.wq, g.wq), where
+
+
+@pytest.mark.parametrize("track,wq", [(False, False), (True, True), (False, True)])
+def test_adam_into_equals_in_place_step(track, wq):
+    """Six steps from zero moments, chunks with ragged ends, an empty chunk and
+    a chunk of zero gradients (whose scales never change): the out-of-place
+    state equals the in-place state after every step; step 1 redoes every
+    chunk whose moments change scale, the zero-gradient chunk keeps its
+    prediction from step 2 on."""
+    sizes = [65536, 4099, 1, 0, 300000, 8192]
+    base = make_adam_state(sizes, ("adam-into", track, wq))
+    base[5].g.zero_()
+    if track or wq:
+        base = _with_tracking(base, wq=wq, track=track)
+    ref, into = base, IntoRunner(_clone(base))
+    ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(sizes)) // 4, **F32)
+    held = 0
+    for step in range(1, 7):
+        fp8.fp8_adam_step(ref, step=step, margin=0, workspace=ws, **HP)
+        into.step(step)
+        assert fp8.fp8_get_status() == 0
+        assert_same_state(ref, into.chunks, step)
+        r = into.redone()
+        if step == 1:
+            assert r[0] and r[1] and r[4]
+        if step >= 2:
+            assert not r[5]
+        held += int(np.count_nonzero(~r[[0, 1, 2, 4]]))
+    assert held > 0  # some chunks with a moving state also kept their prediction
+
+
+def test_adam_into_held_predictions_with_unchanged_moments():
+    """beta1 = beta2 = 0 and a fixed gradient: from step 2 on the new moments
+    equal the old ones, the master moves by ~lr, and every chunk keeps its
+    scales (one pass only); the state still equals the in-place step's."""
+    hp = dict(HP, beta1=0.0, beta2=0.0, lr=1e-6)
+    sizes = [65536 + 7, 4096, 300000]
+    base = _with_tracking(make_adam_state(sizes, ("adam-into-held",)), wq=True)
+    ref, into = base, IntoRunner(_clone(base))
+    ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(sizes)) // 4, **F32)
+    for step in (1, 2, 3):
+        fp8.fp8_adam_step(ref, step=step, margin=0, workspace=ws, **hp)
+        into.step(step, hp=hp)
+        assert fp8.fp8_get_status() == 0
+        assert_same_state(ref, into.chunks, step)
+        assert into.redone().all() if step == 1 else not into.redone().any(), step
+
+
+def test_adam_into_many_chunks_two_launch_groups():
+    """300 chunks (more than one launch's chunk table): the workspace offsets
+    of the second group and its redo pass."""
+    sizes = [37 + 16 * i for i in range(300)]
+    base = _with_tracking(make_adam_state(sizes, ("adam-into-many",)), wq=True)
+    ref, into = base, IntoRunner(_clone(base))
+    ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(sizes)) // 4, **F32)
+    for step in (1, 2):
+        fp8.fp8_adam_step(ref, step=step, margin=0, workspace=ws, **HP)
+        into.step(step)
+        assert fp8.fp8_get_status() == 0
+        assert_same_state(ref, into.chunks, step)
+
+
+def test_adam_into_vs_oracle():
+    """Two steps (the second from the GPU's own first-step state), each
+    against the oracle."""
+    sizes = [65536, 4099, 300000]
+    into = IntoRunner(make_adam_state(sizes, ("adam-into-oracle",), steps_done=4))
+    ties = []
+    for step in (5, 6):
+        before = [snapshot(c) for c in into.chunks]
+        into.step(step)
+        assert fp8.fp8_get_status() == 0
+        for b, c in zip(before, into.chunks):
+            check_adam_chunk(b, c, step, ties=ties)
+    assert len(ties) <= MAX_TIES, ties
+
+
+def test_adam_into_rejects_bad_destinations():
+    chunks = make_adam_state([64], ("adam-into-bad",))
+    c = chunks[0]
+    ws = torch.zeros(16, **F32)
+    with pytest.raises(fp8.FP8Error):  # the new m over the old one
+        fp8.fp8_adam_step_into(chunks, [(c.m, torch.empty_like(c.v), torch.empty_like(c.w))], step=1, margin=0,
+                               workspace=ws, **HP)
+    with pytest.raises(fp8.FP8Error):  # unaligned
+        buf = torch.empty(80, dtype=torch.uint8, device="cuda")
+        fp8.fp8_adam_step_into(chunks, [(buf[8:72], torch.empty_like(c.v), torch.empty_like(c.w))], step=1,
+                               margin=0, workspace=ws, **HP)
+    with pytest.raises(ValueError):
+        fp8.fp8_adam_step_into(chunks, [], step=1, margin=0, workspace=ws, **HP)
+    assert scalar().item() == 0.0  # the device is still usable

@@ -74,9 +74,11 @@ def test_gpt175b_linears_full_size(name, K, N):
 def test_bench_step_three_streams_equals_one_stream(workload):
     """The benchmark step's overlapped schedule (casts, fwd/dgrad and wgrad on
     three streams, each tensor's Adam beside the next linears) computes exactly
-    what the one-stream order computes: the same scalars, gradient codes, Adam
+    what the one-stream order computes, and the out-of-place Adam step exactly
+    what the in-place one computes: the same scalars, gradient codes, Adam
     state and E4M3 weight copies after three steps (the second and third
-    steps' GEMMs read the weights that the previous step's Adam wrote)."""
+    steps' GEMMs read the weights that the previous step's Adam wrote; out of
+    place, the state after step 3 is in the second buffer set)."""
     import importlib.util
     import os
 
@@ -85,18 +87,24 @@ def test_bench_step_three_streams_equals_one_stream(workload):
     bench = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(bench)
     dev = torch.device("cuda", 0)
-    a = bench.BlockStep(dev, seed=3, workload=workload)
-    b = bench.BlockStep(dev, seed=3, workload=workload)
+    a = bench.BlockStep(dev, seed=3, workload=workload, adam="in_place")
+    b = bench.BlockStep(dev, seed=3, workload=workload, adam="into")
+    c = bench.BlockStep(dev, seed=3, workload=workload, adam="into")
     for _ in range(3):
         a.step()
         b.step_overlapped()
+        c.step()
     torch.cuda.synchronize()
     assert fp8.fp8_get_status() == 0
     assert torch.equal(a.result_scalars(), b.result_scalars())
-    for da, db in zip(a.L, b.L):
-        for k in ("gq", "m", "v", "wh", "wq", "y", "dx", "dw"):
-            assert torch.equal(da[k], db[k]), (da["name"], k)
-    del a, b
+    assert torch.equal(a.result_scalars(), c.result_scalars())
+    for da, db, dc in zip(a.L, b.L, c.L):
+        for k in ("gq", "wq", "y", "dx", "dw"):
+            assert torch.equal(da[k], db[k]) and torch.equal(da[k], dc[k]), (da["name"], k)
+        for ka, kb in (("m", "m2"), ("v", "v2"), ("wh", "wh2")):
+            assert torch.equal(da[ka], db[kb]) and torch.equal(da[ka], dc[kb]), (da["name"], ka)
+            assert torch.equal(db[ka], dc[ka]), (da["name"], ka)  # the state after step 2
+    del a, b, c
     torch.cuda.empty_cache()
 
 
