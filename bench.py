@@ -9,13 +9,16 @@ GPT-7B block (tokens 4096, hidden 4096).  Per step:
   for each linear:  amax + fused scale/cast of X (E4M3) and dY (E5M2, mu-scaled)
                     fwd   Y  = Xq Wq^T     (bf16 out, fused next-amax)
                     dgrad dX = dYq Wq      (bf16 out, fused next-amax)
-                    wgrad dW = dYq^T Xq    (fp32 out, fused amax)
+                    wgrad dW = dYq^T Xq    (bf16 rounded to odd, fused amax)
                     grad  gq = E5M2(mu s_g dW)
   then the precision-decoupled FP8 Adam step over the 4 weight tensors
   (E5M2 grad, E4M3 m1, FP16 m2, FP16 master; 1,811,939,328 parameters for
   GPT-175B), which also writes the E4M3 copy of each new master: the next
   step's forward and dgrad read the weight from that copy, so no weight cast
-  runs in the step.  The master's amax is tracked between steps.
+  runs in the step.  The master's amax is tracked between steps.  The step
+  is out of place (`--adam into`, the default): each step writes the new
+  state into the other of two buffer sets, in one pass while the scales
+  hold; `--adam in_place` runs the in-place step (stats pass + update).
 
 `value` is the step's algorithmic GEMM work (3 x 2MNK per linear; 89.06 TFLOP
 for GPT-175B) divided by the device time of the whole step, inputs resident
@@ -39,6 +42,7 @@ overlapped step for timeline profilers.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--workload gpt175b_block|gpt7b_block] [--schedule serial]
+                    [--adam into|in_place]
 """
 from __future__ import annotations
 

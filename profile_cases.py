@@ -8,8 +8,8 @@
     python profile_cases.py castcount --n 268435456
     python profile_cases.py adam7b --iters 10 [--track] [--copy] [--into]
 
-Each case runs `--iters` passes after one warm-up pass on seeded synthetic
-inputs and prints the CUDA-event time per pass.  Launch order per pass:
+Each case runs `--iters` passes after one warm-up pass (and `--skip` more) on
+seeded synthetic inputs and prints the CUDA-event time per pass.  Launch order per pass:
 linear: amax and fused scale+cast of X, W, dY (6 launches), then fwd, dgrad,
 wgrad; cast: amax, fused scale+cast; adam: stats pass, finalize, update pass
 (with --into the out-of-place step: update with the predicted scales,
@@ -269,12 +269,16 @@ def main():
     ap.add_argument("--track", action="store_true", help="adam: track the master amax across steps")
     ap.add_argument("--copy", action="store_true", help="adam7b: write the E4M3 weight copy")
     ap.add_argument("--into", action="store_true", help="adam, adam7b: the out-of-place step")
+    ap.add_argument("--skip", type=int, default=0,
+                    help="passes run before the timed ones besides the one warm-up pass (adam: steps "
+                         "after which the moments' scales have settled)")
     ap.add_argument("--rto", action="store_true", help="linear: dW as bfloat16 rounded to odd")
     a = ap.parse_args()
     one = {"linear": case_linear, "cast": case_cast, "castsweep": case_castsweep, "adam": case_adam,
            "allreduce": case_allreduce,
            "castcount": case_castcount, "adam7b": case_adam7b}[a.case](a)
-    one()
+    for _ in range(1 + a.skip):
+        one()
     torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s.record()

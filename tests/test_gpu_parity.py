@@ -564,7 +564,7 @@ def test_adam_three_steps_stage_parity():
 
 
 def test_adam_many_chunks_multiple_launches():
-    sizes = [37 + 16 * i for i in range(300)]  # > 256 chunks: two launch groups
+    sizes = [37 + 16 * i for i in range(300)]  # > 224 chunks: two launch groups
     chunks = make_adam_state(sizes, ("adam-many",))
     ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(chunks)) // 4, **F32)
     before = [snapshot(c) for c in chunks]

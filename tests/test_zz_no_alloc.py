@@ -7,7 +7,7 @@ device-wide synchronisation that cudaMalloc/cudaFree can cause.
 fp8_adam_step_noalloc serves them from a fixed scratch array inside the
 library.  It runs the same kernels with the same arithmetic as fp8_adam_step,
 so through the C ABI two consecutive calls must leave bit for bit the same
-state: codes, FP16 values and scales.  One case has more than 256 chunks, so
+state: codes, FP16 values and scales.  One case has more than 224 chunks, so
 the step runs as two launch groups that use different parts of the scratch
 array.
 
