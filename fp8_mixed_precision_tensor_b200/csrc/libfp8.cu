@@ -455,15 +455,18 @@ size_t fp8_adam_workspace_bytes(int nchunks) {
 namespace {
 
 // The Adam step in phases: PH_STATS runs the stats pass into the workspace,
-// PH_APPLY finalizes the scales from it and runs the update, PH_ALL both;
-// PH_INTO is the out-of-place step (dest holds the new buffers).
+// PH_APPLY finalizes the scales from it and runs the update, PH_ALL both.
+// With PH_INTO the step is out of place (dest holds the new buffers):
+// PH_STATS is then the update with the predicted scales, which leaves the
+// exact new amaxes in the workspace, and PH_APPLY the scale decision and the
+// redo of the chunks whose prediction was wrong.
 enum { PH_STATS = 1, PH_APPLY = 2, PH_ALL = 3, PH_INTO = 4 };
 
 bool same_buffer(const void *a, const void *b) { return a != nullptr && a == b; }
 
 int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp, void *workspace,
              size_t ws_bytes, void *stream, int phases, const fp8_adam_dest *dest = nullptr) {
-  if ((phases == PH_INTO) != (dest != nullptr)) return FP8_ERR_INVALID_ARG;
+  if (((phases & PH_INTO) != 0) != (dest != nullptr)) return FP8_ERR_INVALID_ARG;
   if (!chunks || !hp || nchunks <= 0 || !workspace) return FP8_ERR_INVALID_ARG;
   if (ws_bytes < fp8_adam_workspace_bytes(nchunks)) return FP8_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FP8_ERR_UNALIGNED;
@@ -484,7 +487,7 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
     // the E4M3 copy is asked for by wq_scale; its codes may be NULL only for an empty chunk
     if ((c.wq || c.wq_scale || c.wq_inv) && (!c.wq_scale || !c.wq_inv)) return FP8_ERR_INVALID_ARG;
     if (c.wq_scale && c.n > 0 && !c.wq) return FP8_ERR_INVALID_ARG;
-    if ((phases == PH_STATS || phases == PH_APPLY) && c.w_amax)
+    if ((phases & PH_ALL) != PH_ALL && c.w_amax)
       return FP8_ERR_INVALID_ARG;  // tracking needs the whole step
     if (c.n > 0 && (!c.g || !c.m || !c.v || !c.w)) return FP8_ERR_INVALID_ARG;
     if (c.n > 0 && (!aligned16(c.g) || !aligned16(c.m) || !aligned16(c.v) || !aligned16(c.w) ||
@@ -504,7 +507,7 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
   int rc = device_info(&d);
   if (rc) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if ((phases & (PH_STATS | PH_INTO)) &&
+  if ((phases & PH_STATS) &&
       (rc = cuda_rc(cudaMemsetAsync(workspace, 0, fp8_adam_workspace_bytes(nchunks), s))))
     return rc;
 
@@ -552,7 +555,15 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
     const unsigned grid6 = tiles == 0 ? 1u : (unsigned)(tiles < cap6 ? tiles : cap6);
     bool tracked = false;
     for (int i = 0; i < cnt; i++) tracked |= L.c[i].w_amax != nullptr;
-    if (phases & PH_STATS) {
+    if (phases & PH_INTO) {
+      if (phases & PH_STATS)
+        k_adam<6><<<grid6, kAdamThreads, 0, s>>>(L);   // update with the predicted scales
+      if (phases & PH_APPLY) {
+        k_adam_finalize<6><<<1, 256, 0, s>>>(L);       // the right scales; wrong predictions flagged
+        k_adam<7><<<grid6, kAdamThreads, 0, s>>>(L);   // flagged chunks again, from the inputs
+        k_adam_finalize<7><<<1, 256, 0, s>>>(L);
+      }
+    } else if (phases & PH_STATS) {
       // stats of the chunks without a known tracked amax (whether a tracking
       // chunk's amax is known yet is only visible on the device): estimated
       // (whole step) or exact (phased step); those with one: estimated
@@ -560,20 +571,15 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
       else            k_adam<1><<<grid1, kAdamThreads, 0, s>>>(L);
       if (tracked) k_adam<4><<<grid4, kAdamThreads, 0, s>>>(L);
     }
-    if (phases == PH_ALL) {
+    if (phases == PH_ALL) {  // in place, whole step
       k_adam_finalize<1><<<1, 256, 0, s>>>(L);
       k_adam<3><<<grid1, kAdamThreads, 0, s>>>(L);  // exact master amax, flagged chunks only
       k_adam_finalize<2><<<1, 256, 0, s>>>(L);
       k_adam<2><<<grid, kAdamThreads, 0, s>>>(L);    // update
       k_adam_finalize<3><<<1, 256, 0, s>>>(L);       // check of the decided scales; tracked amax
-    } else if (phases & PH_APPLY) {
+    } else if (phases == PH_APPLY) {
       k_adam_finalize<12><<<1, 256, 0, s>>>(L);
       k_adam<2><<<grid, kAdamThreads, 0, s>>>(L);    // update
-    } else if (phases == PH_INTO) {
-      k_adam<6><<<grid6, kAdamThreads, 0, s>>>(L);   // update with the predicted scales
-      k_adam_finalize<6><<<1, 256, 0, s>>>(L);       // the right scales; wrong predictions flagged
-      k_adam<7><<<grid6, kAdamThreads, 0, s>>>(L);   // flagged chunks again, from the inputs
-      k_adam_finalize<7><<<1, 256, 0, s>>>(L);
     }
     if ((rc = launch_rc())) return rc;
   }
@@ -592,7 +598,19 @@ int fp8_adam_step(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hpar
 int fp8_adam_step_into(const fp8_adam_chunk *chunks, const fp8_adam_dest *dest, int nchunks,
                        const fp8_adam_hparams *hp, void *workspace, size_t ws_bytes, void *stream) {
   if (!dest) return FP8_ERR_INVALID_ARG;
-  return adam_run(chunks, nchunks, hp, workspace, ws_bytes, stream, PH_INTO, dest);
+  return adam_run(chunks, nchunks, hp, workspace, ws_bytes, stream, PH_INTO | PH_ALL, dest);
+}
+
+int fp8_adam_stats_into(const fp8_adam_chunk *chunks, const fp8_adam_dest *dest, int nchunks,
+                        const fp8_adam_hparams *hp, void *workspace, size_t ws_bytes, void *stream) {
+  if (!dest) return FP8_ERR_INVALID_ARG;
+  return adam_run(chunks, nchunks, hp, workspace, ws_bytes, stream, PH_INTO | PH_STATS, dest);
+}
+
+int fp8_adam_apply_into(const fp8_adam_chunk *chunks, const fp8_adam_dest *dest, int nchunks,
+                        const fp8_adam_hparams *hp, void *workspace, size_t ws_bytes, void *stream) {
+  if (!dest) return FP8_ERR_INVALID_ARG;
+  return adam_run(chunks, nchunks, hp, workspace, ws_bytes, stream, PH_INTO | PH_APPLY, dest);
 }
 
 int fp8_adam_stats(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp,

@@ -31,7 +31,8 @@ _DT = {torch.float32: FP8_DT_F32, torch.bfloat16: FP8_DT_BF16, torch.float16: FP
 SYMBOLS = ("fp8_amax", "fp8_compute_scale", "fp8_cast", "fp8_scale_cast", "fp8_cast_count", "fp8_grad_cast",
            "fp8_sum_codes", "fp8_mu_update", "fp8_linear_fwd", "fp8_linear_dgrad",
            "fp8_linear_wgrad", "fp8_adam_workspace_bytes", "fp8_adam_step", "fp8_adam_stats",
-           "fp8_adam_apply", "fp8_adam_step_noalloc", "fp8_adam_step_into",
+           "fp8_adam_apply", "fp8_adam_step_noalloc", "fp8_adam_step_into", "fp8_adam_stats_into",
+           "fp8_adam_apply_into",
            "fp8_selftest_wait_timeout", "fp8_get_status", "fp8_strerror")
 
 
@@ -90,7 +91,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     for name in ("fp8_adam_step", "fp8_adam_stats", "fp8_adam_apply"):
         getattr(lib, name).argtypes = [ctypes.POINTER(_Chunk), i, ctypes.POINTER(_HParams), p, sz, p]
     lib.fp8_adam_step_noalloc.argtypes = [ctypes.POINTER(_Chunk), i, ctypes.POINTER(_HParams), p]
-    lib.fp8_adam_step_into.argtypes = [ctypes.POINTER(_Chunk), ctypes.POINTER(_Dest), i,
+    for name in ("fp8_adam_step_into", "fp8_adam_stats_into", "fp8_adam_apply_into"):
+        getattr(lib, name).argtypes = [ctypes.POINTER(_Chunk), ctypes.POINTER(_Dest), i,
                                        ctypes.POINTER(_HParams), p, sz, p]
     lib.fp8_selftest_wait_timeout.argtypes = [ctypes.c_uint, p]
     lib.fp8_get_status.argtypes = [ctypes.POINTER(ctypes.c_uint), p]
@@ -280,20 +282,38 @@ def pack_adam_dests(dests) -> ctypes.Array:
     return arr
 
 
+def _adam_into(name, chunks, dests, lr, beta1, beta2, eps, step, margin, workspace, stream):
+    arr = chunks if isinstance(chunks, ctypes.Array) else pack_adam_chunks(chunks)
+    darr = dests if isinstance(dests, ctypes.Array) else pack_adam_dests(dests)
+    if len(darr) != len(arr):
+        raise ValueError("one dest per chunk")
+    hp = _HParams(lr, beta1, beta2, eps, step, margin)
+    _check(getattr(load_library(), name)(arr, darr, len(arr), ctypes.byref(hp), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream(stream)), name)
+
+
 def fp8_adam_step_into(chunks, dests, lr: float, beta1: float, beta2: float, eps: float, step: int,
                        margin: int, workspace: torch.Tensor, stream=None) -> None:
     """The step of fp8_adam_step with the new m, v, w written into `dests`
     (a list of (m, v, w) tensors per chunk, or pack_adam_dests' array); the
     chunks' own m, v, w are only read.  Bit for bit the in-place step's
     results, in one pass over the state when the scales do not change."""
-    arr = chunks if isinstance(chunks, ctypes.Array) else pack_adam_chunks(chunks)
-    darr = dests if isinstance(dests, ctypes.Array) else pack_adam_dests(dests)
-    if len(darr) != len(arr):
-        raise ValueError("one dest per chunk")
-    hp = _HParams(lr, beta1, beta2, eps, step, margin)
-    _check(load_library().fp8_adam_step_into(arr, darr, len(arr), ctypes.byref(hp), _ptr(workspace),
-                                             workspace.numel() * workspace.element_size(), _stream(stream)),
-           "fp8_adam_step_into")
+    _adam_into("fp8_adam_step_into", chunks, dests, lr, beta1, beta2, eps, step, margin, workspace, stream)
+
+
+def fp8_adam_stats_into(chunks, dests, lr: float, beta1: float, beta2: float, eps: float, step: int,
+                        margin: int, workspace: torch.Tensor, stream=None) -> None:
+    """First half of the element-sharded out-of-place step: this rank's new
+    slices into `dests` with the predicted scales, the exact new amaxes into
+    `workspace` (to be MAX-reduced over the ranks)."""
+    _adam_into("fp8_adam_stats_into", chunks, dests, lr, beta1, beta2, eps, step, margin, workspace, stream)
+
+
+def fp8_adam_apply_into(chunks, dests, lr: float, beta1: float, beta2: float, eps: float, step: int,
+                        margin: int, workspace: torch.Tensor, stream=None) -> None:
+    """Second half: the new scales from the reduced workspace, and the slices
+    of the tensors whose scales changed written again."""
+    _adam_into("fp8_adam_apply_into", chunks, dests, lr, beta1, beta2, eps, step, margin, workspace, stream)
 
 
 def _adam_half(name, chunks, lr, beta1, beta2, eps, step, margin, workspace, stream):

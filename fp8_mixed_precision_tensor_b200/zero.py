@@ -6,7 +6,9 @@ contiguous slice of every tensor and runs the decoupled Adam step
 (提案手法 O2) on its slices only.  The one coupling between ranks is the
 per-tensor scale of m, v and w, which comes from the amax of the whole new
 tensor: three scalars per tensor, combined by a single MAX all-reduce
-between the two halves of the step (fp8_adam_stats, fp8_adam_apply).
+between the two halves of the step (fp8_adam_stats, fp8_adam_apply; out of
+place, fp8_adam_stats_into and fp8_adam_apply_into, which read the state
+once while the scales hold).
 
 Slice boundaries sit on multiples of 16 elements, so every slice of the
 1- and 2-byte state arrays starts 16-byte aligned as the kernels require.
@@ -59,32 +61,84 @@ def shard_chunk(c: fp8.AdamChunk, lo: int, hi: int) -> fp8.AdamChunk:
                          None if c.wq is None else view(c.wq), own(c.wq_scale), own(c.wq_inv))
 
 
+def shard_dest(bufs, lo: int, hi: int) -> tuple:
+    """This rank's slice [lo, hi) of a tensor's second set of state buffers
+    (m, v, w), for the out-of-place step."""
+    if (hi > lo and lo % SHARD_ALIGN) or not 0 <= lo <= hi <= bufs[0].numel():
+        raise ValueError(f"bad slice [{lo}, {hi}) of {bufs[0].numel()} elements")
+    return tuple(t.reshape(-1)[lo:hi] for t in bufs)
+
+
 class ShardedAdam:
     """The decoupled FP8 Adam step over this rank's slices.  `chunks` holds
     slice i of tensor i on every rank, in the same order; `group` is the
-    data-parallel process group (None: the default group)."""
+    data-parallel process group (None: the default group).  With `dests`
+    (per chunk the matching slices (m, v, w) of a second set of buffers) the
+    step is out of place: each step writes the new state into the other set
+    and `current` follows it."""
 
-    def __init__(self, chunks: list[fp8.AdamChunk], group=None):
+    def __init__(self, chunks: list[fp8.AdamChunk], group=None, dests: list[tuple] | None = None):
         if any(c.w_amax is not None for c in chunks):
             raise ValueError("tracked master amax is not available in the sharded step")
-        self.chunks = fp8.pack_adam_chunks(chunks)
-        self._keep = chunks
+        if dests is not None and len(dests) != len(chunks):
+            raise ValueError("one dest per chunk")
+        self.current = list(chunks)
+        self.spare = None if dests is None else [tuple(d) for d in dests]
+        self._packs, self._parity = [None, None], 0
+        self._pack()
         self.group = group
         device = chunks[0].g_inv.device
         self.workspace = torch.zeros(fp8.fp8_adam_workspace_bytes(len(chunks)) // 4, dtype=torch.float32,
                                      device=device)
 
-    def step(self, lr: float, beta1: float, beta2: float, eps: float, t: int, margin: int = 0,
-             stream=None) -> None:
-        """stats -> MAX all-reduce of the workspace -> apply, all on `stream`
-        (a torch.cuda.Stream; the current stream by default), which the
-        collective also uses."""
-        args = (lr, beta1, beta2, eps, t, margin, self.workspace)
-        fp8.fp8_adam_stats(self.chunks, *args, stream=stream)
+    def _pack(self) -> None:
+        k = self._parity
+        if self._packs[k] is None:
+            self._packs[k] = (fp8.pack_adam_chunks(self.current),
+                              None if self.spare is None else fp8.pack_adam_dests(self.spare))
+        self.chunks, self.dests = self._packs[k]
+
+    def _reduce(self, stream) -> None:
         if dist.is_available() and dist.is_initialized():  # a group of one rank too
             if stream is None:
                 reduce_workspace(self.workspace, self.group)
             else:
                 with torch.cuda.stream(stream):
                     reduce_workspace(self.workspace, self.group)
-        fp8.fp8_adam_apply(self.chunks, *args, stream=stream)
+
+    def stats(self, lr: float, beta1: float, beta2: float, eps: float, t: int, margin: int = 0,
+              stream=None) -> None:
+        """First half of the step on this rank's slices: the workspace then
+        holds their exact new amaxes (out of place, the new slices are also
+        written with the predicted scales)."""
+        args = (lr, beta1, beta2, eps, t, margin, self.workspace)
+        if self.spare is None:
+            fp8.fp8_adam_stats(self.chunks, *args, stream=stream)
+        else:
+            fp8.fp8_adam_stats_into(self.chunks, self.dests, *args, stream=stream)
+
+    def apply(self, lr: float, beta1: float, beta2: float, eps: float, t: int, margin: int = 0,
+              stream=None) -> None:
+        """Second half, after the workspace was MAX-reduced over the ranks:
+        the new scales and the new slices (out of place, the buffer sets then
+        swap: `current` holds the new state)."""
+        args = (lr, beta1, beta2, eps, t, margin, self.workspace)
+        if self.spare is None:
+            fp8.fp8_adam_apply(self.chunks, *args, stream=stream)
+            return
+        fp8.fp8_adam_apply_into(self.chunks, self.dests, *args, stream=stream)
+        new = [fp8.AdamChunk(c.g, c.g_inv, m, c.m_scale, v, c.v_scale, w, c.w_scale, None, c.wq, c.wq_scale,
+                             c.wq_inv) for c, (m, v, w) in zip(self.current, self.spare)]
+        self.spare = [(c.m, c.v, c.w) for c in self.current]
+        self.current = new
+        self._parity ^= 1
+        self._pack()
+
+    def step(self, lr: float, beta1: float, beta2: float, eps: float, t: int, margin: int = 0,
+             stream=None) -> None:
+        """stats -> MAX all-reduce of the workspace -> apply, all on `stream`
+        (a torch.cuda.Stream; the current stream by default), which the
+        collective also uses."""
+        self.stats(lr, beta1, beta2, eps, t, margin, stream)
+        self._reduce(stream)
+        self.apply(lr, beta1, beta2, eps, t, margin, stream)

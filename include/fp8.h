@@ -385,6 +385,30 @@ int fp8_adam_apply(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hpa
                    void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * The element-sharded step out of place: fp8_adam_step_into in two halves,
+ * with the same MAX reduction of the workspace over the ranks in between.
+ *   fp8_adam_stats_into  clears the workspace, writes this rank's new slices
+ *                        into dest with the predicted (old) scales and the
+ *                        exact amax of the new m, v, w into the workspace;
+ *   <caller>             the element-wise int32 MAX of the workspace, as
+ *                        for fp8_adam_stats;
+ *   fp8_adam_apply_into  derives the new scales from the reduced amaxes
+ *                        (the same on every rank), publishes them, and
+ *                        writes again, from the unchanged inputs, the
+ *                        slices of every tensor whose scales changed.
+ * One pass over this rank's state while the scales hold (two for a tensor
+ * whose scales change), the one collective of the in-place halves, and
+ * every slice ends up bit for bit as fp8_adam_step over the whole tensor
+ * would leave it.  Arguments and errors as for fp8_adam_stats /
+ * fp8_adam_apply plus dest as for fp8_adam_step_into; both calls take the
+ * same chunks, dest, hparams and workspace.
+ */
+int fp8_adam_stats_into(const fp8_adam_chunk *chunks, const fp8_adam_dest *dest, int nchunks,
+                        const fp8_adam_hparams *hp, void *workspace, size_t ws_bytes, void *stream);
+int fp8_adam_apply_into(const fp8_adam_chunk *chunks, const fp8_adam_dest *dest, int nchunks,
+                        const fp8_adam_hparams *hp, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * fp8_adam_step_noalloc -- the same step as fp8_adam_step, for callers that
  * cannot hand the library any device memory of their own: code running under
  * a host framework whose caching allocator owns (and has already reserved)

@@ -173,6 +173,16 @@ def test_adam_step_into_rejects_missing_or_aliased_destinations(lib):
         assert fn(arr, dst, 1, ctypes.byref(hp), S, 64, None) == fp8.FP8_ERR_INVALID_ARG, d
     dst[0] = fp8._Dest(0x60008, 0x70000, 0x80000)
     assert fn(arr, dst, 1, ctypes.byref(hp), S, 64, None) == fp8.FP8_ERR_UNALIGNED
+    # the sharded halves: the same checks, and no tracked master amax
+    dst[0] = fp8._Dest(0x60000, 0x70000, 0x80000)
+    for name in ("fp8_adam_stats_into", "fp8_adam_apply_into"):
+        half = getattr(lib, name)
+        half.argtypes = fn.argtypes
+        assert half(arr, None, 1, ctypes.byref(hp), S, 64, None) == fp8.FP8_ERR_INVALID_ARG
+        arr[0] = fp8._Chunk(G, S, M, S, V, S, W, S, 64, S, None, None, None)
+        assert half(arr, dst, 1, ctypes.byref(hp), S, 64, None) == fp8.FP8_ERR_INVALID_ARG
+        arr[0] = fp8._Chunk(G, S, M, S, V, S, W, S, 64, None, None, None, None)
+        assert half(arr, dst, 1, ctypes.byref(hp), S, 32, None) == fp8.FP8_ERR_INVALID_ARG  # workspace
 
 
 def test_wait_selftest_rejects_limits_outside_its_range(lib):

@@ -163,3 +163,48 @@ def test_adam_into_rejects_bad_destinations():
     with pytest.raises(ValueError):
         fp8.fp8_adam_step_into(chunks, [], step=1, margin=0, workspace=ws, **HP)
     assert scalar().item() == 0.0  # the device is still usable
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 8])
+def test_adam_sharded_into_ranks_equal_whole_tensor_step(world):
+    """"FP8-LM", 提案手法 O3 out of place: ranks holding slices of every
+    tensor, run one after another on this GPU (stats_into on each, a max over
+    their workspaces, apply_into on each, then the buffer sets swap), end
+    with exactly the state, scales and E4M3 copy of the whole-tensor in-place
+    step, over three steps (step 1 redoes every tensor whose moments change
+    scale), through ShardedAdam's two halves (its step puts the collective
+    between them)."""
+    from fp8_mixed_precision_tensor_b200 import zero
+    from test_gpu_parity import _reduce_max_int32
+
+    sizes = [65536 + 5, 4099, 16, 300000]
+    ref = _with_tracking(make_adam_state(sizes, ("adam-shard-into",)), wq=True, track=False)
+    full = _clone(ref)
+    spare = [(torch.empty_like(c.m), torch.empty_like(c.v), torch.empty_like(c.w)) for c in full]
+    bounds = [[zero.shard_bounds(n, world, r) for n in sizes] for r in range(world)]
+    opts = [zero.ShardedAdam([zero.shard_chunk(c, lo, hi) for c, (lo, hi) in zip(full, bounds[r])],
+                             dests=[zero.shard_dest(d, lo, hi) for d, (lo, hi) in zip(spare, bounds[r])])
+            for r in range(world)]
+    ws_ref = torch.zeros(fp8.fp8_adam_workspace_bytes(len(sizes)) // 4, **F32)
+    sets = [[(c.m, c.v, c.w) for c in full], spare]
+    for step in (1, 2, 3):
+        fp8.fp8_adam_step(ref, step=step, margin=0, workspace=ws_ref, **HP)
+        for o in opts:
+            o.stats(t=step, margin=0, **HP)
+        _reduce_max_int32([o.workspace for o in opts])
+        for o in opts:
+            o.apply(t=step, margin=0, **HP)
+        assert fp8.fp8_get_status() == 0
+        new = sets[step % 2]  # the whole tensors behind this step's destination slices
+        for k, c in enumerate(ref):
+            s = snapshot(c)
+            m, v, w = new[k]
+            assert np.array_equal(m.cpu().numpy(), s["m"]), (step, k)
+            assert np.array_equal(v.cpu().numpy().view(np.uint16), s["v"]), (step, k)
+            assert np.array_equal(w.cpu().numpy().view(np.uint16), s["w"]), (step, k)
+            assert torch.equal(full[k].wq, c.wq)
+            for o in opts:
+                mine = o.current[k]
+                assert (mine.m_scale.item(), mine.v_scale.item(), mine.w_scale.item()) == \
+                    (s["s_m"], s["s_v"], s["s_w"]), (step, k)
+                assert (mine.wq_scale.item(), mine.wq_inv.item()) == (c.wq_scale.item(), c.wq_inv.item())

@@ -53,19 +53,21 @@ def _check_allreduce(scaling):
     assert fp8.fp8_get_status() == 0
 
 
-def _check_sharded_adam():
+def _check_sharded_adam(out_of_place=False):
     sizes = [65536 + 5, 4099]
     ref = make_adam_state(sizes, ("mod-zero",))
     mine = make_adam_state(sizes, ("mod-zero",))
-    opt = zero.ShardedAdam([zero.shard_chunk(c, 0, c.g.numel()) for c in mine])
+    dests = ([zero.shard_dest((torch.empty_like(c.m), torch.empty_like(c.v), torch.empty_like(c.w)), 0,
+                              c.g.numel()) for c in mine] if out_of_place else None)
+    opt = zero.ShardedAdam([zero.shard_chunk(c, 0, c.g.numel()) for c in mine], dests=dests)
     ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(ref)) // 4, dtype=torch.float32, device="cuda")
-    for step in (1, 2):
+    for step in (1, 2, 3):
         fp8.fp8_adam_step(ref, step=step, margin=0, workspace=ws, **HP)
         opt.step(t=step, margin=0, **HP)
-        for r, c, full in zip(ref, opt._keep, mine):
-            sr, sf = snapshot(r), snapshot(full)
+        for r, c in zip(ref, opt.current):
+            sr, sc = snapshot(r), snapshot(c)
             for k in ("m", "v", "w"):
-                assert np.array_equal(sr[k], sf[k]), (step, k)
+                assert np.array_equal(sr[k], sc[k]), (step, k)
             assert (c.m_scale.item(), c.v_scale.item(), c.w_scale.item()) == (sr["s_m"], sr["s_v"], sr["s_w"])
     assert fp8.fp8_get_status() == 0
 
@@ -75,10 +77,12 @@ def test_allreduce_module_without_process_group(scaling):
     _check_allreduce(scaling)
 
 
-def test_sharded_adam_module_without_process_group():
-    _check_sharded_adam()
+@pytest.mark.parametrize("out_of_place", [False, True])
+def test_sharded_adam_module_without_process_group(out_of_place):
+    _check_sharded_adam(out_of_place)
 
 
 def test_modules_inside_a_one_rank_nccl_group(nccl_one_rank):
     _check_allreduce("auto")
     _check_sharded_adam()
+    _check_sharded_adam(out_of_place=True)

@@ -155,6 +155,77 @@ def test_sharded_adam_over_gloo_equals_the_whole_tensor_step():
     mp.spawn(_sharded_worker, args=(2, _free_port()), nprocs=2)
 
 
+def _fake_stats_into(chunks, dests, lr, beta1, beta2, eps, t, margin, ws, stream=None):
+    _fake_stats(chunks, lr, beta1, beta2, eps, t, margin, ws)
+    for m, v, w in dests:  # the predicted-scale state: overwritten by the apply half here
+        m.fill_(0x55), v.fill_(0x55), w.fill_(0x55)
+
+
+def _fake_apply_into(chunks, dests, lr, beta1, beta2, eps, t, margin, ws, stream=None):
+    for i, (c, (m, v, w)) in enumerate(zip(chunks, dests)):
+        amax = tuple(float(x) for x in ws[i * WS_FLOATS:i * WS_FLOATS + 3])
+        out = oracle.adam_step(*_chunk_args(c), lr, beta1, beta2, eps, t, margin, amax_in=amax)
+        m.copy_(torch.from_numpy(out["mq"]))
+        v.copy_(torch.from_numpy(out["vh"].view(np.int16)))
+        w.copy_(torch.from_numpy(out["wh"].view(np.int16)))
+        c.m_scale.fill_(out["s_m"])
+        c.v_scale.fill_(out["s_v"])
+        c.w_scale.fill_(out["s_w"])
+
+
+def _sharded_into_worker(rank, world, port):
+    """The out-of-place halves: stats_into -> MAX reduce -> apply_into, then
+    the new buffers become the state and the old ones the next step's
+    destination (the inputs of a step are never its outputs)."""
+    _init(rank, world, port)
+    try:
+        fp8.pack_adam_chunks = lambda chunks: chunks
+        fp8.pack_adam_dests = lambda dests: dests
+        fp8.fp8_adam_workspace_bytes = lambda n: 4 * WS_FLOATS * n
+        fp8.fp8_adam_stats_into = _fake_stats_into
+        fp8.fp8_adam_apply_into = _fake_apply_into
+        states = [_stored_state(n, str(n)) for n in SIZES]
+        bounds = [zero.shard_bounds(n, world, rank) for n in SIZES]
+        mine = [_to_chunk(st, lo, hi) for st, (lo, hi) in zip(states, bounds)]
+        spare = [zero.shard_dest((torch.empty(n, dtype=torch.uint8), torch.empty(n, dtype=torch.int16),
+                                  torch.empty(n, dtype=torch.int16)), lo, hi)
+                 for n, (lo, hi) in zip(SIZES, bounds)]
+        opt = zero.ShardedAdam(mine, dests=spare)
+        whole = [list(st) for st in states]
+        for t in (1, 2, 3):
+            before = [(c.m, c.v, c.w) for c in opt.current]
+            opt.step(t=t, margin=0, **HP)
+            for k, st in enumerate(whole):
+                out = oracle.adam_step(*st, t=t, margin=0, **HP)
+                st[2], st[3], st[4], st[5], st[6], st[7] = (out["mq"], out["s_m"], out["vh"], out["s_v"],
+                                                            out["wh"], out["s_w"])
+                lo, hi = bounds[k]
+                c = opt.current[k]
+                assert all(a is not b for a, b in zip((c.m, c.v, c.w), before[k]))
+                assert all(a is b for a, b in zip(opt.spare[k], before[k]))
+                assert (c.m_scale.item(), c.v_scale.item(), c.w_scale.item()) == (out["s_m"], out["s_v"],
+                                                                                   out["s_w"])
+                assert np.array_equal(c.m.numpy(), out["mq"][lo:hi])
+                assert np.array_equal(c.v.numpy().view(np.uint16), out["vh"][lo:hi])
+                assert np.array_equal(c.w.numpy().view(np.uint16), out["wh"][lo:hi])
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_adam_out_of_place_over_gloo_equals_the_whole_tensor_step():
+    mp.spawn(_sharded_into_worker, args=(2, _free_port()), nprocs=2)
+
+
+def test_shard_dest_checks_its_slice():
+    bufs = (torch.empty(100, dtype=torch.uint8), torch.empty(100, dtype=torch.int16),
+            torch.empty(100, dtype=torch.int16))
+    assert [t.numel() for t in zero.shard_dest(bufs, 16, 48)] == [32, 32, 32]
+    with pytest.raises(ValueError):
+        zero.shard_dest(bufs, 8, 48)
+    with pytest.raises(ValueError):
+        zero.shard_dest(bufs, 96, 112)
+
+
 def test_sharded_adam_rejects_tracked_master_amax():
     st = _stored_state(64, "trk")
     c = _to_chunk(st, 0, 64)
