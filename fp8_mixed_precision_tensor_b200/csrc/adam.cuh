@@ -138,12 +138,44 @@ __device__ __forceinline__ AdamScalars adam_scalars(const AdamLaunch &L, float g
   return s;
 }
 
+// MUFU approximations (flush-to-zero) of the square root and the reciprocal.
+__device__ __forceinline__ float sqrt_approx(float x) {
+  float r;
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// The reciprocal rounded to nearest for the arguments the step gives it,
+// 2^-39 <= b <= 2^66 (the range of sqrt(v_hat) + eps) and +inf: the MUFU
+// approximation y and one Newton-Raphson correction y + y*e whose residual
+// e = 1 - b*y is formed in a fused multiply-add (P. Markstein, "Computation
+// of elementary functions on the IBM RISC System/6000 processor", IBM J.
+// Res. Develop. 34(1), 1990), without a branch; +inf is selected.  Bit for
+// bit CUDA's __frcp_rn on every binary32 argument of that range
+// (fp8_selftest_step_reciprocal checks all of them) and cheaper in the
+// update pass: 10 % at full clock, 15-20 % of the Adam step's time at the
+// power-capped clock of a training step.  (The same construction for the
+// square root needs a scaled residual and a final Tuckerman test to be
+// correctly rounded everywhere, and was slower than __fsqrt_rn.)
+__device__ __forceinline__ float rcp_rn_step(float b) {
+  const float y = rcp_approx(b);
+  const float e = __fmaf_rn(-b, y, 1.0f);
+  const float r = __fmaf_rn(e, y, y);
+  return b == __int_as_float(0x7f800000) ? 0.0f : r;
+}
+
 // The new moments and the master step dw = -lr m_hat / (sqrt(v_hat) + eps)
 // of two parameters, binary32, from decoded codes.  Every operation rounds to
-// nearest (the square root and the reciprocal are CUDA's correctly rounded
-// __fsqrt_rn / __frcp_rn, subnormals kept; the quotient is m times that
-// reciprocal, two roundings, 3 % faster in the update pass than __fdiv_rn;
-// 2^-39 <= eps <= 2^64 keeps the reciprocal a normal number), so the step's
+// nearest (the square root CUDA's correctly rounded __fsqrt_rn, subnormals
+// kept; the reciprocal correctly rounded by rcp_rn_step; the quotient is m
+// times that reciprocal, two roundings, 3 % faster in the update pass than a
+// correctly rounded division; 2^-39 <= eps <= 2^64 keeps the reciprocal a
+// normal number), so the step's
 // error is a fixed number of binary32 roundings:
 // |dw - dw_exact| <= 24 * 2^-24 * dw_abs, where
 // dw_abs is the step with |m| replaced by b1 |m0| + (1 - b1) |g| (which also
@@ -157,7 +189,7 @@ __device__ __forceinline__ void adam_moments(const AdamLaunch &L, float2 gd, flo
   v = __ffma2_rn(s.cv, vd, __fmul2_rn(__fmul2_rn(s.cgv, gd), __fmul2_rn(s.g_inv, gd)));
   const float2 vh = __fmul2_rn(v, both(L.inv_bc2));
   const float2 den = __fadd2_rn(make_float2(__fsqrt_rn(vh.x), __fsqrt_rn(vh.y)), both(L.eps));
-  dw = __fmul2_rn(both(L.neg_lr_bc1), __fmul2_rn(m, make_float2(__frcp_rn(den.x), __frcp_rn(den.y))));
+  dw = __fmul2_rn(both(L.neg_lr_bc1), __fmul2_rn(m, make_float2(rcp_rn_step(den.x), rcp_rn_step(den.y))));
 }
 
 // The same moments and an estimate of the step, with the MUFU square root and
@@ -169,16 +201,6 @@ __device__ __forceinline__ void adam_moments(const AdamLaunch &L, float2 gd, flo
 // because eps >= 2^-39 makes sqrt(v_hat) + eps round to eps for every
 // subnormal v_hat.  The update pass checks every scale decided this way
 // against the exact new amax.
-__device__ __forceinline__ float sqrt_approx(float x) {
-  float r;
-  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-  return r;
-}
-__device__ __forceinline__ float rcp_approx(float x) {
-  float r;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-  return r;
-}
 __device__ __forceinline__ void adam_moments_bound(const AdamLaunch &L, float2 gd, float2 md, float2 vd,
                                                    const AdamScalars &s, float2 &m, float2 &v, float2 &dw) {
   m = __ffma2_rn(s.cm, md, __fmul2_rn(s.cgm, gd));
@@ -673,6 +695,29 @@ __global__ void k_adam_finalize(const __grid_constant__ AdamLaunch L) {
         atomicOr(&g_status, FP8_STATUS_INTERNAL);
       if (C.w_amax != nullptr) *C.w_amax = __fmul_rn(ws[WS_STORED_W], 1.0f / ws[WS_NEW_W]);
     }
+  }
+}
+
+// Self-test of rcp_rn_step against CUDA's correctly rounded __frcp_rn on the
+// binary32 arguments with bit patterns in [lo, hi): counts the arguments
+// where the two differ (two NaNs agree) and keeps the smallest such pattern.
+__global__ void k_step_reciprocal_selftest(uint32_t lo, unsigned long long hi, unsigned long long *bad,
+                                           uint32_t *first) {
+  const unsigned long long stride = (unsigned long long)gridDim.x * blockDim.x;
+  unsigned long long nbad = 0;
+  uint32_t lowest = 0xffffffffu;
+  for (unsigned long long u = lo + (unsigned long long)blockIdx.x * blockDim.x + threadIdx.x; u < hi;
+       u += stride) {
+    const float x = __uint_as_float((uint32_t)u);
+    const float a = rcp_rn_step(x), b = __frcp_rn(x);
+    if (__float_as_uint(a) != __float_as_uint(b) && !(a != a && b != b)) {
+      nbad++;
+      lowest = min(lowest, (uint32_t)u);
+    }
+  }
+  if (nbad) {
+    atomicAdd(bad, nbad);
+    atomicMin(first, lowest);
   }
 }
 

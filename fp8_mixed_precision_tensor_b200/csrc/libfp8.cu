@@ -661,6 +661,17 @@ int fp8_selftest_wait_timeout(unsigned limit_us, void *stream) {
   return launch_rc();
 }
 
+int fp8_selftest_step_reciprocal(unsigned lo_bits, unsigned long long hi_bits, unsigned long long *bad_dev,
+                                 unsigned *first_dev, void *stream) {
+  if (hi_bits > 0x100000000ull || lo_bits >= hi_bits || !bad_dev || !first_dev) return FP8_ERR_INVALID_ARG;
+  DeviceInfo *d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  k_step_reciprocal_selftest<<<d->sms * 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(lo_bits, hi_bits,
+                                                                                        bad_dev, first_dev);
+  return launch_rc();
+}
+
 int fp8_get_status(unsigned *host_out, void *stream) {
   if (!host_out) return FP8_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

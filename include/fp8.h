@@ -459,6 +459,20 @@ int fp8_get_status(unsigned *host_out, void *stream);
  */
 int fp8_selftest_wait_timeout(unsigned limit_us, void *stream);
 
+/*
+ * fp8_selftest_step_reciprocal -- numerics self-test of the Adam step's own
+ * correctly rounded reciprocal, which the library computes without CUDA's
+ * __frcp_rn.  Compares the two on every binary32 argument whose bit pattern
+ * lies in [lo_bits, hi_bits) (hi_bits <= 2^32; the step's arguments are
+ * 2^-39 <= b <= 2^66 and +inf, where they must agree).  Two NaNs agree.
+ * Adds the number of arguments that differ to *bad_dev (dev, one uint64)
+ * and lowers *first_dev (dev, one uint32) to the smallest such bit pattern;
+ * the caller initialises both.  FP8_ERR_INVALID_ARG for an empty or too wide
+ * range or NULL outputs.
+ */
+int fp8_selftest_step_reciprocal(unsigned lo_bits, unsigned long long hi_bits, unsigned long long *bad_dev,
+                                 unsigned *first_dev, void *stream);
+
 /* Human-readable message of a status code (static string). */
 const char *fp8_strerror(int code);
 

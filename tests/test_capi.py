@@ -185,6 +185,15 @@ def test_adam_step_into_rejects_missing_or_aliased_destinations(lib):
         assert half(arr, dst, 1, ctypes.byref(hp), S, 32, None) == fp8.FP8_ERR_INVALID_ARG  # workspace
 
 
+def test_reciprocal_selftest_rejects_bad_arguments_on_the_host(lib):
+    fn = lib.fp8_selftest_step_reciprocal
+    fn.argtypes = [ctypes.c_uint, ctypes.c_ulonglong, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    fake = 0x10000
+    assert fn(16, 16, fake, fake, None) == 1           # empty range
+    assert fn(0, (1 << 32) + 1, fake, fake, None) == 1  # beyond the 2^32 patterns
+    assert fn(0, 16, None, fake, None) == 1            # no counter
+
+
 def test_wait_selftest_rejects_limits_outside_its_range(lib):
     lib.fp8_selftest_wait_timeout.argtypes = [ctypes.c_uint, ctypes.c_void_p]
     assert lib.fp8_selftest_wait_timeout(0, None) == 1
