@@ -6,7 +6,8 @@ block's four linears.  The default workload is the GPT-175B block (tokens
 12288->12288, FFN 12288->49152->12288); `--workload gpt7b_block` runs the
 GPT-7B block (tokens 4096, hidden 4096).  Per step:
 
-  for each linear:  amax + fused scale/cast of X (E4M3) and dY (E5M2, mu-scaled)
+  for each linear:  amax + scale + cast of X (E4M3) and dY (E5M2, mu-scaled), one
+                    pass over each while its scale holds
                     fwd   Y  = Xq Wq^T     (bf16 out, fused next-amax)
                     dgrad dX = dYq Wq      (bf16 out, fused next-amax)
                     wgrad dW = dYq^T Xq    (bf16 rounded to odd, fused amax)
@@ -72,7 +73,7 @@ WORKLOADS = {
 MU = 2.0 ** 10
 HP = dict(lr=1e-4, beta1=0.9, beta2=0.95, eps=1e-8)
 # Algorithmic bytes per element / parameter (reads + writes of the definition).
-CAST_BYTES_BF16 = 2 + 2 + 1   # amax read + cast read + code write
+CAST_BYTES_BF16 = 2 + 1       # x read once + code written (amax and cast in one pass while the scale holds)
 GRAD_CAST_BYTES = 2 + 1       # round-to-odd bf16 dW read (amax fused in the GEMM) + code write
 ADAM_BYTES = 11               # read g1 m1 v2 w2, write m1 v2 w2
 
@@ -281,12 +282,13 @@ class BlockStep:
         self.flops = sum(3 * 2 * d["M"] * d["N"] * d["K"] for d in self.L)
         self.cast_elems = sum(d["M"] * d["K"] + d["M"] * d["N"] for d in self.L)
         self.params = sum(d["N"] * d["K"] for d in self.L)
-        # per linear: (amax, scale+cast) x2, 3 GEMMs, grad scale+cast; Adam out of
-        # place: update, finalize, redo, finalize; in place with a tracked master:
-        # stats, finalize 1, exact-master pass, finalize 2, update, finalize 3
+        # per linear: (amax+cast pass, redo, scale) x2, 3 GEMMs, grad scale+cast;
+        # Adam out of place: update, finalize, redo, finalize; in place with a
+        # tracked master: stats, finalize 1, exact-master pass, finalize 2,
+        # update, finalize 3
         na = 4 if adam == "into" else 6
-        self.launches_per_step = 4 * (2 * 2 + 3 + 1) + na
-        self.launches_per_step_overlapped = 4 * (2 * 2 + 3 + 1 + na)
+        self.launches_per_step = 4 * (2 * 3 + 3 + 1) + na
+        self.launches_per_step_overlapped = 4 * (2 * 3 + 3 + 1 + na)
 
     def adam_step(self, pack, t, ws):
         """Adam step t over the tensors of one packed (chunks, dests) pair."""
@@ -297,9 +299,9 @@ class BlockStep:
             self.fp8.fp8_adam_step(chunks, step=t, margin=0, workspace=ws, **HP)
 
     def quantise(self, x, fmt, sc, i, mu=1.0, out=None):
-        fp8 = self.fp8
-        fp8.fp8_amax(x, sc[i:i + 1])
-        fp8.fp8_scale_cast(x, fmt, sc[i:i + 1], 0, mu, sc[i + 1:i + 2], sc[i + 2:i + 3], out)
+        """amax, scale and cast of x in one call: one pass over x while the
+        scale (sc[i + 1], the previous step's) holds."""
+        self.fp8.fp8_amax_scale_cast(x, fmt, sc[i:i + 1], 0, mu, sc[i + 1:i + 2], sc[i + 2:i + 3], out)
 
     def step(self, ev=None):
         """Enqueue one step on the current stream.  ev: optional dict name ->

@@ -275,4 +275,93 @@ __global__ void __launch_bounds__(kStreamThreads) k_cast(const void *__restrict_
   }
 }
 
+// ---------------------------------------------------------------------------
+// amax and cast in one pass over x.  The cast uses a predicted scale -- the
+// tensor's previous one, which per-tensor scales of activations and
+// gradients keep from step to step unless the amax crosses a power of two --
+// while the pass reduces the tensor's own amax; k_cast_redo then compares
+// the scale of that amax with the prediction and, only where they differ,
+// casts the tensor again with it (every block takes the same decision and
+// returns at once when the prediction held).  k_compute_scale publishes the
+// scale last, so no block of the redo reads a half-updated prediction.  The
+// codes, amax and scales are those of k_amax followed by the fused
+// scale + cast, bit for bit; the tensor is read once instead of twice when
+// the prediction holds.
+template <int DT, int FMT>
+__device__ __forceinline__ uint32_t amax_cast_group(const void *x, size_t g, float s, void *q) {
+  float f[16];
+  load16<DT>(x, g, f);
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < 16; j++) {
+    m = max(m, absbits_f32(f[j]));
+    f[j] *= s;
+  }
+  if constexpr (FMT == FP8_F16S) {
+    uint4 lo = make_uint4(f16x2(f[0], f[1]), f16x2(f[2], f[3]), f16x2(f[4], f[5]), f16x2(f[6], f[7]));
+    uint4 hi = make_uint4(f16x2(f[8], f[9]), f16x2(f[10], f[11]), f16x2(f[12], f[13]), f16x2(f[14], f[15]));
+    uint4 *p = reinterpret_cast<uint4 *>(q) + g * 2;
+    __stcs(p, lo);
+    __stcs(p + 1, hi);
+  } else {
+    uint4 o = make_uint4(enc4<FMT>(f[0], f[1], f[2], f[3]), enc4<FMT>(f[4], f[5], f[6], f[7]),
+                         enc4<FMT>(f[8], f[9], f[10], f[11]), enc4<FMT>(f[12], f[13], f[14], f[15]));
+    __stcs(reinterpret_cast<uint4 *>(q) + g, o);
+  }
+  return m;
+}
+
+// One element of the ragged tail, cast as k_cast casts it.
+template <int FMT>
+__device__ __forceinline__ void cast_one(float y, void *q, size_t i) {
+  if constexpr (FMT == FP8_F16S)
+    reinterpret_cast<uint16_t *>(q)[i] = __half_as_ushort(__float2half_rn(y));
+  else
+    reinterpret_cast<uint8_t *>(q)[i] = (uint8_t)(enc2<FMT>(y, 0.0f) & 0xffu);
+}
+
+template <int DT, int FMT>
+__global__ void __launch_bounds__(kStreamThreads) k_amax_cast(const void *__restrict__ x, size_t n,
+                                                              const float *__restrict__ pred,
+                                                              float *__restrict__ amax, void *__restrict__ q) {
+  __shared__ uint32_t red[32];
+  const float s = *pred;
+  const size_t groups = n / 16;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  uint32_t m0 = 0, m1 = 0;
+  for (; g + stride < groups; g += 2 * stride) {
+    m0 = max(m0, amax_cast_group<DT, FMT>(x, g, s, q));
+    m1 = max(m1, amax_cast_group<DT, FMT>(x, g + stride, s, q));
+  }
+  if (g < groups) m0 = max(m0, amax_cast_group<DT, FMT>(x, g, s, q));
+  uint32_t m = max(m0, m1);
+  if (blockIdx.x == 0) {  // ragged tail (< 16 elements)
+    for (size_t i = groups * 16 + threadIdx.x; i < n; i += blockDim.x) {
+      const float xi = load1<DT>(x, i);
+      m = max(m, absbits_f32(xi));
+      cast_one<FMT>(xi * s, q, i);
+    }
+  }
+  m = block_max_u32(m, red);
+  if (threadIdx.x == 0) atomic_max_bits(amax, m);
+}
+
+template <int DT, int FMT>
+__global__ void __launch_bounds__(kStreamThreads) k_cast_redo(const void *__restrict__ x, size_t n,
+                                                              const float *__restrict__ pred,
+                                                              const float *__restrict__ amax, float fmax,
+                                                              int margin, int log2mu, void *__restrict__ q) {
+  int k;
+  scale_exponent(*amax, fmax, margin, log2mu, k);
+  const float s = pow2f(k);
+  if (s == *pred) return;  // the same for every block: the pass already cast with s
+  const size_t groups = n / 16;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x; g < groups; g += stride)
+    cast_group<DT, FMT>(x, g, s, q);
+  if (blockIdx.x == 0)
+    for (size_t i = groups * 16 + threadIdx.x; i < n; i += blockDim.x) cast_one<FMT>(load1<DT>(x, i) * s, q, i);
+}
+
 }  // namespace fp8lib

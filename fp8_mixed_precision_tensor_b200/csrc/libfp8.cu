@@ -304,6 +304,28 @@ int cast_common(const void *x, int dtype, size_t n, int fmt, const CastScale &cs
   return launch_rc();
 }
 
+// The one-pass amax + cast: the pass with the predicted scale, the redo
+// where the scale of the amax differs, then the scale published.
+template <int DT, int FMT>
+void launch_amax_cast(const void *x, size_t n, float *amax, int margin, int log2mu, float *scale, float *inv,
+                      void *q, cudaStream_t s, int sms) {
+  const unsigned grid = grid_for(n / 16, kStreamThreads * 2, sms * 8);
+  const float fmax = FMT == FP8_E4M3 ? 448.0f : (FMT == FP8_E5M2 ? 57344.0f : 65504.0f);
+  if (n > 0) {
+    k_amax_cast<DT, FMT><<<grid, kStreamThreads, 0, s>>>(x, n, scale, amax, q);
+    k_cast_redo<DT, FMT><<<grid, kStreamThreads, 0, s>>>(x, n, scale, amax, fmax, margin, log2mu, q);
+  }
+  k_compute_scale<<<1, 1, 0, s>>>(amax, fmax, margin, log2mu, scale, inv);
+}
+
+template <int DT>
+void launch_amax_cast_dt(int fmt, const void *x, size_t n, float *amax, int margin, int log2mu, float *scale,
+                         float *inv, void *q, cudaStream_t s, int sms) {
+  if (fmt == FP8_E4M3) launch_amax_cast<DT, FP8_E4M3>(x, n, amax, margin, log2mu, scale, inv, q, s, sms);
+  else if (fmt == FP8_E5M2) launch_amax_cast<DT, FP8_E5M2>(x, n, amax, margin, log2mu, scale, inv, q, s, sms);
+  else launch_amax_cast<DT, FP8_F16S>(x, n, amax, margin, log2mu, scale, inv, q, s, sms);
+}
+
 // mu must be a power of two in [2^-32, 2^32]; its log2 on success.
 bool mu_log2(float mu, int *log2mu) {
   int e2;
@@ -420,6 +442,28 @@ int fp8_scale_cast(const void *x, int dtype, size_t n, int fmt, const float *ama
   if (n > 0 && (!aligned16(x) || !aligned16(q))) return FP8_ERR_UNALIGNED;
   CastScale cs = {nullptr, amax_dev, fmt_max_of(fmt), margin, log2mu, scale_dev, inv_scale_dev, nullptr};
   return cast_common(x, dtype, n, fmt, cs, q, static_cast<cudaStream_t>(stream));
+}
+
+int fp8_amax_scale_cast(const void *x, int dtype, size_t n, int fmt, float *amax_dev, int margin, float mu,
+                        float *scale_dev, float *inv_scale_dev, void *q, void *stream) {
+  int log2mu;
+  if (!valid_dtype(dtype) || !valid_fmt(fmt) || !amax_dev || !scale_dev || !inv_scale_dev)
+    return FP8_ERR_INVALID_ARG;
+  if (margin < 0 || margin > 64 || !mu_log2(mu, &log2mu)) return FP8_ERR_INVALID_ARG;
+  if (n > 0 && (!x || !q)) return FP8_ERR_INVALID_ARG;
+  if (n > 0 && (!aligned16(x) || !aligned16(q))) return FP8_ERR_UNALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int rc = cuda_rc(cudaMemsetAsync(amax_dev, 0, sizeof(float), s));
+  if (rc) return rc;
+  DeviceInfo *d;
+  if ((rc = device_info(&d))) return rc;
+  if (dtype == FP8_DT_F32)
+    launch_amax_cast_dt<FP8_DT_F32>(fmt, x, n, amax_dev, margin, log2mu, scale_dev, inv_scale_dev, q, s, d->sms);
+  else if (dtype == FP8_DT_BF16)
+    launch_amax_cast_dt<FP8_DT_BF16>(fmt, x, n, amax_dev, margin, log2mu, scale_dev, inv_scale_dev, q, s, d->sms);
+  else
+    launch_amax_cast_dt<FP8_DT_F16>(fmt, x, n, amax_dev, margin, log2mu, scale_dev, inv_scale_dev, q, s, d->sms);
+  return launch_rc();
 }
 
 int fp8_linear_fwd(const uint8_t *xq, const float *x_inv, const uint8_t *wq, const float *w_inv,

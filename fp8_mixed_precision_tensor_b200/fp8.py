@@ -28,7 +28,8 @@ FP8_E4M3, FP8_E5M2, FP8_F16S = 0, 1, 2
 
 _DT = {torch.float32: FP8_DT_F32, torch.bfloat16: FP8_DT_BF16, torch.float16: FP8_DT_F16}
 
-SYMBOLS = ("fp8_amax", "fp8_compute_scale", "fp8_cast", "fp8_scale_cast", "fp8_cast_count", "fp8_grad_cast",
+SYMBOLS = ("fp8_amax", "fp8_compute_scale", "fp8_cast", "fp8_scale_cast", "fp8_amax_scale_cast", "fp8_cast_count",
+           "fp8_grad_cast",
            "fp8_sum_codes", "fp8_mu_update", "fp8_linear_fwd", "fp8_linear_dgrad",
            "fp8_linear_wgrad", "fp8_adam_workspace_bytes", "fp8_adam_step", "fp8_adam_stats",
            "fp8_adam_apply", "fp8_adam_step_noalloc", "fp8_adam_step_into", "fp8_adam_stats_into",
@@ -80,6 +81,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fp8_compute_scale.argtypes = [p, i, i, f, p, p, p]
     lib.fp8_cast.argtypes = [p, i, sz, i, p, p, p]
     lib.fp8_scale_cast.argtypes = [p, i, sz, i, p, i, f, p, p, p, p]
+    lib.fp8_amax_scale_cast.argtypes = [p, i, sz, i, p, i, f, p, p, p, p]
     lib.fp8_cast_count.argtypes = [p, i, sz, i, p, p, p, p]
     lib.fp8_grad_cast.argtypes = [p, i, sz, i, p, i, p, p, p, p, p, p]
     lib.fp8_sum_codes.argtypes = [p, i, sz, sz, i, p, p, p, p, p]
@@ -154,6 +156,17 @@ def fp8_scale_cast(x: torch.Tensor, fmt: int, amax: torch.Tensor, margin: int, m
     _check(load_library().fp8_scale_cast(_ptr(x), _DT[x.dtype], x.numel(), fmt, _ptr(amax), margin, mu,
                                          _ptr(scale_out), _ptr(inv_scale_out), _ptr(q_out),
                                          _stream(stream)), "fp8_scale_cast")
+
+
+def fp8_amax_scale_cast(x: torch.Tensor, fmt: int, amax_out: torch.Tensor, margin: int, mu: float,
+                        scale: torch.Tensor, inv_scale_out: torch.Tensor, q_out: torch.Tensor,
+                        stream=None) -> None:
+    """fp8_amax + fp8_scale_cast in one pass over x when the scale holds:
+    `scale` holds the predicted scale on entry (the tensor's previous one) and
+    the new scale on return."""
+    _check(load_library().fp8_amax_scale_cast(_ptr(x), _DT[x.dtype], x.numel(), fmt, _ptr(amax_out), margin, mu,
+                                              _ptr(scale), _ptr(inv_scale_out), _ptr(q_out), _stream(stream)),
+           "fp8_amax_scale_cast")
 
 
 # ---------------------------------------------------------------- scaling variants, FP8 all-reduce

@@ -133,6 +133,24 @@ int fp8_scale_cast(const void *x, int dtype, size_t n, int fmt, const float *ama
                    float mu, float *scale_dev, float *inv_scale_dev, void *q, void *stream);
 
 /*
+ * fp8_amax_scale_cast -- fp8_amax, then fp8_scale_cast on that amax (same
+ * definitions, bit for bit the same amax, scales and codes), reading x once
+ * when the scale does not change: *scale_dev holds a predicted scale on entry
+ * (the tensor's scale from its previous step; any float), x is cast with it
+ * while its amax is reduced, and x is cast a second time, with the scale of
+ * the amax, only if that scale differs from the prediction.  Per-tensor
+ * scales of activations and gradients change only when the amax crosses a
+ * power of two, so most steps take the single pass: 3 instead of 5 bytes of
+ * HBM traffic per bf16 element.
+ *   amax_dev       dev, one float (out)
+ *   scale_dev      dev, one float: the prediction (in), the new scale (out)
+ *   inv_scale_dev  dev, one float (out)
+ * Other arguments and errors as fp8_scale_cast.
+ */
+int fp8_amax_scale_cast(const void *x, int dtype, size_t n, int fmt, float *amax_dev, int margin, float mu,
+                        float *scale_dev, float *inv_scale_dev, void *q, void *stream);
+
+/*
  * fp8_cast_count -- fp8_cast plus its underflow and overflow counts, the
  * measure by which [FP8-LM] アブレーション研究 compares scaling variants
  * (and [FP8-AMAX] 실험 결과, RQ3, dynamic against constant scaling): an

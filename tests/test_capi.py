@@ -98,6 +98,10 @@ def test_host_side_validation_of_the_next_rows(lib):
     reject bad arguments on the host, before any device work."""
     p, i, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
     fake = 0x10000
+    lib.fp8_amax_scale_cast.argtypes = [p, i, sz, i, p, i, f, p, p, p, p]
+    assert lib.fp8_amax_scale_cast(fake, 1, 32, 0, fake, 0, 3.0, fake, fake, fake, None) == 1   # mu
+    assert lib.fp8_amax_scale_cast(fake, 1, 32, 0, None, 0, 1.0, fake, fake, fake, None) == 1   # no amax
+    assert lib.fp8_amax_scale_cast(fake + 8, 1, 32, 0, fake, 0, 1.0, fake, fake, fake, None) == 2  # unaligned
     lib.fp8_cast_count.argtypes = [p, i, sz, i, p, p, p, p]
     assert lib.fp8_cast_count(fake, 1, 32, 0, fake, fake, None, None) == 1       # no counters
     lib.fp8_grad_cast.argtypes = [p, i, sz, i, p, i, p, p, p, p, p, p]

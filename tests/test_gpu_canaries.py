@@ -67,7 +67,13 @@ def test_amax_scale_cast_family_writes_only_its_outputs(dtype, n):
         fp8.fp8_cast(x, fmt, s.t, q.t)
         s2, inv2, q2 = _f32(), _f32(), Guarded(n, qdt)
         fp8.fp8_scale_cast(x, fmt, amax.t, 1, 2.0 ** 4, s2.t, inv2.t, q2.t)
-        _all_intact(amax=amax, s=s, inv=inv, q=q, s2=s2, inv2=inv2, q2=q2)
+        a5, s5, inv5, q5 = _f32(), _f32(1, torch.tensor([0.5])), _f32(), Guarded(n, qdt)
+        fp8.fp8_amax_scale_cast(x, fmt, a5.t, 0, 1.0, s5.t, inv5.t, q5.t)  # a wrong prediction: the redo runs
+        a6, s6, inv6, q6 = _f32(), _f32(1, s5.t.cpu()), _f32(), Guarded(n, qdt)
+        fp8.fp8_amax_scale_cast(x, fmt, a6.t, 0, 1.0, s6.t, inv6.t, q6.t)  # the right one: one pass
+        _all_intact(amax=amax, s=s, inv=inv, q=q, s2=s2, inv2=inv2, q2=q2, a5=a5, s5=s5, inv5=inv5, q5=q5,
+                    a6=a6, s6=s6, inv6=inv6, q6=q6)
+        assert torch.equal(q5.t, q.t) and torch.equal(q6.t, q.t)
         if fmt != fp8.FP8_F16S:
             q3, counts = Guarded(n, torch.uint8), Guarded(2, torch.int64, torch.zeros(2, dtype=torch.int64))
             fp8.fp8_cast_count(x, fmt, s.t, q3.t, counts.t)
