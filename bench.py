@@ -97,18 +97,32 @@ def config_of(wl: dict, schedule: str, world: int, adam: str = "into") -> dict:
             "parallelism": f"replicas{world}" if world > 1 else "single"}
 
 
+def gemm_source_digest() -> str | None:
+    """sha256 of what decides the GEMM's DRAM traffic: the kernel sources
+    (gemm.cuh, pipeline.cuh) and the library's GEMM launch set-up (the text
+    of libfp8.cu from its tensor-map builder to the end of run_gemm, which
+    picks the kernel, the tiles and the tile order).  None when that text
+    cannot be found."""
+    import hashlib
+
+    csrc = os.path.join(ROOT, "fp8_mixed_precision_tensor_b200", "csrc")
+    lib = open(os.path.join(csrc, "libfp8.cu"), "rb").read()
+    lo, hi = lib.find(b"int make_map("), lib.find(b"void launch_amax(")
+    if lo < 0 or hi < lo:
+        return None
+    src = b"".join(open(os.path.join(csrc, f), "rb").read() for f in ("gemm.cuh", "pipeline.cuh")) + lib[lo:hi]
+    return hashlib.sha256(src).hexdigest()
+
+
 def gemm_traffic(workload: str):
     """Mean DRAM bytes per GEMM launch of this step from the committed ncu
     capture, valid while the GEMM kernel source and its launch set-up (tile
     order) are the ones that were measured and the capture is of this
     workload."""
-    import hashlib
-
     try:
         rec = json.load(open(os.path.join(ROOT, "profiles", "gemm_step_traffic.json")))
-        csrc = os.path.join(ROOT, "fp8_mixed_precision_tensor_b200", "csrc")
-        src = b"".join(open(os.path.join(csrc, f), "rb").read() for f in ("gemm.cuh", "libfp8.cu"))
-        if hashlib.sha256(src).hexdigest() == rec["gemm_source_sha256"] and rec.get("workload") == workload:
+        digest = gemm_source_digest()
+        if digest is not None and digest == rec["gemm_source_sha256"] and rec.get("workload") == workload:
             return rec["dram_bytes_per_launch_mean"]
     except Exception:
         pass
