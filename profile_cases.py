@@ -1,7 +1,7 @@
 """Run one kernel family of the hot path on a chosen case (for profilers).
 
     python profile_cases.py linear --M 4096 --N 16384 --K 4096 [--rto]
-    python profile_cases.py cast --n 268435456
+    python profile_cases.py cast --n 268435456 [--onepass]
     python profile_cases.py castsweep
     python profile_cases.py adam --n 67108864 [--track] [--into]
     python profile_cases.py allreduce --n 268435456 --world 8
@@ -76,8 +76,11 @@ def case_cast(a):
     sc = _scalars(3)
 
     def one():
-        fp8.fp8_amax(x, sc[0:1])
-        fp8.fp8_scale_cast(x, fp8.FP8_E4M3, sc[0:1], 0, 1.0, sc[1:2], sc[2:3], q)
+        if a.onepass:  # amax, scale and cast reading x once (the scale of the previous pass as the guess)
+            fp8.fp8_amax_scale_cast(x, fp8.FP8_E4M3, sc[0:1], 0, 1.0, sc[1:2], sc[2:3], q)
+        else:
+            fp8.fp8_amax(x, sc[0:1])
+            fp8.fp8_scale_cast(x, fp8.FP8_E4M3, sc[0:1], 0, 1.0, sc[1:2], sc[2:3], q)
 
     return one
 
@@ -273,6 +276,7 @@ def main():
                     help="passes run before the timed ones besides the one warm-up pass (adam: steps "
                          "after which the moments' scales have settled)")
     ap.add_argument("--rto", action="store_true", help="linear: dW as bfloat16 rounded to odd")
+    ap.add_argument("--onepass", action="store_true", help="cast: amax, scale and cast in one call")
     a = ap.parse_args()
     one = {"linear": case_linear, "cast": case_cast, "castsweep": case_castsweep, "adam": case_adam,
            "allreduce": case_allreduce,
