@@ -32,6 +32,7 @@ struct DeviceInfo {
   int adam_bound_blocks_per_sm = 1;  // of the estimated stats pass of tracking chunks
   int adam_est_blocks_per_sm = 1;    // of the estimated stats pass of the other chunks
   int adam_into_blocks_per_sm = 1;   // of the out-of-place update (and its redo)
+  int cast_blocks_per_sm = 8;        // resident blocks of the streaming cast kernels
   int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair GEMM
   int wide_clusters = 0;  // co-resident 2-CTA clusters of the wide pair GEMM
 };
@@ -87,6 +88,24 @@ int device_info(DeviceInfo **out) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k_adam<6>, kAdamThreads, 0) != cudaSuccess)
       return FP8_ERR_CUDA;
     d.adam_into_blocks_per_sm = bps > 0 ? bps : 1;
+    // the cast kernels' grids are one wave of resident blocks (a grid-stride
+    // loop gives each block an equal share; a partial second wave would run
+    // a third of the work on a few SMs): the fewest resident blocks of the
+    // instantiations the training step runs
+    {
+      int lo = 8;
+      const void *casts[] = {(const void *)k_cast<FP8_DT_BF16, FP8_E4M3, false>,
+                             (const void *)k_cast<FP8_DT_BF16, FP8_E5M2, false>,
+                             (const void *)k_amax_cast<FP8_DT_BF16, FP8_E4M3>,
+                             (const void *)k_amax_cast<FP8_DT_BF16, FP8_E5M2>,
+                             (const void *)k_cast_redo<FP8_DT_BF16, FP8_E4M3>};
+      for (const void *k : casts) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k, kStreamThreads, 0) != cudaSuccess)
+          return FP8_ERR_CUDA;
+        if (bps > 0 && bps < lo) lo = bps;
+      }
+      d.cast_blocks_per_sm = lo;
+    }
     int rc = FP8_OK;
     rc |= set_smem(gemm::k_gemm<256, false, false>, gemm::Cfg<256>::SMEM_BYTES);
     rc |= set_smem(gemm::k_gemm<256, false, true>, gemm::Cfg<256>::SMEM_BYTES);
@@ -279,18 +298,18 @@ void launch_amax(const void *x, size_t n, float *amax, cudaStream_t s, int sms) 
 
 template <int DT, int FMT>
 void launch_cast(const void *x, size_t n, const CastScale &cs, void *q, unsigned long long *counts,
-                 cudaStream_t s, int sms) {
-  unsigned grid = grid_for(n / 16, kStreamThreads * 2, sms * 8);
+                 cudaStream_t s, int max_blocks) {
+  unsigned grid = grid_for(n / 16, kStreamThreads * 2, max_blocks);
   if (counts) k_cast<DT, FMT, true><<<grid, kStreamThreads, 0, s>>>(x, n, cs, q, counts);
   else k_cast<DT, FMT, false><<<grid, kStreamThreads, 0, s>>>(x, n, cs, q, nullptr);
 }
 
 template <int DT>
 void launch_cast_dt(int fmt, const void *x, size_t n, const CastScale &cs, void *q, unsigned long long *counts,
-                    cudaStream_t s, int sms) {
-  if (fmt == FP8_E4M3) launch_cast<DT, FP8_E4M3>(x, n, cs, q, counts, s, sms);
-  else if (fmt == FP8_E5M2) launch_cast<DT, FP8_E5M2>(x, n, cs, q, counts, s, sms);
-  else launch_cast<DT, FP8_F16S>(x, n, cs, q, counts, s, sms);
+                    cudaStream_t s, int max_blocks) {
+  if (fmt == FP8_E4M3) launch_cast<DT, FP8_E4M3>(x, n, cs, q, counts, s, max_blocks);
+  else if (fmt == FP8_E5M2) launch_cast<DT, FP8_E5M2>(x, n, cs, q, counts, s, max_blocks);
+  else launch_cast<DT, FP8_F16S>(x, n, cs, q, counts, s, max_blocks);
 }
 
 int cast_common(const void *x, int dtype, size_t n, int fmt, const CastScale &cs, void *q, cudaStream_t s,
@@ -298,9 +317,10 @@ int cast_common(const void *x, int dtype, size_t n, int fmt, const CastScale &cs
   DeviceInfo *d;
   int rc = device_info(&d);
   if (rc) return rc;
-  if (dtype == FP8_DT_F32) launch_cast_dt<FP8_DT_F32>(fmt, x, n, cs, q, counts, s, d->sms);
-  else if (dtype == FP8_DT_BF16) launch_cast_dt<FP8_DT_BF16>(fmt, x, n, cs, q, counts, s, d->sms);
-  else launch_cast_dt<FP8_DT_F16>(fmt, x, n, cs, q, counts, s, d->sms);
+  const int cap = d->sms * d->cast_blocks_per_sm;  // one wave of resident blocks
+  if (dtype == FP8_DT_F32) launch_cast_dt<FP8_DT_F32>(fmt, x, n, cs, q, counts, s, cap);
+  else if (dtype == FP8_DT_BF16) launch_cast_dt<FP8_DT_BF16>(fmt, x, n, cs, q, counts, s, cap);
+  else launch_cast_dt<FP8_DT_F16>(fmt, x, n, cs, q, counts, s, cap);
   return launch_rc();
 }
 
@@ -308,8 +328,8 @@ int cast_common(const void *x, int dtype, size_t n, int fmt, const CastScale &cs
 // where the scale of the amax differs, then the scale published.
 template <int DT, int FMT>
 void launch_amax_cast(const void *x, size_t n, float *amax, int margin, int log2mu, float *scale, float *inv,
-                      void *q, cudaStream_t s, int sms) {
-  const unsigned grid = grid_for(n / 16, kStreamThreads * 2, sms * 8);
+                      void *q, cudaStream_t s, int max_blocks) {
+  const unsigned grid = grid_for(n / 16, kStreamThreads * 2, max_blocks);
   const float fmax = FMT == FP8_E4M3 ? 448.0f : (FMT == FP8_E5M2 ? 57344.0f : 65504.0f);
   if (n > 0) {
     k_amax_cast<DT, FMT><<<grid, kStreamThreads, 0, s>>>(x, n, scale, amax, q);
@@ -320,10 +340,10 @@ void launch_amax_cast(const void *x, size_t n, float *amax, int margin, int log2
 
 template <int DT>
 void launch_amax_cast_dt(int fmt, const void *x, size_t n, float *amax, int margin, int log2mu, float *scale,
-                         float *inv, void *q, cudaStream_t s, int sms) {
-  if (fmt == FP8_E4M3) launch_amax_cast<DT, FP8_E4M3>(x, n, amax, margin, log2mu, scale, inv, q, s, sms);
-  else if (fmt == FP8_E5M2) launch_amax_cast<DT, FP8_E5M2>(x, n, amax, margin, log2mu, scale, inv, q, s, sms);
-  else launch_amax_cast<DT, FP8_F16S>(x, n, amax, margin, log2mu, scale, inv, q, s, sms);
+                         float *inv, void *q, cudaStream_t s, int max_blocks) {
+  if (fmt == FP8_E4M3) launch_amax_cast<DT, FP8_E4M3>(x, n, amax, margin, log2mu, scale, inv, q, s, max_blocks);
+  else if (fmt == FP8_E5M2) launch_amax_cast<DT, FP8_E5M2>(x, n, amax, margin, log2mu, scale, inv, q, s, max_blocks);
+  else launch_amax_cast<DT, FP8_F16S>(x, n, amax, margin, log2mu, scale, inv, q, s, max_blocks);
 }
 
 // mu must be a power of two in [2^-32, 2^32]; its log2 on success.
@@ -457,12 +477,13 @@ int fp8_amax_scale_cast(const void *x, int dtype, size_t n, int fmt, float *amax
   if (rc) return rc;
   DeviceInfo *d;
   if ((rc = device_info(&d))) return rc;
+  const int cap = d->sms * d->cast_blocks_per_sm;  // one wave of resident blocks
   if (dtype == FP8_DT_F32)
-    launch_amax_cast_dt<FP8_DT_F32>(fmt, x, n, amax_dev, margin, log2mu, scale_dev, inv_scale_dev, q, s, d->sms);
+    launch_amax_cast_dt<FP8_DT_F32>(fmt, x, n, amax_dev, margin, log2mu, scale_dev, inv_scale_dev, q, s, cap);
   else if (dtype == FP8_DT_BF16)
-    launch_amax_cast_dt<FP8_DT_BF16>(fmt, x, n, amax_dev, margin, log2mu, scale_dev, inv_scale_dev, q, s, d->sms);
+    launch_amax_cast_dt<FP8_DT_BF16>(fmt, x, n, amax_dev, margin, log2mu, scale_dev, inv_scale_dev, q, s, cap);
   else
-    launch_amax_cast_dt<FP8_DT_F16>(fmt, x, n, amax_dev, margin, log2mu, scale_dev, inv_scale_dev, q, s, d->sms);
+    launch_amax_cast_dt<FP8_DT_F16>(fmt, x, n, amax_dev, margin, log2mu, scale_dev, inv_scale_dev, q, s, cap);
   return launch_rc();
 }
 
