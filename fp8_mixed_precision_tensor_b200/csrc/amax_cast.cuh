@@ -364,4 +364,27 @@ __global__ void __launch_bounds__(kStreamThreads) k_cast_redo(const void *__rest
     for (size_t i = groups * 16 + threadIdx.x; i < n; i += blockDim.x) cast_one<FMT>(load1<DT>(x, i) * s, q, i);
 }
 
+// Self-test of enc2 against enc2_checked on the binary32 values with bit
+// patterns in [lo, hi), each in the low lane (the other 0) and in the high
+// lane (the other 0): counts the values whose codes differ and keeps the
+// smallest such pattern.
+template <int FMT>
+__global__ void k_encode_selftest(uint32_t lo, unsigned long long hi, unsigned long long *bad, uint32_t *first) {
+  const unsigned long long stride = (unsigned long long)gridDim.x * blockDim.x;
+  unsigned long long nbad = 0;
+  uint32_t lowest = 0xffffffffu;
+  for (unsigned long long u = lo + (unsigned long long)blockIdx.x * blockDim.x + threadIdx.x; u < hi;
+       u += stride) {
+    const float x = __uint_as_float((uint32_t)u);
+    if (enc2<FMT>(x, 0.0f) != enc2_checked<FMT>(x, 0.0f) || enc2<FMT>(0.0f, x) != enc2_checked<FMT>(0.0f, x)) {
+      nbad++;
+      lowest = min(lowest, (uint32_t)u);
+    }
+  }
+  if (nbad) {
+    atomicAdd(bad, nbad);
+    atomicMin(first, lowest);
+  }
+}
+
 }  // namespace fp8lib

@@ -96,9 +96,10 @@ __device__ __forceinline__ uint32_t fix_special(uint32_t code, float y, int fmt)
   return code;
 }
 
-// Two floats -> two codes in the low 16 bits (a in bits 0-7, b in bits 8-15).
+// Two floats -> two codes in the low 16 bits (a in bits 0-7, b in bits 8-15),
+// with an explicit test for the special values.  The reference of enc2.
 template <int FMT>
-__device__ __forceinline__ uint32_t enc2(float a, float b) {
+__device__ __forceinline__ uint32_t enc2_checked(float a, float b) {
   __nv_fp8x2_storage_t r = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE,
                                                     FMT == FP8_E4M3 ? __NV_E4M3 : __NV_E5M2);
   uint32_t c = (uint32_t)r;
@@ -109,6 +110,20 @@ __device__ __forceinline__ uint32_t enc2(float a, float b) {
     c = ca | (cb << 8);
   }
   return c;
+}
+
+// The same two codes without a test or a branch: the saturating cvt already
+// maps +-inf to +-max; a NaN code of either sign is made 0x7F with byte-wise
+// SIMD compares (E4M3: the one NaN pattern S.1111.111; E5M2: S.11111.mm with
+// mm != 0).  fp8_selftest_encode checks enc2 against enc2_checked on every
+// binary32 value in each lane.
+template <int FMT>
+__device__ __forceinline__ uint32_t enc2(float a, float b) {
+  const uint32_t c = (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE,
+                                                         FMT == FP8_E4M3 ? __NV_E4M3 : __NV_E5M2);
+  const uint32_t mag = c & 0x7f7fu;
+  const uint32_t nan = FMT == FP8_E4M3 ? __vcmpeq4(mag, 0x7f7fu) : __vcmpgtu4(mag, 0x7c7cu);
+  return (c & ~nan) | (nan & 0x7f7fu);
 }
 
 // Four floats -> four codes packed little-endian in a 32-bit word.

@@ -737,6 +737,22 @@ int fp8_selftest_step_reciprocal(unsigned lo_bits, unsigned long long hi_bits, u
   return launch_rc();
 }
 
+int fp8_selftest_encode(int fmt, unsigned lo_bits, unsigned long long hi_bits, unsigned long long *bad_dev,
+                        unsigned *first_dev, void *stream) {
+  if ((fmt != FP8_E4M3 && fmt != FP8_E5M2) || hi_bits > 0x100000000ull || lo_bits >= hi_bits || !bad_dev ||
+      !first_dev)
+    return FP8_ERR_INVALID_ARG;
+  DeviceInfo *d;
+  int rc = device_info(&d);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (fmt == FP8_E4M3)
+    k_encode_selftest<FP8_E4M3><<<d->sms * 8, 256, 0, s>>>(lo_bits, hi_bits, bad_dev, first_dev);
+  else
+    k_encode_selftest<FP8_E5M2><<<d->sms * 8, 256, 0, s>>>(lo_bits, hi_bits, bad_dev, first_dev);
+  return launch_rc();
+}
+
 int fp8_get_status(unsigned *host_out, void *stream) {
   if (!host_out) return FP8_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

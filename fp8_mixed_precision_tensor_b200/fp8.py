@@ -34,7 +34,7 @@ SYMBOLS = ("fp8_amax", "fp8_compute_scale", "fp8_cast", "fp8_scale_cast", "fp8_a
            "fp8_linear_wgrad", "fp8_adam_workspace_bytes", "fp8_adam_step", "fp8_adam_stats",
            "fp8_adam_apply", "fp8_adam_step_noalloc", "fp8_adam_step_into", "fp8_adam_stats_into",
            "fp8_adam_apply_into",
-           "fp8_selftest_wait_timeout", "fp8_selftest_step_reciprocal", "fp8_get_status", "fp8_strerror")
+           "fp8_selftest_wait_timeout", "fp8_selftest_step_reciprocal", "fp8_selftest_encode", "fp8_get_status", "fp8_strerror")
 
 
 class FP8Error(RuntimeError):
@@ -98,6 +98,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                        ctypes.POINTER(_HParams), p, sz, p]
     lib.fp8_selftest_wait_timeout.argtypes = [ctypes.c_uint, p]
     lib.fp8_selftest_step_reciprocal.argtypes = [ctypes.c_uint, ctypes.c_ulonglong, p, p, p]
+    lib.fp8_selftest_encode.argtypes = [i, ctypes.c_uint, ctypes.c_ulonglong, p, p, p]
     lib.fp8_get_status.argtypes = [ctypes.POINTER(ctypes.c_uint), p]
     lib.fp8_strerror.argtypes, lib.fp8_strerror.restype = [i], ctypes.c_char_p
     for name in SYMBOLS:
@@ -380,6 +381,16 @@ def fp8_selftest_step_reciprocal(lo_bits: int, hi_bits: int, bad: torch.Tensor, 
     initialised by the caller)."""
     _check(load_library().fp8_selftest_step_reciprocal(lo_bits, hi_bits, _ptr(bad), _ptr(first),
                                                        _stream(stream)), "fp8_selftest_step_reciprocal")
+
+
+def fp8_selftest_encode(fmt: int, lo_bits: int, hi_bits: int, bad: torch.Tensor, first: torch.Tensor,
+                        stream=None) -> None:
+    """Compare the library's branch-free FP8 encoder with the explicitly
+    checked one on the binary32 bit patterns [lo_bits, hi_bits), in both
+    lanes; bad (1 x int64) counts differences, first (1 x int32) gets the
+    smallest differing pattern (both initialised by the caller)."""
+    _check(load_library().fp8_selftest_encode(fmt, lo_bits, hi_bits, _ptr(bad), _ptr(first), _stream(stream)),
+           "fp8_selftest_encode")
 
 
 def fp8_get_status(stream=None) -> int:

@@ -491,6 +491,21 @@ int fp8_selftest_wait_timeout(unsigned limit_us, void *stream);
 int fp8_selftest_step_reciprocal(unsigned lo_bits, unsigned long long hi_bits, unsigned long long *bad_dev,
                                  unsigned *first_dev, void *stream);
 
+/*
+ * fp8_selftest_encode -- numerics self-test of the library's FP8 encoder
+ * (fmt FP8_E4M3 or FP8_E5M2): the saturating hardware conversion with a
+ * branch-free canonicalisation of NaN codes, against the same conversion
+ * with an explicit test of each value for inf and NaN (+-inf -> +-max, NaN
+ * -> 0x7F, as fp8_cast defines), on every binary32 value whose bit pattern
+ * lies in [lo_bits, hi_bits) (hi_bits <= 2^32), in either lane of the
+ * two-value conversion.  Adds the number of values whose codes differ to
+ * *bad_dev (dev, one uint64) and lowers *first_dev (dev, one uint32) to the
+ * smallest such pattern; the caller initialises both.  FP8_ERR_INVALID_ARG
+ * for another format, an empty or too wide range or NULL outputs.
+ */
+int fp8_selftest_encode(int fmt, unsigned lo_bits, unsigned long long hi_bits, unsigned long long *bad_dev,
+                        unsigned *first_dev, void *stream);
+
 /* Human-readable message of a status code (static string). */
 const char *fp8_strerror(int code);
 

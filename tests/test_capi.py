@@ -198,6 +198,17 @@ def test_reciprocal_selftest_rejects_bad_arguments_on_the_host(lib):
     assert fn(0, 16, None, fake, None) == 1            # no counter
 
 
+def test_encode_selftest_rejects_bad_arguments_on_the_host(lib):
+    fn = lib.fp8_selftest_encode
+    fn.argtypes = [ctypes.c_int, ctypes.c_uint, ctypes.c_ulonglong, ctypes.c_void_p, ctypes.c_void_p,
+                   ctypes.c_void_p]
+    fake = 0x10000
+    assert fn(2, 0, 16, fake, fake, None) == 1              # FP16 is not an FP8 format
+    assert fn(0, 16, 16, fake, fake, None) == 1             # empty range
+    assert fn(1, 0, (1 << 32) + 1, fake, fake, None) == 1   # beyond the 2^32 patterns
+    assert fn(0, 0, 16, fake, None, None) == 1              # no first-pattern output
+
+
 def test_wait_selftest_rejects_limits_outside_its_range(lib):
     lib.fp8_selftest_wait_timeout.argtypes = [ctypes.c_uint, ctypes.c_void_p]
     assert lib.fp8_selftest_wait_timeout(0, None) == 1
