@@ -16,10 +16,11 @@ GPT-7B block (tokens 4096, hidden 4096).  Per step:
   (E5M2 grad, E4M3 m1, FP16 m2, FP16 master; 1,811,939,328 parameters for
   GPT-175B), which also writes the E4M3 copy of each new master: the next
   step's forward and dgrad read the weight from that copy, so no weight cast
-  runs in the step.  The master's amax is tracked between steps.  The step
+  runs in the step.  The step
   is out of place (`--adam into`, the default): each step writes the new
   state into the other of two buffer sets, in one pass while the scales
-  hold; `--adam in_place` runs the in-place step (stats pass + update).
+  hold; `--adam in_place` runs the in-place step (stats pass + update, the
+  master's amax tracked between steps so that the stats pass skips it).
 
 `value` is the step's algorithmic GEMM work (3 x 2MNK per linear; 89.06 TFLOP
 for GPT-175B) divided by the device time of the whole step, inputs resident
@@ -91,7 +92,8 @@ def config_of(wl: dict, schedule: str, world: int, adam: str = "into") -> dict:
     return {"workload": wl["workload"], "tokens": wl["tokens"], "hidden": wl["hidden"],
             "linears": [l[0] for l in wl["linears"]], "adam_params": sum(N * K for _, K, N in wl["linears"]),
             "gemm_flops_per_step": flops, "l2": "inputs larger than L2 (no flush)", "schedule": schedule,
-            "weight_operand": "E4M3 copy written by the previous Adam step", "master_amax": "tracked",
+            "weight_operand": "E4M3 copy written by the previous Adam step",
+            "master_amax": "tracked" if adam == "in_place" else "not tracked (no stats pass to skip)",
             "weight_gradient": "bf16 rounded to odd (its E5M2 cast equals the float32 dW's)",
             "adam_step": ADAM_MODES[adam],
             "parallelism": f"replicas{world}" if world > 1 else "single"}
@@ -274,9 +276,11 @@ class BlockStep:
         sets = (("m", "v", "wh"), ("m2", "v2", "wh2")) if adam == "into" else (("m", "v", "wh"),)
 
         def chunk(d, k):
+            # the in-place step tracks the master's amax (its stats pass then
+            # skips the master); the out-of-place step has no stats pass to spare
             m, v, w = (d[x] for x in sets[k])
             return fp8.AdamChunk(d["gq"], d["sc"][11:12], m, d["st"][0:1], v, d["st"][1:2], w, d["st"][2:3],
-                                 d["st"][3:4], d["wq"], d["sc"][4:5], d["sc"][5:6])
+                                 d["st"][3:4] if adam == "in_place" else None, d["wq"], d["sc"][4:5], d["sc"][5:6])
 
         def dest(d, k):
             return tuple(d[x] for x in sets[1 - k])

@@ -96,8 +96,9 @@ def test_bench_step_three_streams_equals_one_stream(workload):
         c.step()
     torch.cuda.synchronize()
     assert fp8.fp8_get_status() == 0
-    assert torch.equal(a.result_scalars(), b.result_scalars())
-    assert torch.equal(a.result_scalars(), c.result_scalars())
+    assert torch.equal(b.result_scalars(), c.result_scalars())
+    for da, db in zip(a.L, b.L):  # the in-place step also tracks the master's amax (st[3])
+        assert torch.equal(da["sc"], db["sc"]) and torch.equal(da["st"][:3], db["st"][:3]), da["name"]
     for da, db, dc in zip(a.L, b.L, c.L):
         for k in ("gq", "wq", "y", "dx", "dw"):
             assert torch.equal(da[k], db[k]) and torch.equal(da[k], dc[k]), (da["name"], k)
