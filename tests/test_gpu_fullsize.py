@@ -65,6 +65,32 @@ def test_gpt7b_linears_full_size(name, K, N):
     _check_linear(synth.GPT7B_TOKENS, K, N, synth.GPT7B_W_STD, 100)
 
 
+@pytest.mark.parametrize("fmt,std", [(fp8.FP8_E4M3, synth.ACT_STD), (fp8.FP8_E5M2, synth.GRAD_STD)])
+def test_one_pass_cast_at_the_largest_step_tensor(fmt, std):
+    """The GPT-175B step's largest activation / output gradient (8192 x 49152
+    bf16, 403 M elements): the one-pass amax + cast the benchmark runs gives
+    the amax, scales and codes of the amax pass and fused scale + cast, bit
+    for bit, with its guess right (one pass) and wrong (the redo)."""
+    M, K = synth.GPT175B_TOKENS, 49152
+    x = synth.device_normal((M, K), std, 4242 + fmt, torch.bfloat16, "cuda")
+    mu = 2.0 ** 10 if fmt == fp8.FP8_E5M2 else 1.0
+    f32 = dict(dtype=torch.float32, device="cuda")
+    a, s, inv = (torch.zeros(1, **f32) for _ in range(3))
+    q = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    fp8.fp8_amax(x, a)
+    fp8.fp8_scale_cast(x, fmt, a, 0, mu, s, inv, q)
+    for guess in (s.item(), s.item() * 2.0):
+        a1, inv1 = torch.zeros(1, **f32), torch.zeros(1, **f32)
+        s1 = torch.full((1,), guess, **f32)
+        q1 = torch.empty_like(q)
+        fp8.fp8_amax_scale_cast(x, fmt, a1, 0, mu, s1, inv1, q1)
+        assert (a1.item(), s1.item(), inv1.item()) == (a.item(), s.item(), inv.item()), guess
+        assert torch.equal(q1, q), guess
+    assert fp8.fp8_get_status() == 0
+    del x, q, q1
+    torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("name,K,N", synth.GPT175B_LINEARS)
 def test_gpt175b_linears_full_size(name, K, N):
     _check_linear(synth.GPT175B_TOKENS, K, N, synth.GPT175B_W_STD, 200)
@@ -122,9 +148,11 @@ def _stored_max(t, fmt):
     return view.float().abs().max().item()
 
 
-def test_gpt7b_adam_full_model_ten_steps():
+@pytest.mark.parametrize("out_of_place", [False, True])
+def test_gpt7b_adam_full_model_ten_steps(out_of_place):
     """The decoupled Adam over all 129 per-tensor chunks of GPT-7B
-    (6,648,496,128 parameters, one call per step) for ten steps, each step
+    (6,648,496,128 parameters, one call per step; in place, and out of place
+    as the benchmark runs it, alternating two buffer sets) for ten steps, each step
     with fresh E5M2 gradients ~N(0, 1e-3) x mu for every chunk.  After every
     step the chunks of ADAM_7B_CHECKS are checked whole against the oracle,
     fed the GPU's own state from the step before (scales bit-equal, master
@@ -135,14 +163,14 @@ def test_gpt7b_adam_full_model_ten_steps():
     for FP16, or the tensor is zero with scale 1)."""
     from profile_cases import build_adam_state
     from test_gpu_parity import HP, MAX_TIES, check_adam_chunk, snapshot
+    from fp8_mixed_precision_tensor_b200.adam_state import FP8Adam
 
     specs = synth.gpt7b_adam_chunks()
     assert sum(n for _, n in specs) == 6648496128 and len(specs) == 129
     names = [name for name, _ in specs]
-    states = build_adam_state(specs)
+    states = build_adam_state(specs, spare=out_of_place)
     chunks = [st.chunk for st in states]
-    arr = fp8.pack_adam_chunks(chunks)
-    ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(chunks)) // 4, dtype=torch.float32, device="cuda")
+    opt = FP8Adam(states, margin=0, out_of_place=out_of_place, **HP)
     ties = []
     for step in range(1, 11):
         if step > 1:  # fresh gradients for every chunk
@@ -152,8 +180,10 @@ def test_gpt7b_adam_full_model_ten_steps():
                 del g
         picks = [names.index(x) for x in ADAM_7B_CHECKS[step]]
         before = {i: snapshot(chunks[i]) for i in picks}
-        fp8.fp8_adam_step(arr, step=step, margin=0, workspace=ws, **HP)
+        opt.step()  # step `step` (out of place: into the other buffer set, which then holds the state)
+        assert opt.t == step
         assert fp8.fp8_get_status() == 0, step
+        chunks = [st.chunk for st in states]
         for i in picks:
             check_adam_chunk(before[i], chunks[i], step, ties=ties, slices=-(-specs[i][1] // ADAM_7B_SLICE))
         before.clear()
