@@ -86,7 +86,13 @@ ADAM_MODES = {
 }
 
 
-def config_of(wl: dict, schedule: str, world: int, adam: str = "into") -> dict:
+GRAD_CAST_MODES = {
+    "fused": "in the out-of-place Adam pass (E5M2 codes formed in registers from the bf16 dW, never stored)",
+    "separate": "a fused scale + cast kernel writing the E5M2 gradient, which Adam reads",
+}
+
+
+def config_of(wl: dict, schedule: str, world: int, adam: str = "into", grad_cast: str = "fused") -> dict:
     """The `config` object of the JSON line (the same for both arms)."""
     flops = sum(3 * 2 * wl["tokens"] * N * K for _, K, N in wl["linears"])
     return {"workload": wl["workload"], "tokens": wl["tokens"], "hidden": wl["hidden"],
@@ -96,6 +102,7 @@ def config_of(wl: dict, schedule: str, world: int, adam: str = "into") -> dict:
             "master_amax": "tracked" if adam == "in_place" else "not tracked (no stats pass to skip)",
             "weight_gradient": "bf16 rounded to odd (its E5M2 cast equals the float32 dW's)",
             "adam_step": ADAM_MODES[adam],
+            "gradient_cast": GRAD_CAST_MODES[grad_cast if adam == "into" else "separate"],
             "parallelism": f"replicas{world}" if world > 1 else "single"}
 
 
@@ -227,7 +234,8 @@ class BlockStep:
     FP16 masters (the Adam state) and the first E4M3 weight operands; from
     then on each step's Adam writes the next step's E4M3 weights."""
 
-    def __init__(self, device, seed: int = 0, workload: str = "gpt175b_block", adam: str = "into"):
+    def __init__(self, device, seed: int = 0, workload: str = "gpt175b_block", adam: str = "into",
+                 grad_cast: str = "fused"):
         from fp8_mixed_precision_tensor_b200 import fp8
 
         wl = WORKLOADS[workload]
@@ -273,25 +281,30 @@ class BlockStep:
         # state buffers of parity t % 2 (0: m, v, wh; 1: m2, v2, wh2) and writes
         # the other set
         self.adam = adam
+        # the gradient cast in the Adam pass needs the out-of-place step
+        self.fused_gcast = adam == "into" and grad_cast == "fused"
         sets = (("m", "v", "wh"), ("m2", "v2", "wh2")) if adam == "into" else (("m", "v", "wh"),)
 
         def chunk(d, k):
             # the in-place step tracks the master's amax (its stats pass then
             # skips the master); the out-of-place step has no stats pass to spare
             m, v, w = (d[x] for x in sets[k])
-            return fp8.AdamChunk(d["gq"], d["sc"][11:12], m, d["st"][0:1], v, d["st"][1:2], w, d["st"][2:3],
+            g = d["dw"] if self.fused_gcast else d["gq"]
+            return fp8.AdamChunk(g, d["sc"][11:12], m, d["st"][0:1], v, d["st"][1:2], w, d["st"][2:3],
                                  d["st"][3:4] if adam == "in_place" else None, d["wq"], d["sc"][4:5], d["sc"][5:6])
 
         def dest(d, k):
             return tuple(d[x] for x in sets[1 - k])
 
         self.packs, self.packs_each = [], []
+        gamax = lambda ds: fp8.pack_grad_amax([d["sc"][14:15] for d in ds]) if self.fused_gcast else None
         for k in range(len(sets)):
             self.packs.append((fp8.pack_adam_chunks([chunk(d, k) for d in self.L]),
-                               fp8.pack_adam_dests([dest(d, k) for d in self.L]) if adam == "into" else None))
+                               fp8.pack_adam_dests([dest(d, k) for d in self.L]) if adam == "into" else None,
+                               gamax(self.L)))
             # one Adam call per tensor (overlapped schedule)
             self.packs_each.append([(fp8.pack_adam_chunks([chunk(d, k)]),
-                                     fp8.pack_adam_dests([dest(d, k)]) if adam == "into" else None)
+                                     fp8.pack_adam_dests([dest(d, k)]) if adam == "into" else None, gamax([d]))
                                     for d in self.L])
         self.ws = torch.zeros(fp8.fp8_adam_workspace_bytes(len(self.L)) // 4 + 64, **f32)
         # a 256-byte-aligned workspace slice per tensor for the per-tensor calls
@@ -305,13 +318,17 @@ class BlockStep:
         # tracked master: stats, finalize 1, exact-master pass, finalize 2,
         # update, finalize 3
         na = 4 if adam == "into" else 6
-        self.launches_per_step = 4 * (2 * 3 + 3 + 1) + na
-        self.launches_per_step_overlapped = 4 * (2 * 3 + 3 + 1 + na)
+        ng = 0 if self.fused_gcast else 1  # the gradient cast kernel
+        self.launches_per_step = 4 * (2 * 3 + 3 + ng) + na
+        self.launches_per_step_overlapped = 4 * (2 * 3 + 3 + ng + na)
 
     def adam_step(self, pack, t, ws):
-        """Adam step t over the tensors of one packed (chunks, dests) pair."""
-        chunks, dests = pack
-        if self.adam == "into":
+        """Adam step t over the tensors of one packed (chunks, dests, gradient
+        amaxes) triple."""
+        chunks, dests, gamax = pack
+        if self.fused_gcast:
+            self.fp8.fp8_adam_step_into_castgrad(chunks, dests, gamax, MU, 0, step=t, margin=0, workspace=ws, **HP)
+        elif self.adam == "into":
             self.fp8.fp8_adam_step_into(chunks, dests, step=t, margin=0, workspace=ws, **HP)
         else:
             self.fp8.fp8_adam_step(chunks, step=t, margin=0, workspace=ws, **HP)
@@ -348,9 +365,10 @@ class BlockStep:
             fp8.fp8_linear_dgrad(d["dyq"], sc[8:9], d["wq"], sc[5:6], d["dx"], sc[13:14])
             fp8.fp8_linear_wgrad(d["dyq"], sc[8:9], d["xq"], sc[2:3], d["dw"], sc[14:15], rto=True)
             if e: e[1].record()
-            e = mark("grad_cast")
-            fp8.fp8_scale_cast(d["dw"], fp8.FP8_E5M2, sc[14:15], 0, MU, sc[10:11], sc[11:12], d["gq"])
-            if e: e[1].record()
+            if not self.fused_gcast:
+                e = mark("grad_cast")
+                fp8.fp8_scale_cast(d["dw"], fp8.FP8_E5M2, sc[14:15], 0, MU, sc[10:11], sc[11:12], d["gq"])
+                if e: e[1].record()
             nvtx.range_pop()
         self.t += 1
         nvtx.range_push("adam")
@@ -405,7 +423,8 @@ class BlockStep:
             self.s_aux.wait_event(e)
             with torch.cuda.stream(self.s_aux):
                 fp8.fp8_linear_wgrad(d["dyq"], sc[8:9], d["xq"], sc[2:3], d["dw"], sc[14:15], rto=True)
-                fp8.fp8_scale_cast(d["dw"], fp8.FP8_E5M2, sc[14:15], 0, MU, sc[10:11], sc[11:12], d["gq"])
+                if not self.fused_gcast:
+                    fp8.fp8_scale_cast(d["dw"], fp8.FP8_E5M2, sc[14:15], 0, MU, sc[10:11], sc[11:12], d["gq"])
                 self.s_aux.wait_event(self.ev_dgrad[i])
                 self.adam_step(self.packs_each[self.t % len(self.packs_each)][i], self.t + 1,
                                self.ws_each[64 * i:64 * (i + 1)])
@@ -510,7 +529,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     wl = WORKLOADS[args.workload]
-    cfg = config_of(wl, args.schedule, args.gpus, args.adam)
+    cfg = config_of(wl, args.schedule, args.gpus, args.adam, args.grad_cast)
     sample = OracleSample(wl)
     t_s, t_f = [], []
     for i in range(args.warmup + args.steps):
@@ -554,7 +573,7 @@ def run_gpu(args):
 
     peaks = load_peaks()
     wl = WORKLOADS[args.workload]
-    runner = BlockStep(dev, seed=rank, workload=args.workload, adam=args.adam)
+    runner = BlockStep(dev, seed=rank, workload=args.workload, adam=args.adam, grad_cast=args.grad_cast)
     overlap = args.schedule == "overlap"
     for _ in range(args.warmup):
         runner.step_overlapped() if overlap else runner.step()
@@ -658,13 +677,15 @@ def run_gpu(args):
     peak, peak_src = fp8_peak(peaks, clocks)
     gemm_tflops = runner.flops / (t_gemm * 1e-3) / 1e12
     cast_gbs = runner.cast_elems * CAST_BYTES_BF16 / (t_cast * 1e-3) / 1e9
-    gcast_gbs = runner.params * GRAD_CAST_BYTES / (t_gcast * 1e-3) / 1e9
-    adam_gbs = runner.params * ADAM_BYTES / (t_adam * 1e-3) / 1e9
+    gcast_gbs = runner.params * GRAD_CAST_BYTES / (t_gcast * 1e-3) / 1e9 if t_gcast > 0 else None
+    # with the gradient cast in the pass, Adam reads the bf16 dW (2 B) instead of the E5M2 code
+    adam_bytes = ADAM_BYTES + (1 if runner.fused_gcast else 0)
+    adam_gbs = runner.params * adam_bytes / (t_adam * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp8(e4m3/e5m2)->f32 accum; f32 elementwise", "data": "synthetic",
-        "config": config_of(wl, args.schedule, world, args.adam),
+        "config": config_of(wl, args.schedule, world, args.adam, args.grad_cast),
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": gemm_tflops / peak, "traffic": gemm_traffic(wl["workload"]),
                      "kernel": "k_gemm3 (fwd+dgrad+wgrad; achieved = GEMM flops per step / summed GEMM "
@@ -674,9 +695,10 @@ def run_gpu(args):
             "gemm": {"ms": t_gemm, "TFLOP/s": gemm_tflops, "frac_fp8_peak": gemm_tflops / peak},
             "amax_scale_cast": {"ms": t_cast, "GB/s": cast_gbs, "frac_hbm": cast_gbs / peaks["hbm"],
                                 "tensors": "X and dY of every linear (the weight operand comes from Adam)"},
-            "grad_cast": {"ms": t_gcast, "GB/s": gcast_gbs, "frac_hbm": gcast_gbs / peaks["hbm"]},
+            "grad_cast": ({"ms": t_gcast, "GB/s": gcast_gbs, "frac_hbm": gcast_gbs / peaks["hbm"]}
+                          if gcast_gbs is not None else {"ms": 0.0, "fused": "in the Adam pass"}),
             "adam": {"ms": t_adam, "GB/s": adam_gbs, "frac_hbm": adam_gbs / peaks["hbm"],
-                     "bytes_per_param_algorithmic": ADAM_BYTES,
+                     "bytes_per_param_algorithmic": adam_bytes,
                      "bytes_per_param_moved": ("11 (one pass while the scales hold; 22 for a chunk whose "
                                                "scales change) + 1 for the E4M3 weight copy"
                                                if args.adam == "into" else
@@ -715,6 +737,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--schedule", default="overlap", choices=["overlap", "serial"],
                     help="overlap: casts / GEMMs / wgrad on three streams; serial: one stream")
+    ap.add_argument("--grad-cast", dest="grad_cast", default="fused", choices=sorted(GRAD_CAST_MODES),
+                    help="fused: the E5M2 gradient cast inside the out-of-place Adam pass; separate: its own kernel")
     ap.add_argument("--adam", default="into", choices=sorted(ADAM_MODES),
                     help="into: out-of-place Adam step (two state buffers); in_place: stats + update passes")
     args = ap.parse_args()

@@ -42,6 +42,10 @@
 //   finalize 7:       tracked amax of the redone chunks.
 // One pass of 6 B read and 5-6 B written per parameter when the scales hold,
 // the same results as the in-place step in every case.
+// Passes 8 and 9 are passes 6 and 7 reading the gradient as the wgrad left
+// it, bfloat16, and casting it to E5M2 in registers with the scale of its
+// amax (the codes the separate gradient cast would store), so the E5M2
+// gradient is never written or read back.
 // All chunks of one call share each launch: the chunk table travels in the
 // kernel parameters and tiles of 4096 parameters are mapped to chunks by a
 // binary search over the chunks' first-tile indices.
@@ -91,6 +95,7 @@ struct AdamChunkDev {
   uint8_t *m_out;    // where the update writes the new state: m, v, w
   uint16_t *v_out;   // themselves (in place) or the out-of-place step's
   uint16_t *w_out;   // new buffers
+  const float *g_amax;  // passes 8, 9: amax of the bfloat16 gradient at g
   unsigned long long n;
   unsigned long long tile_begin;
 };
@@ -104,6 +109,8 @@ struct AdamLaunch {
   float neg_lr_bc1;  // -lr / (1 - beta1^t)
   float inv_bc2;     // 1 / (1 - beta2^t)
   int estimate;      // 1: untracked chunks take the estimated stats pass (PASS 5)
+  int g_hp;          // passes 8, 9: the gradient is bfloat16, cast to E5M2 in the pass
+  int g_margin, g_log2mu;  // its scale rule: margin and log2(mu)
   float *ws;         // kAdamWsFloatsPerChunk floats per chunk of this launch
 };
 static_assert(sizeof(AdamLaunch) <= 32764, "kernel parameters are limited to 32,764 bytes");
@@ -268,6 +275,19 @@ struct AdamNewScales {
   float2 q;        // s_q / s_w: stored master -> its E4M3 copy (powers of two, ~2^-7)
 };
 
+// Passes 8 and 9 run the code of passes 6 and 7 with the gradient cast in
+// the pass: the pass number the rest of the code branches on, and the flag.
+template <int PASS>
+__host__ __device__ constexpr int base_pass() { return PASS >= 8 ? PASS - 2 : PASS; }
+template <int PASS>
+__host__ __device__ constexpr bool cast_grad_pass() { return PASS >= 8; }
+
+// The gradient's E5M2 scale exponent from its amax (the rule of the fused
+// scale + cast, fmt_max 57344); false for a non-finite amax (then 2^log2mu).
+__device__ __forceinline__ bool grad_scale_exponent(const AdamLaunch &L, const AdamChunkDev &C, int &k) {
+  return scale_exponent(*C.g_amax, 57344.0f, L.g_margin, L.g_log2mu, k);
+}
+
 // One thread's full group of 16 parameters: 16 B of g, 16 B of m, 32 B of v,
 // 32 B of w.  Whether the chunk tracks its master amax and whether the E4M3
 // copy is written are per chunk: the stats passes take them as template
@@ -277,13 +297,22 @@ struct AdamNewScales {
 // wq_rt the chunk's flags).  The update passes (2 in place; 6 and 7 out of
 // place, which also reduce the exact amaxes of the new m and v) write the
 // new state through m_out, v_out, w_out.
-template <int PASS, bool TRACK, bool WQ>
+template <int PASS_, bool TRACK, bool WQ>
 __device__ __forceinline__ void adam_group(const AdamLaunch &L, const AdamChunkDev &C, size_t grp,
                                            const AdamScalars &sc, const AdamNewScales &ns, float &am, float &av,
-                                           float &aw, float &au, bool track_rt = TRACK, bool wq_rt = WQ) {
+                                           float &aw, float &au, bool track_rt = TRACK, bool wq_rt = WQ,
+                                           float2 sg = make_float2(1.0f, 1.0f)) {
+  constexpr int PASS = base_pass<PASS_>();
+  constexpr bool kCastG = cast_grad_pass<PASS_>();
   constexpr bool kReadW = PASS != 1 || !TRACK;
   const bool track = TRACK && track_rt, wq = WQ && wq_rt;
-  const uint4 gq = __ldcs(reinterpret_cast<const uint4 *>(C.g) + grp);
+  uint4 gq, gh1 = make_uint4(0, 0, 0, 0);  // E5M2 codes, or the first and second 8 bfloat16
+  if constexpr (kCastG) {
+    gq = __ldcs(reinterpret_cast<const uint4 *>(C.g) + 2 * grp);
+    gh1 = __ldcs(reinterpret_cast<const uint4 *>(C.g) + 2 * grp + 1);
+  } else {
+    gq = __ldcs(reinterpret_cast<const uint4 *>(C.g) + grp);
+  }
   const uint4 mq = __ldcs(reinterpret_cast<const uint4 *>(C.m) + grp);
   const uint4 vq0 = __ldcs(reinterpret_cast<const uint4 *>(C.v) + 2 * grp);
   const uint4 vq1 = __ldcs(reinterpret_cast<const uint4 *>(C.v) + 2 * grp + 1);
@@ -293,13 +322,21 @@ __device__ __forceinline__ void adam_group(const AdamLaunch &L, const AdamChunkD
     wq1 = __ldcs(reinterpret_cast<const uint4 *>(C.w) + 2 * grp + 1);
   }
   const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
+  const uint32_t gb[4] = {gh1.x, gh1.y, gh1.z, gh1.w};
   const uint32_t mw[4] = {mq.x, mq.y, mq.z, mq.w};
   const uint32_t vw[8] = {vq0.x, vq0.y, vq0.z, vq0.w, vq1.x, vq1.y, vq1.z, vq1.w};
   const uint32_t ww[8] = {wq0.x, wq0.y, wq0.z, wq0.w, wq1.x, wq1.y, wq1.z, wq1.w};
   uint32_t mo[4], vo[8], wo[8], qo[4];
 #pragma unroll
   for (int p = 0; p < 8; p++) {  // pairs of parameters
-    const uint32_t g2 = (gw[p >> 1] >> ((p & 1) * 16)) & 0xffffu;
+    uint32_t g2;
+    if constexpr (kCastG) {  // the gradient cast: bfloat16 pair p, times its scale, to E5M2
+      const uint32_t b2 = p < 4 ? gw[p] : gb[p - 4];
+      const float2 y = __fmul2_rn(make_float2(__uint_as_float(b2 << 16), __uint_as_float(b2 & 0xffff0000u)), sg);
+      g2 = enc2<FP8_E5M2>(y.x, y.y);
+    } else {
+      g2 = (gw[p >> 1] >> ((p & 1) * 16)) & 0xffffu;
+    }
     const uint32_t m2 = (mw[p >> 1] >> ((p & 1) * 16)) & 0xffffu;
     float2 m, v, d;
     if constexpr ((PASS == 1 && TRACK) || PASS == 5)  // the step is only estimated
@@ -362,10 +399,12 @@ struct AdamChunkState {
   bool tracked = false, active = true, want_wq = false;
   AdamScalars sc{};
   AdamNewScales ns{both(1.f), both(1.f), both(1.f), both(1.f)};
+  float sg = 1.0f;  // passes 8, 9: the E5M2 scale of the bfloat16 gradient
 };
 
-template <int PASS>
+template <int PASS_>
 __device__ __forceinline__ void adam_chunk_flush(const AdamLaunch &L, AdamChunkState &S) {
+  constexpr int PASS = base_pass<PASS_>();
   constexpr bool kStats = PASS == 1 || PASS == 4;
   if constexpr (kStats)
     if (S.active) flush_max3(L, S.cur, WS_AMAX_M, S.am, WS_AMAX_V, S.av, S.tracked ? WS_STEP_MAX : WS_AMAX_W, S.aw);
@@ -385,8 +424,24 @@ __device__ __forceinline__ void adam_chunk_flush(const AdamLaunch &L, AdamChunkS
   S.am = S.av = S.aw = S.au = 0.f;
 }
 
-template <int PASS>
+// The gradient's descale: stored with its E5M2 codes, or (passes 8, 9) from
+// the scale of its amax, as the gradient cast derives it (that scale kept
+// for the cast in the pass).
+template <int PASS_>
+__device__ __forceinline__ float chunk_grad_inv(const AdamLaunch &L, const AdamChunkDev &C, AdamChunkState &S) {
+  if constexpr (cast_grad_pass<PASS_>()) {
+    int k;
+    grad_scale_exponent(L, C, k);
+    S.sg = pow2f(k);
+    return pow2f(-k);
+  } else {
+    return *C.g_inv;
+  }
+}
+
+template <int PASS_>
 __device__ __forceinline__ void adam_chunk_enter(const AdamLaunch &L, int ci, AdamChunkState &S) {
+  constexpr int PASS = base_pass<PASS_>();
   constexpr bool kStats = PASS == 1 || PASS == 4 || PASS == 5;
   const AdamChunkDev &C = L.c[ci];
   S.cur = ci;
@@ -400,7 +455,7 @@ __device__ __forceinline__ void adam_chunk_enter(const AdamLaunch &L, int ci, Ad
     S.tracked = C.w_amax != nullptr;
     S.active = true;
     const float sm = *C.m_scale, sv = *C.v_scale, sw = *C.w_scale;
-    S.sc = adam_scalars(L, *C.g_inv, 1.0f / sm, 1.0f / sv, 1.0f / sw);
+    S.sc = adam_scalars(L, chunk_grad_inv<PASS_>(L, C, S), 1.0f / sm, 1.0f / sv, 1.0f / sw);
     S.ns.m = both(sm);
     S.ns.v = both(sv);
     S.ns.w = both(sw);
@@ -412,8 +467,8 @@ __device__ __forceinline__ void adam_chunk_enter(const AdamLaunch &L, int ci, Ad
     // chunk that tracks it, including the step that first establishes it
     S.tracked = PASS == 3 ? (fl & FLAG_TRACKED) != 0 : C.w_amax != nullptr;
     S.active = PASS == 2 || (fl & (PASS == 7 ? FLAG_REDO : FLAG_EXACT)) != 0;
-    S.sc = adam_scalars(L, *C.g_inv, ws_get(L, ci, WS_OLDINV_M), ws_get(L, ci, WS_OLDINV_V),
-                        ws_get(L, ci, WS_OLDINV_W));
+    S.sc = adam_scalars(L, chunk_grad_inv<PASS_>(L, C, S), ws_get(L, ci, WS_OLDINV_M),
+                        ws_get(L, ci, WS_OLDINV_V), ws_get(L, ci, WS_OLDINV_W));
     S.ns.m = both(ws_get(L, ci, WS_NEW_M));
     S.ns.v = both(ws_get(L, ci, WS_NEW_V));
     S.ns.w = both(ws_get(L, ci, WS_NEW_W));
@@ -427,15 +482,22 @@ __device__ __forceinline__ void adam_chunk_enter(const AdamLaunch &L, int ci, Ad
 
 // The ragged end of a chunk, [base, n) with n - base < 16: element by element
 // from global memory (lane y of the packed arithmetic unused).
-template <int PASS>
+template <int PASS_>
 __device__ __forceinline__ void adam_tail(const AdamLaunch &L, const AdamChunkDev &C, unsigned long long base,
                                        AdamChunkState &S) {
+  constexpr int PASS = base_pass<PASS_>();
   constexpr bool kStats = PASS == 1 || PASS == 4 || PASS == 5;
   const bool read_w = PASS != 4;
   const AdamScalars &sc = S.sc;
   const AdamNewScales &ns = S.ns;
   for (unsigned long long i = base; i < C.n; i++) {
-    const float2 gd = dec2<FP8_E5M2>(C.g[i]), md = dec2<FP8_E4M3>(C.m[i]);
+    uint32_t gc;
+    if constexpr (cast_grad_pass<PASS_>())  // bfloat16 element i, times its scale, to E5M2
+      gc = enc2<FP8_E5M2>(__fmul_rn(__uint_as_float((uint32_t)reinterpret_cast<const uint16_t *>(C.g)[i] << 16),
+                                    S.sg), 0.0f) & 0xffu;
+    else
+      gc = C.g[i];
+    const float2 gd = dec2<FP8_E5M2>(gc), md = dec2<FP8_E4M3>(C.m[i]);
     const float2 vd = make_float2(__half2float(__ushort_as_half(C.v[i])), 0.0f);
     const float2 wd = make_float2(read_w ? __half2float(__ushort_as_half(C.w[i])) : 0.0f, 0.0f);
     float2 m, v, d;
@@ -509,6 +571,9 @@ __device__ __forceinline__ void adam_pass(const AdamLaunch &L) {
         adam_group<1, false, false>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw, S.au);
       } else if constexpr (PASS == 3) {
         adam_group<3, false, false>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw, S.au);
+      } else if constexpr (cast_grad_pass<PASS>()) {  // 8 or 9
+        adam_group<PASS, true, true>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw, S.au, S.tracked, S.want_wq,
+                                     both(S.sg));
       } else {  // an update pass: 2, 6 or 7
         adam_group<PASS, true, true>(L, C, grp, S.sc, S.ns, S.am, S.av, S.aw, S.au, S.tracked, S.want_wq);
       }
@@ -524,14 +589,15 @@ template <int PASS>
 __global__ void __launch_bounds__(kAdamThreads) k_adam(const __grid_constant__ AdamLaunch L) {
   adam_pass<PASS>(L);
 }
-// The update pass, latency-bound on its loads, is held to 48 registers: five
-// resident blocks per SM instead of four keep more loads in flight.  (A
-// variant fed through a shared-memory ring by bulk copies, one producer warp
-// and eight consumer warps per block, two blocks per SM, was correct but 12 %
-// slower at 64 M parameters: too few warps left to hide the update's
-// arithmetic.)
+// The in-place update pass: 64 registers and four resident blocks per SM.
+// (Held to five blocks' 48 registers it spilled, 64 bytes per thread with the
+// branch-free FP8 encoder; four and five blocks had measured the same when
+// both were spill-free.  A variant fed through a shared-memory ring by bulk
+// copies, one producer warp and eight consumer warps per block, two blocks
+// per SM, was correct but 12 % slower at 64 M parameters: too few warps left
+// to hide the update's arithmetic.)
 template <>
-__global__ void __launch_bounds__(kAdamThreads, 5) k_adam<2>(const __grid_constant__ AdamLaunch L) {
+__global__ void __launch_bounds__(kAdamThreads, 4) k_adam<2>(const __grid_constant__ AdamLaunch L) {
   adam_pass<2>(L);
 }
 // The out-of-place update and its redo: 64 registers and four resident
@@ -545,6 +611,15 @@ __global__ void __launch_bounds__(kAdamThreads, 4) k_adam<6>(const __grid_consta
 template <>
 __global__ void __launch_bounds__(kAdamThreads, 4) k_adam<7>(const __grid_constant__ AdamLaunch L) {
   adam_pass<7>(L);
+}
+// The same two passes with the gradient cast in the pass.
+template <>
+__global__ void __launch_bounds__(kAdamThreads, 4) k_adam<8>(const __grid_constant__ AdamLaunch L) {
+  adam_pass<8>(L);
+}
+template <>
+__global__ void __launch_bounds__(kAdamThreads, 4) k_adam<9>(const __grid_constant__ AdamLaunch L) {
+  adam_pass<9>(L);
 }
 // The estimated stats passes: six resident blocks per SM.
 template <>
@@ -682,6 +757,11 @@ __global__ void k_adam_finalize(const __grid_constant__ AdamLaunch L) {
         *C.wq_inv = 1.0f / nq;
       }
       if (held && C.w_amax != nullptr) *C.w_amax = __fmul_rn(ws[WS_STORED_W], 1.0f / nw);
+      if (L.g_hp) {  // passes 8, 9: publish the gradient's descale, as the gradient cast would
+        int kg;
+        if (!grad_scale_exponent(L, C, kg)) atomicOr(&g_status, FP8_STATUS_NONFINITE);
+        *const_cast<float *>(C.g_inv) = pow2f(-kg);
+      }
     }
     if constexpr (STAGE == 7) {
       if ((flags & FLAG_REDO) && C.w_amax != nullptr)

@@ -32,6 +32,7 @@ struct DeviceInfo {
   int adam_bound_blocks_per_sm = 1;  // of the estimated stats pass of tracking chunks
   int adam_est_blocks_per_sm = 1;    // of the estimated stats pass of the other chunks
   int adam_into_blocks_per_sm = 1;   // of the out-of-place update (and its redo)
+  int adam_castg_blocks_per_sm = 1;  // of the same with the gradient cast in the pass
   int cast_blocks_per_sm = 8;        // resident blocks of the streaming cast kernels
   int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair GEMM
   int wide_clusters = 0;  // co-resident 2-CTA clusters of the wide pair GEMM
@@ -88,6 +89,9 @@ int device_info(DeviceInfo **out) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k_adam<6>, kAdamThreads, 0) != cudaSuccess)
       return FP8_ERR_CUDA;
     d.adam_into_blocks_per_sm = bps > 0 ? bps : 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k_adam<8>, kAdamThreads, 0) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    d.adam_castg_blocks_per_sm = bps > 0 ? bps : 1;
     // the cast kernels' grids are one wave of resident blocks (a grid-stride
     // loop gives each block an equal share; a partial second wave would run
     // a third of the work on a few SMs): the fewest resident blocks of the
@@ -530,8 +534,17 @@ enum { PH_STATS = 1, PH_APPLY = 2, PH_ALL = 3, PH_INTO = 4 };
 bool same_buffer(const void *a, const void *b) { return a != nullptr && a == b; }
 
 int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *hp, void *workspace,
-             size_t ws_bytes, void *stream, int phases, const fp8_adam_dest *dest = nullptr) {
+             size_t ws_bytes, void *stream, int phases, const fp8_adam_dest *dest = nullptr,
+             const fp8_adam_grad_cast *gc = nullptr) {
   if (((phases & PH_INTO) != 0) != (dest != nullptr)) return FP8_ERR_INVALID_ARG;
+  int g_log2mu = 0;
+  if (gc) {  // the gradient cast in the pass: the whole out-of-place step only
+    if (phases != (PH_INTO | PH_ALL) || !gc->amax || !mu_log2(gc->mu, &g_log2mu) || gc->margin < 0 ||
+        gc->margin > 64)
+      return FP8_ERR_INVALID_ARG;
+    for (int i = 0; i < nchunks; i++)
+      if (!gc->amax[i]) return FP8_ERR_INVALID_ARG;
+  }
   if (!chunks || !hp || nchunks <= 0 || !workspace) return FP8_ERR_INVALID_ARG;
   if (ws_bytes < fp8_adam_workspace_bytes(nchunks)) return FP8_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FP8_ERR_UNALIGNED;
@@ -587,11 +600,14 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
   // chunks whose interval is ambiguous); the phased step reduces the exact
   // amaxes over ranks between its two calls
   L.estimate = phases == PH_ALL ? 1 : 0;
+  L.g_hp = gc ? 1 : 0;
+  L.g_margin = gc ? gc->margin : 0;
+  L.g_log2mu = g_log2mu;
   const unsigned cap = (unsigned)(d->sms * d->adam_blocks_per_sm);
   const unsigned cap1 = (unsigned)(d->sms * d->adam_stats_blocks_per_sm);
   const unsigned cap4 = (unsigned)(d->sms * d->adam_bound_blocks_per_sm);
   const unsigned cap5 = (unsigned)(d->sms * d->adam_est_blocks_per_sm);
-  const unsigned cap6 = (unsigned)(d->sms * d->adam_into_blocks_per_sm);
+  const unsigned cap6 = (unsigned)(d->sms * (gc ? d->adam_castg_blocks_per_sm : d->adam_into_blocks_per_sm));
   for (int first = 0; first < nchunks; first += kAdamMaxChunksPerLaunch) {
     const int cnt = nchunks - first < kAdamMaxChunksPerLaunch ? nchunks - first : kAdamMaxChunksPerLaunch;
     unsigned long long tiles = 0;
@@ -606,6 +622,7 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
       } else {
         e.m_out = c.m; e.v_out = c.v; e.w_out = c.w;
       }
+      e.g_amax = gc ? gc->amax[first + i] : nullptr;
       e.n = c.n;
       e.tile_begin = tiles;
       tiles += (c.n + kAdamTile - 1) / kAdamTile;
@@ -621,11 +638,14 @@ int adam_run(const fp8_adam_chunk *chunks, int nchunks, const fp8_adam_hparams *
     bool tracked = false;
     for (int i = 0; i < cnt; i++) tracked |= L.c[i].w_amax != nullptr;
     if (phases & PH_INTO) {
-      if (phases & PH_STATS)
-        k_adam<6><<<grid6, kAdamThreads, 0, s>>>(L);   // update with the predicted scales
+      if (phases & PH_STATS) {  // update with the predicted scales
+        if (gc) k_adam<8><<<grid6, kAdamThreads, 0, s>>>(L);
+        else    k_adam<6><<<grid6, kAdamThreads, 0, s>>>(L);
+      }
       if (phases & PH_APPLY) {
         k_adam_finalize<6><<<1, 256, 0, s>>>(L);       // the right scales; wrong predictions flagged
-        k_adam<7><<<grid6, kAdamThreads, 0, s>>>(L);   // flagged chunks again, from the inputs
+        if (gc) k_adam<9><<<grid6, kAdamThreads, 0, s>>>(L);   // flagged chunks again, from the inputs
+        else    k_adam<7><<<grid6, kAdamThreads, 0, s>>>(L);
         k_adam_finalize<7><<<1, 256, 0, s>>>(L);
       }
     } else if (phases & PH_STATS) {
@@ -664,6 +684,13 @@ int fp8_adam_step_into(const fp8_adam_chunk *chunks, const fp8_adam_dest *dest, 
                        const fp8_adam_hparams *hp, void *workspace, size_t ws_bytes, void *stream) {
   if (!dest) return FP8_ERR_INVALID_ARG;
   return adam_run(chunks, nchunks, hp, workspace, ws_bytes, stream, PH_INTO | PH_ALL, dest);
+}
+
+int fp8_adam_step_into_castgrad(const fp8_adam_chunk *chunks, const fp8_adam_dest *dest,
+                                const fp8_adam_grad_cast *gc, int nchunks, const fp8_adam_hparams *hp,
+                                void *workspace, size_t ws_bytes, void *stream) {
+  if (!dest || !gc) return FP8_ERR_INVALID_ARG;
+  return adam_run(chunks, nchunks, hp, workspace, ws_bytes, stream, PH_INTO | PH_ALL, dest, gc);
 }
 
 int fp8_adam_stats_into(const fp8_adam_chunk *chunks, const fp8_adam_dest *dest, int nchunks,

@@ -32,7 +32,8 @@ SYMBOLS = ("fp8_amax", "fp8_compute_scale", "fp8_cast", "fp8_scale_cast", "fp8_a
            "fp8_grad_cast",
            "fp8_sum_codes", "fp8_mu_update", "fp8_linear_fwd", "fp8_linear_dgrad",
            "fp8_linear_wgrad", "fp8_adam_workspace_bytes", "fp8_adam_step", "fp8_adam_stats",
-           "fp8_adam_apply", "fp8_adam_step_noalloc", "fp8_adam_step_into", "fp8_adam_stats_into",
+           "fp8_adam_apply", "fp8_adam_step_noalloc", "fp8_adam_step_into", "fp8_adam_step_into_castgrad",
+           "fp8_adam_stats_into",
            "fp8_adam_apply_into",
            "fp8_selftest_wait_timeout", "fp8_selftest_step_reciprocal", "fp8_selftest_encode", "fp8_get_status", "fp8_strerror")
 
@@ -53,6 +54,10 @@ class _Chunk(ctypes.Structure):
 
 class _Dest(ctypes.Structure):
     _fields_ = [("m", ctypes.c_void_p), ("v", ctypes.c_void_p), ("w", ctypes.c_void_p)]
+
+
+class _GradCast(ctypes.Structure):
+    _fields_ = [("amax", ctypes.POINTER(ctypes.c_void_p)), ("mu", ctypes.c_float), ("margin", ctypes.c_int)]
 
 
 class _MuRule(ctypes.Structure):
@@ -93,6 +98,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     for name in ("fp8_adam_step", "fp8_adam_stats", "fp8_adam_apply"):
         getattr(lib, name).argtypes = [ctypes.POINTER(_Chunk), i, ctypes.POINTER(_HParams), p, sz, p]
     lib.fp8_adam_step_noalloc.argtypes = [ctypes.POINTER(_Chunk), i, ctypes.POINTER(_HParams), p]
+    lib.fp8_adam_step_into_castgrad.argtypes = [ctypes.POINTER(_Chunk), ctypes.POINTER(_Dest),
+                                                ctypes.POINTER(_GradCast), i, ctypes.POINTER(_HParams), p, sz, p]
     for name in ("fp8_adam_step_into", "fp8_adam_stats_into", "fp8_adam_apply_into"):
         getattr(lib, name).argtypes = [ctypes.POINTER(_Chunk), ctypes.POINTER(_Dest), i,
                                        ctypes.POINTER(_HParams), p, sz, p]
@@ -314,6 +321,34 @@ def fp8_adam_step_into(chunks, dests, lr: float, beta1: float, beta2: float, eps
     chunks' own m, v, w are only read.  Bit for bit the in-place step's
     results, in one pass over the state when the scales do not change."""
     _adam_into("fp8_adam_step_into", chunks, dests, lr, beta1, beta2, eps, step, margin, workspace, stream)
+
+
+def pack_grad_amax(amaxes) -> ctypes.Array:
+    """Host array of the dev pointers of per-chunk gradient amaxes."""
+    arr = (ctypes.c_void_p * len(amaxes))()
+    for i, a in enumerate(amaxes):
+        arr[i] = _ptr(a)
+    return arr
+
+
+def fp8_adam_step_into_castgrad(chunks, dests, grad_amax, mu: float, grad_margin: int, lr: float, beta1: float,
+                                beta2: float, eps: float, step: int, margin: int, workspace: torch.Tensor,
+                                stream=None) -> None:
+    """fp8_adam_step_into with the gradient cast in the pass: each chunk's g is
+    the bfloat16 dW (the wgrad's output), cast to E5M2 with the scale of its
+    amax (grad_amax: per chunk a device scalar, or pack_grad_amax's array),
+    mu and grad_margin -- the codes fp8_scale_cast would write, never
+    stored; each chunk's g_inv receives the gradient's inverse scale."""
+    arr = chunks if isinstance(chunks, ctypes.Array) else pack_adam_chunks(chunks)
+    darr = dests if isinstance(dests, ctypes.Array) else pack_adam_dests(dests)
+    amax = grad_amax if isinstance(grad_amax, ctypes.Array) else pack_grad_amax(grad_amax)
+    if len(darr) != len(arr) or len(amax) != len(arr):
+        raise ValueError("one dest and one gradient amax per chunk")
+    gc = _GradCast(ctypes.cast(amax, ctypes.POINTER(ctypes.c_void_p)), mu, grad_margin)
+    hp = _HParams(lr, beta1, beta2, eps, step, margin)
+    _check(load_library().fp8_adam_step_into_castgrad(arr, darr, ctypes.byref(gc), len(arr), ctypes.byref(hp),
+                                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                                      _stream(stream)), "fp8_adam_step_into_castgrad")
 
 
 def fp8_adam_stats_into(chunks, dests, lr: float, beta1: float, beta2: float, eps: float, step: int,

@@ -375,6 +375,34 @@ typedef struct {
 int fp8_adam_step_into(const fp8_adam_chunk *chunks, const fp8_adam_dest *dest, int nchunks,
                        const fp8_adam_hparams *hp, void *workspace, size_t ws_bytes, void *stream);
 
+/* The gradient cast of fp8_adam_step_into_castgrad. */
+typedef struct {
+  const float *const *amax;  /* HOST array of nchunks dev pointers: amax|dW| of each chunk's
+                                gradient (e.g. the wgrad's fused output amax); none NULL */
+  float mu;                  /* gradient auto-scaling factor, a power of two in [2^-32, 2^32] */
+  int margin;                /* scale margin, 0..64 */
+} fp8_adam_grad_cast;
+
+/*
+ * fp8_adam_step_into_castgrad -- the gradient cast and the out-of-place step
+ * in one pass: for every chunk, chunks[i].g points to the gradient as the wgrad
+ * wrote it, n bfloat16 values (FP8_DT_BF16 or FP8_DT_BF16_RTO), dev, 16-byte
+ * aligned; the step casts it to E5M2 in registers with the scale
+ * fp8_scale_cast(dW, FP8_E5M2, amax[i], margin, mu, ...) would derive --
+ * the same codes that call would store -- and runs fp8_adam_step_into on
+ * them.  The E5M2 gradient is never written: 2 B per parameter less traffic
+ * than the cast followed by the step, and one kernel less per tensor.
+ * chunks[i].g_inv (dev float) receives the gradient's inverse scale (what
+ * the cast writes to inv_scale_dev); its scale itself is not written.  A
+ * non-finite amax sets FP8_STATUS_NONFINITE (as the cast does).  All
+ * results are bit for bit those of fp8_scale_cast then fp8_adam_step_into.
+ * Arguments and errors otherwise as fp8_adam_step_into; FP8_ERR_INVALID_ARG
+ * also for a NULL gc, a NULL amax entry, a bad mu or margin.
+ */
+int fp8_adam_step_into_castgrad(const fp8_adam_chunk *chunks, const fp8_adam_dest *dest,
+                                const fp8_adam_grad_cast *gc, int nchunks, const fp8_adam_hparams *hp,
+                                void *workspace, size_t ws_bytes, void *stream);
+
 /*
  * Element-sharded step ([FP8-LM] 提案手法 O3: FP8 optimizer state under a
  * ZeRO-style partition).  fp8_adam_step in two halves so that ranks which

@@ -189,6 +189,32 @@ def test_adam_step_into_rejects_missing_or_aliased_destinations(lib):
         assert half(arr, dst, 1, ctypes.byref(hp), S, 32, None) == fp8.FP8_ERR_INVALID_ARG  # workspace
 
 
+def test_adam_castgrad_rejects_bad_arguments_on_the_host(lib):
+    """The step with the gradient cast in its pass: a NULL gc or amax array, a
+    NULL amax entry, a bad mu or margin are refused before any launch."""
+    from fp8_mixed_precision_tensor_b200 import fp8
+
+    p, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    G, M, V, W, S = 0x10000, 0x20000, 0x30000, 0x40000, 0x50000
+    arr = (fp8._Chunk * 1)()
+    arr[0] = fp8._Chunk(G, S, M, S, V, S, W, S, 64, None, None, None, None)
+    dst = (fp8._Dest * 1)()
+    dst[0] = fp8._Dest(0x60000, 0x70000, 0x80000)
+    hp = fp8._HParams(1e-4, 0.9, 0.95, 1e-8, 1, 0)
+    fn = lib.fp8_adam_step_into_castgrad
+    fn.argtypes = [ctypes.POINTER(fp8._Chunk), ctypes.POINTER(fp8._Dest), ctypes.POINTER(fp8._GradCast), i,
+                   ctypes.POINTER(fp8._HParams), p, sz, p]
+    amax = (ctypes.c_void_p * 1)(S)
+    none = (ctypes.c_void_p * 1)(None)
+    good = fp8._GradCast(ctypes.cast(amax, ctypes.POINTER(ctypes.c_void_p)), 1024.0, 0)
+    assert fn(arr, dst, None, 1, ctypes.byref(hp), S, 64, None) == fp8.FP8_ERR_INVALID_ARG
+    assert fn(arr, None, ctypes.byref(good), 1, ctypes.byref(hp), S, 64, None) == fp8.FP8_ERR_INVALID_ARG
+    for gc in (fp8._GradCast(None, 1024.0, 0), fp8._GradCast(ctypes.cast(none, ctypes.POINTER(ctypes.c_void_p)), 1024.0, 0),
+               fp8._GradCast(ctypes.cast(amax, ctypes.POINTER(ctypes.c_void_p)), 3.0, 0),
+               fp8._GradCast(ctypes.cast(amax, ctypes.POINTER(ctypes.c_void_p)), 1024.0, 65)):
+        assert fn(arr, dst, ctypes.byref(gc), 1, ctypes.byref(hp), S, 64, None) == fp8.FP8_ERR_INVALID_ARG
+
+
 def test_reciprocal_selftest_rejects_bad_arguments_on_the_host(lib):
     fn = lib.fp8_selftest_step_reciprocal
     fn.argtypes = [ctypes.c_uint, ctypes.c_ulonglong, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]

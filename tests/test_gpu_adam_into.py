@@ -15,7 +15,7 @@ import numpy as np
 import pytest
 import torch
 
-from fp8_mixed_precision_tensor_b200 import fp8
+from fp8_mixed_precision_tensor_b200 import fp8, synth
 
 from test_gpu_parity import (F32, HP, MAX_TIES, _stored_amax, _with_tracking, check_adam_chunk, make_adam_state,
                              scalar, snapshot)
@@ -208,3 +208,59 @@ def test_adam_sharded_into_ranks_equal_whole_tensor_step(world):
                 assert (mine.m_scale.item(), mine.v_scale.item(), mine.w_scale.item()) == \
                     (s["s_m"], s["s_v"], s["s_w"]), (step, k)
                 assert (mine.wq_scale.item(), mine.wq_inv.item()) == (c.wq_scale.item(), c.wq_inv.item())
+
+
+@pytest.mark.parametrize("grad_margin,mu", [(0, 2.0 ** 10), (1, 1.0)])
+def test_adam_into_castgrad_equals_cast_then_step(grad_margin, mu):
+    """The gradient cast in the out-of-place pass (each chunk's g the bf16 dW,
+    its amax given): over three steps with fresh gradients, the new state,
+    scales, E4M3 copy and the gradient's inverse scale equal those of
+    fp8_scale_cast (bf16 dW -> E5M2, mu, margin) followed by the
+    out-of-place step on the stored codes, bit for bit -- chunks with ragged
+    ends, an empty chunk and a gradient of zeros; step 1 from zero moments
+    (every chunk redone)."""
+    sizes = [65536, 4099, 1, 0, 300000, 8192]
+    base = _with_tracking(make_adam_state(sizes, ("adam-castgrad", grad_margin)), wq=True, track=False)
+    ref, fus = IntoRunner(_clone(base)), IntoRunner(_clone(base))
+    f32 = dict(dtype=torch.float32, device="cuda")
+    for step in (1, 2, 3):
+        dws = [synth.device_normal((n,), 1e-3, 77 * step + i, torch.bfloat16, "cuda") for i, n in enumerate(sizes)]
+        dws[5].zero_()
+        amax = [torch.zeros(1, **f32) for _ in sizes]
+        for dw, a in zip(dws, amax):
+            fp8.fp8_amax(dw, a)
+        # reference: the gradient cast kernel, then the step on the stored codes
+        for c, dw, a in zip(ref.chunks, dws, amax):
+            s = torch.zeros(1, **f32)
+            fp8.fp8_scale_cast(dw, fp8.FP8_E5M2, a, grad_margin, mu, s, c.g_inv, c.g)
+        ref.step(step)
+        # fused: the same step reading the bf16 gradients
+        chunks = [fp8.AdamChunk(dw, c.g_inv, c.m, c.m_scale, c.v, c.v_scale, c.w, c.w_scale, None, c.wq,
+                                c.wq_scale, c.wq_inv) for c, dw in zip(fus.chunks, dws)]
+        fp8.fp8_adam_step_into_castgrad(chunks, fus.spare, amax, mu, grad_margin, step=step, margin=0,
+                                        workspace=fus.ws, **HP)
+        fus.chunks = [fp8.AdamChunk(c.g, c.g_inv, m, c.m_scale, v, c.v_scale, w, c.w_scale, None, c.wq, c.wq_scale,
+                                    c.wq_inv) for c, (m, v, w) in zip(fus.chunks, fus.spare)]
+        fus.spare = [(c.m, c.v, c.w) for c in chunks]
+        assert fp8.fp8_get_status() == 0
+        assert_same_state(ref.chunks, fus.chunks, step)
+        for r, f in zip(ref.chunks, fus.chunks):
+            assert r.g_inv.item() == f.g_inv.item(), step
+        if step == 1:
+            assert fus.redone()[[0, 1, 4]].all()
+
+
+def test_adam_into_castgrad_rejects_bad_arguments():
+    chunks = make_adam_state([64], ("adam-castgrad-bad",))
+    c = chunks[0]
+    dw = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
+    ch = [fp8.AdamChunk(dw, c.g_inv, c.m, c.m_scale, c.v, c.v_scale, c.w, c.w_scale)]
+    dst = [(torch.empty_like(c.m), torch.empty_like(c.v), torch.empty_like(c.w))]
+    ws = torch.zeros(16, **F32)
+    a = scalar()
+    with pytest.raises(fp8.FP8Error):  # mu not a power of two
+        fp8.fp8_adam_step_into_castgrad(ch, dst, [a], 3.0, 0, step=1, margin=0, workspace=ws, **HP)
+    with pytest.raises(fp8.FP8Error):  # margin out of range
+        fp8.fp8_adam_step_into_castgrad(ch, dst, [a], 1.0, 65, step=1, margin=0, workspace=ws, **HP)
+    with pytest.raises(ValueError):
+        fp8.fp8_adam_step_into_castgrad(ch, dst, [], 1.0, 0, step=1, margin=0, workspace=ws, **HP)

@@ -152,7 +152,16 @@ def test_adam_steps_write_only_their_outputs():
                                         for c, (m, v, w) in zip(chunks, dests)]
         dst = [(m.t, v.t, w.t) for m, v, w in dests] if step == 3 else [(c.m, c.v, c.w) for c in chunks]
         fp8.fp8_adam_step_into(src, dst, step=step, margin=0, workspace=ws.t, **HP)
+    # step 5 with the gradient cast in the pass (bf16 gradients): writes the first set again
+    dws = [torch.full((c.g.numel(),), 1e-3, dtype=torch.bfloat16, device="cuda") for c in chunks]
+    amax = [_f32(1, torch.tensor([1e-3])) for _ in chunks]
+    ginv = [_f32() for _ in chunks]
+    src = [fp8.AdamChunk(dw, gi.t, m.t, c.m_scale, v.t, c.v_scale, w.t, c.w_scale, None, c.wq, c.wq_scale,
+                         c.wq_inv) for c, dw, gi, (m, v, w) in zip(chunks, dws, ginv, dests)]
+    fp8.fp8_adam_step_into_castgrad(src, [(c.m, c.v, c.w) for c in chunks], [a.t for a in amax], 1024.0, 0,
+                                    step=5, margin=0, workspace=ws.t, **HP)
     assert fp8.fp8_get_status() == 0
     assert all(g.intact() for g in guards)
     assert all(b.intact() for d in dests for b in d)
+    assert all(g.intact() for g in ginv + amax)
     assert ws.intact()
